@@ -1,0 +1,572 @@
+"""Benchmark of one paged decode step on B200.
+
+A step is the whole hot path for one batch: copy-on-write block copies,
+the cache write of each sequence's new token, and paged decode attention.
+Default workload: Llama-2-7B-shaped single-layer decode (64 sequences,
+32 q / 32 kv heads, head_dim 128, block size 16, lengths U{128..2048},
+16384-block pool, placement by a seeded permutation).
+
+Prints one JSON line.  ``value`` is the step's algorithmic HBM bytes per
+second (inputs resident in HBM, timed on the device with CUDA events, max
+over ranks); ``e2e`` is the same metric measured through the public API
+with pinned host buffers (host allocator append, host->device copies of
+the step's inputs, the three launches, device->host read of the output).
+``roofline`` reports the decode call against the measured HBM copy peak;
+``cpu_baseline`` is the fp64 oracle timed on this host's cores on a
+bounded sample of the same workload.
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--config 1..5]
+    python bench.py --impl reference ...   (the oracle arm)
+"""
+from __future__ import annotations
+
+import argparse
+import hashlib
+import json
+import os
+import statistics
+import subprocess
+import sys
+import threading
+import time
+
+import numpy as np
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+if ROOT not in sys.path:
+    sys.path.insert(0, ROOT)
+
+import workloads as W  # noqa: E402
+
+METRIC = "paged decode: achieved HBM GB/s (% of B200 peak) and KV tokens attended/sec"
+NOMINAL_HBM_GBS = 8000.0
+FALLBACK_HBM_GBS = 6650.0
+
+WORKLOAD_NAMES = {
+    1: "tiny paged decode: B=4, lens {1,16,33,47}, 4 q / 2 kv heads, d=64, bs=16, 32-block pool",
+    2: "Llama-2-7B-shaped decode: B=64, 32 q / 32 kv heads, d=128, bs=16, lens U[128,2048], 16384-block pool",
+    3: "Llama-2-13B-shaped chat mix: B=128 (32 groups x n=4), 40/40 heads, d=128, bs=16, "
+       "len=U[100,2000]+U[50,500], 512-token shared prefix, CoW copies",
+    4: "Llama-3-8B-shaped GQA decode: B=256, 32 q / 8 kv heads, d=128, bs=32, lognormal lens (median 800, cap 4096)",
+    5: "long-context split-K decode: B=8, 64 q / 8 kv heads, d=128, bs=16, L=32768, 512-token partitions, "
+       "1024 copy pairs",
+}
+
+
+# ---------------------------------------------------------------------------
+# helpers
+# ---------------------------------------------------------------------------
+
+def _measured_peak():
+    path = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    try:
+        with open(path) as f:
+            d = json.load(f)
+        return float(d["hbm_gbs"]), "measured"
+    except Exception:
+        return FALLBACK_HBM_GBS, "fallback"
+
+
+def _decode_traffic_record():
+    """ncu DRAM traffic of the decode kernel for this workload, if taken on the current source."""
+    path = os.path.join(ROOT, "profiles", "decode_traffic.json")
+    try:
+        with open(path) as f:
+            rec = json.load(f)
+    except Exception:
+        return None
+    src = os.path.join(ROOT, "paged_kv_cache_349_b200", "csrc", "decode.cu")
+    with open(src, "rb") as f:
+        digest = hashlib.sha256(f.read()).hexdigest()
+    if rec.get("decode_cu_sha256") != digest:
+        return None
+    return rec
+
+
+def step_bytes(case):
+    """Algorithmic bytes of one step: (copy, write, decode)."""
+    bs, d, Hkv = case.block_size, case.head_dim, case.num_kv_heads
+    block_bytes = Hkv * bs * d * 2
+    copy = int(case.copy_pairs.shape[0]) * block_bytes * 2 * 2 + case.copy_pairs.size * 4
+    T = int(case.slot_mapping.size)
+    write = T * Hkv * d * 2 * 2 * 2 + T * 4
+    dec = W.algorithmic_decode_bytes(case)
+    return copy, write, dec
+
+
+class ClockSampler:
+    """nvidia-smi clocks and throttle reasons sampled every 200 ms in the background."""
+
+    FIELDS = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+              "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+              "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, device_index: int):
+        self.device_index = device_index
+        self.samples = []
+        self._stop = threading.Event()
+        self._proc = None
+
+    def start(self):
+        try:
+            self._proc = subprocess.Popen(
+                ["nvidia-smi", f"--id={self.device_index}", f"--query-gpu={self.FIELDS}",
+                 "--format=csv,noheader,nounits", "-lms", "200"],
+                stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
+        except Exception:
+            self._proc = None
+            return self
+        self._thread = threading.Thread(target=self._read, daemon=True)
+        self._thread.start()
+        return self
+
+    def _read(self):
+        for line in self._proc.stdout:
+            parts = [p.strip() for p in line.split(",")]
+            if len(parts) >= 9:
+                self.samples.append(parts)
+            if self._stop.is_set():
+                break
+
+    def stop(self):
+        self._stop.set()
+        if self._proc is not None:
+            self._proc.terminate()
+            try:
+                self._proc.wait(timeout=5)
+            except Exception:
+                self._proc.kill()
+        return self.summary()
+
+    def summary(self):
+        if not self.samples:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["unavailable"], "samples": 0}
+        sm = [float(s[1]) for s in self.samples if s[1].replace(".", "").isdigit()]
+        mx = [float(s[2]) for s in self.samples if s[2].replace(".", "").isdigit()]
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        reasons = set()
+        for s in self.samples:
+            for name, val in zip(names, s[5:9]):
+                if val.lower().startswith("active"):
+                    reasons.add(name)
+        return {"sm_mhz": statistics.median(sm) if sm else None, "sm_max_mhz": max(mx) if mx else None,
+                "reasons": sorted(reasons), "samples": len(self.samples)}
+
+
+def _dist_setup():
+    import torch
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    if world > 1:
+        import datetime
+        import torch.distributed as dist
+        backend = "nccl" if torch.cuda.is_available() else "gloo"
+        if torch.cuda.is_available():
+            torch.cuda.set_device(local)
+        dist.init_process_group(backend, timeout=datetime.timedelta(seconds=120))
+    elif torch.cuda.is_available():
+        torch.cuda.set_device(local)
+    return world, rank, local
+
+
+def _max_over_ranks(x: float, world: int) -> float:
+    if world == 1:
+        return x
+    import torch
+    import torch.distributed as dist
+    t = torch.tensor([x], dtype=torch.float64, device="cuda" if torch.cuda.is_available() else "cpu")
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
+
+
+def _sum_over_ranks(x: float, world: int) -> float:
+    if world == 1:
+        return x
+    import torch
+    import torch.distributed as dist
+    t = torch.tensor([x], dtype=torch.float64, device="cuda" if torch.cuda.is_available() else "cpu")
+    dist.all_reduce(t, op=dist.ReduceOp.SUM)
+    return float(t.item())
+
+
+def _barrier(world: int):
+    if world > 1:
+        import torch.distributed as dist
+        dist.barrier()
+
+
+# ---------------------------------------------------------------------------
+# CPU oracle baseline (the only place the bench runs the oracle)
+# ---------------------------------------------------------------------------
+
+def cpu_baseline(case, budget_s: float = 12.0):
+    """Time the fp64 oracle on a bounded sample of (sequence, kv head) units of ``case``.
+
+    Returns the oracle's throughput in the bench's unit (algorithmic GB/s),
+    the threads it used and what the sample was.
+    """
+    import oracle
+    threads = len(os.sched_getaffinity(0))
+    oracle.set_num_threads(threads)
+    G = case.group_size
+    rng = np.random.default_rng(7)
+    units = [(int(b), int(h)) for b in rng.permutation(case.batch) for h in rng.permutation(case.num_kv_heads)]
+    # calibrate on a few units, then size the sample to the budget
+    done_units, done_bytes, elapsed = 0, 0, 0.0
+    chunk = max(1, threads)
+    while done_units < len(units) and elapsed < budget_s:
+        sel = units[done_units:done_units + chunk]
+        rows = np.array([(b, h * G + g) for b, h in sel for g in range(G)], np.int32)
+        t0 = time.perf_counter()
+        oracle.decode(case.q, case.k_cache, case.v_cache, case.block_tables, case.seq_lens,
+                      num_kv_heads=case.num_kv_heads, block_size=case.block_size, scale=case.scale, rows=rows)
+        dt = time.perf_counter() - t0
+        elapsed += dt
+        done_units += len(sel)
+        done_bytes += sum(int(case.seq_lens[b]) * case.head_dim * 4 + G * case.head_dim * 6 for b, _ in sel)
+        if dt < budget_s / 20:
+            chunk *= 2
+    gbs = done_bytes / elapsed / 1e9
+    sample = (f"{done_units} of {len(units)} (sequence, kv head) units of the same workload "
+              f"({done_units * G} query-head rows, {done_bytes / 1e6:.1f} MB of K/V/q/out), "
+              f"{elapsed:.1f} s of oracle time")
+    return gbs, threads, sample, elapsed, done_bytes
+
+
+# ---------------------------------------------------------------------------
+# native arm
+# ---------------------------------------------------------------------------
+
+def run_native(args):
+    import torch
+
+    import paged_kv_cache_349_b200 as pa
+
+    world, rank, local = _dist_setup()
+    torch.cuda.set_device(local)
+    cfg = args.config
+    seed = 1000 + cfg + 7919 * rank  # weak scaling: every rank owns its own batch
+    case = W.make_case(cfg, seed=seed, fill=W.BF16_ZERO)
+    copy_b, write_b, dec_b = step_bytes(case)
+    total_b = copy_b + write_b + dec_b
+    kv_tokens = int(case.seq_lens.sum())
+
+    def bf16(a):
+        return torch.from_numpy(np.ascontiguousarray(a).view(np.int16)).view(torch.bfloat16).cuda()
+
+    def i32(a):
+        return torch.from_numpy(np.ascontiguousarray(a, dtype=np.int32)).cuda()
+
+    k, v = bf16(case.k_cache), bf16(case.v_cache)
+    q = bf16(case.q)
+    k_new, v_new = bf16(case.k_new), bf16(case.v_new)
+    slots = i32(case.slot_mapping)
+    pairs = i32(case.copy_pairs.reshape(-1, 2))
+    tables, lens = i32(case.block_tables), i32(case.seq_lens)
+    out = torch.empty(case.q.shape, dtype=torch.float32, device="cuda")
+    flag = torch.zeros(1, dtype=torch.int32, device="cuda")
+    pt = case.partition_tokens
+    resolved_pt = pa.pa_decode_partition_tokens(case.batch, case.num_q_heads, case.num_kv_heads,
+                                                case.head_dim, case.block_size, case.max_seq_len, pt)
+    ws_bytes = pa.pa_decode_workspace_size(case.batch, case.num_q_heads, case.num_kv_heads, case.head_dim,
+                                           case.block_size, case.max_seq_len, pt)
+    ws = torch.empty(max(ws_bytes, 16), dtype=torch.uint8, device="cuda")
+    stream = torch.cuda.current_stream()
+
+    dec_ev = []
+
+    def step(record=False):
+        if case.copy_pairs.shape[0]:
+            pa.pa_copy_blocks(k, v, pairs, err_flag=flag, stream=stream)
+        pa.pa_reshape_and_cache(k_new, v_new, k, v, slots, err_flag=flag, stream=stream)
+        if record:
+            e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+            e0.record(stream)
+        pa.pa_decode(out, q, k, v, tables, lens, max_seq_len=case.max_seq_len, scale=float(case.scale),
+                     partition_tokens=pt, workspace=ws, err_flag=flag, stream=stream)
+        if record:
+            e1.record(stream)
+            dec_ev.append((e0, e1))
+
+    for _ in range(args.warmup):
+        step()
+    torch.cuda.synchronize()
+    assert int(flag.item()) == 0, f"error flag {int(flag.item()):#x}"
+
+    sampler = ClockSampler(torch.cuda.current_device()).start() if rank == 0 else None
+    time.sleep(0.3 if sampler else 0)
+    _barrier(world)
+    torch.cuda.synchronize()
+    launches0 = pa.launch_count()
+    t0 = torch.cuda.Event(enable_timing=True)
+    t1 = torch.cuda.Event(enable_timing=True)
+    t0.record(stream)
+    for _ in range(args.steps):
+        step(record=True)
+    t1.record(stream)
+    torch.cuda.synchronize()
+    _barrier(world)
+    launches = pa.launch_count() - launches0
+    clocks = sampler.stop() if sampler else None
+    ms_local = t0.elapsed_time(t1)
+    ms = _max_over_ranks(ms_local, world)
+    dec_ms = statistics.mean(a.elapsed_time(b) for a, b in dec_ev)
+    dec_ms = _max_over_ranks(dec_ms, world)
+    assert int(flag.item()) == 0, f"error flag {int(flag.item()):#x}"
+
+    all_bytes = _sum_over_ranks(float(total_b), world)
+    all_tokens = _sum_over_ranks(float(kv_tokens), world)
+    step_s = ms / 1e3 / args.steps
+    value = all_bytes / step_s / 1e9
+    peak, peak_kind = _measured_peak()
+    achieved = dec_b / (dec_ms / 1e3) / 1e9
+
+    e2e = run_e2e(args, case, pa, stream, world, k, v) if not args.no_e2e else None
+
+    traffic = None
+    rec = _decode_traffic_record()
+    if rec and rec.get("config") == cfg:
+        traffic = rec.get("traffic_bytes_per_launch")
+
+    line = {
+        "metric": METRIC,
+        "value": round(value, 1),
+        "unit": "GB/s",
+        "n_gpus": world,
+        "steps": args.steps,
+        "warmup": args.warmup,
+        "ms_per_step": round(ms / args.steps, 4),
+        "higher_is_better": True,
+        "scaling": "weak",
+        "vs_baseline": None,
+        "dtype": "bf16",
+        "accumulate": "fp32",
+        "data": "synthetic (seeded bf16 N(0,1) K/V/q, seeded placement)",
+        "config": {
+            "workload": WORKLOAD_NAMES[cfg],
+            "config_index": cfg,
+            "batch_per_gpu": case.batch,
+            "global_batch": case.batch * world,
+            "kv_tokens_per_gpu": kv_tokens,
+            "partition_tokens": resolved_pt,
+            "parallelism": f"dp{world} (independent sequences per GPU, no collective)",
+            "l2": f"inputs larger than L2: {dec_b / 1e9:.2f} GB of K/V per step vs 126 MB L2; no flush",
+        },
+        "pct_of_peak": {"nominal_8TBps": round(100 * value / NOMINAL_HBM_GBS, 1),
+                        f"{peak_kind}_{peak:.0f}GBps": round(100 * value / peak, 1)},
+        "kv_tokens_per_s": round(all_tokens / step_s, 1),
+        "kv_head_tokens_per_s": round(all_tokens * case.num_kv_heads / step_s, 1),
+        "step_bytes": {"copy": copy_b, "write": write_b, "decode": dec_b},
+        "gpu_launches": launches,
+        "roofline": {
+            "kernel": "pa_decode" + (" (split kernel + LSE reduce)" if resolved_pt > 0 else " (single pass)"),
+            "bound": "hbm",
+            "achieved": round(achieved, 1),
+            "peak": peak,
+            "peak_kind": f"{peak_kind} (HBM copy)",
+            "unit": "GB/s",
+            "frac": round(achieved / peak, 4),
+            "traffic": traffic,
+            "algorithmic_bytes_per_launch": dec_b,
+            "launch_ms": round(dec_ms, 5),
+        },
+        "e2e": e2e,
+        "clocks": clocks,
+    }
+    if rank == 0 and world == 1 and not args.no_cpu_baseline:
+        gbs, cores, sample, _, _ = cpu_baseline(case, budget_s=args.cpu_budget)
+        line["cpu_baseline"] = {"value": round(gbs, 4), "unit": "GB/s", "cores": cores, "kind": "oracle",
+                                "sample": sample}
+    if rank == 0:
+        print(json.dumps(line), flush=True)
+    if world > 1:
+        import torch.distributed as dist
+        dist.destroy_process_group()
+
+
+def replay_allocator(pa, case):
+    """Rebuild the workload's tables with the host allocator (state before the step's append).
+
+    Blocks are dealt in the generator's order; for the n=4 chat workload each
+    group's prompt prefix is appended once, forked three times, and every
+    member then appends its own tokens (members 0..2 copy the partial shared
+    block on their first write, member 3 writes in place).
+    """
+    alloc = pa.Allocator(case.num_blocks, case.block_size, order=case.free_order)
+    sids = np.zeros(case.batch, np.int32)
+    if case.groups is None:
+        for b, L in enumerate(case.seq_lens):
+            s = alloc.create()
+            sids[b] = s
+            for _ in range(max(int(L) - 1, 0)):
+                alloc.append(s)
+        return alloc, sids
+    for g in range(int(case.groups.max()) + 1):
+        members = np.nonzero(case.groups == g)[0]
+        root = alloc.create()
+        for _ in range(int(case.shared_tokens[members[0]])):
+            alloc.append(root)
+        ids = [alloc.fork(root) for _ in range(len(members) - 1)] + [root]
+        for b, s in zip(members, ids):
+            sids[b] = s
+            for _ in range(int(case.seq_lens[b]) - 1 - int(case.shared_tokens[b])):
+                alloc.append(s)
+    return alloc, sids
+
+
+def run_e2e(args, case, pa, stream, world, k_pool, v_pool):
+    """The same step through the public API with host buffers (pinned), timed end to end."""
+    import torch
+    bs = case.block_size
+    steps, warm = args.steps, args.warmup
+    grow = steps + warm + 1
+    alloc, sids = replay_allocator(pa, case)
+    max_blocks = case.max_blocks_per_seq + (grow + bs - 1) // bs + 1
+    max_len_cap = case.max_seq_len + grow
+
+    h_q = torch.from_numpy(np.ascontiguousarray(case.q).view(np.int16)).view(torch.bfloat16).pin_memory()
+    h_k = torch.from_numpy(np.ascontiguousarray(case.k_new).view(np.int16)).view(torch.bfloat16).pin_memory()
+    h_v = torch.from_numpy(np.ascontiguousarray(case.v_new).view(np.int16)).view(torch.bfloat16).pin_memory()
+    h_tables = torch.empty((case.batch, max_blocks), dtype=torch.int32).pin_memory()
+    h_lens = torch.empty(case.batch, dtype=torch.int32).pin_memory()
+    h_slots = torch.empty(case.batch, dtype=torch.int32).pin_memory()
+    h_pairs = torch.empty((case.batch, 2), dtype=torch.int32).pin_memory()
+    h_out = torch.empty(case.q.shape, dtype=torch.float32).pin_memory()
+    d_q = torch.empty_like(h_q, device="cuda")
+    d_k = torch.empty_like(h_k, device="cuda")
+    d_v = torch.empty_like(h_v, device="cuda")
+    d_tables = torch.empty_like(h_tables, device="cuda")
+    d_lens = torch.empty_like(h_lens, device="cuda")
+    d_slots = torch.empty_like(h_slots, device="cuda")
+    d_pairs = torch.empty_like(h_pairs, device="cuda")
+    d_out = torch.empty_like(h_out, device="cuda")
+    ws_bytes = pa.pa_decode_workspace_size(case.batch, case.num_q_heads, case.num_kv_heads, case.head_dim,
+                                           bs, max_len_cap, case.partition_tokens)
+    ws = torch.empty(max(ws_bytes, 16), dtype=torch.uint8, device="cuda")
+    # the pools stay resident: they are the cache, not an input of the step
+    tables_np = h_tables.numpy()
+    lens_np = h_lens.numpy()
+    flag = torch.zeros(1, dtype=torch.int32, device="cuda")
+    bytes_acc = {"h2d": 0, "d2h": 0, "alg": 0, "tokens": 0}
+
+    def e2e_step(count):
+        slots, pairs = alloc.append_batch(sids)
+        t, lens = alloc.export(sids, max_blocks)
+        tables_np[:] = t
+        lens_np[:] = lens
+        h_slots.numpy()[:] = slots
+        n_pairs = pairs.shape[0]
+        if n_pairs:
+            h_pairs.numpy()[:n_pairs] = pairs
+        max_len = int(lens.max())
+        d_q.copy_(h_q, non_blocking=True)
+        d_k.copy_(h_k, non_blocking=True)
+        d_v.copy_(h_v, non_blocking=True)
+        d_slots.copy_(h_slots, non_blocking=True)
+        d_tables.copy_(h_tables, non_blocking=True)
+        d_lens.copy_(h_lens, non_blocking=True)
+        if n_pairs:
+            d_pairs[:n_pairs].copy_(h_pairs[:n_pairs], non_blocking=True)
+            pa.pa_copy_blocks(k_pool, v_pool, d_pairs[:n_pairs], err_flag=flag, stream=stream)
+        pa.pa_reshape_and_cache(d_k, d_v, k_pool, v_pool, d_slots, err_flag=flag, stream=stream)
+        pa.pa_decode(d_out, d_q, k_pool, v_pool, d_tables, d_lens, max_seq_len=max_len, scale=float(case.scale),
+                     partition_tokens=case.partition_tokens, workspace=ws, err_flag=flag, stream=stream)
+        h_out.copy_(d_out, non_blocking=True)
+        stream.synchronize()  # the step's result is on the host
+        if count:
+            bytes_acc["h2d"] += sum(t.numel() * t.element_size() for t in (h_q, h_k, h_v, h_slots, h_tables, h_lens))
+            bytes_acc["h2d"] += n_pairs * 8
+            bytes_acc["d2h"] += h_out.numel() * 4
+            bytes_acc["tokens"] += int(lens.sum())
+            c, w, d = step_bytes_from(case, lens, n_pairs)
+            bytes_acc["alg"] += c + w + d
+
+    for _ in range(warm):
+        e2e_step(False)
+    _barrier(world)
+    torch.cuda.synchronize()
+    t0 = time.perf_counter()
+    for _ in range(steps):
+        e2e_step(True)
+    dt = time.perf_counter() - t0
+    dt = _max_over_ranks(dt, world)
+    assert int(flag.item()) == 0
+    alg = _sum_over_ranks(float(bytes_acc["alg"]), world)
+    alloc.close()
+    return {"value": round(alg / dt / 1e9, 1), "unit": "GB/s",
+            "ms_per_step": round(dt * 1e3 / steps, 4),
+            "h2d_bytes_per_step": bytes_acc["h2d"] // steps, "d2h_bytes_per_step": bytes_acc["d2h"] // steps,
+            "kv_tokens_per_s": round(_sum_over_ranks(float(bytes_acc["tokens"]), world) / dt, 1),
+            "includes": "host allocator append + table export, H2D of q/k_new/v_new/slots/tables/lens, "
+                        "copy/write/decode launches, D2H of out"}
+
+
+def step_bytes_from(case, lens, n_pairs):
+    bs, d, Hkv = case.block_size, case.head_dim, case.num_kv_heads
+    copy = n_pairs * Hkv * bs * d * 2 * 2 * 2
+    T = int(lens.size)
+    write = T * Hkv * d * 2 * 2 * 2 + T * 4
+    dec = W.algorithmic_decode_bytes(lens, num_q_heads=case.num_q_heads, num_kv_heads=Hkv, head_dim=d,
+                                     block_size=bs)
+    return copy, write, dec
+
+
+# ---------------------------------------------------------------------------
+# reference arm: the fp64 oracle on the host cores
+# ---------------------------------------------------------------------------
+
+def run_reference(args):
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    if rank != 0:
+        return
+    cfg = args.config
+    case = W.make_case(cfg, fill=W.BF16_ZERO)
+    per_step = max(1.0, args.cpu_budget / max(1, args.steps + args.warmup))
+    for _ in range(args.warmup):
+        cpu_baseline(case, budget_s=per_step / 4)
+    vals, secs, nbytes = [], 0.0, 0
+    sample = ""
+    cores = 0
+    for _ in range(args.steps):
+        gbs, cores, sample, el, by = cpu_baseline(case, budget_s=per_step)
+        vals.append(gbs)
+        secs += el
+        nbytes += by
+    value = nbytes / secs / 1e9
+    line = {
+        "metric": METRIC, "value": round(value, 4), "unit": "GB/s", "n_gpus": world,
+        "steps": args.steps, "warmup": args.warmup, "ms_per_step": round(secs * 1e3 / args.steps, 2),
+        "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64",
+        "data": "synthetic (seeded bf16 N(0,1) K/V/q, seeded placement)",
+        "config": {"workload": WORKLOAD_NAMES[cfg], "config_index": cfg, "batch_per_gpu": case.batch},
+        "impl": "reference",
+        "cpu_baseline": {"value": round(value, 4), "unit": "GB/s", "cores": cores, "kind": "oracle",
+                         "sample": "per step: " + sample},
+        "e2e": {"value": round(value, 4), "unit": "GB/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
+    }
+    print(json.dumps(line), flush=True)
+
+
+def main():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=20)
+    ap.add_argument("--warmup", type=int, default=5)
+    ap.add_argument("--config", type=int, default=2, choices=[1, 2, 3, 4, 5])
+    ap.add_argument("--impl", choices=["native", "reference"], default="native")
+    ap.add_argument("--no-e2e", action="store_true")
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--cpu-budget", type=float, default=12.0, help="seconds of oracle time")
+    args = ap.parse_args()
+    if args.warmup < 3:
+        ap.error("--warmup must be at least 3")
+    if args.impl == "reference":
+        run_reference(args)
+    else:
+        run_native(args)
+
+
+if __name__ == "__main__":
+    main()

@@ -1,0 +1,221 @@
+/*
+ * pa.h -- C ABI of the paged KV-cache decode library (NVIDIA B200, sm_100a).
+ *
+ * The library implements the data-parallel hot path of PagedAttention:
+ *
+ *   - a shared pool of fixed-size KV blocks addressed through per-request
+ *     block tables ("PagedAttention & vLLM" (fp-ai-systems.pages.dev),
+ *     section "The insight: KV cache as virtual memory"),
+ *   - the cache-append write through a slot mapping ("Walk through paged
+ *     attention end to end" (zenaique.com), conceptual
+ *     paged_attention_decode, append step),
+ *   - single-query decode attention that dereferences the block table for
+ *     every attended position (same page, attention step; "What is
+ *     PagedAttention and how does it manage KV cache" (n4n.ai), section
+ *     "How PagedAttention works": two-level indirection, tokens contiguous
+ *     inside a block),
+ *   - the copy-on-write block copy ("PagedAttention & vLLM", section
+ *     "Copy-on-write sharing"),
+ *   - a host-side refcounted block allocator with fork and copy-on-write.
+ *
+ * Conventions shared by every entry point
+ * ---------------------------------------
+ *  - Every function returns an int status (pa_status).  Argument errors are
+ *    detected on the host, before any launch, and nothing is launched.
+ *    A failed launch returns PA_ERR_CUDA.
+ *  - Device pointers are caller-owned device memory of the current CUDA
+ *    device.  The library allocates no device memory; the caller provides
+ *    the decode workspace (size from pa_decode_workspace_size).
+ *  - `stream` is a cudaStream_t passed as void*; NULL is the legacy default
+ *    stream.  Device work is asynchronous on that stream.
+ *  - Data-dependent index errors (a slot, block id or copy pair out of range,
+ *    a sequence longer than its table) never fault: the offending access is
+ *    skipped and a PA_FLAG_* bit is OR-ed into *err_flag (an int32 in device
+ *    memory; may be NULL to skip reporting).  The caller reads it when it
+ *    chooses to.  Bounded waits inside kernels that run out set
+ *    PA_FLAG_TIMEOUT the same way.  Kernels never trap.
+ *  - Pool layout (both K and V, separate allocations):
+ *        bf16 [num_blocks, num_kv_heads, block_size, head_dim], row-major,
+ *    base address 16-byte aligned.  One (block, kv head) tile of
+ *    block_size x head_dim values is contiguous.
+ *  - Supported shapes: bf16 only; head_dim in {64, 128}; block_size in
+ *    {16, 32}; num_q_heads / num_kv_heads in {1, 2, 4, 8}.
+ *  - A slot is physical_block * block_size + row_in_block.
+ */
+#ifndef PA_H
+#define PA_H
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef enum {
+    PA_OK = 0,
+    PA_ERR_INVALID_ARG = 1, /* null pointer, bad size, misaligned buffer, ... */
+    PA_ERR_UNSUPPORTED = 2, /* shape outside the supported set */
+    PA_ERR_CUDA = 3,        /* a CUDA runtime call or launch failed */
+    PA_ERR_BAD_INDEX = 4,   /* host allocator: unknown sequence / block id */
+    PA_ERR_TIMEOUT = 5,     /* reserved for host-side waits */
+    PA_ERR_OOM = 6,         /* host allocator: pool exhausted (state unchanged) */
+    PA_ERR_STATE = 7        /* operation not valid in the current state */
+} pa_status;
+
+/* Bits OR-ed into the device error flag by kernels. */
+#define PA_FLAG_BAD_SLOT 0x1    /* reshape: slot outside [0, num_blocks*block_size), not -1 */
+#define PA_FLAG_BAD_BLOCK 0x2   /* decode: block id outside [0, num_blocks) */
+#define PA_FLAG_BAD_PAIR 0x4    /* copy: src or dst outside [0, num_blocks) */
+#define PA_FLAG_BAD_LEN 0x8     /* decode: seq_len < 0, > max_seq_len, or > table capacity */
+#define PA_FLAG_TIMEOUT 0x10    /* a bounded in-kernel wait ran out */
+
+/* Human-readable name of a status code (static string, never NULL). */
+const char *pa_status_string(int status);
+
+/* Library version, major*10000 + minor*100 + patch. */
+int pa_version(void);
+
+/* Number of kernels this library has launched in the process so far. */
+uint64_t pa_launch_count(void);
+
+/* ------------------------------------------------------------------------
+ * Cache write ("Walk through paged attention end to end", conceptual
+ * paged_attention_decode: the new token's K and V go to block
+ * table[-1] at offset next_pos % block_size).
+ *
+ *   k_cache[s / bs, h, s % bs, :] = k_new[t, h, :]   for s = slot_mapping[t]
+ *   v_cache[s / bs, h, s % bs, :] = v_new[t, h, :]
+ *
+ * k_new, v_new   : device bf16 [num_tokens, num_kv_heads, head_dim], 16-byte aligned
+ * k_cache,v_cache: device bf16 pools (layout above)
+ * slot_mapping   : device int32 [num_tokens]; -1 = skip (padding token);
+ *                  other values outside [0, num_blocks*block_size) set
+ *                  PA_FLAG_BAD_SLOT and are skipped.
+ * Distinct tokens must name distinct slots (otherwise the winner is
+ * unspecified).  num_tokens == 0 launches nothing.  Bit-exact copy.
+ * ---------------------------------------------------------------------- */
+int pa_reshape_and_cache(const void *k_new, const void *v_new, void *k_cache, void *v_cache,
+                         const int32_t *slot_mapping, int num_tokens, int64_t num_blocks,
+                         int num_kv_heads, int block_size, int head_dim, int32_t *err_flag,
+                         void *stream);
+
+/* ------------------------------------------------------------------------
+ * Copy-on-write block copy ("PagedAttention & vLLM", Copy-on-write sharing:
+ * duplicate just that one block, then write).
+ *
+ * For each pair i: block pairs[2i+1] of both pools becomes a bit copy of
+ * block pairs[2i] (all heads, rows and dims).
+ *
+ * pairs : device int32 [num_pairs, 2] = (src, dst).  Destinations must be
+ *         distinct and must not appear as sources in the same call (a source
+ *         may repeat).  Ids outside [0, num_blocks) set PA_FLAG_BAD_PAIR and
+ *         the pair is skipped.  num_pairs == 0 launches nothing.
+ * ---------------------------------------------------------------------- */
+int pa_copy_blocks(void *k_cache, void *v_cache, const int32_t *pairs, int num_pairs,
+                   int64_t num_blocks, int num_kv_heads, int block_size, int head_dim,
+                   int32_t *err_flag, void *stream);
+
+/* ------------------------------------------------------------------------
+ * Paged decode attention.  For every sequence b and query head g, with
+ * kv head h = g / (num_q_heads / num_kv_heads) and L = seq_lens[b]:
+ *
+ *   s_p   = scale * q[b,g,:] . K_h[p,:]          p = 0 .. L-1
+ *   out   = sum_p exp(s_p - max s) V_h[p,:] / sum_p exp(s_p - max s)
+ *
+ * where row p of sequence b is pool[block_tables[b, p / bs], h, p % bs, :]
+ * ("Walk through paged attention end to end", attention step; the math is
+ * standard attention, only the addressing changes).  L = 0 yields zeros.
+ * seq_lens counts the token appended in this step (append, then attend).
+ *
+ * out           : device fp32 [batch, num_q_heads, head_dim]
+ * q             : device bf16 [batch, num_q_heads, head_dim], 16-byte aligned
+ * block_tables  : device int32 [batch, max_blocks_per_seq]; only entries
+ *                 j < ceil(L/bs) are read (padding may hold anything)
+ * seq_lens      : device int32 [batch]
+ * max_seq_len   : host-side upper bound of seq_lens (sizes the split grid);
+ *                 longer sequences set PA_FLAG_BAD_LEN and are truncated.
+ * scale         : softmax scale (usually 1/sqrt(head_dim))
+ * partition_tokens : 0 = library default for this shape, -1 = one pass per
+ *                 (sequence, kv head), > 0 = split each sequence into
+ *                 partitions of this many tokens (a multiple of block_size)
+ *                 whose partial softmax states are merged by a second
+ *                 log-sum-exp reduce kernel.
+ * workspace     : device scratch of at least pa_decode_workspace_size(...)
+ *                 bytes, 16-byte aligned (may be NULL if that size is 0).
+ * Each (sequence, kv head) is processed by one CTA (per partition) that
+ * serves all query heads of the group, so every K/V byte is read once.
+ * ---------------------------------------------------------------------- */
+size_t pa_decode_workspace_size(int batch, int num_q_heads, int num_kv_heads, int head_dim,
+                                int block_size, int max_seq_len, int partition_tokens);
+
+/* The partition size pa_decode will use for these arguments (-1 = one pass). */
+int pa_decode_partition_tokens(int batch, int num_q_heads, int num_kv_heads, int head_dim,
+                               int block_size, int max_seq_len, int partition_tokens);
+
+int pa_decode(float *out, const void *q, const void *k_cache, const void *v_cache,
+              const int32_t *block_tables, int max_blocks_per_seq, const int32_t *seq_lens,
+              int batch, int max_seq_len, int num_q_heads, int num_kv_heads, int head_dim,
+              int block_size, int64_t num_blocks, float scale, int partition_tokens,
+              void *workspace, size_t workspace_bytes, int32_t *err_flag, void *stream);
+
+/* ------------------------------------------------------------------------
+ * Host block allocator (owns host memory only; not thread-safe).
+ *
+ * append  : the token at position n of a sequence goes to logical block
+ *           n / block_size, row n % block_size; a fresh block is taken from
+ *           the free pool when n % block_size == 0 ("Walk through paged
+ *           attention end to end", append step; "What is PagedAttention",
+ *           BlockTable.append_token).  Writing into a block whose refcount
+ *           is above one first moves the sequence to a fresh copy and
+ *           reports the (src, dst) pair the caller must pass to
+ *           pa_copy_blocks before the cache write ("PagedAttention & vLLM",
+ *           Copy-on-write sharing).  The last owner writes in place.
+ * fork    : the child references every block of the parent, the partially
+ *           filled last one included; each refcount grows by one.
+ * free    : refcounts drop; blocks that reach zero return to the pool at
+ *           once, no compaction ("What is PagedAttention", chat workload
+ *           example).
+ * On PA_ERR_OOM the allocator state is unchanged.
+ * ---------------------------------------------------------------------- */
+typedef struct pa_allocator pa_allocator;
+
+/* Pool of num_blocks blocks handed out in id order 0, 1, 2, ... */
+int pa_alloc_create(int num_blocks, int block_size, pa_allocator **out);
+/* Same, but fresh blocks are handed out in the order order[0], order[1], ...
+ * (order must be a permutation of 0..num_blocks-1; host memory, copied). */
+int pa_alloc_create_ordered(int num_blocks, int block_size, const int32_t *order,
+                            pa_allocator **out);
+void pa_alloc_destroy(pa_allocator *alloc);
+
+int pa_seq_create(pa_allocator *alloc, int *seq_id);
+/* Append one token.  *slot_out = slot of the new token; (*cow_src, *cow_dst)
+ * = the block copy required first, or (-1, -1).  cow_* may be NULL only if
+ * the caller knows no copy can be needed (no forks). */
+int pa_seq_append(pa_allocator *alloc, int seq_id, int32_t *slot_out, int32_t *cow_src,
+                  int32_t *cow_dst);
+/* Append one token to each of seq_ids[0..n) in order (a decode step).
+ * slots_out[i] receives the slot of seq_ids[i]; cow_pairs_out (capacity n
+ * pairs, int32 [n,2]) receives the required copies, *n_cow their count.
+ * All-or-nothing: on PA_ERR_OOM nothing changed. */
+int pa_seq_append_batch(pa_allocator *alloc, const int32_t *seq_ids, int n, int32_t *slots_out,
+                        int32_t *cow_pairs_out, int *n_cow);
+int pa_seq_fork(pa_allocator *alloc, int parent_id, int *child_id);
+int pa_seq_free(pa_allocator *alloc, int seq_id);
+/* Copy a sequence's block table into out[0..cap); *n_blocks and *n_tokens
+ * receive its sizes.  PA_ERR_INVALID_ARG if cap < *n_blocks. */
+int pa_seq_block_table(const pa_allocator *alloc, int seq_id, int32_t *out, int cap,
+                       int *n_blocks, int *n_tokens);
+/* Export tables of seq_ids[0..n) as a padded int32 [n, max_blocks] array
+ * (unused entries = pad) plus int32 seq_lens[n]; host memory. */
+int pa_alloc_export(const pa_allocator *alloc, const int32_t *seq_ids, int n, int32_t *tables,
+                    int max_blocks, int32_t pad, int32_t *seq_lens);
+int pa_alloc_num_free(const pa_allocator *alloc);
+/* Reference count of a block (0 = free), or -1 for an id out of range. */
+int pa_block_refcount(const pa_allocator *alloc, int32_t block);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* PA_H */

@@ -1,0 +1,252 @@
+"""B200-native paged KV-cache decode: Python binding of ``libpa.so``.
+
+Argument marshalling only: every function below turns torch tensors (or
+host numpy arrays for the allocator) into the plain pointers and sizes of
+the C ABI declared in ``include/pa.h`` and raises ``PaError`` on a non-zero
+status.  All device work runs in the library's CUDA kernels.
+
+Device ops (names as in the C ABI):
+    pa_reshape_and_cache, pa_copy_blocks, pa_decode,
+    pa_decode_workspace_size, pa_decode_partition_tokens
+Host allocator:
+    Allocator (pa_alloc_* / pa_seq_* / pa_block_refcount)
+"""
+from __future__ import annotations
+
+import ctypes
+from typing import Optional, Sequence, Tuple
+
+import numpy as np
+
+from ._lib import lib
+
+PA_OK = 0
+PA_ERR_INVALID_ARG = 1
+PA_ERR_UNSUPPORTED = 2
+PA_ERR_CUDA = 3
+PA_ERR_BAD_INDEX = 4
+PA_ERR_TIMEOUT = 5
+PA_ERR_OOM = 6
+PA_ERR_STATE = 7
+
+PA_FLAG_BAD_SLOT = 0x1
+PA_FLAG_BAD_BLOCK = 0x2
+PA_FLAG_BAD_PAIR = 0x4
+PA_FLAG_BAD_LEN = 0x8
+PA_FLAG_TIMEOUT = 0x10
+
+
+class PaError(RuntimeError):
+    def __init__(self, status: int, where: str):
+        self.status = status
+        super().__init__(f"{where}: {lib.pa_status_string(status).decode()} ({status})")
+
+
+def _check(status: int, where: str) -> None:
+    if status != PA_OK:
+        raise PaError(status, where)
+
+
+def status_string(status: int) -> str:
+    return lib.pa_status_string(status).decode()
+
+
+def version() -> int:
+    return lib.pa_version()
+
+
+def launch_count() -> int:
+    """Kernels the library has launched in this process."""
+    return int(lib.pa_launch_count())
+
+
+# ---------------------------------------------------------------------------
+# Device ops (torch tensors in, pointers out)
+# ---------------------------------------------------------------------------
+
+def _torch():
+    import torch
+    return torch
+
+
+def _dev(t, dtype, name):
+    torch = _torch()
+    if not isinstance(t, torch.Tensor) or not t.is_cuda:
+        raise TypeError(f"{name} must be a CUDA tensor")
+    if t.dtype != dtype:
+        raise TypeError(f"{name} must be {dtype}, got {t.dtype}")
+    if not t.is_contiguous():
+        raise ValueError(f"{name} must be contiguous")
+    return ctypes.c_void_p(t.data_ptr())
+
+
+def _opt_flag(err_flag):
+    if err_flag is None:
+        return None
+    return _dev(err_flag, _torch().int32, "err_flag")
+
+
+def _stream(stream):
+    torch = _torch()
+    if stream is None:
+        return ctypes.c_void_p(torch.cuda.current_stream().cuda_stream)
+    if isinstance(stream, int):
+        return ctypes.c_void_p(stream)
+    return ctypes.c_void_p(stream.cuda_stream)
+
+
+def pa_reshape_and_cache(k_new, v_new, k_cache, v_cache, slot_mapping, err_flag=None, stream=None) -> None:
+    """Write k_new/v_new [T, Hkv, d] into the pools [NB, Hkv, bs, d] at slot_mapping [T]."""
+    torch = _torch()
+    T, Hkv, d = k_new.shape
+    NB, Hkv2, bs, d2 = k_cache.shape
+    if (Hkv2, d2) != (Hkv, d) or v_new.shape != k_new.shape or v_cache.shape != k_cache.shape:
+        raise ValueError("shape mismatch")
+    if slot_mapping.numel() != T:
+        raise ValueError("slot_mapping must have one entry per token")
+    _check(lib.pa_reshape_and_cache(
+        _dev(k_new, torch.bfloat16, "k_new"), _dev(v_new, torch.bfloat16, "v_new"),
+        _dev(k_cache, torch.bfloat16, "k_cache"), _dev(v_cache, torch.bfloat16, "v_cache"),
+        _dev(slot_mapping, torch.int32, "slot_mapping"), T, NB, Hkv, bs, d,
+        _opt_flag(err_flag), _stream(stream)), "pa_reshape_and_cache")
+
+
+def pa_copy_blocks(k_cache, v_cache, pairs, err_flag=None, stream=None) -> None:
+    """Copy whole blocks src -> dst in both pools; pairs is int32 [n, 2] on the device."""
+    torch = _torch()
+    NB, Hkv, bs, d = k_cache.shape
+    n = pairs.shape[0] if pairs.dim() == 2 else pairs.numel() // 2
+    if n and (pairs.numel() != 2 * n):
+        raise ValueError("pairs must be [n, 2]")
+    _check(lib.pa_copy_blocks(
+        _dev(k_cache, torch.bfloat16, "k_cache"), _dev(v_cache, torch.bfloat16, "v_cache"),
+        _dev(pairs, torch.int32, "pairs") if n else None, n, NB, Hkv, bs, d,
+        _opt_flag(err_flag), _stream(stream)), "pa_copy_blocks")
+
+
+def pa_decode_workspace_size(batch, num_q_heads, num_kv_heads, head_dim, block_size, max_seq_len,
+                             partition_tokens=0) -> int:
+    return int(lib.pa_decode_workspace_size(batch, num_q_heads, num_kv_heads, head_dim, block_size,
+                                            max_seq_len, partition_tokens))
+
+
+def pa_decode_partition_tokens(batch, num_q_heads, num_kv_heads, head_dim, block_size, max_seq_len,
+                               partition_tokens=0) -> int:
+    return int(lib.pa_decode_partition_tokens(batch, num_q_heads, num_kv_heads, head_dim, block_size,
+                                              max_seq_len, partition_tokens))
+
+
+def pa_decode(out, q, k_cache, v_cache, block_tables, seq_lens, *, max_seq_len: int, scale: float,
+              partition_tokens: int = 0, workspace=None, err_flag=None, stream=None) -> None:
+    """Paged decode: out fp32 [B, Hq, d] <- attention of q bf16 [B, Hq, d] over the pools.
+
+    block_tables int32 [B, max_blocks], seq_lens int32 [B] (device tensors);
+    ``workspace`` is a uint8 CUDA tensor of at least ``pa_decode_workspace_size`` bytes.
+    """
+    torch = _torch()
+    B, Hq, d = q.shape
+    NB, Hkv, bs, d2 = k_cache.shape
+    if d2 != d or out.shape != q.shape or v_cache.shape != k_cache.shape:
+        raise ValueError("shape mismatch")
+    if block_tables.dim() != 2 or block_tables.shape[0] != B or seq_lens.numel() != B:
+        raise ValueError("block_tables must be [B, max_blocks] and seq_lens [B]")
+    ws_ptr, ws_bytes = None, 0
+    if workspace is not None:
+        ws_ptr = _dev(workspace, workspace.dtype, "workspace")
+        ws_bytes = workspace.numel() * workspace.element_size()
+    _check(lib.pa_decode(
+        _dev(out, torch.float32, "out"), _dev(q, torch.bfloat16, "q"),
+        _dev(k_cache, torch.bfloat16, "k_cache"), _dev(v_cache, torch.bfloat16, "v_cache"),
+        _dev(block_tables, torch.int32, "block_tables"), block_tables.shape[1],
+        _dev(seq_lens, torch.int32, "seq_lens"), B, int(max_seq_len), Hq, Hkv, d, bs, NB,
+        float(scale), int(partition_tokens), ws_ptr, ws_bytes, _opt_flag(err_flag),
+        _stream(stream)), "pa_decode")
+
+
+# ---------------------------------------------------------------------------
+# Host allocator
+# ---------------------------------------------------------------------------
+
+def _np_ptr(a: np.ndarray):
+    return a.ctypes.data_as(ctypes.c_void_p)
+
+
+class Allocator:
+    """Refcounted block allocator with fork and copy-on-write (host memory only)."""
+
+    def __init__(self, num_blocks: int, block_size: int, order: Optional[Sequence[int]] = None):
+        h = ctypes.c_void_p()
+        if order is None:
+            _check(lib.pa_alloc_create(num_blocks, block_size, ctypes.byref(h)), "pa_alloc_create")
+        else:
+            o = np.ascontiguousarray(order, dtype=np.int32)
+            if o.size != num_blocks:
+                raise ValueError("order must list every block once")
+            _check(lib.pa_alloc_create_ordered(num_blocks, block_size, _np_ptr(o), ctypes.byref(h)),
+                   "pa_alloc_create_ordered")
+        self._h = h
+        self.num_blocks = num_blocks
+        self.block_size = block_size
+
+    def close(self) -> None:
+        if self._h:
+            lib.pa_alloc_destroy(self._h)
+            self._h = ctypes.c_void_p()
+
+    def __del__(self):
+        try:
+            self.close()
+        except Exception:
+            pass
+
+    def create(self) -> int:
+        sid = ctypes.c_int()
+        _check(lib.pa_seq_create(self._h, ctypes.byref(sid)), "pa_seq_create")
+        return sid.value
+
+    def append(self, seq_id: int) -> Tuple[int, Optional[Tuple[int, int]]]:
+        slot, src, dst = ctypes.c_int32(), ctypes.c_int32(), ctypes.c_int32()
+        _check(lib.pa_seq_append(self._h, seq_id, ctypes.byref(slot), ctypes.byref(src), ctypes.byref(dst)),
+               "pa_seq_append")
+        return slot.value, ((src.value, dst.value) if src.value >= 0 else None)
+
+    def append_batch(self, seq_ids) -> Tuple[np.ndarray, np.ndarray]:
+        ids = np.ascontiguousarray(seq_ids, dtype=np.int32)
+        slots = np.empty(ids.size, dtype=np.int32)
+        pairs = np.empty((max(ids.size, 1), 2), dtype=np.int32)
+        n = ctypes.c_int()
+        _check(lib.pa_seq_append_batch(self._h, _np_ptr(ids), ids.size, _np_ptr(slots), _np_ptr(pairs),
+                                       ctypes.byref(n)), "pa_seq_append_batch")
+        return slots, pairs[:n.value].copy()
+
+    def fork(self, parent: int) -> int:
+        c = ctypes.c_int()
+        _check(lib.pa_seq_fork(self._h, parent, ctypes.byref(c)), "pa_seq_fork")
+        return c.value
+
+    def free(self, seq_id: int) -> None:
+        _check(lib.pa_seq_free(self._h, seq_id), "pa_seq_free")
+
+    def block_table(self, seq_id: int) -> Tuple[np.ndarray, int]:
+        nb, nt = ctypes.c_int(), ctypes.c_int()
+        st = lib.pa_seq_block_table(self._h, seq_id, None, 0, ctypes.byref(nb), ctypes.byref(nt))
+        if st not in (PA_OK, PA_ERR_INVALID_ARG):
+            _check(st, "pa_seq_block_table")
+        out = np.empty(max(nb.value, 1), dtype=np.int32)
+        _check(lib.pa_seq_block_table(self._h, seq_id, _np_ptr(out), out.size, ctypes.byref(nb),
+                                      ctypes.byref(nt)), "pa_seq_block_table")
+        return out[:nb.value].copy(), nt.value
+
+    def export(self, seq_ids, max_blocks: int, pad: int = -1) -> Tuple[np.ndarray, np.ndarray]:
+        ids = np.ascontiguousarray(seq_ids, dtype=np.int32)
+        tables = np.empty((ids.size, max_blocks), dtype=np.int32)
+        lens = np.empty(ids.size, dtype=np.int32)
+        _check(lib.pa_alloc_export(self._h, _np_ptr(ids), ids.size, _np_ptr(tables), max_blocks, pad,
+                                   _np_ptr(lens)), "pa_alloc_export")
+        return tables, lens
+
+    def num_free(self) -> int:
+        return int(lib.pa_alloc_num_free(self._h))
+
+    def refcount(self, block: int) -> int:
+        return int(lib.pa_block_refcount(self._h, block))

@@ -1,0 +1,58 @@
+"""ctypes loader for ``libpa.so`` (the CUDA library built from ``csrc/``).
+
+There is no fallback: if the library cannot be loaded (or built with nvcc
+when it is missing), importing the package fails.
+"""
+from __future__ import annotations
+
+import ctypes
+import os
+
+from . import build as _build
+
+_P = ctypes.c_void_p
+_I = ctypes.c_int
+_I64 = ctypes.c_int64
+_U64 = ctypes.c_uint64
+_SZ = ctypes.c_size_t
+_F = ctypes.c_float
+_PI = ctypes.POINTER(ctypes.c_int)
+
+# name -> (restype, argtypes); mirrors include/pa.h
+SIGNATURES = {
+    "pa_status_string": (ctypes.c_char_p, [_I]),
+    "pa_version": (_I, []),
+    "pa_launch_count": (_U64, []),
+    "pa_reshape_and_cache": (_I, [_P, _P, _P, _P, _P, _I, _I64, _I, _I, _I, _P, _P]),
+    "pa_copy_blocks": (_I, [_P, _P, _P, _I, _I64, _I, _I, _I, _P, _P]),
+    "pa_decode_workspace_size": (_SZ, [_I, _I, _I, _I, _I, _I, _I]),
+    "pa_decode_partition_tokens": (_I, [_I, _I, _I, _I, _I, _I, _I]),
+    "pa_decode": (_I, [_P, _P, _P, _P, _P, _I, _P, _I, _I, _I, _I, _I, _I, _I64, _F, _I, _P, _SZ, _P, _P]),
+    "pa_alloc_create": (_I, [_I, _I, ctypes.POINTER(_P)]),
+    "pa_alloc_create_ordered": (_I, [_I, _I, _P, ctypes.POINTER(_P)]),
+    "pa_alloc_destroy": (None, [_P]),
+    "pa_seq_create": (_I, [_P, _PI]),
+    "pa_seq_append": (_I, [_P, _I, _P, _P, _P]),
+    "pa_seq_append_batch": (_I, [_P, _P, _I, _P, _P, _PI]),
+    "pa_seq_fork": (_I, [_P, _I, _PI]),
+    "pa_seq_free": (_I, [_P, _I]),
+    "pa_seq_block_table": (_I, [_P, _I, _P, _I, _PI, _PI]),
+    "pa_alloc_export": (_I, [_P, _P, _I, _P, _I, ctypes.c_int32, _P]),
+    "pa_alloc_num_free": (_I, [_P]),
+    "pa_block_refcount": (_I, [_P, ctypes.c_int32]),
+}
+
+
+def load() -> ctypes.CDLL:
+    path = _build.LIB
+    if not os.path.exists(path):
+        _build.build()
+    lib = ctypes.CDLL(path)
+    for name, (res, args) in SIGNATURES.items():
+        fn = getattr(lib, name)
+        fn.restype = res
+        fn.argtypes = args
+    return lib
+
+
+lib = load()

@@ -1,0 +1,124 @@
+// Cache write (slot mapping) and copy-on-write block copy.
+//
+// Both are pure data movement and HBM-bound: 16-byte vector loads and
+// stores, several in flight per thread, grids sized from the work.
+#include "pa_common.cuh"
+
+namespace pa {
+namespace {
+
+// One thread moves one 16-byte chunk of one (token, kv head) row of K and of V
+// to slot_mapping[token] ("Walk through paged attention end to end", append
+// step: write_kv_to_pool(last_block, offset)).
+__global__ void __launch_bounds__(256) reshape_and_cache_kernel(
+    const uint4 *__restrict__ k_new, const uint4 *__restrict__ v_new, uint4 *__restrict__ k_cache,
+    uint4 *__restrict__ v_cache, const int32_t *__restrict__ slot_mapping, int num_tokens,
+    int64_t num_slots, int num_kv_heads, int block_size, int chunks_per_row,
+    int32_t *__restrict__ err_flag) {
+    const int64_t idx = (int64_t)blockIdx.x * blockDim.x + threadIdx.x;
+    const int64_t per_token = (int64_t)num_kv_heads * chunks_per_row;
+    if (idx >= (int64_t)num_tokens * per_token) return;
+    const int t = (int)(idx / per_token);
+    const int rem = (int)(idx - (int64_t)t * per_token);
+    const int h = rem / chunks_per_row;
+    const int c = rem - h * chunks_per_row;
+    const int64_t slot = __ldg(slot_mapping + t);
+    if (slot == -1) return;
+    if (slot < 0 || slot >= num_slots) {
+        if (rem == 0) raise_flag(err_flag, PA_FLAG_BAD_SLOT);
+        return;
+    }
+    const int64_t blk = slot / block_size;
+    const int64_t row = slot - blk * block_size;
+    const int64_t dst = ((blk * num_kv_heads + h) * block_size + row) * chunks_per_row + c;
+    const uint4 kv = __ldg(k_new + idx);
+    const uint4 vv = __ldg(v_new + idx);
+    k_cache[dst] = kv;
+    v_cache[dst] = vv;
+}
+
+constexpr int kCopyThreads = 256;
+constexpr int kCopyUnroll = 4;  // 16-byte chunks in flight per thread
+
+// grid.x: pair * groups_per_block + chunk group, grid.y: 0 = K pool, 1 = V pool.
+// Copies block src -> dst ("PagedAttention & vLLM", Copy-on-write sharing).
+__global__ void __launch_bounds__(kCopyThreads) copy_blocks_kernel(
+    uint4 *__restrict__ k_cache, uint4 *__restrict__ v_cache, const int32_t *__restrict__ pairs,
+    int64_t num_blocks, int64_t chunks_per_block, int groups_per_block,
+    int32_t *__restrict__ err_flag) {
+    const int pair = blockIdx.x / groups_per_block;
+    const int group = blockIdx.x - pair * groups_per_block;
+    const int64_t src = __ldg(pairs + 2 * pair);
+    const int64_t dst = __ldg(pairs + 2 * pair + 1);
+    if (src < 0 || src >= num_blocks || dst < 0 || dst >= num_blocks) {
+        if (group == 0 && blockIdx.y == 0 && threadIdx.x == 0) raise_flag(err_flag, PA_FLAG_BAD_PAIR);
+        return;
+    }
+    uint4 *pool = blockIdx.y == 0 ? k_cache : v_cache;
+    const uint4 *from = pool + src * chunks_per_block;
+    uint4 *to = pool + dst * chunks_per_block;
+    const int64_t base = (int64_t)group * (kCopyThreads * kCopyUnroll) + threadIdx.x;
+    uint4 buf[kCopyUnroll];
+#pragma unroll
+    for (int u = 0; u < kCopyUnroll; ++u) {
+        const int64_t i = base + (int64_t)u * kCopyThreads;
+        if (i < chunks_per_block) buf[u] = __ldcs(from + i);
+    }
+#pragma unroll
+    for (int u = 0; u < kCopyUnroll; ++u) {
+        const int64_t i = base + (int64_t)u * kCopyThreads;
+        if (i < chunks_per_block) __stcs(to + i, buf[u]);
+    }
+}
+
+}  // namespace
+}  // namespace pa
+
+extern "C" {
+
+int pa_reshape_and_cache(const void *k_new, const void *v_new, void *k_cache, void *v_cache,
+                         const int32_t *slot_mapping, int num_tokens, int64_t num_blocks,
+                         int num_kv_heads, int block_size, int head_dim, int32_t *err_flag,
+                         void *stream) {
+    if (num_tokens < 0 || num_blocks <= 0 || num_kv_heads <= 0) return PA_ERR_INVALID_ARG;
+    if (head_dim != 64 && head_dim != 128) return PA_ERR_UNSUPPORTED;
+    if (block_size != 16 && block_size != 32) return PA_ERR_UNSUPPORTED;
+    if (num_tokens == 0) return PA_OK;
+    if (!k_new || !v_new || !k_cache || !v_cache || !slot_mapping) return PA_ERR_INVALID_ARG;
+    if (!pa::aligned16(k_new) || !pa::aligned16(v_new) || !pa::aligned16(k_cache) ||
+        !pa::aligned16(v_cache))
+        return PA_ERR_INVALID_ARG;
+    const int chunks = head_dim / 8;
+    const int64_t total = (int64_t)num_tokens * num_kv_heads * chunks;
+    const int threads = 256;
+    const int64_t grid = (total + threads - 1) / threads;
+    if (grid > 0x7fffffffLL) return PA_ERR_INVALID_ARG;
+    pa::reshape_and_cache_kernel<<<(unsigned)grid, threads, 0, (cudaStream_t)stream>>>(
+        (const uint4 *)k_new, (const uint4 *)v_new, (uint4 *)k_cache, (uint4 *)v_cache,
+        slot_mapping, num_tokens, num_blocks * block_size, num_kv_heads, block_size, chunks,
+        err_flag);
+    pa::count_launch();
+    return pa::launch_status();
+}
+
+int pa_copy_blocks(void *k_cache, void *v_cache, const int32_t *pairs, int num_pairs,
+                   int64_t num_blocks, int num_kv_heads, int block_size, int head_dim,
+                   int32_t *err_flag, void *stream) {
+    if (num_pairs < 0 || num_blocks <= 0 || num_kv_heads <= 0) return PA_ERR_INVALID_ARG;
+    if (head_dim != 64 && head_dim != 128) return PA_ERR_UNSUPPORTED;
+    if (block_size != 16 && block_size != 32) return PA_ERR_UNSUPPORTED;
+    if (num_pairs == 0) return PA_OK;
+    if (!k_cache || !v_cache || !pairs) return PA_ERR_INVALID_ARG;
+    if (!pa::aligned16(k_cache) || !pa::aligned16(v_cache)) return PA_ERR_INVALID_ARG;
+    const int64_t chunks = (int64_t)num_kv_heads * block_size * head_dim / 8;
+    const int64_t per_cta = pa::kCopyThreads * pa::kCopyUnroll;
+    const int64_t groups = (chunks + per_cta - 1) / per_cta;
+    if (groups * num_pairs > 0x7fffffffLL) return PA_ERR_INVALID_ARG;
+    dim3 grid((unsigned)(groups * num_pairs), 2);
+    pa::copy_blocks_kernel<<<grid, pa::kCopyThreads, 0, (cudaStream_t)stream>>>(
+        (uint4 *)k_cache, (uint4 *)v_cache, pairs, num_blocks, chunks, (int)groups, err_flag);
+    pa::count_launch();
+    return pa::launch_status();
+}
+
+}  // extern "C"

@@ -1,0 +1,544 @@
+// Paged decode attention for sm_100a.
+//
+// What it computes ("Walk through paged attention end to end", attention
+// step): for each sequence b and query head g, softmax(scale * q K^T) V over
+// the sequence's L tokens, where token p lives in block
+// block_tables[b][p / bs] at row p % bs of the pool ("What is PagedAttention
+// and how does it manage KV cache", How PagedAttention works: two-level
+// indirection, tokens contiguous inside a block).
+//
+// How it runs on B200:
+//  * One CTA per (kv head h, sequence b[, sequence partition]) serves all G
+//    query heads of the group, so each K/V byte leaves HBM once.
+//  * The sequence is cut into 16-token tiles.  A producer warp dereferences
+//    the block table and stages each tile's K and V (16 rows x head_dim
+//    bf16, contiguous in the pool) into shared memory with TMA tile loads
+//    (128-byte swizzle, no multicast) through an 8-deep mbarrier ring.
+//  * Four consumer warps take tiles round-robin.  Per tile a warp computes
+//    S^T = K_tile Q^T with bf16 mma.sync (M = 16 tokens, N = 8 query-head
+//    columns, K = head_dim), runs an online softmax in fp32 (log2 domain),
+//    and accumulates O^T += V_tile^T P^T with a second mma (M = 16 dims,
+//    N = 8 heads, K = 16 tokens).  P is split into bf16 hi + lo parts so the
+//    PV product keeps ~16 mantissa bits.
+//  * Warps merge their (max, sum, O) states through shared memory.  In the
+//    split variant each CTA writes its partition's state to the workspace
+//    and a log-sum-exp reduce kernel combines the partitions.
+#include <mutex>
+
+#include "pa_common.cuh"
+
+namespace pa {
+namespace {
+
+constexpr int kTileTokens = 16;
+constexpr int kConsumerWarps = 4;
+constexpr int kThreads = (kConsumerWarps + 1) * 32;
+constexpr int kStages = 8;
+constexpr int kBoxBytes = kTileTokens * 128;  // one 64-wide bf16 column box of a tile
+constexpr float kLog2e = 1.4426950408889634f;
+
+template <int HEAD_DIM>
+struct Cfg {
+    static constexpr int kBoxes = HEAD_DIM / 64;
+    static constexpr int kTileBytes = kBoxes * kBoxBytes;  // K or V of one tile
+    static constexpr int kStageBytes = 2 * kTileBytes;
+    static constexpr int kRingBytes = kStages * kStageBytes;
+    static constexpr int kMergeBytes = kConsumerWarps * 8 * (HEAD_DIM + 2) * 4;
+    static_assert(kMergeBytes <= kRingBytes, "merge area reuses the ring");
+    static constexpr int kSmemBytes = 1024 /*align slack*/ + kRingBytes + kStages * 8 * 2 + kStages * 4;
+};
+
+struct DecodeParams {
+    float *out;                 // [B, Hq, d]            (single pass)
+    float *part_o;              // [B, Hq, P, d]         (split)
+    float *part_ml;             // [B, Hq, P, 2]         (split)
+    const uint16_t *q;          // [B, Hq, d] bf16
+    const int32_t *block_tables;
+    const int32_t *seq_lens;
+    int32_t *err_flag;
+    int64_t num_blocks;
+    int max_blocks;
+    int max_seq_len;
+    int num_q_heads;
+    int num_kv_heads;
+    int group;
+    int block_size;
+    int part_tokens;            // tokens per CTA along the sequence
+    int num_parts;
+    float scale_log2;           // softmax scale * log2(e)
+};
+
+// Sequence length as every kernel of one call sees it: out-of-contract values
+// are clamped (and reported once by the caller of this helper).
+__device__ __forceinline__ int clamp_len(int L, const DecodeParams &p) {
+    const int cap = min(p.max_seq_len, p.max_blocks * p.block_size);
+    return L < 0 ? 0 : (L > cap ? cap : L);
+}
+
+// Byte offset of 16-byte chunk c of token row r inside one TMA-swizzled tile.
+__device__ __forceinline__ uint32_t tile_offset(int r, int c) {
+    return (uint32_t)((c >> 3) * kBoxBytes + r * 128 + (((c & 7) ^ (r & 7)) << 4));
+}
+
+template <int HEAD_DIM, bool SPLIT>
+__global__ void __launch_bounds__(kThreads) paged_decode_kernel(
+    const __grid_constant__ CUtensorMap k_map, const __grid_constant__ CUtensorMap v_map,
+    const DecodeParams p) {
+    using C = Cfg<HEAD_DIM>;
+    extern __shared__ uint8_t smem_raw[];
+    uint8_t *smem = reinterpret_cast<uint8_t *>(
+        (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~static_cast<uintptr_t>(1023));
+    uint64_t *full = reinterpret_cast<uint64_t *>(smem + C::kRingBytes);
+    uint64_t *empty = full + kStages;
+    int *tile_ok = reinterpret_cast<int *>(empty + kStages);
+
+    const int part = blockIdx.x;
+    const int h = blockIdx.y;
+    const int b = blockIdx.z;
+    const int warp = threadIdx.x >> 5;
+    const int lane = threadIdx.x & 31;
+
+    const int L_raw = __ldg(p.seq_lens + b);
+    const int L = clamp_len(L_raw, p);
+    const int tok_begin = part * p.part_tokens;
+    const int tok_end = min(L, tok_begin + p.part_tokens);
+    const int n_tiles = tok_end > tok_begin ? (tok_end - tok_begin + kTileTokens - 1) / kTileTokens : 0;
+    if (SPLIT && n_tiles == 0) return;  // empty partition: the reduce skips it
+    if (threadIdx.x == 0 && part == 0 && h == 0 && L != L_raw) raise_flag(p.err_flag, PA_FLAG_BAD_LEN);
+
+    if (threadIdx.x == 0) {
+        for (int s = 0; s < kStages; ++s) {
+            mbar_init(&full[s], 1);
+            mbar_init(&empty[s], 1);
+        }
+        fence_mbar_init();
+    }
+    __syncthreads();
+
+    // Per consumer thread: softmax state of query-head columns 2t, 2t+1.
+    const int gid = lane >> 2;  // mma group id
+    const int tig = lane & 3;   // thread in group
+    float m_run[2] = {-INFINITY, -INFINITY};
+    float l_run[2] = {0.f, 0.f};
+    float o[HEAD_DIM / 16][4];
+#pragma unroll
+    for (int mt = 0; mt < HEAD_DIM / 16; ++mt) o[mt][0] = o[mt][1] = o[mt][2] = o[mt][3] = 0.f;
+
+    if (warp == kConsumerWarps) {
+        // ---------------- producer: block-table dereference + TMA ----------------
+        if (lane == 0) {
+            prefetch_tensormap(&k_map);
+            prefetch_tensormap(&v_map);
+            const uint64_t policy = l2_policy_evict_first();
+            const int32_t *table = p.block_tables + (int64_t)b * p.max_blocks;
+            int issued = 0;
+            for (int i = 0; i < n_tiles; ++i) {
+                const int s = i % kStages;
+                if (i >= kStages && !mbar_wait_bounded(&empty[s], ((i / kStages) - 1) & 1, p.err_flag))
+                    break;
+                const int tok0 = tok_begin + i * kTileTokens;
+                const int j = tok0 / p.block_size;
+                const int row = tok0 - j * p.block_size;
+                const int64_t phys = __ldg(table + j);
+                issued = i + 1;
+                if (phys < 0 || phys >= p.num_blocks) {
+                    raise_flag(p.err_flag, PA_FLAG_BAD_BLOCK);
+                    tile_ok[s] = 0;
+                    mbar_arrive(&full[s]);
+                    continue;
+                }
+                tile_ok[s] = 1;
+                const int y = (int)((phys * p.num_kv_heads + h) * p.block_size + row);
+                uint8_t *dst = smem + s * C::kStageBytes;
+                mbar_arrive_expect_tx(&full[s], C::kStageBytes);
+#pragma unroll
+                for (int bx = 0; bx < C::kBoxes; ++bx)
+                    tma_load_2d(dst + bx * kBoxBytes, &k_map, bx * 64, y, &full[s], policy);
+#pragma unroll
+                for (int bx = 0; bx < C::kBoxes; ++bx)
+                    tma_load_2d(dst + C::kTileBytes + bx * kBoxBytes, &v_map, bx * 64, y, &full[s],
+                                policy);
+            }
+            // Drain: every issued tile has landed before the ring is reused or the CTA exits.
+            for (int i = max(0, issued - kStages); i < issued; ++i)
+                if (!mbar_wait_bounded(&full[i % kStages], (i / kStages) & 1, p.err_flag)) break;
+        }
+    } else {
+        // ---------------- consumers ----------------
+        const int G = p.group;
+        // Q^T as mma B fragments (k = head dim, permuted; n = query head column gid).
+        uint32_t qf[HEAD_DIM / 16][2];
+        if (gid < G) {
+            const uint4 *qrow = reinterpret_cast<const uint4 *>(
+                p.q + ((int64_t)b * p.num_q_heads + (int64_t)h * G + gid) * HEAD_DIM);
+#pragma unroll
+            for (int j = 0; j < HEAD_DIM / 32; ++j) {
+                const uint4 v = __ldg(qrow + 4 * j + tig);
+                qf[2 * j][0] = v.x;
+                qf[2 * j][1] = v.y;
+                qf[2 * j + 1][0] = v.z;
+                qf[2 * j + 1][1] = v.w;
+            }
+        } else {
+#pragma unroll
+            for (int k = 0; k < HEAD_DIM / 16; ++k) qf[k][0] = qf[k][1] = 0u;
+        }
+        // Token row of mma row gid (gid+8 -> +8): this order keeps both the K
+        // fragment loads and the V ldmatrix reads free of bank conflicts.
+        const int tau = (gid >> 1) | ((gid & 1) << 2);
+        // ldmatrix row address pattern for V: matrix (lane>>3), row (lane&7).
+        const int v_row = ((lane & 7) >> 1 | ((lane & 1) << 2)) + (((lane >> 4) & 1) << 3);
+        const int v_chunk_hi = (lane >> 3) & 1;
+
+        for (int i = warp; i < n_tiles; i += kConsumerWarps) {
+            const int s = i % kStages;
+            const bool got = mbar_wait_bounded(&full[s], (i / kStages) & 1, p.err_flag);
+            if (!__all_sync(0xffffffffu, got)) break;
+            const int valid = min(kTileTokens, tok_end - (tok_begin + i * kTileTokens));
+            if (tile_ok[s]) {
+                const uint32_t kbase = smem_addr(smem + s * C::kStageBytes);
+                const uint32_t vbase = kbase + C::kTileBytes;
+                if (valid < kTileTokens) {
+                    // Rows past the sequence end hold stale data: zero them so
+                    // that P = 0 times V cannot produce NaN.
+                    const int lines = (kTileTokens - valid) * C::kBoxes;
+                    for (int x = lane; x < lines * 8; x += 32) {
+                        const int line = x >> 3;
+                        const int r = valid + line / C::kBoxes;
+                        const int bx = line % C::kBoxes;
+                        const uint32_t a = vbase + bx * kBoxBytes + r * 128 + ((x & 7) << 4);
+                        asm volatile("st.shared.v4.u32 [%0], {%1, %1, %1, %1};" ::"r"(a), "r"(0u)
+                                     : "memory");
+                    }
+                    __syncwarp();
+                }
+                // ---- S^T = K Q^T ----
+                float sacc[4] = {0.f, 0.f, 0.f, 0.f};
+#pragma unroll
+                for (int j = 0; j < HEAD_DIM / 32; ++j) {
+                    const int c = 4 * j + tig;
+                    const uint4 ka = lds128(kbase + tile_offset(tau, c));
+                    const uint4 kb = lds128(kbase + tile_offset(tau + 8, c));
+                    mma_bf16_16816(sacc, ka.x, kb.x, ka.y, kb.y, qf[2 * j][0], qf[2 * j][1]);
+                    mma_bf16_16816(sacc, ka.z, kb.z, ka.w, kb.w, qf[2 * j + 1][0], qf[2 * j + 1][1]);
+                }
+                // sacc: (token tau, col 2t), (tau, 2t+1), (tau+8, 2t), (tau+8, 2t+1)
+                const float s0 = tau < valid ? sacc[0] * p.scale_log2 : -INFINITY;
+                const float s1 = tau < valid ? sacc[1] * p.scale_log2 : -INFINITY;
+                const float s2 = tau + 8 < valid ? sacc[2] * p.scale_log2 : -INFINITY;
+                const float s3 = tau + 8 < valid ? sacc[3] * p.scale_log2 : -INFINITY;
+                float mx0 = fmaxf(s0, s2), mx1 = fmaxf(s1, s3);
+#pragma unroll
+                for (int off = 4; off < 32; off <<= 1) {
+                    mx0 = fmaxf(mx0, __shfl_xor_sync(0xffffffffu, mx0, off));
+                    mx1 = fmaxf(mx1, __shfl_xor_sync(0xffffffffu, mx1, off));
+                }
+                const float mn0 = fmaxf(m_run[0], mx0), mn1 = fmaxf(m_run[1], mx1);
+                const float a0 = fast_exp2(m_run[0] - mn0), a1 = fast_exp2(m_run[1] - mn1);
+                m_run[0] = mn0;
+                m_run[1] = mn1;
+                const float p0 = fast_exp2(s0 - mn0), p1 = fast_exp2(s1 - mn1);
+                const float p2 = fast_exp2(s2 - mn0), p3 = fast_exp2(s3 - mn1);
+                l_run[0] = l_run[0] * a0 + (p0 + p2);
+                l_run[1] = l_run[1] * a1 + (p1 + p3);
+                if (__any_sync(0xffffffffu, a0 != 1.f || a1 != 1.f)) {
+#pragma unroll
+                    for (int mt = 0; mt < HEAD_DIM / 16; ++mt) {
+                        o[mt][0] *= a0;
+                        o[mt][1] *= a1;
+                        o[mt][2] *= a0;
+                        o[mt][3] *= a1;
+                    }
+                }
+                // ---- P^T as B fragments: hi + lo bf16 parts ----
+                const uint32_t h01 = pack_bf16x2(p0, p1);
+                const uint32_t h23 = pack_bf16x2(p2, p3);
+                const uint32_t l01 = pack_bf16x2(p0 - bf16_lo_to_float(h01), p1 - bf16_hi_to_float(h01));
+                const uint32_t l23 = pack_bf16x2(p2 - bf16_lo_to_float(h23), p3 - bf16_hi_to_float(h23));
+                const uint32_t bh0 = movmatrix_trans(h01), bh1 = movmatrix_trans(h23);
+                const uint32_t bl0 = movmatrix_trans(l01), bl1 = movmatrix_trans(l23);
+                // ---- O^T += V^T P^T ----
+#pragma unroll
+                for (int mt = 0; mt < HEAD_DIM / 16; ++mt) {
+                    uint32_t a0r, a1r, a2r, a3r;
+                    ldmatrix_x4_trans(vbase + tile_offset(v_row, 2 * mt + v_chunk_hi), a0r, a1r, a2r, a3r);
+                    mma_bf16_16816(o[mt], a0r, a1r, a2r, a3r, bh0, bh1);
+                    mma_bf16_16816(o[mt], a0r, a1r, a2r, a3r, bl0, bl1);
+                }
+                if (valid < kTileTokens) fence_proxy_async_smem();
+            }
+            __syncwarp();
+            if (lane == 0) mbar_arrive(&empty[s]);
+        }
+        // Row sums over this warp's tokens (lanes with the same tig share a column).
+#pragma unroll
+        for (int off = 4; off < 32; off <<= 1) {
+            l_run[0] += __shfl_xor_sync(0xffffffffu, l_run[0], off);
+            l_run[1] += __shfl_xor_sync(0xffffffffu, l_run[1], off);
+        }
+    }
+
+    // ---------------- merge the warps' states (ring memory is free now) ----------------
+    __syncthreads();
+    float *mo = reinterpret_cast<float *>(smem);                      // [W][8][HEAD_DIM]
+    float *mm = mo + kConsumerWarps * 8 * HEAD_DIM;                   // [W][8]
+    float *ml = mm + kConsumerWarps * 8;                              // [W][8]
+    if (warp < kConsumerWarps) {
+        const int gid = lane >> 2, tig = lane & 3;
+        float *w0 = mo + (warp * 8 + 2 * tig) * HEAD_DIM;
+        float *w1 = w0 + HEAD_DIM;
+#pragma unroll
+        for (int mt = 0; mt < HEAD_DIM / 16; ++mt) {
+            w0[16 * mt + gid] = o[mt][0];
+            w1[16 * mt + gid] = o[mt][1];
+            w0[16 * mt + gid + 8] = o[mt][2];
+            w1[16 * mt + gid + 8] = o[mt][3];
+        }
+        if (gid == 0) {
+            mm[warp * 8 + 2 * tig] = m_run[0];
+            mm[warp * 8 + 2 * tig + 1] = m_run[1];
+            ml[warp * 8 + 2 * tig] = l_run[0];
+            ml[warp * 8 + 2 * tig + 1] = l_run[1];
+        }
+    }
+    __syncthreads();
+    const int G = p.group;
+    for (int x = threadIdx.x; x < G * HEAD_DIM; x += kThreads) {
+        const int n = x / HEAD_DIM;
+        const int d = x - n * HEAD_DIM;
+        float M = -INFINITY;
+#pragma unroll
+        for (int w = 0; w < kConsumerWarps; ++w) M = fmaxf(M, mm[w * 8 + n]);
+        float num = 0.f, den = 0.f;
+        if (M != -INFINITY) {
+#pragma unroll
+            for (int w = 0; w < kConsumerWarps; ++w) {
+                const float f = fast_exp2(mm[w * 8 + n] - M);
+                num += f * mo[(w * 8 + n) * HEAD_DIM + d];
+                den += f * ml[w * 8 + n];
+            }
+        }
+        const int64_t row = (int64_t)b * p.num_q_heads + (int64_t)h * G + n;
+        if (SPLIT) {
+            p.part_o[(row * p.num_parts + part) * HEAD_DIM + d] = num / den;
+            if (d == 0) {
+                p.part_ml[(row * p.num_parts + part) * 2] = M;
+                p.part_ml[(row * p.num_parts + part) * 2 + 1] = den;
+            }
+        } else {
+            p.out[row * HEAD_DIM + d] = den > 0.f ? num / den : 0.f;
+        }
+    }
+}
+
+// Log-sum-exp merge of the partitions of one (sequence, query head):
+//   out = sum_p 2^(m_p - M) l_p o_p / sum_p 2^(m_p - M) l_p,  M = max_p m_p.
+template <int HEAD_DIM>
+__global__ void __launch_bounds__(HEAD_DIM) lse_reduce_kernel(const DecodeParams p) {
+    const int hq = blockIdx.x;
+    const int b = blockIdx.y;
+    const int d = threadIdx.x;
+    const int L = clamp_len(__ldg(p.seq_lens + b), p);
+    const int n = (L + p.part_tokens - 1) / p.part_tokens;
+    const int64_t row = (int64_t)b * p.num_q_heads + hq;
+    const float *ml = p.part_ml + row * p.num_parts * 2;
+    const float *po = p.part_o + row * p.num_parts * HEAD_DIM + d;
+    float M = -INFINITY;
+    for (int i = 0; i < n; ++i) M = fmaxf(M, __ldg(ml + 2 * i));
+    float num = 0.f, den = 0.f;
+    if (M != -INFINITY) {
+        for (int i = 0; i < n; ++i) {
+            const float w = fast_exp2(__ldg(ml + 2 * i) - M) * __ldg(ml + 2 * i + 1);
+            num += w * __ldg(po + (int64_t)i * HEAD_DIM);
+            den += w;
+        }
+    }
+    p.out[row * HEAD_DIM + d] = den > 0.f ? num / den : 0.f;
+}
+
+// ---------------------------------------------------------------------------
+// Host helpers
+// ---------------------------------------------------------------------------
+
+using EncodeTiledFn = decltype(&cuTensorMapEncodeTiled);
+
+EncodeTiledFn encode_fn() {
+    static EncodeTiledFn fn = nullptr;
+    static std::once_flag once;
+    std::call_once(once, [] {
+        void *ptr = nullptr;
+        cudaDriverEntryPointQueryResult q;
+        if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &ptr, cudaEnableDefault, &q) ==
+                cudaSuccess &&
+            q == cudaDriverEntryPointSuccess)
+            fn = reinterpret_cast<EncodeTiledFn>(ptr);
+    });
+    return fn;
+}
+
+struct MapKey {
+    const void *ptr;
+    uint64_t rows;
+    int head_dim;
+    int device;
+};
+
+// Small cache of pool tensor maps: a decode step re-uses the same pools.
+bool pool_tensor_map(const void *pool, uint64_t rows, int head_dim, CUtensorMap *out) {
+    static std::mutex mu;
+    static MapKey keys[8];
+    static CUtensorMap maps[8];
+    static int used = 0, next = 0;
+    int dev = 0;
+    cudaGetDevice(&dev);
+    std::lock_guard<std::mutex> lock(mu);
+    for (int i = 0; i < used; ++i) {
+        if (keys[i].ptr == pool && keys[i].rows == rows && keys[i].head_dim == head_dim &&
+            keys[i].device == dev) {
+            *out = maps[i];
+            return true;
+        }
+    }
+    EncodeTiledFn enc = encode_fn();
+    if (!enc) return false;
+    CUtensorMap m;
+    cuuint64_t dims[2] = {(cuuint64_t)head_dim, (cuuint64_t)rows};
+    cuuint64_t strides[1] = {(cuuint64_t)head_dim * 2};
+    cuuint32_t box[2] = {64, (cuuint32_t)kTileTokens};
+    cuuint32_t estr[2] = {1, 1};
+    CUresult r = enc(&m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void *>(pool), dims, strides,
+                     box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+                     CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+    if (r != CUDA_SUCCESS) return false;
+    const int slot = used < 8 ? used++ : (next++ & 7);
+    keys[slot] = MapKey{pool, rows, head_dim, dev};
+    maps[slot] = m;
+    *out = m;
+    return true;
+}
+
+// Resolve the partition size: -1 = single pass, else tokens per partition.
+int resolve_partition(int batch, int num_kv_heads, int block_size, int max_seq_len, int requested) {
+    if (requested < 0) return -1;
+    if (requested > 0) return requested >= max_seq_len ? -1 : requested;
+    // Default: split only when (sequence, kv head) units cannot fill the GPU.
+    const int sms = device_sm_count();
+    const int64_t units = (int64_t)batch * num_kv_heads;
+    if (units >= 2LL * sms || max_seq_len <= 1024) return -1;
+    const int64_t want_parts = (3LL * sms + units - 1) / units;
+    int64_t pt = ((int64_t)max_seq_len + want_parts - 1) / want_parts;
+    pt = ((pt + 511) / 512) * 512;
+    if (pt < 512) pt = 512;
+    return pt >= max_seq_len ? -1 : (int)pt;
+}
+
+template <int HEAD_DIM, bool SPLIT>
+int launch_decode(const CUtensorMap &km, const CUtensorMap &vm, const DecodeParams &p, int batch,
+                  cudaStream_t stream) {
+    using C = Cfg<HEAD_DIM>;
+    auto kern = paged_decode_kernel<HEAD_DIM, SPLIT>;
+    static std::once_flag once;
+    static cudaError_t attr_err = cudaSuccess;
+    std::call_once(once, [&] {
+        attr_err = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, C::kSmemBytes);
+    });
+    if (attr_err != cudaSuccess) return PA_ERR_CUDA;
+    dim3 grid((unsigned)p.num_parts, (unsigned)p.num_kv_heads, (unsigned)batch);
+    kern<<<grid, kThreads, C::kSmemBytes, stream>>>(km, vm, p);
+    count_launch();
+    int st = launch_status();
+    if (st != PA_OK || !SPLIT) return st;
+    dim3 rgrid((unsigned)p.num_q_heads, (unsigned)batch);
+    lse_reduce_kernel<HEAD_DIM><<<rgrid, HEAD_DIM, 0, stream>>>(p);
+    count_launch();
+    return launch_status();
+}
+
+}  // namespace
+}  // namespace pa
+
+extern "C" {
+
+int pa_decode_partition_tokens(int batch, int num_q_heads, int num_kv_heads, int head_dim,
+                               int block_size, int max_seq_len, int partition_tokens) {
+    (void)num_q_heads;
+    (void)head_dim;
+    if (batch <= 0 || max_seq_len <= 0) return -1;
+    return pa::resolve_partition(batch, num_kv_heads, block_size, max_seq_len, partition_tokens);
+}
+
+size_t pa_decode_workspace_size(int batch, int num_q_heads, int num_kv_heads, int head_dim,
+                                int block_size, int max_seq_len, int partition_tokens) {
+    if (batch <= 0 || num_q_heads <= 0 || num_kv_heads <= 0 || max_seq_len <= 0) return 0;
+    const int pt = pa::resolve_partition(batch, num_kv_heads, block_size, max_seq_len, partition_tokens);
+    if (pt <= 0) return 0;
+    const int64_t parts = ((int64_t)max_seq_len + pt - 1) / pt;
+    const int64_t rows = (int64_t)batch * num_q_heads * parts;
+    const int64_t o_bytes = ((rows * head_dim * 4) + 255) / 256 * 256;
+    return (size_t)(o_bytes + rows * 2 * 4);
+}
+
+int pa_decode(float *out, const void *q, const void *k_cache, const void *v_cache,
+              const int32_t *block_tables, int max_blocks_per_seq, const int32_t *seq_lens,
+              int batch, int max_seq_len, int num_q_heads, int num_kv_heads, int head_dim,
+              int block_size, int64_t num_blocks, float scale, int partition_tokens,
+              void *workspace, size_t workspace_bytes, int32_t *err_flag, void *stream) {
+    if (batch < 0 || max_seq_len < 0 || num_blocks <= 0 || max_blocks_per_seq < 0)
+        return PA_ERR_INVALID_ARG;
+    if (!pa::supported_shape(num_q_heads, num_kv_heads, head_dim, block_size)) return PA_ERR_UNSUPPORTED;
+    if (batch == 0) return PA_OK;
+    if (!out || !q || !k_cache || !v_cache || !block_tables || !seq_lens) return PA_ERR_INVALID_ARG;
+    if (!pa::aligned16(q) || !pa::aligned16(k_cache) || !pa::aligned16(v_cache) || !pa::aligned16(out))
+        return PA_ERR_INVALID_ARG;
+    if (partition_tokens > 0 && partition_tokens % block_size) return PA_ERR_INVALID_ARG;
+    if (batch > 65535 || num_kv_heads > 65535) return PA_ERR_UNSUPPORTED;
+    const uint64_t rows = (uint64_t)num_blocks * (uint64_t)num_kv_heads * (uint64_t)block_size;
+    if (rows >= (1ull << 31)) return PA_ERR_UNSUPPORTED;  // TMA row coordinate is int32
+
+    pa::DecodeParams p{};
+    p.out = out;
+    p.q = static_cast<const uint16_t *>(q);
+    p.block_tables = block_tables;
+    p.seq_lens = seq_lens;
+    p.err_flag = err_flag;
+    p.num_blocks = num_blocks;
+    p.max_blocks = max_blocks_per_seq;
+    p.max_seq_len = max_seq_len;
+    p.num_q_heads = num_q_heads;
+    p.num_kv_heads = num_kv_heads;
+    p.group = num_q_heads / num_kv_heads;
+    p.block_size = block_size;
+    p.scale_log2 = scale * pa::kLog2e;
+
+    const int pt = max_seq_len > 0
+                       ? pa::resolve_partition(batch, num_kv_heads, block_size, max_seq_len, partition_tokens)
+                       : -1;
+    const bool split = pt > 0;
+    if (split) {
+        const size_t need = pa_decode_workspace_size(batch, num_q_heads, num_kv_heads, head_dim,
+                                                     block_size, max_seq_len, partition_tokens);
+        if (!workspace || workspace_bytes < need || !pa::aligned16(workspace)) return PA_ERR_INVALID_ARG;
+        p.part_tokens = pt;
+        p.num_parts = (max_seq_len + pt - 1) / pt;
+        const int64_t prow = (int64_t)batch * num_q_heads * p.num_parts;
+        p.part_o = static_cast<float *>(workspace);
+        p.part_ml = reinterpret_cast<float *>(static_cast<char *>(workspace) +
+                                              ((prow * head_dim * 4) + 255) / 256 * 256);
+        if (p.num_parts > 65535) return PA_ERR_UNSUPPORTED;
+    } else {
+        p.part_tokens = max_seq_len > 0 ? max_seq_len : 1;
+        p.num_parts = 1;
+    }
+
+    CUtensorMap km, vm;
+    if (!pa::pool_tensor_map(k_cache, rows, head_dim, &km) || !pa::pool_tensor_map(v_cache, rows, head_dim, &vm))
+        return PA_ERR_CUDA;
+    cudaStream_t s = static_cast<cudaStream_t>(stream);
+    if (head_dim == 128)
+        return split ? pa::launch_decode<128, true>(km, vm, p, batch, s)
+                     : pa::launch_decode<128, false>(km, vm, p, batch, s);
+    return split ? pa::launch_decode<64, true>(km, vm, p, batch, s)
+                 : pa::launch_decode<64, false>(km, vm, p, batch, s);
+}
+
+}  // extern "C"

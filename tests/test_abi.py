@@ -1,0 +1,95 @@
+"""The C ABI: the library loads on a CPU-only host, exports every declared symbol,
+and rejects bad arguments synchronously, before any launch."""
+import ctypes
+import os
+import re
+
+import pytest
+
+from tests.conftest import ROOT
+
+import paged_kv_cache_349_b200 as pa
+from paged_kv_cache_349_b200._lib import SIGNATURES, lib
+
+
+def _declared_functions():
+    src = open(os.path.join(ROOT, "include", "pa.h")).read()
+    src = re.sub(r"/\*.*?\*/", "", src, flags=re.S)
+    names = re.findall(r"\b(pa_[a-z0-9_]+)\s*\(", src)
+    return sorted(set(names))
+
+
+def test_header_and_binding_agree():
+    declared = _declared_functions()
+    assert len(declared) >= 20
+    assert sorted(SIGNATURES) == declared
+
+
+def test_every_declared_symbol_is_exported():
+    for name in _declared_functions():
+        assert hasattr(lib, name), name
+
+
+def test_status_strings():
+    assert pa.status_string(0) == "PA_OK"
+    assert pa.status_string(pa.PA_ERR_OOM) == "PA_ERR_OOM"
+    assert pa.status_string(999) == "PA_ERR_UNKNOWN"
+    assert pa.version() >= 100
+
+
+P = ctypes.c_void_p
+
+
+def _fake(addr=0x10000):
+    return P(addr)
+
+
+def test_decode_argument_errors_need_no_gpu():
+    f = lib.pa_decode
+    ok_args = dict(out=_fake(), q=_fake(), k=_fake(), v=_fake(), bt=_fake(), maxb=4, lens=_fake(),
+                   B=2, maxlen=64, Hq=8, Hkv=2, d=128, bs=16, NB=64, scale=0.1, pt=-1,
+                   ws=None, wsb=0, flag=None, stream=None)
+
+    def call(**kw):
+        a = dict(ok_args, **kw)
+        return f(a["out"], a["q"], a["k"], a["v"], a["bt"], a["maxb"], a["lens"], a["B"], a["maxlen"],
+                 a["Hq"], a["Hkv"], a["d"], a["bs"], a["NB"], a["scale"], a["pt"], a["ws"], a["wsb"],
+                 a["flag"], a["stream"])
+
+    assert call(B=0) == pa.PA_OK                         # nothing to do, nothing launched
+    assert call(d=96) == pa.PA_ERR_UNSUPPORTED
+    assert call(bs=8) == pa.PA_ERR_UNSUPPORTED
+    assert call(Hq=6, Hkv=4) == pa.PA_ERR_UNSUPPORTED    # not a whole group
+    assert call(Hq=32, Hkv=2) == pa.PA_ERR_UNSUPPORTED   # group of 16
+    assert call(q=None) == pa.PA_ERR_INVALID_ARG
+    assert call(q=_fake(0x10008)) == pa.PA_ERR_INVALID_ARG  # misaligned
+    assert call(pt=24) == pa.PA_ERR_INVALID_ARG          # not a multiple of block_size
+    assert call(pt=16, ws=None) == pa.PA_ERR_INVALID_ARG  # split needs a workspace
+    assert call(NB=0) == pa.PA_ERR_INVALID_ARG
+    assert call(NB=1 << 30) == pa.PA_ERR_UNSUPPORTED     # TMA row coordinate overflow
+
+
+def test_cache_op_argument_errors_need_no_gpu():
+    assert lib.pa_reshape_and_cache(None, None, None, None, None, 0, 8, 2, 16, 128, None, None) == pa.PA_OK
+    assert lib.pa_reshape_and_cache(_fake(), _fake(), _fake(), _fake(), None, 3, 8, 2, 16, 128, None,
+                                    None) == pa.PA_ERR_INVALID_ARG
+    assert lib.pa_reshape_and_cache(_fake(), _fake(), _fake(), _fake(), _fake(), 3, 8, 2, 16, 80, None,
+                                    None) == pa.PA_ERR_UNSUPPORTED
+    assert lib.pa_copy_blocks(None, None, None, 0, 8, 2, 16, 128, None, None) == pa.PA_OK
+    assert lib.pa_copy_blocks(_fake(), _fake(), None, 2, 8, 2, 16, 128, None, None) == pa.PA_ERR_INVALID_ARG
+    assert lib.pa_copy_blocks(_fake(0x10004), _fake(), _fake(), 2, 8, 2, 16, 128, None,
+                              None) == pa.PA_ERR_INVALID_ARG
+
+
+@pytest.mark.parametrize("pt,maxlen,parts", [(512, 32768, 64), (512, 512, 0), (16, 40, 3), (-1, 4096, 0)])
+def test_workspace_size_explicit_partitions(pt, maxlen, parts):
+    B, Hq, Hkv, d = 8, 64, 8, 128
+    size = pa.pa_decode_workspace_size(B, Hq, Hkv, d, 16, maxlen, pt)
+    if parts == 0:
+        assert size == 0
+        assert pa.pa_decode_partition_tokens(B, Hq, Hkv, d, 16, maxlen, pt) == -1
+    else:
+        rows = B * Hq * parts
+        o_bytes = -(-rows * d * 4 // 256) * 256
+        assert size == o_bytes + rows * 8
+        assert pa.pa_decode_partition_tokens(B, Hq, Hkv, d, 16, maxlen, pt) == pt

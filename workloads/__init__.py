@@ -299,6 +299,25 @@ def make_case(config: int, *, seed: Optional[int] = None, fill=BF16_QNAN,
     raise ValueError(f"unknown workload {config}")
 
 
+def make_custom_case(lens, *, num_q_heads: int, num_kv_heads: int, head_dim: int, block_size: int,
+                     num_blocks: Optional[int] = None, seed: int = 0, fill=BF16_QNAN,
+                     poison_padding: bool = True, extra_table_cols: int = 0,
+                     partition_tokens: int = 0, scale=None) -> DecodeCase:
+    """A decode step with the given lengths and shape, blocks placed by a seeded permutation."""
+    rng = np.random.default_rng(seed)
+    lens = np.asarray(lens, dtype=np.int64)
+    bs = block_size
+    used = int((-(-lens // bs)).sum())
+    NB = num_blocks if num_blocks is not None else max(8, 2 * used + 8)
+    order = rng.permutation(NB)
+    max_blocks = max(1, int((-(-lens // bs)).max()) if lens.size else 1) + extra_table_cols
+    pad = _padding_ids(order, used, rng, poison_padding)
+    tables = _deal_tables(lens, order, bs, max_blocks, pad)
+    return _finish("custom", rng, seed, Hq=num_q_heads, Hkv=num_kv_heads, d=head_dim, bs=bs, NB=NB,
+                   lens=lens, tables=tables, fill=fill, free_order=order.astype(np.int32),
+                   partition_tokens=partition_tokens, scale=scale)
+
+
 def gqa_lengths(rng: np.random.Generator, batch: int, cap: int = 4096) -> np.ndarray:
     """Lengths of workload 4: lognormal with median 800 and sigma 1.0, rounded, clamped to [1, cap]."""
     return np.clip(np.rint(rng.lognormal(np.log(800.0), 1.0, size=batch)), 1, cap).astype(np.int64)
