@@ -30,10 +30,25 @@
 namespace pa {
 namespace {
 
+// Compile-time shape of the decode CTA (overridable for tuning builds).
+#ifndef PA_DECODE_CONSUMER_WARPS
+#define PA_DECODE_CONSUMER_WARPS 4
+#endif
+#ifndef PA_DECODE_STAGES
+#define PA_DECODE_STAGES 8
+#endif
+#ifndef PA_DECODE_PRODUCER_LANES
+#define PA_DECODE_PRODUCER_LANES 8
+#endif
+
 constexpr int kTileTokens = 16;
-constexpr int kConsumerWarps = 4;
+constexpr int kConsumerWarps = PA_DECODE_CONSUMER_WARPS;
 constexpr int kThreads = (kConsumerWarps + 1) * 32;
-constexpr int kStages = 8;
+constexpr int kStages = PA_DECODE_STAGES;
+// Producer lanes issue tiles round-robin; lane k owns ring slots k, k+P, ...
+constexpr int kProducerLanes = PA_DECODE_PRODUCER_LANES;
+static_assert(kStages % kProducerLanes == 0, "each producer lane owns whole ring slots");
+static_assert(kProducerLanes >= 1 && kProducerLanes <= 8, "window indexing assumes <= 8 lanes");
 constexpr int kBoxBytes = kTileTokens * 128;  // one 64-wide bf16 column box of a tile
 constexpr float kLog2e = 1.4426950408889634f;
 
@@ -126,42 +141,75 @@ __global__ void __launch_bounds__(kThreads) paged_decode_kernel(
 
     if (warp == kConsumerWarps) {
         // ---------------- producer: block-table dereference + TMA ----------------
-        if (lane == 0) {
-            prefetch_tensormap(&k_map);
-            prefetch_tensormap(&v_map);
-            const uint64_t policy = l2_policy_evict_first();
-            const int32_t *table = p.block_tables + (int64_t)b * p.max_blocks;
-            int issued = 0;
-            for (int i = 0; i < n_tiles; ++i) {
-                const int s = i % kStages;
-                if (i >= kStages && !mbar_wait_bounded(&empty[s], ((i / kStages) - 1) & 1, p.err_flag))
-                    break;
-                const int tok0 = tok_begin + i * kTileTokens;
-                const int j = tok0 / p.block_size;
-                const int row = tok0 - j * p.block_size;
-                const int64_t phys = __ldg(table + j);
-                issued = i + 1;
-                if (phys < 0 || phys >= p.num_blocks) {
-                    raise_flag(p.err_flag, PA_FLAG_BAD_BLOCK);
-                    tile_ok[s] = 0;
-                    mbar_arrive(&full[s]);
-                    continue;
-                }
-                tile_ok[s] = 1;
-                const int y = (int)((phys * p.num_kv_heads + h) * p.block_size + row);
-                uint8_t *dst = smem + s * C::kStageBytes;
-                mbar_arrive_expect_tx(&full[s], C::kStageBytes);
-#pragma unroll
-                for (int bx = 0; bx < C::kBoxes; ++bx)
-                    tma_load_2d(dst + bx * kBoxBytes, &k_map, bx * 64, y, &full[s], policy);
-#pragma unroll
-                for (int bx = 0; bx < C::kBoxes; ++bx)
-                    tma_load_2d(dst + C::kTileBytes + bx * kBoxBytes, &v_map, bx * 64, y, &full[s],
-                                policy);
+        // The whole warp walks the tiles so that block-table entries arrive 32 at a
+        // time (one coalesced load per window, the next window loaded ahead).
+        // kProducerLanes lanes wait on the ring and issue copies in parallel:
+        // lane k handles tiles k, k+P, k+2P, ... and therefore ring slots k, k+P, ...
+        const int32_t *table = p.block_tables + (int64_t)b * p.max_blocks;
+        const int j_end = (tok_end + p.block_size - 1) / p.block_size;  // blocks this CTA reads
+        int win = tok_begin / p.block_size;                             // first entry of the window
+        int32_t cur = win + lane < j_end ? __ldg(table + win + lane) : -1;
+        int32_t nxt = win + 32 + lane < j_end ? __ldg(table + win + 32 + lane) : -1;
+        uint64_t policy = 0;
+        if (lane < kProducerLanes) {
+            if (lane == 0) {
+                prefetch_tensormap(&k_map);
+                prefetch_tensormap(&v_map);
             }
-            // Drain: every issued tile has landed before the ring is reused or the CTA exits.
-            for (int i = max(0, issued - kStages); i < issued; ++i)
-                if (!mbar_wait_bounded(&full[i % kStages], (i / kStages) & 1, p.err_flag)) break;
+            policy = l2_policy_evict_first();
+        }
+        int issued = 0;  // tiles issued by this lane's rounds (max over lanes below)
+        bool stop = false;
+        for (int i0 = 0; i0 < n_tiles; i0 += kProducerLanes) {
+            const int j0 = (tok_begin + i0 * kTileTokens) / p.block_size;
+            if (j0 >= win + 32) {  // warp-uniform: slide the window
+                win += 32;
+                cur = nxt;
+                nxt = win + 32 + lane < j_end ? __ldg(table + win + 32 + lane) : -1;
+            }
+            const int i = i0 + lane;
+            const bool mine = lane < kProducerLanes && i < n_tiles;
+            const int tok0 = tok_begin + i * kTileTokens;
+            const int j = mine ? tok0 / p.block_size : win;
+            const int row = tok0 - j * p.block_size;
+            const int idx = j - win;  // in [0, 32 + kProducerLanes)
+            const int32_t from_cur = __shfl_sync(0xffffffffu, cur, idx & 31);
+            const int32_t from_nxt = __shfl_sync(0xffffffffu, nxt, idx & 31);
+            const int64_t phys = idx < 32 ? from_cur : from_nxt;
+            if (mine) {
+                const int s = i % kStages;
+                if (i >= kStages && !mbar_wait_bounded(&empty[s], ((i / kStages) - 1) & 1, p.err_flag)) {
+                    stop = true;
+                } else {
+                    issued = i + 1;
+                    if (phys < 0 || phys >= p.num_blocks) {
+                        raise_flag(p.err_flag, PA_FLAG_BAD_BLOCK);
+                        tile_ok[s] = 0;
+                        mbar_arrive(&full[s]);
+                    } else {
+                        tile_ok[s] = 1;
+                        const int y = (int)((phys * p.num_kv_heads + h) * p.block_size + row);
+                        uint8_t *dst = smem + s * C::kStageBytes;
+                        mbar_arrive_expect_tx(&full[s], C::kStageBytes);
+#pragma unroll
+                        for (int bx = 0; bx < C::kBoxes; ++bx)
+                            tma_load_2d(dst + bx * kBoxBytes, &k_map, bx * 64, y, &full[s], policy);
+#pragma unroll
+                        for (int bx = 0; bx < C::kBoxes; ++bx)
+                            tma_load_2d(dst + C::kTileBytes + bx * kBoxBytes, &v_map, bx * 64, y,
+                                        &full[s], policy);
+                    }
+                }
+            }
+            if (__any_sync(0xffffffffu, stop)) break;
+        }
+        // Drain: every issued tile has landed before the ring is reused or the CTA exits.
+        // A tile is the last user of its slot when no tile kStages later was issued.
+        const int issued_all = __reduce_max_sync(0xffffffffu, issued);
+        if (lane < kProducerLanes) {
+            for (int i = lane; i < issued_all; i += kProducerLanes)
+                if (i + kStages >= issued_all && i < issued)
+                    if (!mbar_wait_bounded(&full[i % kStages], (i / kStages) & 1, p.err_flag)) break;
         }
     } else {
         // ---------------- consumers ----------------
@@ -418,18 +466,22 @@ bool pool_tensor_map(const void *pool, uint64_t rows, int head_dim, CUtensorMap 
 }
 
 // Resolve the partition size: -1 = single pass, else tokens per partition.
+//
+// Default (measured on B200, decode of bf16 d=128 pools): one CTA per
+// (sequence, kv head) is best when there are enough of them to fill the GPU
+// several times over and no sequence can be much longer than the rest;
+// otherwise 1024-token partitions keep the CTAs short enough that the last
+// wave does not leave SMs idle (long-tailed length mixes, few sequences).
 int resolve_partition(int batch, int num_kv_heads, int block_size, int max_seq_len, int requested) {
+    (void)block_size;
     if (requested < 0) return -1;
     if (requested > 0) return requested >= max_seq_len ? -1 : requested;
-    // Default: split only when (sequence, kv head) units cannot fill the GPU.
-    const int sms = device_sm_count();
+    constexpr int kDefaultPartition = 1024;
+    if (max_seq_len <= kDefaultPartition) return -1;
     const int64_t units = (int64_t)batch * num_kv_heads;
-    if (units >= 2LL * sms || max_seq_len <= 1024) return -1;
-    const int64_t want_parts = (3LL * sms + units - 1) / units;
-    int64_t pt = ((int64_t)max_seq_len + want_parts - 1) / want_parts;
-    pt = ((pt + 511) / 512) * 512;
-    if (pt < 512) pt = 512;
-    return pt >= max_seq_len ? -1 : (int)pt;
+    const int64_t resident = 3LL * device_sm_count();  // CTAs resident at once
+    if (units >= 2 * resident && max_seq_len < 3 * kDefaultPartition) return -1;
+    return kDefaultPartition;
 }
 
 template <int HEAD_DIM, bool SPLIT>

@@ -36,17 +36,17 @@ inline bool supported_shape(int num_q_heads, int num_kv_heads, int head_dim, int
 // Device side
 // ---------------------------------------------------------------------------
 
-// A bounded wait gives up after this many nanoseconds (about one second).
-constexpr unsigned long long kWaitLimitNs = 1000000000ull;
+// A bounded wait gives up after this many SM clock cycles (about one second).
+constexpr long long kWaitLimitCycles = 2000000000LL;
+
+// Wait style: 0 = mbarrier.try_wait (the thread may be suspended by the
+// hardware until the phase completes), 1 = mbarrier.test_wait spin.
+#ifndef PA_WAIT_SPIN
+#define PA_WAIT_SPIN 0
+#endif
 
 __device__ __forceinline__ uint32_t smem_addr(const void *p) {
     return static_cast<uint32_t>(__cvta_generic_to_shared(p));
-}
-
-__device__ __forceinline__ unsigned long long global_timer_ns() {
-    unsigned long long t;
-    asm volatile("mov.u64 %0, %%globaltimer;" : "=l"(t));
-    return t;
 }
 
 __device__ __forceinline__ void raise_flag(int32_t *flag, int bits) {
@@ -85,14 +85,30 @@ __device__ __forceinline__ bool mbar_try_wait(uint64_t *bar, uint32_t parity) {
     return done != 0;
 }
 
+__device__ __forceinline__ bool mbar_test_wait(uint64_t *bar, uint32_t parity) {
+    uint32_t done;
+    asm volatile(
+        "{\n\t.reg .pred p;\n\t"
+        "mbarrier.test_wait.parity.acquire.cta.shared::cta.b64 p, [%1], %2;\n\t"
+        "selp.u32 %0, 1, 0, p;\n\t}"
+        : "=r"(done)
+        : "r"(smem_addr(bar)), "r"(parity)
+        : "memory");
+    return done != 0;
+}
+
 // Wait for the phase of `bar` with the given parity to complete.  Returns
-// false (and sets PA_FLAG_TIMEOUT) if that takes longer than kWaitLimitNs.
+// false (and sets PA_FLAG_TIMEOUT) if that takes longer than kWaitLimitCycles.
+// The clock is only read every 64 polls, so the common case costs one poll.
 __device__ __forceinline__ bool mbar_wait_bounded(uint64_t *bar, uint32_t parity, int32_t *flag) {
-    if (mbar_try_wait(bar, parity)) return true;
-    const unsigned long long t0 = global_timer_ns();
+    const long long t0 = clock64();
     for (uint32_t it = 1;; ++it) {
+#if PA_WAIT_SPIN
+        if (mbar_test_wait(bar, parity)) return true;
+#else
         if (mbar_try_wait(bar, parity)) return true;
-        if ((it & 255u) == 0 && global_timer_ns() - t0 > kWaitLimitNs) {
+#endif
+        if ((it & 63u) == 0 && clock64() - t0 > kWaitLimitCycles) {
             raise_flag(flag, PA_FLAG_TIMEOUT);
             return false;
         }
