@@ -24,8 +24,10 @@
  *    detected on the host, before any launch, and nothing is launched.
  *    A failed launch returns PA_ERR_CUDA.
  *  - Device pointers are caller-owned device memory of the current CUDA
- *    device.  The library allocates no device memory; the caller provides
- *    the decode workspace (size from pa_decode_workspace_size).
+ *    device.  The library allocates no device memory at run time; the
+ *    caller provides the decode workspace (size from
+ *    pa_decode_workspace_size).  The one exception is
+ *    pa_decode_builtin_scratch, whose scratch is a static device array.
  *  - `stream` is a cudaStream_t passed as void*; NULL is the legacy default
  *    stream.  Device work is asynchronous on that stream.
  *  - Data-dependent index errors (a slot, block id or copy pair out of range,
@@ -158,6 +160,46 @@ int pa_decode(float *out, const void *q, const void *k_cache, const void *v_cach
               int batch, int max_seq_len, int num_q_heads, int num_kv_heads, int head_dim,
               int block_size, int64_t num_blocks, float scale, int partition_tokens,
               void *workspace, size_t workspace_bytes, int32_t *err_flag, void *stream);
+
+/* ------------------------------------------------------------------------
+ * Decode with library-owned scratch (no workspace argument).
+ *
+ * The pages have no counterpart: this entry point is a convenience of this
+ * library, not a step of PagedAttention.
+ *
+ * Some callers cannot allocate device memory at the moment they decode:
+ * a plugin whose host program owns every device allocation through its own
+ * pool and forbids direct cudaMalloc, a caller from another language
+ * runtime that only hands over pointers to tensors it already owns, or a
+ * latency-critical loop that must not pay for (or synchronise on)
+ * cudaMalloc/cudaFree.  For them this call behaves exactly like pa_decode,
+ * except that the partial softmax states of the split variant go to a
+ * device array owned by the library instead of a caller workspace.
+ *
+ *  - The array is a file-scope device variable of
+ *    PA_DECODE_BUILTIN_SCRATCH_BYTES bytes.  Every GPU on which the library
+ *    is loaded holds it until the process exits.
+ *  - The first call on each device looks up the array's device address
+ *    (cudaGetSymbolAddress) with that device current.  Make that first call
+ *    before any stream capture.
+ *  - If the split this call would use needs more scratch than
+ *    PA_DECODE_BUILTIN_SCRATCH_BYTES (see pa_decode_workspace_size), the
+ *    call returns PA_ERR_UNSUPPORTED and launches nothing.
+ *  - No cudaMalloc, cudaFree or other allocating routine is called.
+ *  - All calls share the one array, and it keeps whatever the last call
+ *    wrote.  Nothing in it has to start at zero: each partition's state is
+ *    written before it is read within the same call.  Calls whose kernels
+ *    can overlap on the GPU (different streams, or several host threads)
+ *    race on the array; issue them on one stream.
+ * Other arguments, layouts and errors: as pa_decode.
+ * ---------------------------------------------------------------------- */
+#define PA_DECODE_BUILTIN_SCRATCH_BYTES ((size_t)32 << 20)
+
+int pa_decode_builtin_scratch(float *out, const void *q, const void *k_cache, const void *v_cache,
+                              const int32_t *block_tables, int max_blocks_per_seq,
+                              const int32_t *seq_lens, int batch, int max_seq_len, int num_q_heads,
+                              int num_kv_heads, int head_dim, int block_size, int64_t num_blocks,
+                              float scale, int partition_tokens, int32_t *err_flag, void *stream);
 
 /* ------------------------------------------------------------------------
  * Host block allocator (owns host memory only; not thread-safe).

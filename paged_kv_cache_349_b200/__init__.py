@@ -163,6 +163,30 @@ def pa_decode(out, q, k_cache, v_cache, block_tables, seq_lens, *, max_seq_len: 
         _stream(stream)), "pa_decode")
 
 
+PA_DECODE_BUILTIN_SCRATCH_BYTES = 32 << 20
+
+
+def pa_decode_builtin_scratch(out, q, k_cache, v_cache, block_tables, seq_lens, *, max_seq_len: int,
+                              scale: float, partition_tokens: int = 0, err_flag=None, stream=None) -> None:
+    """pa_decode for callers that cannot allocate a workspace: split states go to a
+    library-owned device array of PA_DECODE_BUILTIN_SCRATCH_BYTES (shared by all calls;
+    calls that overlap on the GPU race on it)."""
+    torch = _torch()
+    B, Hq, d = q.shape
+    NB, Hkv, bs, d2 = k_cache.shape
+    if d2 != d or out.shape != q.shape or v_cache.shape != k_cache.shape:
+        raise ValueError("shape mismatch")
+    if block_tables.dim() != 2 or block_tables.shape[0] != B or seq_lens.numel() != B:
+        raise ValueError("block_tables must be [B, max_blocks] and seq_lens [B]")
+    _check(lib.pa_decode_builtin_scratch(
+        _dev(out, torch.float32, "out"), _dev(q, torch.bfloat16, "q"),
+        _dev(k_cache, torch.bfloat16, "k_cache"), _dev(v_cache, torch.bfloat16, "v_cache"),
+        _dev(block_tables, torch.int32, "block_tables"), block_tables.shape[1],
+        _dev(seq_lens, torch.int32, "seq_lens"), B, int(max_seq_len), Hq, Hkv, d, bs, NB,
+        float(scale), int(partition_tokens), _opt_flag(err_flag), _stream(stream)),
+        "pa_decode_builtin_scratch")
+
+
 # ---------------------------------------------------------------------------
 # Host allocator
 # ---------------------------------------------------------------------------

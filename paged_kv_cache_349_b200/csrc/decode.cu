@@ -507,6 +507,29 @@ int launch_decode(const CUtensorMap &km, const CUtensorMap &vm, const DecodePara
 }
 
 }  // namespace
+
+// Scratch for pa_decode_builtin_scratch, for callers that cannot allocate a
+// workspace.  In host code the name is only a stand-in: kernels receive the
+// device address that cudaGetSymbolAddress returns for the current device.
+static __device__ __align__(256) unsigned char g_builtin_scratch[PA_DECODE_BUILTIN_SCRATCH_BYTES];
+
+// Device address of the scratch array on the current device, looked up once
+// per device (the first call on a device does the lookup).
+int builtin_scratch_address(void **out) {
+    static std::mutex mu;
+    static void *addr[64] = {};
+    int dev = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) return PA_ERR_CUDA;
+    std::lock_guard<std::mutex> lock(mu);
+    if (!addr[dev]) {
+        void *p = nullptr;
+        if (cudaGetSymbolAddress(&p, g_builtin_scratch) != cudaSuccess || p == nullptr) return PA_ERR_CUDA;
+        addr[dev] = p;
+    }
+    *out = addr[dev];
+    return PA_OK;
+}
+
 }  // namespace pa
 
 extern "C" {
@@ -591,6 +614,24 @@ int pa_decode(float *out, const void *q, const void *k_cache, const void *v_cach
                      : pa::launch_decode<128, false>(km, vm, p, batch, s);
     return split ? pa::launch_decode<64, true>(km, vm, p, batch, s)
                  : pa::launch_decode<64, false>(km, vm, p, batch, s);
+}
+
+int pa_decode_builtin_scratch(float *out, const void *q, const void *k_cache, const void *v_cache,
+                              const int32_t *block_tables, int max_blocks_per_seq,
+                              const int32_t *seq_lens, int batch, int max_seq_len, int num_q_heads,
+                              int num_kv_heads, int head_dim, int block_size, int64_t num_blocks,
+                              float scale, int partition_tokens, int32_t *err_flag, void *stream) {
+    if (batch < 0 || max_seq_len < 0) return PA_ERR_INVALID_ARG;
+    void *scratch = nullptr;
+    const int st = pa::builtin_scratch_address(&scratch);
+    if (st != PA_OK) return st;
+    const size_t need = batch > 0 ? pa_decode_workspace_size(batch, num_q_heads, num_kv_heads, head_dim,
+                                                             block_size, max_seq_len, partition_tokens)
+                                  : 0;
+    if (need > PA_DECODE_BUILTIN_SCRATCH_BYTES) return PA_ERR_UNSUPPORTED;
+    return pa_decode(out, q, k_cache, v_cache, block_tables, max_blocks_per_seq, seq_lens, batch,
+                     max_seq_len, num_q_heads, num_kv_heads, head_dim, block_size, num_blocks, scale,
+                     partition_tokens, scratch, PA_DECODE_BUILTIN_SCRATCH_BYTES, err_flag, stream);
 }
 
 }  // extern "C"
