@@ -203,8 +203,10 @@ def _barrier(world: int):
 def cpu_baseline(case, budget_s: float = 12.0):
     """Time the fp64 oracle on a bounded sample of (sequence, kv head) units of ``case``.
 
+    Units are taken in a seeded order, in chunks, cycling over the whole
+    workload until about ``budget_s`` seconds of oracle time have passed.
     Returns the oracle's throughput in the bench's unit (algorithmic GB/s),
-    the threads it used and what the sample was.
+    the threads it used, what the sample was, the seconds and bytes timed.
     """
     import oracle
     threads = len(os.sched_getaffinity(0))
@@ -212,11 +214,12 @@ def cpu_baseline(case, budget_s: float = 12.0):
     G = case.group_size
     rng = np.random.default_rng(7)
     units = [(int(b), int(h)) for b in rng.permutation(case.batch) for h in rng.permutation(case.num_kv_heads)]
-    # calibrate on a few units, then size the sample to the budget
     done_units, done_bytes, elapsed = 0, 0, 0.0
     chunk = max(1, threads)
-    while done_units < len(units) and elapsed < budget_s:
-        sel = units[done_units:done_units + chunk]
+    pos = 0
+    while elapsed < budget_s:
+        sel = [units[(pos + i) % len(units)] for i in range(min(chunk, len(units)))]
+        pos = (pos + len(sel)) % len(units)
         rows = np.array([(b, h * G + g) for b, h in sel for g in range(G)], np.int32)
         t0 = time.perf_counter()
         oracle.decode(case.q, case.k_cache, case.v_cache, case.block_tables, case.seq_lens,
@@ -228,9 +231,9 @@ def cpu_baseline(case, budget_s: float = 12.0):
         if dt < budget_s / 20:
             chunk *= 2
     gbs = done_bytes / elapsed / 1e9
-    sample = (f"{done_units} of {len(units)} (sequence, kv head) units of the same workload "
-              f"({done_units * G} query-head rows, {done_bytes / 1e6:.1f} MB of K/V/q/out), "
-              f"{elapsed:.1f} s of oracle time")
+    sample = (f"{done_units} (sequence, kv head) units ({done_units / len(units):.2f} passes over the "
+              f"workload's {len(units)}), {done_units * G} query-head rows, {done_bytes / 1e9:.2f} GB of "
+              f"K/V/q/out, {elapsed:.1f} s of oracle time")
     return gbs, threads, sample, elapsed, done_bytes
 
 
