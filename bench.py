@@ -250,7 +250,7 @@ def run_native(args):
     torch.cuda.set_device(local)
     cfg = args.config
     seed = 1000 + cfg + 7919 * rank  # weak scaling: every rank owns its own batch
-    case = W.make_case(cfg, seed=seed, fill=W.BF16_ZERO)
+    case = W.make_case(cfg, seed=seed, fill=W.BF16_ZERO, num_blocks=args.num_blocks)
     copy_b, write_b, dec_b = step_bytes(case)
     total_b = copy_b + write_b + dec_b
     kv_tokens = int(case.seq_lens.sum())
@@ -429,8 +429,9 @@ def run_e2e(args, case, pa, stream, world, k_pool, v_pool):
     max_len_cap = case.max_seq_len + grow
 
     h_q = torch.from_numpy(np.ascontiguousarray(case.q).view(np.int16)).view(torch.bfloat16).pin_memory()
-    h_k = torch.from_numpy(np.ascontiguousarray(case.k_new).view(np.int16)).view(torch.bfloat16).pin_memory()
-    h_v = torch.from_numpy(np.ascontiguousarray(case.v_new).view(np.int16)).view(torch.bfloat16).pin_memory()
+    # one new token per sequence and step (the case may carry extra rows for its first step)
+    h_k = torch.from_numpy(np.ascontiguousarray(case.k_new[:case.batch]).view(np.int16)).view(torch.bfloat16).pin_memory()
+    h_v = torch.from_numpy(np.ascontiguousarray(case.v_new[:case.batch]).view(np.int16)).view(torch.bfloat16).pin_memory()
     h_tables = torch.empty((case.batch, max_blocks), dtype=torch.int32).pin_memory()
     h_lens = torch.empty(case.batch, dtype=torch.int32).pin_memory()
     h_slots = torch.empty(case.batch, dtype=torch.int32).pin_memory()
@@ -562,6 +563,8 @@ def main():
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--cpu-budget", type=float, default=12.0, help="seconds of oracle time")
+    ap.add_argument("--num-blocks", type=int, default=None,
+                    help="pool size override (same decode launch, smaller pool: for profiler captures)")
     args = ap.parse_args()
     if args.warmup < 3:
         ap.error("--warmup must be at least 3")

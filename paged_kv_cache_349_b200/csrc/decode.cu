@@ -58,7 +58,8 @@ struct Cfg {
     static constexpr int kTileBytes = kBoxes * kBoxBytes;  // K or V of one tile
     static constexpr int kStageBytes = 2 * kTileBytes;
     static constexpr int kRingBytes = kStages * kStageBytes;
-    static constexpr int kMergeBytes = kConsumerWarps * 8 * (HEAD_DIM + 2) * 4;
+    static constexpr int kMergeStride = HEAD_DIM + 4;  // padded row: conflict-free merge stores
+    static constexpr int kMergeBytes = kConsumerWarps * 8 * (kMergeStride + 2) * 4;
     static_assert(kMergeBytes <= kRingBytes, "merge area reuses the ring");
     static constexpr int kSmemBytes = 1024 /*align slack*/ + kRingBytes + kStages * 8 * 2 + kStages * 4;
 };
@@ -118,6 +119,9 @@ __global__ void __launch_bounds__(kThreads) paged_decode_kernel(
     const int tok_begin = part * p.part_tokens;
     const int tok_end = min(L, tok_begin + p.part_tokens);
     const int n_tiles = tok_end > tok_begin ? (tok_end - tok_begin + kTileTokens - 1) / kTileTokens : 0;
+    // Let the log-sum-exp reduce (launched as a programmatic dependent) get
+    // scheduled while this grid's last wave runs; it waits for our results.
+    if (SPLIT) asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
     if (SPLIT && n_tiles == 0) return;  // empty partition: the reduce skips it
     if (threadIdx.x == 0 && part == 0 && h == 0 && L != L_raw) raise_flag(p.err_flag, PA_FLAG_BAD_LEN);
 
@@ -328,13 +332,13 @@ __global__ void __launch_bounds__(kThreads) paged_decode_kernel(
 
     // ---------------- merge the warps' states (ring memory is free now) ----------------
     __syncthreads();
-    float *mo = reinterpret_cast<float *>(smem);                      // [W][8][HEAD_DIM]
-    float *mm = mo + kConsumerWarps * 8 * HEAD_DIM;                   // [W][8]
+    float *mo = reinterpret_cast<float *>(smem);                      // [W][8][kMergeStride]
+    float *mm = mo + kConsumerWarps * 8 * C::kMergeStride;            // [W][8]
     float *ml = mm + kConsumerWarps * 8;                              // [W][8]
     if (warp < kConsumerWarps) {
         const int gid = lane >> 2, tig = lane & 3;
-        float *w0 = mo + (warp * 8 + 2 * tig) * HEAD_DIM;
-        float *w1 = w0 + HEAD_DIM;
+        float *w0 = mo + (warp * 8 + 2 * tig) * C::kMergeStride;
+        float *w1 = w0 + C::kMergeStride;
 #pragma unroll
         for (int mt = 0; mt < HEAD_DIM / 16; ++mt) {
             w0[16 * mt + gid] = o[mt][0];
@@ -362,7 +366,7 @@ __global__ void __launch_bounds__(kThreads) paged_decode_kernel(
 #pragma unroll
             for (int w = 0; w < kConsumerWarps; ++w) {
                 const float f = fast_exp2(mm[w * 8 + n] - M);
-                num += f * mo[(w * 8 + n) * HEAD_DIM + d];
+                num += f * mo[(w * 8 + n) * C::kMergeStride + d];
                 den += f * ml[w * 8 + n];
             }
         }
@@ -381,27 +385,73 @@ __global__ void __launch_bounds__(kThreads) paged_decode_kernel(
 
 // Log-sum-exp merge of the partitions of one (sequence, query head):
 //   out = sum_p 2^(m_p - M) l_p o_p / sum_p 2^(m_p - M) l_p,  M = max_p m_p.
+// Four warps split the partitions; each lane owns HEAD_DIM/32 output dims.
+constexpr int kReduceThreads = 128;
+
 template <int HEAD_DIM>
-__global__ void __launch_bounds__(HEAD_DIM) lse_reduce_kernel(const DecodeParams p) {
+__global__ void __launch_bounds__(kReduceThreads) lse_reduce_kernel(const DecodeParams p) {
+    // Launched as a programmatic dependent of the decode grid: wait for its results.
+    asm volatile("griddepcontrol.wait;" ::: "memory");
+    constexpr int kWarps = kReduceThreads / 32;
+    constexpr int V = HEAD_DIM / 32;  // dims per lane: 4 or 2
+    __shared__ float s_max[kWarps];
+    __shared__ float s_den[kWarps];
+    __shared__ float s_acc[kWarps][HEAD_DIM];
     const int hq = blockIdx.x;
     const int b = blockIdx.y;
-    const int d = threadIdx.x;
+    const int warp = threadIdx.x >> 5;
+    const int lane = threadIdx.x & 31;
     const int L = clamp_len(__ldg(p.seq_lens + b), p);
     const int n = (L + p.part_tokens - 1) / p.part_tokens;
     const int64_t row = (int64_t)b * p.num_q_heads + hq;
-    const float *ml = p.part_ml + row * p.num_parts * 2;
-    const float *po = p.part_o + row * p.num_parts * HEAD_DIM + d;
+    const float2 *ml = reinterpret_cast<const float2 *>(p.part_ml + row * p.num_parts * 2);
+    const float *po = p.part_o + row * p.num_parts * HEAD_DIM + lane * V;
+
     float M = -INFINITY;
-    for (int i = 0; i < n; ++i) M = fmaxf(M, __ldg(ml + 2 * i));
-    float num = 0.f, den = 0.f;
+    for (int i = threadIdx.x; i < n; i += kReduceThreads) M = fmaxf(M, __ldg(&ml[i].x));
+#pragma unroll
+    for (int off = 16; off; off >>= 1) M = fmaxf(M, __shfl_xor_sync(0xffffffffu, M, off));
+    if (lane == 0) s_max[warp] = M;
+    __syncthreads();
+#pragma unroll
+    for (int w = 0; w < kWarps; ++w) M = fmaxf(M, s_max[w]);
+
+    float acc[V];
+#pragma unroll
+    for (int k = 0; k < V; ++k) acc[k] = 0.f;
+    float den = 0.f;
     if (M != -INFINITY) {
-        for (int i = 0; i < n; ++i) {
-            const float w = fast_exp2(__ldg(ml + 2 * i) - M) * __ldg(ml + 2 * i + 1);
-            num += w * __ldg(po + (int64_t)i * HEAD_DIM);
+#pragma unroll 4
+        for (int i = warp; i < n; i += kWarps) {
+            const float2 mlv = __ldg(&ml[i]);
+            const float w = fast_exp2(mlv.x - M) * mlv.y;
+            if constexpr (V == 4) {
+                const float4 v = __ldg(reinterpret_cast<const float4 *>(po + (int64_t)i * HEAD_DIM));
+                acc[0] += w * v.x;
+                acc[1] += w * v.y;
+                acc[2] += w * v.z;
+                acc[3] += w * v.w;
+            } else {
+                const float2 v = __ldg(reinterpret_cast<const float2 *>(po + (int64_t)i * HEAD_DIM));
+                acc[0] += w * v.x;
+                acc[1] += w * v.y;
+            }
             den += w;
         }
     }
-    p.out[row * HEAD_DIM + d] = den > 0.f ? num / den : 0.f;
+#pragma unroll
+    for (int k = 0; k < V; ++k) s_acc[warp][lane * V + k] = acc[k];
+    if (lane == 0) s_den[warp] = den;
+    __syncthreads();
+    for (int x = threadIdx.x; x < HEAD_DIM; x += kReduceThreads) {
+        float num = 0.f, dd = 0.f;
+#pragma unroll
+        for (int w = 0; w < kWarps; ++w) {
+            num += s_acc[w][x];
+            dd += s_den[w];
+        }
+        p.out[row * HEAD_DIM + x] = dd > 0.f ? num / dd : 0.f;
+    }
 }
 
 // ---------------------------------------------------------------------------
@@ -500,10 +550,19 @@ int launch_decode(const CUtensorMap &km, const CUtensorMap &vm, const DecodePara
     count_launch();
     int st = launch_status();
     if (st != PA_OK || !SPLIT) return st;
-    dim3 rgrid((unsigned)p.num_q_heads, (unsigned)batch);
-    lse_reduce_kernel<HEAD_DIM><<<rgrid, HEAD_DIM, 0, stream>>>(p);
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = dim3((unsigned)p.num_q_heads, (unsigned)batch);
+    cfg.blockDim = dim3(kReduceThreads);
+    cfg.dynamicSmemBytes = 0;
+    cfg.stream = stream;
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    attr[0].val.programmaticStreamSerializationAllowed = 1;
+    cfg.attrs = attr;
+    cfg.numAttrs = 1;
+    const cudaError_t e = cudaLaunchKernelEx(&cfg, lse_reduce_kernel<HEAD_DIM>, p);
     count_launch();
-    return launch_status();
+    return e == cudaSuccess ? launch_status() : PA_ERR_CUDA;
 }
 
 }  // namespace
