@@ -265,6 +265,13 @@ def run_native(args):
     q = bf16(case.q)
     k_new, v_new = bf16(case.k_new), bf16(case.v_new)
     slots = i32(case.slot_mapping)
+    # Fused step: each sequence's token at L-1 is written by the decode launch itself;
+    # any other new rows of the step (copy-on-write destinations) go through the cache write.
+    k_last_np, v_last_np, other = W.split_last_tokens(case)
+    k_last, v_last = bf16(k_last_np), bf16(v_last_np)
+    k_other, v_other = bf16(case.k_new[other]), bf16(case.v_new[other])
+    slots_other = i32(case.slot_mapping[other])
+    fused = not args.unfused
     pairs = i32(case.copy_pairs.reshape(-1, 2))
     tables, lens = i32(case.block_tables), i32(case.seq_lens)
     out = torch.empty(case.q.shape, dtype=torch.float32, device="cuda")
@@ -282,12 +289,21 @@ def run_native(args):
     def step(record=False):
         if case.copy_pairs.shape[0]:
             pa.pa_copy_blocks(k, v, pairs, err_flag=flag, stream=stream)
-        pa.pa_reshape_and_cache(k_new, v_new, k, v, slots, err_flag=flag, stream=stream)
+        if fused:
+            if other.size:
+                pa.pa_reshape_and_cache(k_other, v_other, k, v, slots_other, err_flag=flag, stream=stream)
+        else:
+            pa.pa_reshape_and_cache(k_new, v_new, k, v, slots, err_flag=flag, stream=stream)
         if record:
             e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
             e0.record(stream)
-        pa.pa_decode(out, q, k, v, tables, lens, max_seq_len=case.max_seq_len, scale=float(case.scale),
-                     partition_tokens=pt, workspace=ws, err_flag=flag, stream=stream)
+        if fused:
+            pa.pa_decode_append(out, q, k_last, v_last, k, v, tables, lens, max_seq_len=case.max_seq_len,
+                                scale=float(case.scale), partition_tokens=pt, workspace=ws, err_flag=flag,
+                                stream=stream)
+        else:
+            pa.pa_decode(out, q, k, v, tables, lens, max_seq_len=case.max_seq_len, scale=float(case.scale),
+                         partition_tokens=pt, workspace=ws, err_flag=flag, stream=stream)
         if record:
             e1.record(stream)
             dec_ev.append((e0, e1))
@@ -355,6 +371,8 @@ def run_native(args):
             "partition_tokens": resolved_pt,
             "parallelism": f"dp{world} (independent sequences per GPU, no collective)",
             "l2": f"inputs larger than L2: {dec_b / 1e9:.2f} GB of K/V per step vs 126 MB L2; no flush",
+            "step": ("block copies, then pa_decode_append (cache write fused into decode)" if fused else
+                     "block copies, pa_reshape_and_cache, pa_decode"),
         },
         "pct_of_peak": {"nominal_8TBps": round(100 * value / NOMINAL_HBM_GBS, 1),
                         f"{peak_kind}_{peak:.0f}GBps": round(100 * value / peak, 1)},
@@ -363,7 +381,8 @@ def run_native(args):
         "step_bytes": {"copy": copy_b, "write": write_b, "decode": dec_b},
         "gpu_launches": launches,
         "roofline": {
-            "kernel": "pa_decode" + (" (split kernel + LSE reduce)" if resolved_pt > 0 else " (single pass)"),
+            "kernel": ("pa_decode_append" if fused else "pa_decode") +
+                      (" (split kernel + LSE reduce)" if resolved_pt > 0 else " (single pass)"),
             "bound": "hbm",
             "achieved": round(achieved, 1),
             "peak": peak,
@@ -467,19 +486,28 @@ def run_e2e(args, case, pa, stream, world, k_pool, v_pool):
         d_q.copy_(h_q, non_blocking=True)
         d_k.copy_(h_k, non_blocking=True)
         d_v.copy_(h_v, non_blocking=True)
-        d_slots.copy_(h_slots, non_blocking=True)
+        if args.unfused:
+            d_slots.copy_(h_slots, non_blocking=True)
         d_tables.copy_(h_tables, non_blocking=True)
         d_lens.copy_(h_lens, non_blocking=True)
         if n_pairs:
             d_pairs[:n_pairs].copy_(h_pairs[:n_pairs], non_blocking=True)
             pa.pa_copy_blocks(k_pool, v_pool, d_pairs[:n_pairs], err_flag=flag, stream=stream)
-        pa.pa_reshape_and_cache(d_k, d_v, k_pool, v_pool, d_slots, err_flag=flag, stream=stream)
-        pa.pa_decode(d_out, d_q, k_pool, v_pool, d_tables, d_lens, max_seq_len=max_len, scale=float(case.scale),
-                     partition_tokens=case.partition_tokens, workspace=ws, err_flag=flag, stream=stream)
+        if args.unfused:
+            pa.pa_reshape_and_cache(d_k, d_v, k_pool, v_pool, d_slots, err_flag=flag, stream=stream)
+            pa.pa_decode(d_out, d_q, k_pool, v_pool, d_tables, d_lens, max_seq_len=max_len,
+                         scale=float(case.scale), partition_tokens=case.partition_tokens, workspace=ws,
+                         err_flag=flag, stream=stream)
+        else:
+            # slots from the allocator are implied by the tables: the fused launch writes at L-1
+            pa.pa_decode_append(d_out, d_q, d_k, d_v, k_pool, v_pool, d_tables, d_lens, max_seq_len=max_len,
+                                scale=float(case.scale), partition_tokens=case.partition_tokens, workspace=ws,
+                                err_flag=flag, stream=stream)
         h_out.copy_(d_out, non_blocking=True)
         stream.synchronize()  # the step's result is on the host
         if count:
-            bytes_acc["h2d"] += sum(t.numel() * t.element_size() for t in (h_q, h_k, h_v, h_slots, h_tables, h_lens))
+            sent = (h_q, h_k, h_v, h_tables, h_lens) + ((h_slots,) if args.unfused else ())
+            bytes_acc["h2d"] += sum(t.numel() * t.element_size() for t in sent)
             bytes_acc["h2d"] += n_pairs * 8
             bytes_acc["d2h"] += h_out.numel() * 4
             bytes_acc["tokens"] += int(lens.sum())
@@ -502,8 +530,8 @@ def run_e2e(args, case, pa, stream, world, k_pool, v_pool):
             "ms_per_step": round(dt * 1e3 / steps, 4),
             "h2d_bytes_per_step": bytes_acc["h2d"] // steps, "d2h_bytes_per_step": bytes_acc["d2h"] // steps,
             "kv_tokens_per_s": round(_sum_over_ranks(float(bytes_acc["tokens"]), world) / dt, 1),
-            "includes": "host allocator append + table export, H2D of q/k_new/v_new/slots/tables/lens, "
-                        "copy/write/decode launches, D2H of out"}
+            "includes": "host allocator append + table export, H2D of q/k_new/v_new/tables/lens "
+                        "(+ slots when unfused), copy/write/decode launches, D2H of out"}
 
 
 def step_bytes_from(case, lens, n_pairs):
@@ -563,6 +591,8 @@ def main():
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--cpu-budget", type=float, default=12.0, help="seconds of oracle time")
+    ap.add_argument("--unfused", action="store_true",
+                    help="time pa_reshape_and_cache + pa_decode instead of the fused pa_decode_append")
     ap.add_argument("--num-blocks", type=int, default=None,
                     help="pool size override (same decode launch, smaller pool: for profiler captures)")
     args = ap.parse_args()

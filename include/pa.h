@@ -162,6 +162,30 @@ int pa_decode(float *out, const void *q, const void *k_cache, const void *v_cach
               void *workspace, size_t workspace_bytes, int32_t *err_flag, void *stream);
 
 /* ------------------------------------------------------------------------
+ * Fused decode step: each sequence's new token is written to the cache and
+ * attended in the same launch ("Walk through paged attention end to end",
+ * conceptual paged_attention_decode: append the new K/V to the block of
+ * position next_pos, then attend over every position).
+ *
+ * Equivalent to pa_reshape_and_cache with
+ *     slot_mapping[b] = block_tables[b][(L-1)/bs] * bs + (L-1) % bs,  L = seq_lens[b]
+ * followed by pa_decode, but in one decode launch (plus the reduce when the
+ * call splits).  k_new, v_new: device bf16 [batch, num_kv_heads, head_dim],
+ * 16-byte aligned; row b is the token at position seq_lens[b] - 1 (seq_lens
+ * counts it).  Sequences with seq_lens[b] == 0, or longer than max_seq_len
+ * or their table (PA_FLAG_BAD_LEN), write nothing.  The block that receives
+ * the new token must belong to this sequence alone (the allocator's
+ * copy-on-write guarantees that; apply its copy pairs first).  Other
+ * arguments, layouts and errors: as pa_decode (the same workspace size).
+ * ---------------------------------------------------------------------- */
+int pa_decode_append(float *out, const void *q, const void *k_new, const void *v_new, void *k_cache,
+                     void *v_cache, const int32_t *block_tables, int max_blocks_per_seq,
+                     const int32_t *seq_lens, int batch, int max_seq_len, int num_q_heads,
+                     int num_kv_heads, int head_dim, int block_size, int64_t num_blocks, float scale,
+                     int partition_tokens, void *workspace, size_t workspace_bytes, int32_t *err_flag,
+                     void *stream);
+
+/* ------------------------------------------------------------------------
  * Decode with library-owned scratch (no workspace argument).
  *
  * The pages have no counterpart: this entry point is a convenience of this

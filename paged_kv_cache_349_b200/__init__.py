@@ -163,6 +163,33 @@ def pa_decode(out, q, k_cache, v_cache, block_tables, seq_lens, *, max_seq_len: 
         _stream(stream)), "pa_decode")
 
 
+def pa_decode_append(out, q, k_new, v_new, k_cache, v_cache, block_tables, seq_lens, *, max_seq_len: int,
+                     scale: float, partition_tokens: int = 0, workspace=None, err_flag=None, stream=None) -> None:
+    """Fused decode step: write each sequence's new token (k_new/v_new bf16 [B, Hkv, d], at
+    position seq_lens[b]-1) into the pools and decode, in one launch."""
+    torch = _torch()
+    B, Hq, d = q.shape
+    NB, Hkv, bs, d2 = k_cache.shape
+    if d2 != d or out.shape != q.shape or v_cache.shape != k_cache.shape:
+        raise ValueError("shape mismatch")
+    if tuple(k_new.shape) != (B, Hkv, d) or v_new.shape != k_new.shape:
+        raise ValueError("k_new/v_new must be [B, Hkv, d]")
+    if block_tables.dim() != 2 or block_tables.shape[0] != B or seq_lens.numel() != B:
+        raise ValueError("block_tables must be [B, max_blocks] and seq_lens [B]")
+    ws_ptr, ws_bytes = None, 0
+    if workspace is not None:
+        ws_ptr = _dev(workspace, workspace.dtype, "workspace")
+        ws_bytes = workspace.numel() * workspace.element_size()
+    _check(lib.pa_decode_append(
+        _dev(out, torch.float32, "out"), _dev(q, torch.bfloat16, "q"),
+        _dev(k_new, torch.bfloat16, "k_new"), _dev(v_new, torch.bfloat16, "v_new"),
+        _dev(k_cache, torch.bfloat16, "k_cache"), _dev(v_cache, torch.bfloat16, "v_cache"),
+        _dev(block_tables, torch.int32, "block_tables"), block_tables.shape[1],
+        _dev(seq_lens, torch.int32, "seq_lens"), B, int(max_seq_len), Hq, Hkv, d, bs, NB,
+        float(scale), int(partition_tokens), ws_ptr, ws_bytes, _opt_flag(err_flag),
+        _stream(stream)), "pa_decode_append")
+
+
 PA_DECODE_BUILTIN_SCRATCH_BYTES = 32 << 20
 
 

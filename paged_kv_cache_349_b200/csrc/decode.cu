@@ -72,6 +72,10 @@ struct DecodeParams {
     const int32_t *block_tables;
     const int32_t *seq_lens;
     int32_t *err_flag;
+    const uint16_t *k_new;      // [B, Hkv, d] bf16 (fused cache write only)
+    const uint16_t *v_new;
+    uint16_t *k_pool;           // pools, written by the fused cache write
+    uint16_t *v_pool;
     int64_t num_blocks;
     int max_blocks;
     int max_seq_len;
@@ -96,7 +100,7 @@ __device__ __forceinline__ uint32_t tile_offset(int r, int c) {
     return (uint32_t)((c >> 3) * kBoxBytes + r * 128 + (((c & 7) ^ (r & 7)) << 4));
 }
 
-template <int HEAD_DIM, bool SPLIT>
+template <int HEAD_DIM, bool SPLIT, bool APPEND>
 __global__ void __launch_bounds__(kThreads) paged_decode_kernel(
     const __grid_constant__ CUtensorMap k_map, const __grid_constant__ CUtensorMap v_map,
     const DecodeParams p) {
@@ -242,6 +246,32 @@ __global__ void __launch_bounds__(kThreads) paged_decode_kernel(
         const int v_row = ((lane & 7) >> 1 | ((lane & 1) << 2)) + (((lane >> 4) & 1) << 3);
         const int v_chunk_hi = (lane >> 3) & 1;
 
+        // Fused cache write ("append, then attend"): the warp that owns the tile
+        // holding position L-1 fetches the new token's K row (lanes 0..15) and
+        // V row (lanes 16..31) up front, stores them to the pool, and patches
+        // them into its staged tile before computing.  The block receiving the
+        // token is owned by this sequence alone (copy-on-write), so no other
+        // CTA reads that row.
+        int i_new = -1;
+        uint4 new_row = make_uint4(0u, 0u, 0u, 0u);
+        int64_t new_dst = -1;  // 16-byte chunk index of the row in the pool
+        if (APPEND && L == L_raw && L > 0 && L - 1 >= tok_begin && L - 1 < tok_end) {
+            const int it = (L - 1 - tok_begin) / kTileTokens;
+            if (it % kConsumerWarps == warp) {
+                i_new = it;
+                const int c = lane & 15;
+                const int64_t phys = __ldg(p.block_tables + (int64_t)b * p.max_blocks + (L - 1) / p.block_size);
+                if (c < HEAD_DIM / 8) {
+                    const uint16_t *src = (lane < 16 ? p.k_new : p.v_new) +
+                                          ((int64_t)b * p.num_kv_heads + h) * HEAD_DIM;
+                    new_row = __ldg(reinterpret_cast<const uint4 *>(src) + c);
+                    if (phys >= 0 && phys < p.num_blocks)
+                        new_dst = ((phys * p.num_kv_heads + h) * p.block_size + (L - 1) % p.block_size) *
+                                      (HEAD_DIM / 8) + c;
+                }
+            }
+        }
+
         for (int i = warp; i < n_tiles; i += kConsumerWarps) {
             const int s = i % kStages;
             const bool got = mbar_wait_bounded(&full[s], (i / kStages) & 1, p.err_flag);
@@ -261,6 +291,19 @@ __global__ void __launch_bounds__(kThreads) paged_decode_kernel(
                         const uint32_t a = vbase + bx * kBoxBytes + r * 128 + ((x & 7) << 4);
                         asm volatile("st.shared.v4.u32 [%0], {%1, %1, %1, %1};" ::"r"(a), "r"(0u)
                                      : "memory");
+                    }
+                    __syncwarp();
+                }
+                if (APPEND && i == i_new) {
+                    const int r = (L - 1) & (kTileTokens - 1);
+                    const int c = lane & 15;
+                    if (c < HEAD_DIM / 8) {
+                        const uint32_t a = (lane < 16 ? kbase : vbase) + tile_offset(r, c);
+                        asm volatile("st.shared.v4.u32 [%0], {%1, %2, %3, %4};" ::"r"(a), "r"(new_row.x),
+                                     "r"(new_row.y), "r"(new_row.z), "r"(new_row.w)
+                                     : "memory");
+                        if (new_dst >= 0)
+                            reinterpret_cast<uint4 *>(lane < 16 ? p.k_pool : p.v_pool)[new_dst] = new_row;
                     }
                     __syncwarp();
                 }
@@ -317,7 +360,7 @@ __global__ void __launch_bounds__(kThreads) paged_decode_kernel(
                     mma_bf16_16816(o[mt], a0r, a1r, a2r, a3r, bh0, bh1);
                     mma_bf16_16816(o[mt], a0r, a1r, a2r, a3r, bl0, bl1);
                 }
-                if (valid < kTileTokens) fence_proxy_async_smem();
+                if (valid < kTileTokens || (APPEND && i == i_new)) fence_proxy_async_smem();
             }
             __syncwarp();
             if (lane == 0) mbar_arrive(&empty[s]);
@@ -534,11 +577,11 @@ int resolve_partition(int batch, int num_kv_heads, int block_size, int max_seq_l
     return kDefaultPartition;
 }
 
-template <int HEAD_DIM, bool SPLIT>
+template <int HEAD_DIM, bool SPLIT, bool APPEND>
 int launch_decode(const CUtensorMap &km, const CUtensorMap &vm, const DecodeParams &p, int batch,
                   cudaStream_t stream) {
     using C = Cfg<HEAD_DIM>;
-    auto kern = paged_decode_kernel<HEAD_DIM, SPLIT>;
+    auto kern = paged_decode_kernel<HEAD_DIM, SPLIT, APPEND>;
     static std::once_flag once;
     static cudaError_t attr_err = cudaSuccess;
     std::call_once(once, [&] {
@@ -589,6 +632,83 @@ int builtin_scratch_address(void **out) {
     return PA_OK;
 }
 
+// Shared body of pa_decode and pa_decode_append (k_new == nullptr: no cache write).
+int decode_impl(float *out, const void *q, const void *k_new, const void *v_new, const void *k_cache,
+                const void *v_cache, const int32_t *block_tables, int max_blocks_per_seq,
+                const int32_t *seq_lens, int batch, int max_seq_len, int num_q_heads, int num_kv_heads,
+                int head_dim, int block_size, int64_t num_blocks, float scale, int partition_tokens,
+                void *workspace, size_t workspace_bytes, int32_t *err_flag, void *stream) {
+    const bool append = k_new != nullptr;
+    if (batch < 0 || max_seq_len < 0 || num_blocks <= 0 || max_blocks_per_seq < 0)
+        return PA_ERR_INVALID_ARG;
+    if (!supported_shape(num_q_heads, num_kv_heads, head_dim, block_size)) return PA_ERR_UNSUPPORTED;
+    if (batch == 0) return PA_OK;
+    if (!out || !q || !k_cache || !v_cache || !block_tables || !seq_lens) return PA_ERR_INVALID_ARG;
+    if (!aligned16(q) || !aligned16(k_cache) || !aligned16(v_cache) || !aligned16(out))
+        return PA_ERR_INVALID_ARG;
+    if (append && (!v_new || !aligned16(k_new) || !aligned16(v_new))) return PA_ERR_INVALID_ARG;
+    if (partition_tokens > 0 && partition_tokens % block_size) return PA_ERR_INVALID_ARG;
+    if (batch > 65535 || num_kv_heads > 65535) return PA_ERR_UNSUPPORTED;
+    const uint64_t rows = (uint64_t)num_blocks * (uint64_t)num_kv_heads * (uint64_t)block_size;
+    if (rows >= (1ull << 31)) return PA_ERR_UNSUPPORTED;  // TMA row coordinate is int32
+
+    DecodeParams p{};
+    p.out = out;
+    p.q = static_cast<const uint16_t *>(q);
+    p.block_tables = block_tables;
+    p.seq_lens = seq_lens;
+    p.err_flag = err_flag;
+    p.num_blocks = num_blocks;
+    p.max_blocks = max_blocks_per_seq;
+    p.max_seq_len = max_seq_len;
+    p.num_q_heads = num_q_heads;
+    p.num_kv_heads = num_kv_heads;
+    p.group = num_q_heads / num_kv_heads;
+    p.block_size = block_size;
+    p.scale_log2 = scale * kLog2e;
+    p.k_new = static_cast<const uint16_t *>(k_new);
+    p.v_new = static_cast<const uint16_t *>(v_new);
+    p.k_pool = static_cast<uint16_t *>(const_cast<void *>(k_cache));
+    p.v_pool = static_cast<uint16_t *>(const_cast<void *>(v_cache));
+
+    const int pt = max_seq_len > 0
+                       ? resolve_partition(batch, num_kv_heads, block_size, max_seq_len, partition_tokens)
+                       : -1;
+    const bool split = pt > 0;
+    if (split) {
+        const size_t need = pa_decode_workspace_size(batch, num_q_heads, num_kv_heads, head_dim,
+                                                     block_size, max_seq_len, partition_tokens);
+        if (!workspace || workspace_bytes < need || !aligned16(workspace)) return PA_ERR_INVALID_ARG;
+        p.part_tokens = pt;
+        p.num_parts = (max_seq_len + pt - 1) / pt;
+        const int64_t prow = (int64_t)batch * num_q_heads * p.num_parts;
+        p.part_o = static_cast<float *>(workspace);
+        p.part_ml = reinterpret_cast<float *>(static_cast<char *>(workspace) +
+                                              ((prow * head_dim * 4) + 255) / 256 * 256);
+        if (p.num_parts > 65535) return PA_ERR_UNSUPPORTED;
+    } else {
+        p.part_tokens = max_seq_len > 0 ? max_seq_len : 1;
+        p.num_parts = 1;
+    }
+
+    CUtensorMap km, vm;
+    if (!pool_tensor_map(k_cache, rows, head_dim, &km) || !pool_tensor_map(v_cache, rows, head_dim, &vm))
+        return PA_ERR_CUDA;
+    cudaStream_t s = static_cast<cudaStream_t>(stream);
+    if (head_dim == 128) {
+        if (append)
+            return split ? launch_decode<128, true, true>(km, vm, p, batch, s)
+                         : launch_decode<128, false, true>(km, vm, p, batch, s);
+        return split ? launch_decode<128, true, false>(km, vm, p, batch, s)
+                     : launch_decode<128, false, false>(km, vm, p, batch, s);
+    }
+    if (append)
+        return split ? launch_decode<64, true, true>(km, vm, p, batch, s)
+                     : launch_decode<64, false, true>(km, vm, p, batch, s);
+    return split ? launch_decode<64, true, false>(km, vm, p, batch, s)
+                 : launch_decode<64, false, false>(km, vm, p, batch, s);
+}
+
 }  // namespace pa
 
 extern "C" {
@@ -617,62 +737,21 @@ int pa_decode(float *out, const void *q, const void *k_cache, const void *v_cach
               int batch, int max_seq_len, int num_q_heads, int num_kv_heads, int head_dim,
               int block_size, int64_t num_blocks, float scale, int partition_tokens,
               void *workspace, size_t workspace_bytes, int32_t *err_flag, void *stream) {
-    if (batch < 0 || max_seq_len < 0 || num_blocks <= 0 || max_blocks_per_seq < 0)
-        return PA_ERR_INVALID_ARG;
-    if (!pa::supported_shape(num_q_heads, num_kv_heads, head_dim, block_size)) return PA_ERR_UNSUPPORTED;
-    if (batch == 0) return PA_OK;
-    if (!out || !q || !k_cache || !v_cache || !block_tables || !seq_lens) return PA_ERR_INVALID_ARG;
-    if (!pa::aligned16(q) || !pa::aligned16(k_cache) || !pa::aligned16(v_cache) || !pa::aligned16(out))
-        return PA_ERR_INVALID_ARG;
-    if (partition_tokens > 0 && partition_tokens % block_size) return PA_ERR_INVALID_ARG;
-    if (batch > 65535 || num_kv_heads > 65535) return PA_ERR_UNSUPPORTED;
-    const uint64_t rows = (uint64_t)num_blocks * (uint64_t)num_kv_heads * (uint64_t)block_size;
-    if (rows >= (1ull << 31)) return PA_ERR_UNSUPPORTED;  // TMA row coordinate is int32
+    return pa::decode_impl(out, q, nullptr, nullptr, k_cache, v_cache, block_tables, max_blocks_per_seq,
+                           seq_lens, batch, max_seq_len, num_q_heads, num_kv_heads, head_dim, block_size,
+                           num_blocks, scale, partition_tokens, workspace, workspace_bytes, err_flag, stream);
+}
 
-    pa::DecodeParams p{};
-    p.out = out;
-    p.q = static_cast<const uint16_t *>(q);
-    p.block_tables = block_tables;
-    p.seq_lens = seq_lens;
-    p.err_flag = err_flag;
-    p.num_blocks = num_blocks;
-    p.max_blocks = max_blocks_per_seq;
-    p.max_seq_len = max_seq_len;
-    p.num_q_heads = num_q_heads;
-    p.num_kv_heads = num_kv_heads;
-    p.group = num_q_heads / num_kv_heads;
-    p.block_size = block_size;
-    p.scale_log2 = scale * pa::kLog2e;
-
-    const int pt = max_seq_len > 0
-                       ? pa::resolve_partition(batch, num_kv_heads, block_size, max_seq_len, partition_tokens)
-                       : -1;
-    const bool split = pt > 0;
-    if (split) {
-        const size_t need = pa_decode_workspace_size(batch, num_q_heads, num_kv_heads, head_dim,
-                                                     block_size, max_seq_len, partition_tokens);
-        if (!workspace || workspace_bytes < need || !pa::aligned16(workspace)) return PA_ERR_INVALID_ARG;
-        p.part_tokens = pt;
-        p.num_parts = (max_seq_len + pt - 1) / pt;
-        const int64_t prow = (int64_t)batch * num_q_heads * p.num_parts;
-        p.part_o = static_cast<float *>(workspace);
-        p.part_ml = reinterpret_cast<float *>(static_cast<char *>(workspace) +
-                                              ((prow * head_dim * 4) + 255) / 256 * 256);
-        if (p.num_parts > 65535) return PA_ERR_UNSUPPORTED;
-    } else {
-        p.part_tokens = max_seq_len > 0 ? max_seq_len : 1;
-        p.num_parts = 1;
-    }
-
-    CUtensorMap km, vm;
-    if (!pa::pool_tensor_map(k_cache, rows, head_dim, &km) || !pa::pool_tensor_map(v_cache, rows, head_dim, &vm))
-        return PA_ERR_CUDA;
-    cudaStream_t s = static_cast<cudaStream_t>(stream);
-    if (head_dim == 128)
-        return split ? pa::launch_decode<128, true>(km, vm, p, batch, s)
-                     : pa::launch_decode<128, false>(km, vm, p, batch, s);
-    return split ? pa::launch_decode<64, true>(km, vm, p, batch, s)
-                 : pa::launch_decode<64, false>(km, vm, p, batch, s);
+int pa_decode_append(float *out, const void *q, const void *k_new, const void *v_new, void *k_cache,
+                     void *v_cache, const int32_t *block_tables, int max_blocks_per_seq,
+                     const int32_t *seq_lens, int batch, int max_seq_len, int num_q_heads,
+                     int num_kv_heads, int head_dim, int block_size, int64_t num_blocks, float scale,
+                     int partition_tokens, void *workspace, size_t workspace_bytes, int32_t *err_flag,
+                     void *stream) {
+    if (batch > 0 && (!k_new || !v_new)) return PA_ERR_INVALID_ARG;
+    return pa::decode_impl(out, q, k_new, v_new, k_cache, v_cache, block_tables, max_blocks_per_seq,
+                           seq_lens, batch, max_seq_len, num_q_heads, num_kv_heads, head_dim, block_size,
+                           num_blocks, scale, partition_tokens, workspace, workspace_bytes, err_flag, stream);
 }
 
 int pa_decode_builtin_scratch(float *out, const void *q, const void *k_cache, const void *v_cache,

@@ -77,3 +77,25 @@ def sample_rows(case, n, seed=0):
     b[0] = int(np.argmax(case.seq_lens))
     b[1] = int(np.argmin(case.seq_lens))
     return np.stack([b, g], axis=1).astype(np.int32)
+
+
+def run_fused_step(dc, partition_tokens=None):
+    """copy_blocks -> (cache write of tokens other than each sequence's last) -> pa_decode_append."""
+    import torch
+    import paged_kv_cache_349_b200 as pa
+    c = dc.case
+    pt = c.partition_tokens if partition_tokens is None else partition_tokens
+    import workloads as W
+    k_last, v_last, other = W.split_last_tokens(c)
+    pa.pa_copy_blocks(dc.k, dc.v, dc.pairs, err_flag=dc.flag)
+    if other.size:
+        pa.pa_reshape_and_cache(bf16_dev(c.k_new[other]), bf16_dev(c.v_new[other]), dc.k, dc.v,
+                                i32_dev(c.slot_mapping[other]), err_flag=dc.flag)
+    ws_bytes = pa.pa_decode_workspace_size(c.batch, c.num_q_heads, c.num_kv_heads, c.head_dim,
+                                           c.block_size, c.max_seq_len, pt)
+    ws = torch.empty(max(ws_bytes, 16), dtype=torch.uint8, device="cuda") if ws_bytes else None
+    pa.pa_decode_append(dc.out, dc.q, bf16_dev(k_last), bf16_dev(v_last), dc.k, dc.v, dc.tables, dc.lens,
+                        max_seq_len=c.max_seq_len, scale=float(c.scale), partition_tokens=pt, workspace=ws,
+                        err_flag=dc.flag)
+    torch.cuda.synchronize()
+    return dc.out.cpu().numpy().astype(np.float64)

@@ -400,6 +400,31 @@ def _make_chat_case(rng, seed, *, fill, batch, max_len, num_blocks, poison_paddi
                    partition_tokens=0 if partition_tokens is None else partition_tokens)
 
 
+def split_last_tokens(case: DecodeCase):
+    """Split a step's new tokens into each sequence's token at position L-1 (ordered by
+    sequence, zero rows for empty sequences) and the remaining token indices.
+
+    Returns (k_last [B, Hkv, d], v_last [B, Hkv, d], other: int64 indices into k_new).
+    """
+    bs = case.block_size
+    want = {}
+    for b, L in enumerate(case.seq_lens):
+        if L > 0:
+            want[int(case.block_tables[b, (L - 1) // bs]) * bs + (int(L) - 1) % bs] = b
+    B, Hkv, d = case.batch, case.num_kv_heads, case.head_dim
+    k_last = np.zeros((B, Hkv, d), np.uint16)
+    v_last = np.zeros((B, Hkv, d), np.uint16)
+    other = []
+    for t, s in enumerate(case.slot_mapping):
+        b = want.get(int(s))
+        if b is None:
+            other.append(t)
+        else:
+            k_last[b] = case.k_new[t]
+            v_last[b] = case.v_new[t]
+    return k_last, v_last, np.array(other, dtype=np.int64)
+
+
 def algorithmic_decode_bytes(case_or_lens, *, num_q_heads=None, num_kv_heads=None,
                              head_dim=None, block_size=None) -> int:
     """Bytes a decode call must move at minimum: K+V rows once, q, fp32 out, table entries, lengths."""
