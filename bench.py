@@ -341,7 +341,7 @@ def run_native(args):
     peak, peak_kind = _measured_peak()
     achieved = dec_b / (dec_ms / 1e3) / 1e9
 
-    e2e = run_e2e(args, case, pa, stream, world, k, v) if not args.no_e2e else None
+    e2e = run_e2e(args, case, pa, stream, world, k, v) if not (args.no_e2e or args.unfused) else None
 
     traffic = None
     rec = _decode_traffic_record()
@@ -438,7 +438,14 @@ def replay_allocator(pa, case):
 
 
 def run_e2e(args, case, pa, stream, world, k_pool, v_pool):
-    """The same step through the public API with host buffers (pinned), timed end to end."""
+    """The same step through the public API with host buffers (pinned), timed end to end.
+
+    Every step: the host allocator appends one token per sequence (and reports
+    copy-on-write pairs), exports the tables into pinned memory, and one
+    ``pa_decode_step_host`` call uploads the step's inputs, applies the copies,
+    runs the fused cache write + decode and copies the output back; the step
+    ends when the output is on the host.
+    """
     import torch
     bs = case.block_size
     steps, warm = args.steps, args.warmup
@@ -446,73 +453,47 @@ def run_e2e(args, case, pa, stream, world, k_pool, v_pool):
     alloc, sids = replay_allocator(pa, case)
     max_blocks = case.max_blocks_per_seq + (grow + bs - 1) // bs + 1
     max_len_cap = case.max_seq_len + grow
+    B = case.batch
 
-    h_q = torch.from_numpy(np.ascontiguousarray(case.q).view(np.int16)).view(torch.bfloat16).pin_memory()
+    def pinned_bf16(a):
+        return torch.from_numpy(np.ascontiguousarray(a).view(np.int16)).view(torch.bfloat16).pin_memory()
+
     # one new token per sequence and step (the case may carry extra rows for its first step)
-    h_k = torch.from_numpy(np.ascontiguousarray(case.k_new[:case.batch]).view(np.int16)).view(torch.bfloat16).pin_memory()
-    h_v = torch.from_numpy(np.ascontiguousarray(case.v_new[:case.batch]).view(np.int16)).view(torch.bfloat16).pin_memory()
-    h_tables = torch.empty((case.batch, max_blocks), dtype=torch.int32).pin_memory()
-    h_lens = torch.empty(case.batch, dtype=torch.int32).pin_memory()
-    h_slots = torch.empty(case.batch, dtype=torch.int32).pin_memory()
-    h_pairs = torch.empty((case.batch, 2), dtype=torch.int32).pin_memory()
+    h_q = pinned_bf16(case.q)
+    h_k = pinned_bf16(case.k_new[:B])
+    h_v = pinned_bf16(case.v_new[:B])
+    h_tables = torch.empty((B, max_blocks), dtype=torch.int32).pin_memory()
+    h_lens = torch.empty(B, dtype=torch.int32).pin_memory()
+    h_pairs = torch.zeros((B, 2), dtype=torch.int32).pin_memory()
     h_out = torch.empty(case.q.shape, dtype=torch.float32).pin_memory()
-    d_q = torch.empty_like(h_q, device="cuda")
-    d_k = torch.empty_like(h_k, device="cuda")
-    d_v = torch.empty_like(h_v, device="cuda")
-    d_tables = torch.empty_like(h_tables, device="cuda")
-    d_lens = torch.empty_like(h_lens, device="cuda")
-    d_slots = torch.empty_like(h_slots, device="cuda")
-    d_pairs = torch.empty_like(h_pairs, device="cuda")
-    d_out = torch.empty_like(h_out, device="cuda")
-    ws_bytes = pa.pa_decode_workspace_size(case.batch, case.num_q_heads, case.num_kv_heads, case.head_dim,
-                                           bs, max_len_cap, case.partition_tokens)
-    ws = torch.empty(max(ws_bytes, 16), dtype=torch.uint8, device="cuda")
-    # the pools stay resident: they are the cache, not an input of the step
-    tables_np = h_tables.numpy()
-    lens_np = h_lens.numpy()
+    tables_np, lens_np, pairs_np = h_tables.numpy(), h_lens.numpy(), h_pairs.numpy()
     flag = torch.zeros(1, dtype=torch.int32, device="cuda")
-    bytes_acc = {"h2d": 0, "d2h": 0, "alg": 0, "tokens": 0}
+    size = pa.pa_decode_step_staging_size(B, max_blocks, B, case.num_q_heads, case.num_kv_heads, case.head_dim, bs,
+                                          max_len_cap, case.partition_tokens)
+    staging = torch.empty(size, dtype=torch.uint8, device="cuda")
+    if args.unfused:
+        raise SystemExit("--unfused applies to the device-resident step only")
+    run = pa.DecodeStepHost(out_host=h_out, q_host=h_q, k_new_host=h_k, v_new_host=h_v, tables_host=h_tables,
+                            lens_host=h_lens, pairs_host=h_pairs, k_cache=k_pool, v_cache=v_pool,
+                            scale=float(case.scale), partition_tokens=case.partition_tokens, staging=staging,
+                            err_flag=flag, stream=stream)
+    acc = {"h2d": 0, "d2h": 0, "alg": 0, "tokens": 0}
 
     def e2e_step(count):
-        slots, pairs = alloc.append_batch(sids)
-        t, lens = alloc.export(sids, max_blocks)
-        tables_np[:] = t
-        lens_np[:] = lens
-        h_slots.numpy()[:] = slots
+        _, pairs = alloc.append_batch(sids)
+        alloc.export(sids, max_blocks, tables=tables_np, lens=lens_np)
         n_pairs = pairs.shape[0]
         if n_pairs:
-            h_pairs.numpy()[:n_pairs] = pairs
-        max_len = int(lens.max())
-        d_q.copy_(h_q, non_blocking=True)
-        d_k.copy_(h_k, non_blocking=True)
-        d_v.copy_(h_v, non_blocking=True)
-        if args.unfused:
-            d_slots.copy_(h_slots, non_blocking=True)
-        d_tables.copy_(h_tables, non_blocking=True)
-        d_lens.copy_(h_lens, non_blocking=True)
-        if n_pairs:
-            d_pairs[:n_pairs].copy_(h_pairs[:n_pairs], non_blocking=True)
-            pa.pa_copy_blocks(k_pool, v_pool, d_pairs[:n_pairs], err_flag=flag, stream=stream)
-        if args.unfused:
-            pa.pa_reshape_and_cache(d_k, d_v, k_pool, v_pool, d_slots, err_flag=flag, stream=stream)
-            pa.pa_decode(d_out, d_q, k_pool, v_pool, d_tables, d_lens, max_seq_len=max_len,
-                         scale=float(case.scale), partition_tokens=case.partition_tokens, workspace=ws,
-                         err_flag=flag, stream=stream)
-        else:
-            # slots from the allocator are implied by the tables: the fused launch writes at L-1
-            pa.pa_decode_append(d_out, d_q, d_k, d_v, k_pool, v_pool, d_tables, d_lens, max_seq_len=max_len,
-                                scale=float(case.scale), partition_tokens=case.partition_tokens, workspace=ws,
-                                err_flag=flag, stream=stream)
-        h_out.copy_(d_out, non_blocking=True)
-        stream.synchronize()  # the step's result is on the host
+            pairs_np[:n_pairs] = pairs
+        max_len = int(lens_np.max())
+        run(max_len, n_pairs)
+        stream.synchronize()  # the step's output is on the host
         if count:
-            sent = (h_q, h_k, h_v, h_tables, h_lens) + ((h_slots,) if args.unfused else ())
-            bytes_acc["h2d"] += sum(t.numel() * t.element_size() for t in sent)
-            bytes_acc["h2d"] += n_pairs * 8
-            bytes_acc["d2h"] += h_out.numel() * 4
-            bytes_acc["tokens"] += int(lens.sum())
-            c, w, d = step_bytes_from(case, lens, n_pairs)
-            bytes_acc["alg"] += c + w + d
+            acc["h2d"] += sum(t.numel() * t.element_size() for t in (h_q, h_k, h_v, h_tables, h_lens)) + n_pairs * 8
+            acc["d2h"] += h_out.numel() * 4
+            acc["tokens"] += int(lens_np.sum())
+            c, w, d = step_bytes_from(case, lens_np, n_pairs)
+            acc["alg"] += c + w + d
 
     for _ in range(warm):
         e2e_step(False)
@@ -524,14 +505,15 @@ def run_e2e(args, case, pa, stream, world, k_pool, v_pool):
     dt = time.perf_counter() - t0
     dt = _max_over_ranks(dt, world)
     assert int(flag.item()) == 0
-    alg = _sum_over_ranks(float(bytes_acc["alg"]), world)
+    alg = _sum_over_ranks(float(acc["alg"]), world)
     alloc.close()
     return {"value": round(alg / dt / 1e9, 1), "unit": "GB/s",
             "ms_per_step": round(dt * 1e3 / steps, 4),
-            "h2d_bytes_per_step": bytes_acc["h2d"] // steps, "d2h_bytes_per_step": bytes_acc["d2h"] // steps,
-            "kv_tokens_per_s": round(_sum_over_ranks(float(bytes_acc["tokens"]), world) / dt, 1),
-            "includes": "host allocator append + table export, H2D of q/k_new/v_new/tables/lens "
-                        "(+ slots when unfused), copy/write/decode launches, D2H of out"}
+            "h2d_bytes_per_step": acc["h2d"] // steps, "d2h_bytes_per_step": acc["d2h"] // steps,
+            "kv_tokens_per_s": round(_sum_over_ranks(float(acc["tokens"]), world) / dt, 1),
+            "includes": "host allocator batched append + table export into pinned memory, then one "
+                        "pa_decode_step_host call: H2D of q/k_new/v_new/tables/lens/copy pairs, block copies, "
+                        "fused cache write + decode, D2H of out; timed until out is on the host"}
 
 
 def step_bytes_from(case, lens, n_pairs):

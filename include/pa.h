@@ -186,6 +186,41 @@ int pa_decode_append(float *out, const void *q, const void *k_new, const void *v
                      void *stream);
 
 /* ------------------------------------------------------------------------
+ * One decode step from host buffers.  Enqueues on `stream`, in order:
+ *   1. host-to-device copies of q, k_new, v_new, the block tables, the
+ *      sequence lengths and the copy pairs into `staging` (one
+ *      cudaMemcpyAsync per input),
+ *   2. pa_copy_blocks of the copy pairs (if any),
+ *   3. pa_decode_append (cache write of each sequence's new token + decode),
+ *   4. a device-to-host copy of the fp32 output into out_host.
+ * The call returns once everything is enqueued; synchronise the stream
+ * before reading out_host.  Host buffers should be page-locked (pinned)
+ * for the copies to be asynchronous, and must stay valid and unchanged
+ * until the stream has passed them.
+ *
+ * Host inputs: q_host bf16 [batch, Hq, d]; k_new_host, v_new_host bf16
+ * [batch, Hkv, d] (the token at position seq_lens[b]-1); block_tables_host
+ * int32 [batch, max_blocks_per_seq]; seq_lens_host int32 [batch];
+ * copy_pairs_host int32 [num_pairs, 2] (may be NULL when num_pairs == 0).
+ * Host output: out_host fp32 [batch, Hq, d].
+ * staging: device memory of at least pa_decode_step_staging_size(...) bytes
+ * (computed with the same batch, max_blocks_per_seq, max_copy_pairs and
+ * shapes, and a max_seq_len at least this call's), 256-byte aligned; it
+ * holds the uploaded inputs, the device output and the decode workspace.
+ * Other arguments, layouts and errors: as pa_decode_append.
+ * ---------------------------------------------------------------------- */
+size_t pa_decode_step_staging_size(int batch, int max_blocks_per_seq, int max_copy_pairs, int num_q_heads,
+                                   int num_kv_heads, int head_dim, int block_size, int max_seq_len,
+                                   int partition_tokens);
+
+int pa_decode_step_host(float *out_host, const void *q_host, const void *k_new_host, const void *v_new_host,
+                        const int32_t *block_tables_host, int max_blocks_per_seq, const int32_t *seq_lens_host,
+                        const int32_t *copy_pairs_host, int num_pairs, int max_copy_pairs, void *k_cache,
+                        void *v_cache, int batch, int max_seq_len, int num_q_heads, int num_kv_heads,
+                        int head_dim, int block_size, int64_t num_blocks, float scale, int partition_tokens,
+                        void *staging, size_t staging_bytes, int32_t *err_flag, void *stream);
+
+/* ------------------------------------------------------------------------
  * Decode with library-owned scratch (no workspace argument).
  *
  * The pages have no counterpart: this entry point is a convenience of this

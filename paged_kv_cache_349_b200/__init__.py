@@ -190,6 +190,53 @@ def pa_decode_append(out, q, k_new, v_new, k_cache, v_cache, block_tables, seq_l
         _stream(stream)), "pa_decode_append")
 
 
+def pa_decode_step_staging_size(batch, max_blocks_per_seq, max_copy_pairs, num_q_heads, num_kv_heads, head_dim,
+                                block_size, max_seq_len, partition_tokens=0) -> int:
+    return int(lib.pa_decode_step_staging_size(batch, max_blocks_per_seq, max_copy_pairs, num_q_heads,
+                                               num_kv_heads, head_dim, block_size, max_seq_len, partition_tokens))
+
+
+class DecodeStepHost:
+    """One decode step from host buffers through ``pa_decode_step_host``.
+
+    Holds the argument tuple for a fixed set of pinned host buffers, pools and
+    staging, so each step only marshals what changes (max_seq_len, the number of
+    copy pairs).  Host arrays are torch CPU tensors (pinned); pools and staging are
+    CUDA tensors.
+    """
+
+    def __init__(self, *, out_host, q_host, k_new_host, v_new_host, tables_host, lens_host, pairs_host,
+                 k_cache, v_cache, scale: float, partition_tokens: int = 0, staging=None, err_flag=None,
+                 stream=None):
+        torch = _torch()
+        B, Hq, d = q_host.shape
+        NB, Hkv, bs, d2 = k_cache.shape
+        if d2 != d or tuple(out_host.shape) != (B, Hq, d) or tuple(k_new_host.shape) != (B, Hkv, d):
+            raise ValueError("shape mismatch")
+        for t, dt, name in ((out_host, torch.float32, "out_host"), (q_host, torch.bfloat16, "q_host"),
+                            (k_new_host, torch.bfloat16, "k_new_host"), (v_new_host, torch.bfloat16, "v_new_host"),
+                            (tables_host, torch.int32, "tables_host"), (lens_host, torch.int32, "lens_host"),
+                            (pairs_host, torch.int32, "pairs_host")):
+            if t.is_cuda or t.dtype != dt or not t.is_contiguous():
+                raise TypeError(f"{name} must be a contiguous host {dt} tensor")
+        self.max_blocks = int(tables_host.shape[1])
+        self.max_pairs = int(pairs_host.shape[0])
+        self.staging = staging
+        self._head = (ctypes.c_void_p(out_host.data_ptr()), ctypes.c_void_p(q_host.data_ptr()),
+                      ctypes.c_void_p(k_new_host.data_ptr()), ctypes.c_void_p(v_new_host.data_ptr()),
+                      ctypes.c_void_p(tables_host.data_ptr()), self.max_blocks,
+                      ctypes.c_void_p(lens_host.data_ptr()), ctypes.c_void_p(pairs_host.data_ptr()))
+        self._kv = (self.max_pairs, _dev(k_cache, torch.bfloat16, "k_cache"), _dev(v_cache, torch.bfloat16, "v_cache"),
+                    B)
+        self._shape = (Hq, Hkv, d, bs, NB, float(scale), int(partition_tokens))
+        self._tail = (ctypes.c_void_p(staging.data_ptr()), staging.numel() * staging.element_size(),
+                      _opt_flag(err_flag), _stream(stream))
+
+    def __call__(self, max_seq_len: int, num_pairs: int = 0) -> None:
+        _check(lib.pa_decode_step_host(*self._head, int(num_pairs), *self._kv, int(max_seq_len), *self._shape,
+                                       *self._tail), "pa_decode_step_host")
+
+
 PA_DECODE_BUILTIN_SCRATCH_BYTES = 32 << 20
 
 
@@ -288,10 +335,18 @@ class Allocator:
                                       ctypes.byref(nt)), "pa_seq_block_table")
         return out[:nb.value].copy(), nt.value
 
-    def export(self, seq_ids, max_blocks: int, pad: int = -1) -> Tuple[np.ndarray, np.ndarray]:
+    def export(self, seq_ids, max_blocks: int, pad: int = -1, tables: Optional[np.ndarray] = None,
+               lens: Optional[np.ndarray] = None) -> Tuple[np.ndarray, np.ndarray]:
+        """Padded int32 tables [n, max_blocks] and lengths [n]; written into ``tables`` /
+        ``lens`` when given (e.g. numpy views of pinned buffers)."""
         ids = np.ascontiguousarray(seq_ids, dtype=np.int32)
-        tables = np.empty((ids.size, max_blocks), dtype=np.int32)
-        lens = np.empty(ids.size, dtype=np.int32)
+        if tables is None:
+            tables = np.empty((ids.size, max_blocks), dtype=np.int32)
+        if lens is None:
+            lens = np.empty(ids.size, dtype=np.int32)
+        if (tables.dtype != np.int32 or not tables.flags.c_contiguous or tables.shape != (ids.size, max_blocks)
+                or lens.dtype != np.int32 or not lens.flags.c_contiguous or lens.shape != (ids.size,)):
+            raise ValueError("tables/lens must be contiguous int32 [n, max_blocks] / [n]")
         _check(lib.pa_alloc_export(self._h, _np_ptr(ids), ids.size, _np_ptr(tables), max_blocks, pad,
                                    _np_ptr(lens)), "pa_alloc_export")
         return tables, lens

@@ -29,6 +29,9 @@ SIGNATURES = {
     "pa_decode_partition_tokens": (_I, [_I, _I, _I, _I, _I, _I, _I]),
     "pa_decode": (_I, [_P, _P, _P, _P, _P, _I, _P, _I, _I, _I, _I, _I, _I, _I64, _F, _I, _P, _SZ, _P, _P]),
     "pa_decode_append": (_I, [_P, _P, _P, _P, _P, _P, _P, _I, _P, _I, _I, _I, _I, _I, _I, _I64, _F, _I, _P, _SZ, _P, _P]),
+    "pa_decode_step_staging_size": (_SZ, [_I, _I, _I, _I, _I, _I, _I, _I, _I]),
+    "pa_decode_step_host": (_I, [_P, _P, _P, _P, _P, _I, _P, _P, _I, _I, _P, _P, _I, _I, _I, _I, _I, _I, _I64, _F,
+                                 _I, _P, _SZ, _P, _P]),
     "pa_decode_builtin_scratch": (_I, [_P, _P, _P, _P, _P, _I, _P, _I, _I, _I, _I, _I, _I, _I64, _F, _I, _P, _P]),
     "pa_alloc_create": (_I, [_I, _I, ctypes.POINTER(_P)]),
     "pa_alloc_create_ordered": (_I, [_I, _I, _P, ctypes.POINTER(_P)]),

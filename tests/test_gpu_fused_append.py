@@ -60,3 +60,48 @@ def test_full_size_llama2_7b_sampled_rows():
     want, k_ref, v_ref = oracle.decode_step(case, rows=rows)
     assert np.array_equal(bits_host(dc.k), k_ref) and np.array_equal(bits_host(dc.v), v_ref)
     assert_close(got[rows[:, 0], rows[:, 1]], want, "cfg2 full fused")
+
+
+@pytest.mark.parametrize("cfg,kw", [
+    (2, dict(batch=6, max_len=300, num_blocks=256)),
+    (4, dict(batch=9, max_len=1500, num_blocks=512)),
+    (5, dict(batch=2, max_len=2048, num_blocks=640, num_copy_pairs=40)),
+])
+def test_host_step_matches_device_path(cfg, kw):
+    """pa_decode_step_host (uploads, copies, fused decode, download) == the device-resident path."""
+    import torch
+    import paged_kv_cache_349_b200 as pa
+    case = W.make_case(cfg, **kw)
+    k_last, v_last, other = W.split_last_tokens(case)
+    assert other.size == 0
+    ref = DeviceCase(case)
+    want = run_fused_step(ref)
+    dc = DeviceCase(case)
+
+    def pinned(a, dtype):
+        t = torch.from_numpy(np.ascontiguousarray(a))
+        return (t.view(dtype) if dtype is torch.bfloat16 else t.to(dtype)).pin_memory()
+
+    out_h = torch.full(case.q.shape, float("nan"), dtype=torch.float32).pin_memory()
+    pairs = case.copy_pairs.reshape(-1, 2)
+    max_pairs = max(1, pairs.shape[0])
+    pairs_h = torch.zeros((max_pairs, 2), dtype=torch.int32)
+    pairs_h[:pairs.shape[0]] = torch.from_numpy(pairs)
+    pairs_h = pairs_h.pin_memory()
+    size = pa.pa_decode_step_staging_size(case.batch, case.max_blocks_per_seq, max_pairs, case.num_q_heads,
+                                          case.num_kv_heads, case.head_dim, case.block_size, case.max_seq_len,
+                                          case.partition_tokens)
+    staging = torch.empty(size, dtype=torch.uint8, device="cuda")
+    step = pa.DecodeStepHost(out_host=out_h, q_host=pinned(case.q.view(np.int16), torch.bfloat16),
+                             k_new_host=pinned(k_last.view(np.int16), torch.bfloat16),
+                             v_new_host=pinned(v_last.view(np.int16), torch.bfloat16),
+                             tables_host=pinned(case.block_tables, torch.int32),
+                             lens_host=pinned(case.seq_lens, torch.int32), pairs_host=pairs_h,
+                             k_cache=dc.k, v_cache=dc.v, scale=float(case.scale),
+                             partition_tokens=case.partition_tokens, staging=staging, err_flag=dc.flag)
+    step(case.max_seq_len, pairs.shape[0])
+    torch.cuda.synchronize()
+    got = out_h.numpy().astype(np.float64)
+    assert np.array_equal(got, want)
+    assert np.array_equal(bits_host(dc.k), bits_host(ref.k)) and np.array_equal(bits_host(dc.v), bits_host(ref.v))
+    assert int(dc.flag.item()) == 0

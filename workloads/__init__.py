@@ -188,6 +188,9 @@ def _deal_tables(lens: np.ndarray, order: np.ndarray, bs: int, max_blocks: int,
     tables = np.empty((B, max_blocks), dtype=np.int64)
     tables[:] = np.resize(pad, (B, max_blocks)) if pad.size else -1
     cursor = 0
+    need = int((-(-lens // bs)).sum())
+    if need > order.size:
+        raise ValueError(f"pool of {order.size} blocks cannot hold {need} blocks of tables")
     for b in range(B):
         n = -(-int(lens[b]) // bs)
         tables[b, :n] = order[cursor:cursor + n]
