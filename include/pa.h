@@ -119,6 +119,28 @@ int pa_copy_blocks(void *k_cache, void *v_cache, const int32_t *pairs, int num_p
                    int32_t *err_flag, void *stream);
 
 /* ------------------------------------------------------------------------
+ * Block swap between two pools ("What is PagedAttention and how does it
+ * manage KV cache", Swapping and preemption: blocks are evicted to CPU
+ * memory when GPU memory runs short and fetched back when the request
+ * resumes).
+ *
+ * For each pair i: block pairs[2i+1] of the destination pools becomes a bit
+ * copy of block pairs[2i] of the source pools (K and V, all heads, rows and
+ * dims).  Either side may be device memory or page-locked host memory that
+ * the device can address (pinned with cudaHostAlloc / cudaHostRegister on a
+ * system with unified addressing): swap-out is device -> host, swap-in is
+ * host -> device.  Both sides use the pool layout above with the same
+ * num_kv_heads, block_size and head_dim; they may differ in block count.
+ * pairs: int32 [num_pairs, 2] = (src block, dst block), device-addressable.
+ * Destinations must be distinct.  Ids out of range set PA_FLAG_BAD_PAIR and
+ * the pair is skipped.  Bandwidth is that of the slower side (PCIe or
+ * NVLink-C2C for host memory).
+ * ---------------------------------------------------------------------- */
+int pa_swap_blocks(void *dst_k_cache, void *dst_v_cache, int64_t dst_num_blocks, const void *src_k_cache,
+                   const void *src_v_cache, int64_t src_num_blocks, const int32_t *pairs, int num_pairs,
+                   int num_kv_heads, int block_size, int head_dim, int32_t *err_flag, void *stream);
+
+/* ------------------------------------------------------------------------
  * Paged decode attention.  For every sequence b and query head g, with
  * kv head h = g / (num_q_heads / num_kv_heads) and L = seq_lens[b]:
  *

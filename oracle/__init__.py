@@ -73,6 +73,8 @@ def _load():
             lib.oracle_reshape_and_cache.restype = i32
             lib.oracle_copy_blocks.argtypes = [P, P, P, i32, i64, i32, i32, i32]
             lib.oracle_copy_blocks.restype = i32
+            lib.oracle_swap_blocks.argtypes = [P, P, i64, P, P, i64, P, i32, i32, i32, i32]
+            lib.oracle_swap_blocks.restype = i32
             _lib = lib
     return _lib
 
@@ -183,6 +185,18 @@ def copy_blocks(k_pool: np.ndarray, v_pool: np.ndarray, pairs) -> int:
     nb, hkv, bs, d = k_pool.shape
     return int(_load().oracle_copy_blocks(_ptr(k_pool), _ptr(v_pool), _ptr(pairs), pairs.shape[0],
                                           nb, hkv, bs, d))
+
+
+def swap_blocks(dst_k: np.ndarray, dst_v: np.ndarray, src_k, src_v, pairs) -> int:
+    """In-place copy of (src, dst) block pairs from the source pools into the destination pools."""
+    assert dst_k.flags.c_contiguous and dst_v.flags.c_contiguous
+    src_k = _c(src_k, np.uint16)
+    src_v = _c(src_v, np.uint16)
+    pairs = _c(pairs, np.int32).reshape(-1, 2)
+    nbd, hkv, bs, d = dst_k.shape
+    assert src_k.shape[1:] == dst_k.shape[1:]
+    return int(_load().oracle_swap_blocks(_ptr(dst_k), _ptr(dst_v), nbd, _ptr(src_k), _ptr(src_v),
+                                          src_k.shape[0], _ptr(pairs), pairs.shape[0], hkv, bs, d))
 
 
 def decode_step(case, rows: Optional[np.ndarray] = None):

@@ -26,6 +26,9 @@
  *    last_block, offset); slot -1 is skipped.
  *  - copy_blocks: copy whole blocks src -> dst, K and V ("PagedAttention &
  *    vLLM", Copy-on-write sharing: duplicate just that one block).
+ *  - swap_blocks: the same copy between two different pools (device pool
+ *    and CPU-side pool), "What is PagedAttention and how does it manage KV
+ *    cache", Swapping and preemption.
  *
  * All floating point is IEEE double (build without -ffast-math).  OpenMP
  * only spreads independent output rows over threads; each row's arithmetic
@@ -235,6 +238,32 @@ int oracle_copy_blocks(uint16_t *k_pool, uint16_t *v_pool, const int32_t *pairs,
         for (int64_t e = 0; e < block_elems; ++e) {
             k_pool[dst * block_elems + e] = k_pool[src * block_elems + e];
             v_pool[dst * block_elems + e] = v_pool[src * block_elems + e];
+        }
+    }
+    return bad;
+}
+
+/*
+ * For each (src, dst) pair in order, copy block src of the source pools to
+ * block dst of the destination pools.  Returns the number of pairs with an
+ * id out of range (skipped).
+ */
+int oracle_swap_blocks(uint16_t *dst_k, uint16_t *dst_v, int64_t dst_num_blocks, const uint16_t *src_k,
+                       const uint16_t *src_v, int64_t src_num_blocks, const int32_t *pairs, int num_pairs,
+                       int num_kv_heads, int block_size, int head_dim)
+{
+    int bad = 0;
+    int64_t block_elems = (int64_t)num_kv_heads * block_size * head_dim;
+    for (int i = 0; i < num_pairs; ++i) {
+        int64_t src = pairs[2 * i];
+        int64_t dst = pairs[2 * i + 1];
+        if (src < 0 || src >= src_num_blocks || dst < 0 || dst >= dst_num_blocks) {
+            ++bad;
+            continue;
+        }
+        for (int64_t e = 0; e < block_elems; ++e) {
+            dst_k[dst * block_elems + e] = src_k[src * block_elems + e];
+            dst_v[dst * block_elems + e] = src_v[src * block_elems + e];
         }
     }
     return bad;

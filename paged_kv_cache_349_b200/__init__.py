@@ -124,6 +124,34 @@ def pa_copy_blocks(k_cache, v_cache, pairs, err_flag=None, stream=None) -> None:
         _opt_flag(err_flag), _stream(stream)), "pa_copy_blocks")
 
 
+def _dev_or_pinned(t, dtype, name):
+    torch = _torch()
+    if not isinstance(t, torch.Tensor) or not (t.is_cuda or t.is_pinned()):
+        raise TypeError(f"{name} must be a CUDA tensor or a pinned host tensor")
+    if t.dtype != dtype:
+        raise TypeError(f"{name} must be {dtype}, got {t.dtype}")
+    if not t.is_contiguous():
+        raise ValueError(f"{name} must be contiguous")
+    return ctypes.c_void_p(t.data_ptr())
+
+
+def pa_swap_blocks(dst_k, dst_v, src_k, src_v, pairs, err_flag=None, stream=None) -> None:
+    """Copy blocks between two pools [NB, Hkv, bs, d]; either side may be pinned host memory.
+
+    pairs: int32 [n, 2] (src block, dst block), a CUDA tensor or a pinned host tensor.
+    """
+    torch = _torch()
+    if dst_k.shape[1:] != src_k.shape[1:] or dst_v.shape != dst_k.shape or src_v.shape != src_k.shape:
+        raise ValueError("pools must share [Hkv, bs, d]")
+    NBd, Hkv, bs, d = dst_k.shape
+    n = pairs.shape[0] if pairs.dim() == 2 else pairs.numel() // 2
+    _check(lib.pa_swap_blocks(
+        _dev_or_pinned(dst_k, torch.bfloat16, "dst_k"), _dev_or_pinned(dst_v, torch.bfloat16, "dst_v"), NBd,
+        _dev_or_pinned(src_k, torch.bfloat16, "src_k"), _dev_or_pinned(src_v, torch.bfloat16, "src_v"),
+        src_k.shape[0], _dev_or_pinned(pairs, torch.int32, "pairs") if n else None, n, Hkv, bs, d,
+        _opt_flag(err_flag), _stream(stream)), "pa_swap_blocks")
+
+
 def pa_decode_workspace_size(batch, num_q_heads, num_kv_heads, head_dim, block_size, max_seq_len,
                              partition_tokens=0) -> int:
     return int(lib.pa_decode_workspace_size(batch, num_q_heads, num_kv_heads, head_dim, block_size,

@@ -25,6 +25,7 @@ SIGNATURES = {
     "pa_launch_count": (_U64, []),
     "pa_reshape_and_cache": (_I, [_P, _P, _P, _P, _P, _I, _I64, _I, _I, _I, _P, _P]),
     "pa_copy_blocks": (_I, [_P, _P, _P, _I, _I64, _I, _I, _I, _P, _P]),
+    "pa_swap_blocks": (_I, [_P, _P, _I64, _P, _P, _I64, _P, _I, _I, _I, _I, _P, _P]),
     "pa_decode_workspace_size": (_SZ, [_I, _I, _I, _I, _I, _I, _I]),
     "pa_decode_partition_tokens": (_I, [_I, _I, _I, _I, _I, _I, _I]),
     "pa_decode": (_I, [_P, _P, _P, _P, _P, _I, _P, _I, _I, _I, _I, _I, _I, _I64, _F, _I, _P, _SZ, _P, _P]),

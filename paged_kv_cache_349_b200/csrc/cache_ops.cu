@@ -41,22 +41,24 @@ constexpr int kCopyThreads = 256;
 constexpr int kCopyUnroll = 4;  // 16-byte chunks in flight per thread
 
 // grid.x: pair * groups_per_block + chunk group, grid.y: 0 = K pool, 1 = V pool.
-// Copies block src -> dst ("PagedAttention & vLLM", Copy-on-write sharing).
+// Copies block src of the source pools to block dst of the destination pools
+// ("PagedAttention & vLLM", Copy-on-write sharing, when both are the same pools;
+// "What is PagedAttention...", swapping to CPU memory, when one side is pinned
+// host memory mapped into the device address space).
 __global__ void __launch_bounds__(kCopyThreads) copy_blocks_kernel(
-    uint4 *__restrict__ k_cache, uint4 *__restrict__ v_cache, const int32_t *__restrict__ pairs,
-    int64_t num_blocks, int64_t chunks_per_block, int groups_per_block,
-    int32_t *__restrict__ err_flag) {
+    uint4 *__restrict__ dst_k, uint4 *__restrict__ dst_v, const uint4 *src_k, const uint4 *src_v,
+    const int32_t *__restrict__ pairs, int64_t src_blocks, int64_t dst_blocks, int64_t chunks_per_block,
+    int groups_per_block, int flag_bit, int32_t *__restrict__ err_flag) {
     const int pair = blockIdx.x / groups_per_block;
     const int group = blockIdx.x - pair * groups_per_block;
     const int64_t src = __ldg(pairs + 2 * pair);
     const int64_t dst = __ldg(pairs + 2 * pair + 1);
-    if (src < 0 || src >= num_blocks || dst < 0 || dst >= num_blocks) {
-        if (group == 0 && blockIdx.y == 0 && threadIdx.x == 0) raise_flag(err_flag, PA_FLAG_BAD_PAIR);
+    if (src < 0 || src >= src_blocks || dst < 0 || dst >= dst_blocks) {
+        if (group == 0 && blockIdx.y == 0 && threadIdx.x == 0) raise_flag(err_flag, flag_bit);
         return;
     }
-    uint4 *pool = blockIdx.y == 0 ? k_cache : v_cache;
-    const uint4 *from = pool + src * chunks_per_block;
-    uint4 *to = pool + dst * chunks_per_block;
+    const uint4 *from = (blockIdx.y == 0 ? src_k : src_v) + src * chunks_per_block;
+    uint4 *to = (blockIdx.y == 0 ? dst_k : dst_v) + dst * chunks_per_block;
     const int64_t base = (int64_t)group * (kCopyThreads * kCopyUnroll) + threadIdx.x;
     uint4 buf[kCopyUnroll];
 #pragma unroll
@@ -69,6 +71,21 @@ __global__ void __launch_bounds__(kCopyThreads) copy_blocks_kernel(
         const int64_t i = base + (int64_t)u * kCopyThreads;
         if (i < chunks_per_block) __stcs(to + i, buf[u]);
     }
+}
+
+int launch_block_copy(void *dst_k, void *dst_v, const void *src_k, const void *src_v, const int32_t *pairs,
+                      int num_pairs, int64_t src_blocks, int64_t dst_blocks, int num_kv_heads, int block_size,
+                      int head_dim, int flag_bit, int32_t *err_flag, void *stream) {
+    const int64_t chunks = (int64_t)num_kv_heads * block_size * head_dim / 8;
+    const int64_t per_cta = kCopyThreads * kCopyUnroll;
+    const int64_t groups = (chunks + per_cta - 1) / per_cta;
+    if (groups * num_pairs > 0x7fffffffLL) return PA_ERR_INVALID_ARG;
+    dim3 grid((unsigned)(groups * num_pairs), 2);
+    copy_blocks_kernel<<<grid, kCopyThreads, 0, (cudaStream_t)stream>>>(
+        (uint4 *)dst_k, (uint4 *)dst_v, (const uint4 *)src_k, (const uint4 *)src_v, pairs, src_blocks,
+        dst_blocks, chunks, (int)groups, flag_bit, err_flag);
+    count_launch();
+    return launch_status();
 }
 
 }  // namespace
@@ -110,15 +127,25 @@ int pa_copy_blocks(void *k_cache, void *v_cache, const int32_t *pairs, int num_p
     if (num_pairs == 0) return PA_OK;
     if (!k_cache || !v_cache || !pairs) return PA_ERR_INVALID_ARG;
     if (!pa::aligned16(k_cache) || !pa::aligned16(v_cache)) return PA_ERR_INVALID_ARG;
-    const int64_t chunks = (int64_t)num_kv_heads * block_size * head_dim / 8;
-    const int64_t per_cta = pa::kCopyThreads * pa::kCopyUnroll;
-    const int64_t groups = (chunks + per_cta - 1) / per_cta;
-    if (groups * num_pairs > 0x7fffffffLL) return PA_ERR_INVALID_ARG;
-    dim3 grid((unsigned)(groups * num_pairs), 2);
-    pa::copy_blocks_kernel<<<grid, pa::kCopyThreads, 0, (cudaStream_t)stream>>>(
-        (uint4 *)k_cache, (uint4 *)v_cache, pairs, num_blocks, chunks, (int)groups, err_flag);
-    pa::count_launch();
-    return pa::launch_status();
+    return pa::launch_block_copy(k_cache, v_cache, k_cache, v_cache, pairs, num_pairs, num_blocks, num_blocks,
+                                 num_kv_heads, block_size, head_dim, PA_FLAG_BAD_PAIR, err_flag, stream);
+}
+
+int pa_swap_blocks(void *dst_k_cache, void *dst_v_cache, int64_t dst_num_blocks, const void *src_k_cache,
+                   const void *src_v_cache, int64_t src_num_blocks, const int32_t *pairs, int num_pairs,
+                   int num_kv_heads, int block_size, int head_dim, int32_t *err_flag, void *stream) {
+    if (num_pairs < 0 || dst_num_blocks <= 0 || src_num_blocks <= 0 || num_kv_heads <= 0)
+        return PA_ERR_INVALID_ARG;
+    if (head_dim != 64 && head_dim != 128) return PA_ERR_UNSUPPORTED;
+    if (block_size != 16 && block_size != 32) return PA_ERR_UNSUPPORTED;
+    if (num_pairs == 0) return PA_OK;
+    if (!dst_k_cache || !dst_v_cache || !src_k_cache || !src_v_cache || !pairs) return PA_ERR_INVALID_ARG;
+    if (!pa::aligned16(dst_k_cache) || !pa::aligned16(dst_v_cache) || !pa::aligned16(src_k_cache) ||
+        !pa::aligned16(src_v_cache))
+        return PA_ERR_INVALID_ARG;
+    return pa::launch_block_copy(dst_k_cache, dst_v_cache, src_k_cache, src_v_cache, pairs, num_pairs,
+                                 src_num_blocks, dst_num_blocks, num_kv_heads, block_size, head_dim,
+                                 PA_FLAG_BAD_PAIR, err_flag, stream);
 }
 
 }  // extern "C"

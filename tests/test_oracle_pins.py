@@ -369,6 +369,20 @@ def test_copy_blocks_literal():
     assert oracle.copy_blocks(k, v, np.array([[4, 0]], np.int32)) == 1
 
 
+def test_swap_blocks_literal():
+    dev_k = np.arange(3 * 1 * 2 * 2, dtype=np.uint16).reshape(3, 1, 2, 2)
+    dev_v = dev_k + 50
+    host_k = np.zeros((5, 1, 2, 2), np.uint16)
+    host_v = np.zeros_like(host_k)
+    assert oracle.swap_blocks(host_k, host_v, dev_k, dev_v, np.array([[2, 4], [0, 1]], np.int32)) == 0
+    want = np.zeros_like(host_k)
+    want[4] = [[[8, 9], [10, 11]]]
+    want[1] = [[[0, 1], [2, 3]]]
+    assert np.array_equal(host_k, want) and np.array_equal(host_v[[1, 4]], want[[1, 4]] + 50)
+    assert not host_v[[0, 2, 3]].any()
+    assert oracle.swap_blocks(host_k, host_v, dev_k, dev_v, np.array([[3, 0], [0, 5]], np.int32)) == 2
+
+
 # ---------------------------------------------------------------------------
 # Allocator model
 # ---------------------------------------------------------------------------
