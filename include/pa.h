@@ -41,7 +41,7 @@
  *    base address 16-byte aligned.  One (block, kv head) tile of
  *    block_size x head_dim values is contiguous.
  *  - Supported shapes: bf16 only; head_dim in {64, 128}; block_size in
- *    {16, 32}; num_q_heads / num_kv_heads in {1, 2, 4, 8}.
+ *    {8, 16, 32, 64}; num_q_heads / num_kv_heads in {1, 2, 4, 8}.
  *  - A slot is physical_block * block_size + row_in_block.
  */
 #ifndef PA_H

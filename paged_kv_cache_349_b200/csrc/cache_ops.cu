@@ -99,7 +99,7 @@ int pa_reshape_and_cache(const void *k_new, const void *v_new, void *k_cache, vo
                          void *stream) {
     if (num_tokens < 0 || num_blocks <= 0 || num_kv_heads <= 0) return PA_ERR_INVALID_ARG;
     if (head_dim != 64 && head_dim != 128) return PA_ERR_UNSUPPORTED;
-    if (block_size != 16 && block_size != 32) return PA_ERR_UNSUPPORTED;
+    if (!pa::supported_block_size(block_size)) return PA_ERR_UNSUPPORTED;
     if (num_tokens == 0) return PA_OK;
     if (!k_new || !v_new || !k_cache || !v_cache || !slot_mapping) return PA_ERR_INVALID_ARG;
     if (!pa::aligned16(k_new) || !pa::aligned16(v_new) || !pa::aligned16(k_cache) ||
@@ -123,7 +123,7 @@ int pa_copy_blocks(void *k_cache, void *v_cache, const int32_t *pairs, int num_p
                    int32_t *err_flag, void *stream) {
     if (num_pairs < 0 || num_blocks <= 0 || num_kv_heads <= 0) return PA_ERR_INVALID_ARG;
     if (head_dim != 64 && head_dim != 128) return PA_ERR_UNSUPPORTED;
-    if (block_size != 16 && block_size != 32) return PA_ERR_UNSUPPORTED;
+    if (!pa::supported_block_size(block_size)) return PA_ERR_UNSUPPORTED;
     if (num_pairs == 0) return PA_OK;
     if (!k_cache || !v_cache || !pairs) return PA_ERR_INVALID_ARG;
     if (!pa::aligned16(k_cache) || !pa::aligned16(v_cache)) return PA_ERR_INVALID_ARG;
@@ -137,7 +137,7 @@ int pa_swap_blocks(void *dst_k_cache, void *dst_v_cache, int64_t dst_num_blocks,
     if (num_pairs < 0 || dst_num_blocks <= 0 || src_num_blocks <= 0 || num_kv_heads <= 0)
         return PA_ERR_INVALID_ARG;
     if (head_dim != 64 && head_dim != 128) return PA_ERR_UNSUPPORTED;
-    if (block_size != 16 && block_size != 32) return PA_ERR_UNSUPPORTED;
+    if (!pa::supported_block_size(block_size)) return PA_ERR_UNSUPPORTED;
     if (num_pairs == 0) return PA_OK;
     if (!dst_k_cache || !dst_v_cache || !src_k_cache || !src_v_cache || !pairs) return PA_ERR_INVALID_ARG;
     if (!pa::aligned16(dst_k_cache) || !pa::aligned16(dst_v_cache) || !pa::aligned16(src_k_cache) ||

@@ -180,17 +180,23 @@ __global__ void __launch_bounds__(kThreads) paged_decode_kernel(
             const int tok0 = tok_begin + i * kTileTokens;
             const int j = mine ? tok0 / p.block_size : win;
             const int row = tok0 - j * p.block_size;
-            const int idx = j - win;  // in [0, 32 + kProducerLanes)
-            const int32_t from_cur = __shfl_sync(0xffffffffu, cur, idx & 31);
-            const int32_t from_nxt = __shfl_sync(0xffffffffu, nxt, idx & 31);
-            const int64_t phys = idx < 32 ? from_cur : from_nxt;
+            // A tile is one slice of a block, or two whole 8-token blocks.
+            const int idx = j - win;  // in [0, 32 + 2 * kProducerLanes)
+            const int32_t a_cur = __shfl_sync(0xffffffffu, cur, idx & 31);
+            const int32_t a_nxt = __shfl_sync(0xffffffffu, nxt, idx & 31);
+            const int32_t b_cur = __shfl_sync(0xffffffffu, cur, (idx + 1) & 31);
+            const int32_t b_nxt = __shfl_sync(0xffffffffu, nxt, (idx + 1) & 31);
+            const int64_t phys = idx < 32 ? a_cur : a_nxt;
+            const int64_t phys2 = idx + 1 < 32 ? b_cur : b_nxt;
+            const bool two_blocks = p.block_size < kTileTokens;
+            const bool second = two_blocks && tok0 + p.block_size < tok_end;
             if (mine) {
                 const int s = i % kStages;
                 if (i >= kStages && !mbar_wait_bounded(&empty[s], ((i / kStages) - 1) & 1, p.err_flag)) {
                     stop = true;
                 } else {
                     issued = i + 1;
-                    if (phys < 0 || phys >= p.num_blocks) {
+                    if (phys < 0 || phys >= p.num_blocks || (second && (phys2 < 0 || phys2 >= p.num_blocks))) {
                         raise_flag(p.err_flag, PA_FLAG_BAD_BLOCK);
                         tile_ok[s] = 0;
                         mbar_arrive(&full[s]);
@@ -198,7 +204,7 @@ __global__ void __launch_bounds__(kThreads) paged_decode_kernel(
                         tile_ok[s] = 1;
                         const int y = (int)((phys * p.num_kv_heads + h) * p.block_size + row);
                         uint8_t *dst = smem + s * C::kStageBytes;
-                        mbar_arrive_expect_tx(&full[s], C::kStageBytes);
+                        mbar_arrive_expect_tx(&full[s], two_blocks && !second ? C::kStageBytes / 2 : C::kStageBytes);
 #pragma unroll
                         for (int bx = 0; bx < C::kBoxes; ++bx)
                             tma_load_2d(dst + bx * kBoxBytes, &k_map, bx * 64, y, &full[s], policy);
@@ -206,6 +212,17 @@ __global__ void __launch_bounds__(kThreads) paged_decode_kernel(
                         for (int bx = 0; bx < C::kBoxes; ++bx)
                             tma_load_2d(dst + C::kTileBytes + bx * kBoxBytes, &v_map, bx * 64, y,
                                         &full[s], policy);
+                        if (second) {  // rows 8..15 of the tile come from the next 8-token block
+                            const int y2 = (int)((phys2 * p.num_kv_heads + h) * p.block_size);
+#pragma unroll
+                            for (int bx = 0; bx < C::kBoxes; ++bx)
+                                tma_load_2d(dst + bx * kBoxBytes + kBoxBytes / 2, &k_map, bx * 64, y2, &full[s],
+                                            policy);
+#pragma unroll
+                            for (int bx = 0; bx < C::kBoxes; ++bx)
+                                tma_load_2d(dst + C::kTileBytes + bx * kBoxBytes + kBoxBytes / 2, &v_map,
+                                            bx * 64, y2, &full[s], policy);
+                        }
                     }
                 }
             }
@@ -295,7 +312,7 @@ __global__ void __launch_bounds__(kThreads) paged_decode_kernel(
                     __syncwarp();
                 }
                 if (APPEND && i == i_new) {
-                    const int r = (L - 1) & (kTileTokens - 1);
+                    const int r = (L - 1 - tok_begin) - i_new * kTileTokens;  // row of L-1 in this tile
                     const int c = lane & 15;
                     if (c < HEAD_DIM / 8) {
                         const uint32_t a = (lane < 16 ? kbase : vbase) + tile_offset(r, c);
@@ -521,11 +538,12 @@ struct MapKey {
     const void *ptr;
     uint64_t rows;
     int head_dim;
+    int box_rows;
     int device;
 };
 
 // Small cache of pool tensor maps: a decode step re-uses the same pools.
-bool pool_tensor_map(const void *pool, uint64_t rows, int head_dim, CUtensorMap *out) {
+bool pool_tensor_map(const void *pool, uint64_t rows, int head_dim, int box_rows, CUtensorMap *out) {
     static std::mutex mu;
     static MapKey keys[8];
     static CUtensorMap maps[8];
@@ -535,7 +553,7 @@ bool pool_tensor_map(const void *pool, uint64_t rows, int head_dim, CUtensorMap 
     std::lock_guard<std::mutex> lock(mu);
     for (int i = 0; i < used; ++i) {
         if (keys[i].ptr == pool && keys[i].rows == rows && keys[i].head_dim == head_dim &&
-            keys[i].device == dev) {
+            keys[i].box_rows == box_rows && keys[i].device == dev) {
             *out = maps[i];
             return true;
         }
@@ -545,14 +563,14 @@ bool pool_tensor_map(const void *pool, uint64_t rows, int head_dim, CUtensorMap 
     CUtensorMap m;
     cuuint64_t dims[2] = {(cuuint64_t)head_dim, (cuuint64_t)rows};
     cuuint64_t strides[1] = {(cuuint64_t)head_dim * 2};
-    cuuint32_t box[2] = {64, (cuuint32_t)kTileTokens};
+    cuuint32_t box[2] = {64, (cuuint32_t)box_rows};
     cuuint32_t estr[2] = {1, 1};
     CUresult r = enc(&m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void *>(pool), dims, strides,
                      box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
                      CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
     if (r != CUDA_SUCCESS) return false;
     const int slot = used < 8 ? used++ : (next++ & 7);
-    keys[slot] = MapKey{pool, rows, head_dim, dev};
+    keys[slot] = MapKey{pool, rows, head_dim, box_rows, dev};
     maps[slot] = m;
     *out = m;
     return true;
@@ -692,7 +710,9 @@ int decode_impl(float *out, const void *q, const void *k_new, const void *v_new,
     }
 
     CUtensorMap km, vm;
-    if (!pool_tensor_map(k_cache, rows, head_dim, &km) || !pool_tensor_map(v_cache, rows, head_dim, &vm))
+    const int box_rows = block_size < kTileTokens ? block_size : kTileTokens;
+    if (!pool_tensor_map(k_cache, rows, head_dim, box_rows, &km) ||
+        !pool_tensor_map(v_cache, rows, head_dim, box_rows, &vm))
         return PA_ERR_CUDA;
     cudaStream_t s = static_cast<cudaStream_t>(stream);
     if (head_dim == 128) {

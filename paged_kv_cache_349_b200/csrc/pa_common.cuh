@@ -35,8 +35,12 @@ inline bool supported_shape(int num_q_heads, int num_kv_heads, int head_dim, int
     const int g = num_q_heads / num_kv_heads;
     if (g != 1 && g != 2 && g != 4 && g != 8) return false;
     if (head_dim != 64 && head_dim != 128) return false;
-    if (block_size != 16 && block_size != 32) return false;
+    if (block_size != 8 && block_size != 16 && block_size != 32 && block_size != 64) return false;
     return true;
+}
+
+inline bool supported_block_size(int block_size) {
+    return block_size == 8 || block_size == 16 || block_size == 32 || block_size == 64;
 }
 
 // ---------------------------------------------------------------------------

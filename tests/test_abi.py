@@ -58,7 +58,8 @@ def test_decode_argument_errors_need_no_gpu():
 
     assert call(B=0) == pa.PA_OK                         # nothing to do, nothing launched
     assert call(d=96) == pa.PA_ERR_UNSUPPORTED
-    assert call(bs=8) == pa.PA_ERR_UNSUPPORTED
+    assert call(bs=12) == pa.PA_ERR_UNSUPPORTED
+    assert call(bs=128) == pa.PA_ERR_UNSUPPORTED
     assert call(Hq=6, Hkv=4) == pa.PA_ERR_UNSUPPORTED    # not a whole group
     assert call(Hq=32, Hkv=2) == pa.PA_ERR_UNSUPPORTED   # group of 16
     assert call(q=None) == pa.PA_ERR_INVALID_ARG

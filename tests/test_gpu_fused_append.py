@@ -41,7 +41,7 @@ def test_workloads(cfg, kw):
 
 
 @pytest.mark.parametrize("d", [64, 128])
-@pytest.mark.parametrize("bs", [16, 32])
+@pytest.mark.parametrize("bs", [8, 16, 32, 64])
 @pytest.mark.parametrize("G", [1, 4, 8])
 def test_ragged_shapes(d, bs, G):
     lens = [0, 1, 2, 15, 16, 17, 31, 32, 33, 48, 49, 257]

@@ -63,7 +63,7 @@ def test_split_and_single_pass_agree_with_oracle(pt):
 
 
 @pytest.mark.parametrize("d", [64, 128])
-@pytest.mark.parametrize("bs", [16, 32])
+@pytest.mark.parametrize("bs", [8, 16, 32, 64])
 @pytest.mark.parametrize("G", [1, 2, 4, 8])
 def test_ragged_lengths_all_shapes(d, bs, G):
     lens = [1, 2, 15, 16, 17, 31, 32, 33, 47, 48, 49, 95, 257]
