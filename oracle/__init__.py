@@ -75,6 +75,18 @@ def _load():
             lib.oracle_copy_blocks.restype = i32
             lib.oracle_swap_blocks.argtypes = [P, P, i64, P, P, i64, P, i32, i32, i32, i32]
             lib.oracle_swap_blocks.restype = i32
+            lib.oracle_e4m3_decode.argtypes = [ctypes.c_uint8]
+            lib.oracle_e4m3_decode.restype = ctypes.c_double
+            lib.oracle_e4m3_encode.argtypes = [ctypes.c_float]
+            lib.oracle_e4m3_encode.restype = ctypes.c_uint8
+            lib.oracle_quantize_e4m3.argtypes = [P, P, i64, ctypes.c_float]
+            lib.oracle_quantize_e4m3.restype = None
+            lib.oracle_reshape_and_cache_fp8.argtypes = [P, P, P, P, P, i32, i64, i32, i32, i32,
+                                                         ctypes.c_float, ctypes.c_float]
+            lib.oracle_reshape_and_cache_fp8.restype = i32
+            lib.oracle_decode_rows_fp8.argtypes = [P, P, P, P, i32, P, i32, i32, i32, i32, i32, i64,
+                                                   ctypes.c_float, ctypes.c_float, ctypes.c_float, P, i32, P]
+            lib.oracle_decode_rows_fp8.restype = i32
             _lib = lib
     return _lib
 
@@ -197,6 +209,76 @@ def swap_blocks(dst_k: np.ndarray, dst_v: np.ndarray, src_k, src_v, pairs) -> in
     assert src_k.shape[1:] == dst_k.shape[1:]
     return int(_load().oracle_swap_blocks(_ptr(dst_k), _ptr(dst_v), nbd, _ptr(src_k), _ptr(src_v),
                                           src_k.shape[0], _ptr(pairs), pairs.shape[0], hkv, bs, d))
+
+
+# ---------------------------------------------------------------------------
+# fp8 (E4M3) pools
+# ---------------------------------------------------------------------------
+
+def e4m3_value(codes) -> np.ndarray:
+    """Value of each E4M3 code (float64; NaN for the NaN codes)."""
+    lib = _load()
+    flat = np.asarray(codes, dtype=np.uint8).ravel()
+    return np.array([lib.oracle_e4m3_decode(int(c)) for c in flat], np.float64).reshape(np.shape(codes))
+
+
+def e4m3_code(x) -> np.ndarray:
+    """Nearest E4M3 code of each fp32 value (ties to even, saturating at 448)."""
+    lib = _load()
+    flat = np.asarray(x, dtype=np.float32).ravel()
+    return np.array([lib.oracle_e4m3_encode(float(v)) for v in flat], np.uint8).reshape(np.shape(x))
+
+
+def inv_scale(scale) -> np.float32:
+    """The fp32 reciprocal both sides quantize with: 1 / scale rounded to fp32."""
+    return np.float32(1.0) / np.float32(scale)
+
+
+def quantize_e4m3(bf16_bits, scale) -> np.ndarray:
+    """Codes E4M3(bf16 * (1/scale)) with the product in fp32."""
+    src = _c(bf16_bits, np.uint16)
+    dst = np.empty(src.shape, np.uint8)
+    _load().oracle_quantize_e4m3(_ptr(src), _ptr(dst), src.size, ctypes.c_float(float(inv_scale(scale))))
+    return dst
+
+
+def reshape_and_cache_fp8(k_new, v_new, k_pool: np.ndarray, v_pool: np.ndarray, slot_mapping, block_size: int,
+                          k_scale, v_scale) -> int:
+    assert k_pool.dtype == np.uint8 and v_pool.dtype == np.uint8
+    assert k_pool.flags.c_contiguous and v_pool.flags.c_contiguous
+    k_new = _c(k_new, np.uint16)
+    v_new = _c(v_new, np.uint16)
+    slots = _c(slot_mapping, np.int32)
+    nb, hkv, bs, d = k_pool.shape
+    assert bs == block_size
+    return int(_load().oracle_reshape_and_cache_fp8(
+        _ptr(k_new), _ptr(v_new), _ptr(k_pool), _ptr(v_pool), _ptr(slots), slots.size, nb, hkv, bs, d,
+        ctypes.c_float(float(inv_scale(k_scale))), ctypes.c_float(float(inv_scale(v_scale)))))
+
+
+def decode_fp8(q, k_pool, v_pool, block_tables, seq_lens, *, num_kv_heads: int, block_size: int, scale,
+               k_scale, v_scale, rows: Optional[np.ndarray] = None) -> np.ndarray:
+    """Paged decode in fp64 over fp8 pools (rows dequantised as E4M3 value * scale)."""
+    q = _c(q, np.uint16)
+    k_pool = _c(k_pool, np.uint8)
+    v_pool = _c(v_pool, np.uint8)
+    tables = _c(block_tables, np.int32)
+    lens = _c(seq_lens, np.int32)
+    B, Hq, d = q.shape
+    if rows is None:
+        rows = np.array([(b, g) for b in range(B) for g in range(Hq)], np.int32).reshape(-1, 2)
+        full = True
+    else:
+        rows = _c(rows, np.int32).reshape(-1, 2)
+        full = False
+    out = np.zeros((rows.shape[0], d), np.float64)
+    st = _load().oracle_decode_rows_fp8(
+        _ptr(q), _ptr(k_pool), _ptr(v_pool), _ptr(tables), tables.shape[1], _ptr(lens), B, Hq, num_kv_heads, d,
+        block_size, k_pool.shape[0], ctypes.c_float(float(scale)), ctypes.c_float(float(k_scale)),
+        ctypes.c_float(float(v_scale)), _ptr(rows), rows.shape[0], _ptr(out))
+    if st:
+        raise IndexError(f"oracle_decode_fp8: status {st}")
+    return out.reshape(B, Hq, d) if full else out
 
 
 def decode_step(case, rows: Optional[np.ndarray] = None):

@@ -268,3 +268,144 @@ int oracle_swap_blocks(uint16_t *dst_k, uint16_t *dst_v, int64_t dst_num_blocks,
     }
     return bad;
 }
+
+/* ------------------------------------------------------------------------
+ * fp8 pools: OCP 8-bit E4M3 ("FN": no infinities, S.1111.111 is NaN, largest
+ * finite 448).  Values are stored as code = E4M3(x * inv_scale), rounded to
+ * nearest with ties to even and saturated to +-448, where x is the bf16 input
+ * widened to fp32 and the product is an fp32 multiply; the value a code
+ * stands for is E4M3_value(code) * scale.  The pages only say paging
+ * composes with KV quantization ("Walk through paged attention end to end",
+ * summary); the format and per-tensor scaling are this library's choice.
+ * ---------------------------------------------------------------------- */
+
+/* Value of an E4M3 code: sign, 4 exponent bits (bias 7), 3 mantissa bits. */
+double oracle_e4m3_decode(uint8_t code)
+{
+    int sign = code >> 7;
+    int e = (code >> 3) & 15;
+    int m = code & 7;
+    double v;
+    if (e == 15 && m == 7) return NAN;
+    if (e == 0)
+        v = ldexp((double)m, -9);            /* subnormal: m/8 * 2^-6 */
+    else
+        v = ldexp(1.0 + m / 8.0, e - 7);     /* normal */
+    return sign ? -v : v;
+}
+
+/* Nearest E4M3 code to an fp32 value: ties to even, saturating at 448. */
+uint8_t oracle_e4m3_encode(float x)
+{
+    double v = (double)x;
+    uint8_t sign = signbit(v) ? 0x80 : 0x00;
+    if (isnan(v)) return (uint8_t)(sign | 0x7F);
+    double a = fabs(v);
+    if (a >= 448.0) return (uint8_t)(sign | 0x7E);
+    if (a < ldexp(1.0, -6)) {                   /* subnormal range, steps of 2^-9 */
+        double q = nearbyint(ldexp(a, 9));     /* ties to even (default rounding mode) */
+        return (uint8_t)(sign | (uint8_t)q);    /* q == 8 is exactly the smallest normal */
+    }
+    int ex;
+    double f = frexp(a, &ex);                   /* a = f * 2^ex, f in [0.5, 1) */
+    int e = ex - 1;                             /* a = (2f) * 2^e, 2f in [1, 2) */
+    double q = nearbyint((2.0 * f - 1.0) * 8.0);
+    if (q == 8.0) {
+        q = 0.0;
+        e += 1;
+    }
+    return (uint8_t)(sign | (uint8_t)(((e + 7) << 3) | (int)q));
+}
+
+/* dst[i] = E4M3(bf16(src[i]) * inv_scale) for n elements. */
+void oracle_quantize_e4m3(const uint16_t *src, uint8_t *dst, int64_t n, float inv_scale)
+{
+    for (int64_t i = 0; i < n; ++i) {
+        float x = (float)oracle_bf16_to_f64(src[i]);
+        float prod = x * inv_scale;
+        dst[i] = oracle_e4m3_encode(prod);
+    }
+}
+
+/* Cache write into fp8 pools: like oracle_reshape_and_cache, quantizing each value. */
+int oracle_reshape_and_cache_fp8(const uint16_t *k_new, const uint16_t *v_new, uint8_t *k_pool,
+                                 uint8_t *v_pool, const int32_t *slot_mapping, int num_tokens,
+                                 int64_t num_blocks, int num_kv_heads, int block_size, int head_dim,
+                                 float k_inv_scale, float v_inv_scale)
+{
+    int bad = 0;
+    for (int t = 0; t < num_tokens; ++t) {
+        int64_t s = slot_mapping[t];
+        if (s == -1) continue;
+        if (s < 0 || s >= num_blocks * block_size) {
+            ++bad;
+            continue;
+        }
+        int64_t blk = s / block_size;
+        int64_t row = s % block_size;
+        for (int h = 0; h < num_kv_heads; ++h) {
+            int64_t dst = ((blk * num_kv_heads + h) * block_size + row) * head_dim;
+            int64_t src = ((int64_t)t * num_kv_heads + h) * head_dim;
+            oracle_quantize_e4m3(k_new + src, k_pool + dst, head_dim, k_inv_scale);
+            oracle_quantize_e4m3(v_new + src, v_pool + dst, head_dim, v_inv_scale);
+        }
+    }
+    return bad;
+}
+
+/* Gather of fp8 rows, dequantised: dst[p][i] = E4M3_value(code) * scale. */
+static int gather_fp8(const uint8_t *pool, int64_t num_blocks, int num_kv_heads, int block_size,
+                      int head_dim, const int32_t *table, int table_len, int seq_len, int h,
+                      double scale, double *dst)
+{
+    for (int p = 0; p < seq_len; ++p) {
+        int j = p / block_size;
+        int row = p % block_size;
+        if (j >= table_len) return -1;
+        int64_t phys = table[j];
+        if (phys < 0 || phys >= num_blocks) return -2;
+        int64_t base = ((phys * num_kv_heads + h) * (int64_t)block_size + row) * head_dim;
+        for (int i = 0; i < head_dim; ++i)
+            dst[(int64_t)p * head_dim + i] = oracle_e4m3_decode(pool[base + i]) * scale;
+    }
+    return 0;
+}
+
+/* Decode over fp8 pools: textbook attention on the dequantised rows. */
+int oracle_decode_rows_fp8(const uint16_t *q, const uint8_t *k_pool, const uint8_t *v_pool,
+                           const int32_t *tables, int max_blocks, const int32_t *seq_lens,
+                           int batch, int num_q_heads, int num_kv_heads, int head_dim,
+                           int block_size, int64_t num_blocks, float scale, float k_scale,
+                           float v_scale, const int32_t *rows, int n_rows, double *out)
+{
+    int status = 0;
+    int group = num_q_heads / num_kv_heads;
+#pragma omp parallel for schedule(dynamic, 1)
+    for (int r = 0; r < n_rows; ++r) {
+        int b = rows[2 * r];
+        int g = rows[2 * r + 1];
+        int h = g / group;
+        int L = (b >= 0 && b < batch) ? seq_lens[b] : 0;
+        double *qd = (double *)malloc(sizeof(double) * (size_t)head_dim);
+        double *K = (double *)malloc(sizeof(double) * (size_t)head_dim * (size_t)(L > 0 ? L : 1));
+        double *V = (double *)malloc(sizeof(double) * (size_t)head_dim * (size_t)(L > 0 ? L : 1));
+        for (int i = 0; i < head_dim; ++i)
+            qd[i] = oracle_bf16_to_f64(q[((int64_t)b * num_q_heads + g) * head_dim + i]);
+        const int32_t *table = tables + (int64_t)b * max_blocks;
+        int st = gather_fp8(k_pool, num_blocks, num_kv_heads, block_size, head_dim, table, max_blocks,
+                            L, h, (double)k_scale, K);
+        if (st == 0)
+            st = gather_fp8(v_pool, num_blocks, num_kv_heads, block_size, head_dim, table, max_blocks,
+                            L, h, (double)v_scale, V);
+        if (st == 0) {
+            oracle_attend(qd, K, V, L, head_dim, (double)scale, out + (int64_t)r * head_dim);
+        } else {
+#pragma omp critical
+            { if (status == 0) status = st; }
+        }
+        free(qd);
+        free(K);
+        free(V);
+    }
+    return status;
+}

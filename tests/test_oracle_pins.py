@@ -487,3 +487,87 @@ def test_model_logical_views_survive_sharing():
         assert len(used) + m.num_free() == NB
         for b in range(NB):
             assert m.ref[b] == sum(t.count(b) for t in m.tables.values())
+
+
+# ---------------------------------------------------------------------------
+# fp8 (E4M3) pools
+# ---------------------------------------------------------------------------
+
+def test_e4m3_known_codes():
+    # worked by hand from the format: sign | exponent (bias 7) | 3-bit mantissa
+    table = {1.0: 0x38, 0.5: 0x30, 448.0: 0x7E, -2.0: 0xC0, 2.0 ** -9: 0x01, 2.0 ** -6: 0x08,
+             7 * 2.0 ** -9: 0x07, 240.0: 0x77, 30.0: 0x5F, 0.0: 0x00, 1.125: 0x39, -448.0: 0xFE}
+    assert list(oracle.e4m3_code(list(table))) == list(table.values())
+    assert list(oracle.e4m3_value(list(table.values()))) == list(table)
+
+
+def test_e4m3_round_trip_every_code():
+    codes = np.array([c for c in range(256) if c not in (0x7F, 0xFF)], np.uint8)
+    vals = oracle.e4m3_value(codes)
+    assert np.all(np.isfinite(vals))
+    assert np.array_equal(oracle.e4m3_code(vals.astype(np.float32)), codes)
+    assert np.isnan(oracle.e4m3_value([0x7F, 0xFF])).all()
+    pos = vals[(codes < 0x80)]
+    assert np.all(np.diff(pos) > 0) and pos.max() == 448.0
+
+
+def test_e4m3_ties_to_even_and_nearest():
+    codes = np.arange(0, 0x7E, dtype=np.uint8)           # adjacent finite positive pairs (c, c+1)
+    lo = oracle.e4m3_value(codes)
+    hi = oracle.e4m3_value(codes + 1)
+    mid = ((lo + hi) / 2).astype(np.float32)
+    assert np.array_equal(mid.astype(np.float64), (lo + hi) / 2)  # midpoints are exact in fp32
+    even = np.where(codes % 2 == 0, codes, codes + 1).astype(np.uint8)
+    assert np.array_equal(oracle.e4m3_code(mid), even)
+    below = np.nextafter(mid, np.float32(0))
+    above = np.nextafter(mid, np.float32(1000))
+    assert np.array_equal(oracle.e4m3_code(below), codes)
+    assert np.array_equal(oracle.e4m3_code(above), (codes + 1).astype(np.uint8))
+
+
+def test_e4m3_saturates():
+    big = np.array([448.5, 463.9, 464.0, 1e6, np.inf], np.float32)
+    assert list(oracle.e4m3_code(big)) == [0x7E] * 5
+    assert list(oracle.e4m3_code(-big)) == [0xFE] * 5
+
+
+def test_quantize_uses_fp32_product():
+    # inv = fp32(1/0.1) = 10.000000149...; 3 * inv in fp32 = 30.0000004 -> code of 30
+    x = W.bf16_bits(np.array([3.0], np.float32))
+    assert oracle.inv_scale(0.1) == np.float32(1) / np.float32(0.1)
+    assert list(oracle.quantize_e4m3(x, 0.1)) == [0x5F]
+    # 1.0625 * 1 is a tie between 1.0 and 1.125 -> even code 0x38
+    assert list(oracle.quantize_e4m3(W.bf16_bits(np.array([1.0625], np.float32)), 1.0)) == [0x38]
+
+
+def test_fp8_decode_equals_bf16_decode_on_dequantised_pool():
+    """With a power-of-two scale the dequantised rows are exact bf16 values: both paths agree bitwise."""
+    case = W.make_case(2, batch=4, max_len=90, num_blocks=64)
+    _, k_pool, v_pool = oracle.decode_step(case)     # pools after the step's cache write
+    k_codes = oracle.quantize_e4m3(k_pool, 0.5)
+    v_codes = oracle.quantize_e4m3(v_pool, 0.25)
+    # rebuild bf16 pools from the codes' values (exact in bf16 after scaling by a power of two)
+    k_deq = W.bf16_bits((oracle.e4m3_value(k_codes) * 0.5).astype(np.float32))
+    v_deq = W.bf16_bits((oracle.e4m3_value(v_codes) * 0.25).astype(np.float32))
+    kw = dict(num_kv_heads=case.num_kv_heads, block_size=case.block_size, scale=case.scale)
+    got = oracle.decode_fp8(case.q, k_codes, v_codes, case.block_tables, case.seq_lens, k_scale=0.5,
+                            v_scale=0.25, **kw)
+    want = oracle.decode(case.q, k_deq, v_deq, case.block_tables, case.seq_lens, **kw)
+    finite = np.isfinite(want).all(axis=-1)  # rows never read poisoned slots
+    assert finite.all()
+    assert np.array_equal(got, want)
+    # v_scale is linear in the output
+    twice = oracle.decode_fp8(case.q, k_codes, v_codes, case.block_tables, case.seq_lens, k_scale=0.5,
+                              v_scale=0.5, **kw)
+    assert np.array_equal(twice, 2 * got)
+
+
+def test_fp8_cache_write_literal():
+    k = np.zeros((2, 1, 2, 2), np.uint8)
+    v = np.zeros_like(k)
+    k_new = W.bf16_bits(np.array([[[1.0, -2.0]]], np.float32))     # [T=1, Hkv=1, d=2]
+    v_new = W.bf16_bits(np.array([[[448.0, 0.5]]], np.float32))
+    assert oracle.reshape_and_cache_fp8(k_new, v_new, k, v, np.array([3], np.int32), 2, 1.0, 2.0) == 0
+    # v: 448 / 2 = 224 = 1.75 * 2^7 -> 0x76; 0.5 / 2 = 0.25 -> 0x28
+    assert list(k[1, 0, 1]) == [0x38, 0xC0] and list(v[1, 0, 1]) == [0x76, 0x28]
+    assert not k[0].any() and not k[1, 0, 0].any()
