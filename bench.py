@@ -83,14 +83,14 @@ def _decode_traffic_record():
     return rec
 
 
-def step_bytes(case):
-    """Algorithmic bytes of one step: (copy, write, decode)."""
+def step_bytes(case, kv_elem_bytes: int = 2):
+    """Algorithmic bytes of one step: (copy, write, decode); fp8 pools hold 1 byte per value."""
     bs, d, Hkv = case.block_size, case.head_dim, case.num_kv_heads
-    block_bytes = Hkv * bs * d * 2
+    block_bytes = Hkv * bs * d * kv_elem_bytes
     copy = int(case.copy_pairs.shape[0]) * block_bytes * 2 * 2 + case.copy_pairs.size * 4
     T = int(case.slot_mapping.size)
-    write = T * Hkv * d * 2 * 2 * 2 + T * 4
-    dec = W.algorithmic_decode_bytes(case)
+    write = T * Hkv * d * (2 + kv_elem_bytes) * 2 + T * 4
+    dec = W.algorithmic_decode_bytes(case, kv_elem_bytes=kv_elem_bytes)
     return copy, write, dec
 
 
@@ -251,7 +251,8 @@ def run_native(args):
     cfg = args.config
     seed = 1000 + cfg + 7919 * rank  # weak scaling: every rank owns its own batch
     case = W.make_case(cfg, seed=seed, fill=W.BF16_ZERO, num_blocks=args.num_blocks)
-    copy_b, write_b, dec_b = step_bytes(case)
+    fp8 = args.kv_dtype == "fp8"
+    copy_b, write_b, dec_b = step_bytes(case, 1 if fp8 else 2)
     total_b = copy_b + write_b + dec_b
     kv_tokens = int(case.seq_lens.sum())
 
@@ -262,6 +263,18 @@ def run_native(args):
         return torch.from_numpy(np.ascontiguousarray(a, dtype=np.int32)).cuda()
 
     k, v = bf16(case.k_cache), bf16(case.v_cache)
+    k_scale = v_scale = 1.0
+    if fp8:
+        # fp8 pools, quantised on the device by the library (per-pool scale = amax / 448)
+        k_scale = max(float(k.float().abs().amax()) / 448.0, 1e-30)
+        v_scale = max(float(v.float().abs().amax()) / 448.0, 1e-30)
+        k8 = torch.empty(k.shape, dtype=torch.uint8, device="cuda")
+        v8 = torch.empty(v.shape, dtype=torch.uint8, device="cuda")
+        pa.pa_quantize_fp8(k, k8, k_scale)
+        pa.pa_quantize_fp8(v, v8, v_scale)
+        torch.cuda.synchronize()
+        del k, v
+        k, v = k8, v8
     q = bf16(case.q)
     k_new, v_new = bf16(case.k_new), bf16(case.v_new)
     slots = i32(case.slot_mapping)
@@ -286,7 +299,25 @@ def run_native(args):
 
     dec_ev = []
 
+    def step_fp8(record):
+        if case.copy_pairs.shape[0]:
+            pa.pa_copy_blocks_fp8(k, v, pairs, err_flag=flag, stream=stream)
+        if other.size:
+            pa.pa_reshape_and_cache_fp8(k_other, v_other, k, v, slots_other, k_scale=k_scale, v_scale=v_scale,
+                                        err_flag=flag, stream=stream)
+        if record:
+            e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+            e0.record(stream)
+        pa.pa_decode_fp8(out, q, k, v, tables, lens, max_seq_len=case.max_seq_len, scale=float(case.scale),
+                         k_scale=k_scale, v_scale=v_scale, partition_tokens=pt, workspace=ws, err_flag=flag,
+                         stream=stream, k_new=k_last, v_new=v_last)
+        if record:
+            e1.record(stream)
+            dec_ev.append((e0, e1))
+
     def step(record=False):
+        if fp8:
+            return step_fp8(record)
         if case.copy_pairs.shape[0]:
             pa.pa_copy_blocks(k, v, pairs, err_flag=flag, stream=stream)
         if fused:
@@ -341,7 +372,7 @@ def run_native(args):
     peak, peak_kind = _measured_peak()
     achieved = dec_b / (dec_ms / 1e3) / 1e9
 
-    e2e = run_e2e(args, case, pa, stream, world, k, v) if not (args.no_e2e or args.unfused) else None
+    e2e = run_e2e(args, case, pa, stream, world, k, v) if not (args.no_e2e or args.unfused or fp8) else None
 
     traffic = None
     rec = _decode_traffic_record()
@@ -359,7 +390,7 @@ def run_native(args):
         "higher_is_better": True,
         "scaling": "weak",
         "vs_baseline": None,
-        "dtype": "bf16",
+        "dtype": "bf16" if not fp8 else "e4m3 K/V (f16 mma), bf16 q",
         "accumulate": "fp32",
         "data": "synthetic (seeded bf16 N(0,1) K/V/q, seeded placement)",
         "config": {
@@ -371,7 +402,9 @@ def run_native(args):
             "partition_tokens": resolved_pt,
             "parallelism": f"dp{world} (independent sequences per GPU, no collective)",
             "l2": f"inputs larger than L2: {dec_b / 1e9:.2f} GB of K/V per step vs 126 MB L2; no flush",
-            "step": ("block copies, then pa_decode_append (cache write fused into decode)" if fused else
+            "step": ("block copies, then pa_decode_append_fp8 (the write quantises to E4M3 and is fused into decode)"
+                     if fp8 else
+                     "block copies, then pa_decode_append (cache write fused into decode)" if fused else
                      "block copies, pa_reshape_and_cache, pa_decode"),
         },
         "pct_of_peak": {"nominal_8TBps": round(100 * value / NOMINAL_HBM_GBS, 1),
@@ -381,7 +414,7 @@ def run_native(args):
         "step_bytes": {"copy": copy_b, "write": write_b, "decode": dec_b},
         "gpu_launches": launches,
         "roofline": {
-            "kernel": ("pa_decode_append" if fused else "pa_decode") +
+            "kernel": ("pa_decode_append_fp8" if fp8 else "pa_decode_append" if fused else "pa_decode") +
                       (" (split kernel + LSE reduce)" if resolved_pt > 0 else " (single pass)"),
             "bound": "hbm",
             "achieved": round(achieved, 1),
@@ -396,7 +429,9 @@ def run_native(args):
         "e2e": e2e,
         "clocks": clocks,
     }
-    if rank == 0 and world == 1 and not args.no_cpu_baseline:
+    if fp8:
+        line["config"]["kv_scales"] = {"k": k_scale, "v": v_scale}
+    if rank == 0 and world == 1 and not args.no_cpu_baseline and not fp8:
         gbs, cores, sample, _, _ = cpu_baseline(case, budget_s=args.cpu_budget)
         line["cpu_baseline"] = {"value": round(gbs, 4), "unit": "GB/s", "cores": cores, "kind": "oracle",
                                 "sample": sample}
@@ -573,6 +608,8 @@ def main():
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--cpu-budget", type=float, default=12.0, help="seconds of oracle time")
+    ap.add_argument("--kv-dtype", choices=["bf16", "fp8"], default="bf16",
+                    help="fp8: E4M3 pools quantised by the library (per-pool scales); e2e is bf16-only")
     ap.add_argument("--unfused", action="store_true",
                     help="time pa_reshape_and_cache + pa_decode instead of the fused pa_decode_append")
     ap.add_argument("--num-blocks", type=int, default=None,

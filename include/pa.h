@@ -283,6 +283,57 @@ int pa_decode_builtin_scratch(float *out, const void *q, const void *k_cache, co
                               float scale, int partition_tokens, int32_t *err_flag, void *stream);
 
 /* ------------------------------------------------------------------------
+ * fp8 KV pools.  "Walk through paged attention end to end" (summary) only
+ * says paging composes with KV quantization; the format is this library's:
+ *
+ *   - Each pool holds OCP 8-bit E4M3 codes (no infinities, S.1111.111 is NaN,
+ *     largest finite 448), 1 byte per value, same [num_blocks, num_kv_heads,
+ *     block_size, head_dim] layout as the bf16 pools.
+ *   - One scale per pool (k_scale, v_scale > 0): a code c stands for
+ *     E4M3_value(c) * scale.
+ *   - Writing quantises: c = E4M3(x * inv), x the bf16 input widened to fp32,
+ *     inv = 1.0f / scale (fp32 division), the product an fp32 multiply,
+ *     rounded to nearest with ties to even and saturated to +-448.
+ *   - Decode computes exactly the pa_decode result on the dequantised rows.
+ *     It runs its mma in f16: q is rescaled by a power of two so its largest
+ *     entry lies in [2^13, 2^14); entries more than 2^37 below that largest
+ *     one are flushed to zero.
+ *
+ * Entry points mirror their bf16 counterparts; copy and swap move bytes.
+ * ---------------------------------------------------------------------- */
+
+/* dst[i] = E4M3(bf16 src[i] * (1/scale)); num_values a multiple of 8;
+ * src 16-byte aligned, dst 8-byte aligned (device memory). */
+int pa_quantize_fp8(const void *src, void *dst, int64_t num_values, float scale, void *stream);
+
+int pa_reshape_and_cache_fp8(const void *k_new, const void *v_new, void *k_cache, void *v_cache,
+                             const int32_t *slot_mapping, int num_tokens, int64_t num_blocks, int num_kv_heads,
+                             int block_size, int head_dim, float k_scale, float v_scale, int32_t *err_flag,
+                             void *stream);
+
+int pa_copy_blocks_fp8(void *k_cache, void *v_cache, const int32_t *pairs, int num_pairs, int64_t num_blocks,
+                       int num_kv_heads, int block_size, int head_dim, int32_t *err_flag, void *stream);
+
+int pa_swap_blocks_fp8(void *dst_k_cache, void *dst_v_cache, int64_t dst_num_blocks, const void *src_k_cache,
+                       const void *src_v_cache, int64_t src_num_blocks, const int32_t *pairs, int num_pairs,
+                       int num_kv_heads, int block_size, int head_dim, int32_t *err_flag, void *stream);
+
+/* pa_decode over fp8 pools (same workspace size as pa_decode). */
+int pa_decode_fp8(float *out, const void *q, const void *k_cache, const void *v_cache,
+                  const int32_t *block_tables, int max_blocks_per_seq, const int32_t *seq_lens, int batch,
+                  int max_seq_len, int num_q_heads, int num_kv_heads, int head_dim, int block_size,
+                  int64_t num_blocks, float scale, float k_scale, float v_scale, int partition_tokens,
+                  void *workspace, size_t workspace_bytes, int32_t *err_flag, void *stream);
+
+/* pa_decode_append over fp8 pools: the bf16 new token is quantised as it is written. */
+int pa_decode_append_fp8(float *out, const void *q, const void *k_new, const void *v_new, void *k_cache,
+                         void *v_cache, const int32_t *block_tables, int max_blocks_per_seq,
+                         const int32_t *seq_lens, int batch, int max_seq_len, int num_q_heads,
+                         int num_kv_heads, int head_dim, int block_size, int64_t num_blocks, float scale,
+                         float k_scale, float v_scale, int partition_tokens, void *workspace,
+                         size_t workspace_bytes, int32_t *err_flag, void *stream);
+
+/* ------------------------------------------------------------------------
  * Host block allocator (owns host memory only; not thread-safe).
  *
  * append  : the token at position n of a sequence goes to logical block

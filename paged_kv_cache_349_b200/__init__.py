@@ -265,6 +265,84 @@ class DecodeStepHost:
                                        *self._tail), "pa_decode_step_host")
 
 
+# ---------------------------------------------------------------------------
+# fp8 (E4M3) pools: uint8 tensors of codes, one scale per pool
+# ---------------------------------------------------------------------------
+
+def pa_quantize_fp8(src, dst, scale: float, stream=None) -> None:
+    """dst (uint8 codes) = E4M3(bf16 src * (1/scale)), element by element."""
+    torch = _torch()
+    if src.numel() != dst.numel():
+        raise ValueError("size mismatch")
+    _check(lib.pa_quantize_fp8(_dev(src, torch.bfloat16, "src"), _dev(dst, torch.uint8, "dst"), src.numel(),
+                               float(scale), _stream(stream)), "pa_quantize_fp8")
+
+
+def pa_reshape_and_cache_fp8(k_new, v_new, k_cache, v_cache, slot_mapping, *, k_scale: float, v_scale: float,
+                             err_flag=None, stream=None) -> None:
+    torch = _torch()
+    T, Hkv, d = k_new.shape
+    NB, Hkv2, bs, d2 = k_cache.shape
+    if (Hkv2, d2) != (Hkv, d) or v_new.shape != k_new.shape or v_cache.shape != k_cache.shape:
+        raise ValueError("shape mismatch")
+    _check(lib.pa_reshape_and_cache_fp8(
+        _dev(k_new, torch.bfloat16, "k_new"), _dev(v_new, torch.bfloat16, "v_new"),
+        _dev(k_cache, torch.uint8, "k_cache"), _dev(v_cache, torch.uint8, "v_cache"),
+        _dev(slot_mapping, torch.int32, "slot_mapping"), T, NB, Hkv, bs, d, float(k_scale), float(v_scale),
+        _opt_flag(err_flag), _stream(stream)), "pa_reshape_and_cache_fp8")
+
+
+def pa_copy_blocks_fp8(k_cache, v_cache, pairs, err_flag=None, stream=None) -> None:
+    torch = _torch()
+    NB, Hkv, bs, d = k_cache.shape
+    n = pairs.shape[0] if pairs.dim() == 2 else pairs.numel() // 2
+    _check(lib.pa_copy_blocks_fp8(
+        _dev(k_cache, torch.uint8, "k_cache"), _dev(v_cache, torch.uint8, "v_cache"),
+        _dev(pairs, torch.int32, "pairs") if n else None, n, NB, Hkv, bs, d, _opt_flag(err_flag),
+        _stream(stream)), "pa_copy_blocks_fp8")
+
+
+def pa_swap_blocks_fp8(dst_k, dst_v, src_k, src_v, pairs, err_flag=None, stream=None) -> None:
+    torch = _torch()
+    if dst_k.shape[1:] != src_k.shape[1:] or dst_v.shape != dst_k.shape or src_v.shape != src_k.shape:
+        raise ValueError("pools must share [Hkv, bs, d]")
+    NBd, Hkv, bs, d = dst_k.shape
+    n = pairs.shape[0] if pairs.dim() == 2 else pairs.numel() // 2
+    _check(lib.pa_swap_blocks_fp8(
+        _dev_or_pinned(dst_k, torch.uint8, "dst_k"), _dev_or_pinned(dst_v, torch.uint8, "dst_v"), NBd,
+        _dev_or_pinned(src_k, torch.uint8, "src_k"), _dev_or_pinned(src_v, torch.uint8, "src_v"), src_k.shape[0],
+        _dev_or_pinned(pairs, torch.int32, "pairs") if n else None, n, Hkv, bs, d, _opt_flag(err_flag),
+        _stream(stream)), "pa_swap_blocks_fp8")
+
+
+def pa_decode_fp8(out, q, k_cache, v_cache, block_tables, seq_lens, *, max_seq_len: int, scale: float,
+                  k_scale: float, v_scale: float, partition_tokens: int = 0, workspace=None, err_flag=None,
+                  stream=None, k_new=None, v_new=None) -> None:
+    """pa_decode over uint8 E4M3 pools; with k_new/v_new, pa_decode_append_fp8 (fused write)."""
+    torch = _torch()
+    B, Hq, d = q.shape
+    NB, Hkv, bs, d2 = k_cache.shape
+    if d2 != d or out.shape != q.shape or v_cache.shape != k_cache.shape:
+        raise ValueError("shape mismatch")
+    ws_ptr, ws_bytes = None, 0
+    if workspace is not None:
+        ws_ptr = _dev(workspace, workspace.dtype, "workspace")
+        ws_bytes = workspace.numel() * workspace.element_size()
+    head = (_dev(out, torch.float32, "out"), _dev(q, torch.bfloat16, "q"))
+    pools = (_dev(k_cache, torch.uint8, "k_cache"), _dev(v_cache, torch.uint8, "v_cache"))
+    tail = (_dev(block_tables, torch.int32, "block_tables"), block_tables.shape[1],
+            _dev(seq_lens, torch.int32, "seq_lens"), B, int(max_seq_len), Hq, Hkv, d, bs, NB, float(scale),
+            float(k_scale), float(v_scale), int(partition_tokens), ws_ptr, ws_bytes, _opt_flag(err_flag),
+            _stream(stream))
+    if k_new is None:
+        _check(lib.pa_decode_fp8(*head, *pools, *tail), "pa_decode_fp8")
+    else:
+        if tuple(k_new.shape) != (B, Hkv, d) or v_new.shape != k_new.shape:
+            raise ValueError("k_new/v_new must be [B, Hkv, d]")
+        new = (_dev(k_new, torch.bfloat16, "k_new"), _dev(v_new, torch.bfloat16, "v_new"))
+        _check(lib.pa_decode_append_fp8(*head, *new, *pools, *tail), "pa_decode_append_fp8")
+
+
 PA_DECODE_BUILTIN_SCRATCH_BYTES = 32 << 20
 
 

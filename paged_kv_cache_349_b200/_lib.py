@@ -34,6 +34,14 @@ SIGNATURES = {
     "pa_decode_step_host": (_I, [_P, _P, _P, _P, _P, _I, _P, _P, _I, _I, _P, _P, _I, _I, _I, _I, _I, _I, _I64, _F,
                                  _I, _P, _SZ, _P, _P]),
     "pa_decode_builtin_scratch": (_I, [_P, _P, _P, _P, _P, _I, _P, _I, _I, _I, _I, _I, _I, _I64, _F, _I, _P, _P]),
+    "pa_quantize_fp8": (_I, [_P, _P, _I64, _F, _P]),
+    "pa_reshape_and_cache_fp8": (_I, [_P, _P, _P, _P, _P, _I, _I64, _I, _I, _I, _F, _F, _P, _P]),
+    "pa_copy_blocks_fp8": (_I, [_P, _P, _P, _I, _I64, _I, _I, _I, _P, _P]),
+    "pa_swap_blocks_fp8": (_I, [_P, _P, _I64, _P, _P, _I64, _P, _I, _I, _I, _I, _P, _P]),
+    "pa_decode_fp8": (_I, [_P, _P, _P, _P, _P, _I, _P, _I, _I, _I, _I, _I, _I, _I64, _F, _F, _F, _I, _P, _SZ, _P,
+                           _P]),
+    "pa_decode_append_fp8": (_I, [_P, _P, _P, _P, _P, _P, _P, _I, _P, _I, _I, _I, _I, _I, _I, _I64, _F, _F, _F, _I,
+                                  _P, _SZ, _P, _P]),
     "pa_alloc_create": (_I, [_I, _I, ctypes.POINTER(_P)]),
     "pa_alloc_create_ordered": (_I, [_I, _I, _P, ctypes.POINTER(_P)]),
     "pa_alloc_destroy": (None, [_P]),

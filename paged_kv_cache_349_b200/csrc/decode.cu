@@ -40,6 +40,10 @@ namespace {
 #ifndef PA_DECODE_PRODUCER_LANES
 #define PA_DECODE_PRODUCER_LANES 8
 #endif
+// fp8 tiles: 1 = expand E4M3 with integer bit moves (value * 2^-8), 0 = hardware cvt.
+#ifndef PA_FP8_BIT_EXPAND
+#define PA_FP8_BIT_EXPAND 0
+#endif
 
 constexpr int kTileTokens = 16;
 constexpr int kConsumerWarps = PA_DECODE_CONSUMER_WARPS;
@@ -49,19 +53,35 @@ constexpr int kStages = PA_DECODE_STAGES;
 constexpr int kProducerLanes = PA_DECODE_PRODUCER_LANES;
 static_assert(kStages % kProducerLanes == 0, "each producer lane owns whole ring slots");
 static_assert(kProducerLanes >= 1 && kProducerLanes <= 8, "window indexing assumes <= 8 lanes");
-constexpr int kBoxBytes = kTileTokens * 128;  // one 64-wide bf16 column box of a tile
+// A 16-bit tile (bf16, or f16 expanded from fp8) is stored as HEAD_DIM/64
+// boxes of 16 rows x 128 bytes with the TMA 128-byte swizzle.
+constexpr int kBox16Bytes = kTileTokens * 128;
 constexpr float kLog2e = 1.4426950408889634f;
 
-template <int HEAD_DIM>
+template <int HEAD_DIM, bool FP8>
 struct Cfg {
-    static constexpr int kBoxes = HEAD_DIM / 64;
+    // What TMA lands in the ring: bf16 tiles in 64-column swizzled boxes, or
+    // fp8 tiles as one unswizzled box of 16 rows x HEAD_DIM bytes.
+    static constexpr int kBoxes = FP8 ? 1 : HEAD_DIM / 64;
+    static constexpr int kBoxCols = FP8 ? HEAD_DIM : 64;
+    static constexpr int kBoxRowBytes = FP8 ? HEAD_DIM : 128;
+    static constexpr int kBoxBytes = kTileTokens * kBoxRowBytes;
     static constexpr int kTileBytes = kBoxes * kBoxBytes;  // K or V of one tile
     static constexpr int kStageBytes = 2 * kTileBytes;
     static constexpr int kRingBytes = kStages * kStageBytes;
+    // fp8, head_dim 128: the ring tile carries the 128-byte swizzle; K fragments
+    // are built straight from it and only V is expanded to a 16-bit tile.
+    // fp8, head_dim 64: the ring tile is unswizzled and both K and V are expanded.
+    static constexpr bool kDirectK = FP8 && HEAD_DIM == 128;
+    static constexpr int kTile16Bytes = (HEAD_DIM / 64) * kBox16Bytes;
+    static constexpr int kStagingBytes = FP8 ? kConsumerWarps * (kDirectK ? 1 : 2) * kTile16Bytes : 0;
+    static constexpr int kDataBytes = kRingBytes + kStagingBytes;
     static constexpr int kMergeStride = HEAD_DIM + 4;  // padded row: conflict-free merge stores
     static constexpr int kMergeBytes = kConsumerWarps * 8 * (kMergeStride + 2) * 4;
-    static_assert(kMergeBytes <= kRingBytes, "merge area reuses the ring");
-    static constexpr int kSmemBytes = 1024 /*align slack*/ + kRingBytes + kStages * 8 * 2 + kStages * 4;
+    static_assert(kMergeBytes <= kDataBytes, "merge area reuses the ring");
+    // + barriers, tile flags, the fused write's row (32 x 16 bytes) and its block id
+    static constexpr int kSmemBytes =
+        1024 /*align slack*/ + kDataBytes + kStages * 8 * 2 + kStages * 4 + 32 * 16 + 16;
 };
 
 struct DecodeParams {
@@ -86,6 +106,10 @@ struct DecodeParams {
     int part_tokens;            // tokens per CTA along the sequence
     int num_parts;
     float scale_log2;           // softmax scale * log2(e)
+    float k_scale;              // fp8 pools: dequantisation multipliers
+    float v_scale;
+    float k_inv_scale;          // fp8 pools: 1 / scale, for the fused cache write
+    float v_inv_scale;
 };
 
 // Sequence length as every kernel of one call sees it: out-of-contract values
@@ -95,22 +119,61 @@ __device__ __forceinline__ int clamp_len(int L, const DecodeParams &p) {
     return L < 0 ? 0 : (L > cap ? cap : L);
 }
 
-// Byte offset of 16-byte chunk c of token row r inside one TMA-swizzled tile.
+// Byte offset of 16-byte chunk c of token row r inside one swizzled 16-bit tile.
 __device__ __forceinline__ uint32_t tile_offset(int r, int c) {
-    return (uint32_t)((c >> 3) * kBoxBytes + r * 128 + (((c & 7) ^ (r & 7)) << 4));
+    return (uint32_t)((c >> 3) * kBox16Bytes + r * 128 + (((c & 7) ^ (r & 7)) << 4));
 }
 
-template <int HEAD_DIM, bool SPLIT, bool APPEND>
-__global__ void __launch_bounds__(kThreads) paged_decode_kernel(
+// Byte offset of byte `byte` of row r in a 128-byte-swizzled fp8 tile (128-byte rows).
+__device__ __forceinline__ uint32_t fp8_tile_offset(int r, int byte) {
+    return (uint32_t)(r * 128 + ((((byte >> 4) ^ (r & 7))) << 4) + (byte & 15));
+}
+
+// Eight E4M3 codes -> four f16x2 words (codes 0,1 | 2,3 | 4,5 | 6,7).
+__device__ __forceinline__ uint4 e4m3x8_to_f16x8(uint32_t lo, uint32_t hi) {
+#if PA_FP8_BIT_EXPAND
+    return make_uint4(e4m3x2_to_f16x2_scaled<0x1404u>(lo), e4m3x2_to_f16x2_scaled<0x3424u>(lo),
+                      e4m3x2_to_f16x2_scaled<0x1404u>(hi), e4m3x2_to_f16x2_scaled<0x3424u>(hi));
+#else
+    uint4 r;
+    e4m3x4_to_f16x4(lo, r.x, r.y);
+    e4m3x4_to_f16x4(hi, r.z, r.w);
+    return r;
+#endif
+}
+
+template <bool FP8>
+__device__ __forceinline__ void mma_16816(float (&d)[4], uint32_t a0, uint32_t a1, uint32_t a2, uint32_t a3,
+                                          uint32_t b0, uint32_t b1) {
+    if constexpr (FP8)
+        mma_f16_16816(d, a0, a1, a2, a3, b0, b1);
+    else
+        mma_bf16_16816(d, a0, a1, a2, a3, b0, b1);
+}
+
+// CTAs per SM the register allocation must allow (bf16 is limited to 3 by shared memory).
+#ifndef PA_DECODE_MIN_CTAS_FP8
+#define PA_DECODE_MIN_CTAS_FP8 3
+#endif
+#ifndef PA_DECODE_MIN_CTAS_BF16
+#define PA_DECODE_MIN_CTAS_BF16 3
+#endif
+
+template <int HEAD_DIM, bool SPLIT, bool APPEND, bool FP8>
+__global__ void __launch_bounds__(kThreads, FP8 ? PA_DECODE_MIN_CTAS_FP8 : PA_DECODE_MIN_CTAS_BF16) paged_decode_kernel(
     const __grid_constant__ CUtensorMap k_map, const __grid_constant__ CUtensorMap v_map,
     const DecodeParams p) {
-    using C = Cfg<HEAD_DIM>;
+    using C = Cfg<HEAD_DIM, FP8>;
     extern __shared__ uint8_t smem_raw[];
     uint8_t *smem = reinterpret_cast<uint8_t *>(
         (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~static_cast<uintptr_t>(1023));
-    uint64_t *full = reinterpret_cast<uint64_t *>(smem + C::kRingBytes);
+    uint64_t *full = reinterpret_cast<uint64_t *>(smem + C::kDataBytes);
     uint64_t *empty = full + kStages;
     int *tile_ok = reinterpret_cast<int *>(empty + kStages);
+    // Fused write: the new token's bf16 K/V row (16 bytes per lane) and its block id,
+    // fetched asynchronously so no registers are held until the tile is reached.
+    uint4 *append_row = reinterpret_cast<uint4 *>(tile_ok + kStages);
+    int *append_phys = reinterpret_cast<int *>(append_row + 32);
 
     const int part = blockIdx.x;
     const int h = blockIdx.y;
@@ -207,21 +270,21 @@ __global__ void __launch_bounds__(kThreads) paged_decode_kernel(
                         mbar_arrive_expect_tx(&full[s], two_blocks && !second ? C::kStageBytes / 2 : C::kStageBytes);
 #pragma unroll
                         for (int bx = 0; bx < C::kBoxes; ++bx)
-                            tma_load_2d(dst + bx * kBoxBytes, &k_map, bx * 64, y, &full[s], policy);
+                            tma_load_2d(dst + bx * C::kBoxBytes, &k_map, bx * C::kBoxCols, y, &full[s], policy);
 #pragma unroll
                         for (int bx = 0; bx < C::kBoxes; ++bx)
-                            tma_load_2d(dst + C::kTileBytes + bx * kBoxBytes, &v_map, bx * 64, y,
+                            tma_load_2d(dst + C::kTileBytes + bx * C::kBoxBytes, &v_map, bx * C::kBoxCols, y,
                                         &full[s], policy);
                         if (second) {  // rows 8..15 of the tile come from the next 8-token block
                             const int y2 = (int)((phys2 * p.num_kv_heads + h) * p.block_size);
 #pragma unroll
                             for (int bx = 0; bx < C::kBoxes; ++bx)
-                                tma_load_2d(dst + bx * kBoxBytes + kBoxBytes / 2, &k_map, bx * 64, y2, &full[s],
-                                            policy);
+                                tma_load_2d(dst + bx * C::kBoxBytes + C::kBoxBytes / 2, &k_map, bx * C::kBoxCols, y2,
+                                            &full[s], policy);
 #pragma unroll
                             for (int bx = 0; bx < C::kBoxes; ++bx)
-                                tma_load_2d(dst + C::kTileBytes + bx * kBoxBytes + kBoxBytes / 2, &v_map,
-                                            bx * 64, y2, &full[s], policy);
+                                tma_load_2d(dst + C::kTileBytes + bx * C::kBoxBytes + C::kBoxBytes / 2, &v_map,
+                                            bx * C::kBoxCols, y2, &full[s], policy);
                         }
                     }
                 }
@@ -256,11 +319,41 @@ __global__ void __launch_bounds__(kThreads) paged_decode_kernel(
 #pragma unroll
             for (int k = 0; k < HEAD_DIM / 16; ++k) qf[k][0] = qf[k][1] = 0u;
         }
+        // fp8 pools run the mma in f16: q is scaled by a power of two 2^qexp so its
+        // largest entry lands just below 2^14 (exact, well inside the f16 range);
+        // 2^-qexp and the K dequantisation scale fold into the softmax scale.
+        float s_scale = p.scale_log2;
+        if constexpr (FP8) {
+            float amax = 0.f;
+#pragma unroll
+            for (int k = 0; k < HEAD_DIM / 16; ++k) {
+                amax = fmaxf(amax, fmaxf(fabsf(bf16_lo_to_float(qf[k][0])), fabsf(bf16_hi_to_float(qf[k][0]))));
+                amax = fmaxf(amax, fmaxf(fabsf(bf16_lo_to_float(qf[k][1])), fabsf(bf16_hi_to_float(qf[k][1]))));
+            }
+#pragma unroll
+            for (int off = 16; off; off >>= 1) amax = fmaxf(amax, __shfl_xor_sync(0xffffffffu, amax, off));
+            // amax in [2^e, 2^(e+1)) -> qexp = 13 - e; amax == 0 -> qexp = 0
+            const int e = amax > 0.f ? (int)((__float_as_uint(amax) >> 23) & 0xff) - 127 : 13;
+            const int qexp = max(-100, min(100, 13 - e));
+            const float up = __uint_as_float((uint32_t)(127 + qexp) << 23);
+            const float down = __uint_as_float((uint32_t)(127 - qexp) << 23);
+#pragma unroll
+            for (int k = 0; k < HEAD_DIM / 16; ++k) {
+                qf[k][0] = pack_f16x2(bf16_lo_to_float(qf[k][0]) * up, bf16_hi_to_float(qf[k][0]) * up);
+                qf[k][1] = pack_f16x2(bf16_lo_to_float(qf[k][1]) * up, bf16_hi_to_float(qf[k][1]) * up);
+            }
+            s_scale = p.scale_log2 * p.k_scale * down;
+#if PA_FP8_BIT_EXPAND
+            s_scale *= 256.f;  // the expanded K tile holds E4M3_value * 2^-8
+#endif
+        }
         // Token row of mma row gid (gid+8 -> +8): this order keeps both the K
         // fragment loads and the V ldmatrix reads free of bank conflicts.
-        const int tau = (gid >> 1) | ((gid & 1) << 2);
+        // (fp8 with K read straight from the swizzled fp8 tile uses 0,2,4,6,1,3,5,7.)
+        auto token_of = [](int g) { return C::kDirectK ? ((g & 3) << 1) | (g >> 2) : (g >> 1) | ((g & 1) << 2); };
+        const int tau = token_of(gid);
         // ldmatrix row address pattern for V: matrix (lane>>3), row (lane&7).
-        const int v_row = ((lane & 7) >> 1 | ((lane & 1) << 2)) + (((lane >> 4) & 1) << 3);
+        const int v_row = token_of(lane & 7) + (((lane >> 4) & 1) << 3);
         const int v_chunk_hi = (lane >> 3) & 1;
 
         // Fused cache write ("append, then attend"): the warp that owns the tile
@@ -270,24 +363,33 @@ __global__ void __launch_bounds__(kThreads) paged_decode_kernel(
         // token is owned by this sequence alone (copy-on-write), so no other
         // CTA reads that row.
         int i_new = -1;
-        uint4 new_row = make_uint4(0u, 0u, 0u, 0u);
-        int64_t new_dst = -1;  // 16-byte chunk index of the row in the pool
         if (APPEND && L == L_raw && L > 0 && L - 1 >= tok_begin && L - 1 < tok_end) {
             const int it = (L - 1 - tok_begin) / kTileTokens;
             if (it % kConsumerWarps == warp) {
                 i_new = it;
                 const int c = lane & 15;
-                const int64_t phys = __ldg(p.block_tables + (int64_t)b * p.max_blocks + (L - 1) / p.block_size);
                 if (c < HEAD_DIM / 8) {
                     const uint16_t *src = (lane < 16 ? p.k_new : p.v_new) +
-                                          ((int64_t)b * p.num_kv_heads + h) * HEAD_DIM;
-                    new_row = __ldg(reinterpret_cast<const uint4 *>(src) + c);
-                    if (phys >= 0 && phys < p.num_blocks)
-                        new_dst = ((phys * p.num_kv_heads + h) * p.block_size + (L - 1) % p.block_size) *
-                                      (HEAD_DIM / 8) + c;
+                                          ((int64_t)b * p.num_kv_heads + h) * HEAD_DIM + c * 8;
+                    cp_async16(smem_addr(append_row + lane), src);
                 }
+                if (lane == 0)
+                    cp_async4(smem_addr(append_phys),
+                              p.block_tables + (int64_t)b * p.max_blocks + (L - 1) / p.block_size);
+                cp_async_commit();
             }
         }
+        // This lane's share of the fused write at the tile that holds L-1: returns the
+        // bf16 row chunk and the pool index of its 8 values (-1 if the block id is bad).
+        auto append_fetch = [&](uint4 &row) -> int64_t {
+            cp_async_wait_all();
+            __syncwarp();
+            const int64_t phys = *reinterpret_cast<volatile int *>(append_phys);
+            row = append_row[lane];
+            if (phys < 0 || phys >= p.num_blocks) return -1;
+            return ((phys * p.num_kv_heads + h) * p.block_size + (L - 1) % p.block_size) * (HEAD_DIM / 8) +
+                   (lane & 15);
+        };
 
         for (int i = warp; i < n_tiles; i += kConsumerWarps) {
             const int s = i % kStages;
@@ -295,32 +397,115 @@ __global__ void __launch_bounds__(kThreads) paged_decode_kernel(
             if (!__all_sync(0xffffffffu, got)) break;
             const int valid = min(kTileTokens, tok_end - (tok_begin + i * kTileTokens));
             if (tile_ok[s]) {
-                const uint32_t kbase = smem_addr(smem + s * C::kStageBytes);
-                const uint32_t vbase = kbase + C::kTileBytes;
+                uint32_t kbase = smem_addr(smem + s * C::kStageBytes);
+                uint32_t vbase = kbase + C::kTileBytes;
+                uint32_t ring_k = kbase;  // fp8 direct-K: K stays in the ring until QK is done
+                if constexpr (C::kDirectK) {
+                    // The fused cache write lands in the (swizzled) fp8 tile first, and in the pool.
+                    if (APPEND && i == i_new) {
+                        const int r = (L - 1 - tok_begin) - i_new * kTileTokens;
+                        const int c = lane & 15;  // 8-byte piece of the 128-byte row
+                        uint4 row;
+                        const int64_t dst = append_fetch(row);
+                        const uint2 q8 = bf16x8_to_e4m3x8(row, lane < 16 ? p.k_inv_scale : p.v_inv_scale);
+                        const uint32_t a = (lane < 16 ? kbase : vbase) + fp8_tile_offset(r, c * 8);
+                        asm volatile("st.shared.v2.u32 [%0], {%1, %2};" ::"r"(a), "r"(q8.x), "r"(q8.y) : "memory");
+                        if (dst >= 0) reinterpret_cast<uint2 *>(lane < 16 ? p.k_pool : p.v_pool)[dst] = q8;
+                        __syncwarp();
+                    }
+                    // Expand V into this warp's 16-bit tile.  Each group of 8 lanes takes rows
+                    // r and r^5 and four 16-byte chunks of one column box, so both the swizzled
+                    // fp8 reads and the swizzled 16-bit writes hit 8 distinct bank groups.
+                    const uint32_t stg_v = smem_addr(smem + C::kRingBytes + warp * C::kTile16Bytes);
+#pragma unroll
+                    for (int x = lane; x < kTileTokens * (HEAD_DIM / 16); x += 32) {
+                        const int grp = x >> 3, pair = grp >> 1, box = grp & 1;
+                        const int r0 = ((pair & 1) << 1) | (((pair >> 1) & 1) << 3) | (pair >> 2);
+                        const int r = (x & 4) ? (r0 ^ 5) : r0;
+                        const int c16 = box * 4 + (x & 3);
+                        const uint4 w = lds128(vbase + fp8_tile_offset(r, c16 * 16));
+                        const uint4 lo = e4m3x8_to_f16x8(w.x, w.y);
+                        const uint4 hi = e4m3x8_to_f16x8(w.z, w.w);
+                        asm volatile("st.shared.v4.u32 [%0], {%1, %2, %3, %4};" ::"r"(stg_v + tile_offset(r, 2 * c16)),
+                                     "r"(lo.x), "r"(lo.y), "r"(lo.z), "r"(lo.w)
+                                     : "memory");
+                        asm volatile("st.shared.v4.u32 [%0], {%1, %2, %3, %4};" ::"r"(stg_v + tile_offset(r, 2 * c16 + 1)),
+                                     "r"(hi.x), "r"(hi.y), "r"(hi.z), "r"(hi.w)
+                                     : "memory");
+                    }
+                    __syncwarp();
+                    vbase = stg_v;
+                } else if constexpr (FP8) {
+                    // head_dim 64: the fused write lands in the unswizzled fp8 tile first.
+                    if (APPEND && i == i_new) {
+                        const int r = (L - 1 - tok_begin) - i_new * kTileTokens;
+                        const int c = lane & 15;
+                        uint4 row;
+                        const int64_t dst = append_fetch(row);
+                        if (c < HEAD_DIM / 8) {
+                            const uint2 q8 = bf16x8_to_e4m3x8(row, lane < 16 ? p.k_inv_scale : p.v_inv_scale);
+                            const uint32_t a = (lane < 16 ? kbase : vbase) + r * HEAD_DIM + c * 8;
+                            asm volatile("st.shared.v2.u32 [%0], {%1, %2};" ::"r"(a), "r"(q8.x), "r"(q8.y)
+                                         : "memory");
+                            if (dst >= 0) reinterpret_cast<uint2 *>(lane < 16 ? p.k_pool : p.v_pool)[dst] = q8;
+                        }
+                        __syncwarp();
+                    }
+                    // Expand K and V into this warp's 16-bit tiles (E4M3 -> f16 is exact),
+                    // laid out like a TMA-swizzled bf16 tile so the code below is shared.
+                    const uint32_t stg_k = smem_addr(smem + C::kRingBytes + warp * 2 * C::kTile16Bytes);
+                    const uint32_t stg_v = stg_k + C::kTile16Bytes;
+                    constexpr int kChunksPerRow = HEAD_DIM / 16;  // 16 fp8 values per 16-byte chunk
+#pragma unroll
+                    for (int x = lane; x < kTileTokens * kChunksPerRow; x += 32) {
+                        const int r = x / kChunksPerRow;
+                        const int c16 = x - r * kChunksPerRow;
+#pragma unroll
+                        for (int kv = 0; kv < 2; ++kv) {
+                            const uint4 w = lds128((kv ? vbase : kbase) + x * 16);
+                            const uint32_t dst = kv ? stg_v : stg_k;
+                            const uint4 lo = e4m3x8_to_f16x8(w.x, w.y);
+                            const uint4 hi = e4m3x8_to_f16x8(w.z, w.w);
+                            asm volatile("st.shared.v4.u32 [%0], {%1, %2, %3, %4};" ::"r"(dst + tile_offset(r, 2 * c16)),
+                                         "r"(lo.x), "r"(lo.y), "r"(lo.z), "r"(lo.w)
+                                         : "memory");
+                            asm volatile("st.shared.v4.u32 [%0], {%1, %2, %3, %4};" ::"r"(dst + tile_offset(r, 2 * c16 + 1)),
+                                         "r"(hi.x), "r"(hi.y), "r"(hi.z), "r"(hi.w)
+                                         : "memory");
+                        }
+                    }
+                    if (APPEND && i == i_new) fence_proxy_async_smem();
+                    __syncwarp();
+                    if (lane == 0) mbar_arrive(&empty[s]);  // the ring slot is free again
+                    kbase = stg_k;
+                    vbase = stg_v;
+                }
                 if (valid < kTileTokens) {
                     // Rows past the sequence end hold stale data: zero them so
                     // that P = 0 times V cannot produce NaN.
-                    const int lines = (kTileTokens - valid) * C::kBoxes;
+                    constexpr int kBoxes16 = HEAD_DIM / 64;  // boxes of the 16-bit tile
+                    const int lines = (kTileTokens - valid) * kBoxes16;
                     for (int x = lane; x < lines * 8; x += 32) {
                         const int line = x >> 3;
-                        const int r = valid + line / C::kBoxes;
-                        const int bx = line % C::kBoxes;
-                        const uint32_t a = vbase + bx * kBoxBytes + r * 128 + ((x & 7) << 4);
+                        const int r = valid + line / kBoxes16;
+                        const int bx = line % kBoxes16;
+                        const uint32_t a = vbase + bx * kBox16Bytes + r * 128 + ((x & 7) << 4);
                         asm volatile("st.shared.v4.u32 [%0], {%1, %1, %1, %1};" ::"r"(a), "r"(0u)
                                      : "memory");
                     }
                     __syncwarp();
                 }
-                if (APPEND && i == i_new) {
+                if (APPEND && !FP8 && i == i_new) {
                     const int r = (L - 1 - tok_begin) - i_new * kTileTokens;  // row of L-1 in this tile
                     const int c = lane & 15;
+                    uint4 row;
+                    const int64_t dst = append_fetch(row);
                     if (c < HEAD_DIM / 8) {
                         const uint32_t a = (lane < 16 ? kbase : vbase) + tile_offset(r, c);
-                        asm volatile("st.shared.v4.u32 [%0], {%1, %2, %3, %4};" ::"r"(a), "r"(new_row.x),
-                                     "r"(new_row.y), "r"(new_row.z), "r"(new_row.w)
+                        asm volatile("st.shared.v4.u32 [%0], {%1, %2, %3, %4};" ::"r"(a), "r"(row.x), "r"(row.y),
+                                     "r"(row.z), "r"(row.w)
                                      : "memory");
-                        if (new_dst >= 0)
-                            reinterpret_cast<uint4 *>(lane < 16 ? p.k_pool : p.v_pool)[new_dst] = new_row;
+                        if (dst >= 0) reinterpret_cast<uint4 *>(lane < 16 ? p.k_pool : p.v_pool)[dst] = row;
                     }
                     __syncwarp();
                 }
@@ -328,17 +513,37 @@ __global__ void __launch_bounds__(kThreads) paged_decode_kernel(
                 float sacc[4] = {0.f, 0.f, 0.f, 0.f};
 #pragma unroll
                 for (int j = 0; j < HEAD_DIM / 32; ++j) {
-                    const int c = 4 * j + tig;
-                    const uint4 ka = lds128(kbase + tile_offset(tau, c));
-                    const uint4 kb = lds128(kbase + tile_offset(tau + 8, c));
-                    mma_bf16_16816(sacc, ka.x, kb.x, ka.y, kb.y, qf[2 * j][0], qf[2 * j][1]);
-                    mma_bf16_16816(sacc, ka.z, kb.z, ka.w, kb.w, qf[2 * j + 1][0], qf[2 * j + 1][1]);
+                    uint4 ka, kb;
+                    if constexpr (C::kDirectK) {
+                        // 8 fp8 codes (dims 32j+8t .. +7) of rows tau and tau+8, expanded in registers
+                        uint32_t a0, a1, b0, b1;
+                        asm volatile("ld.shared.v2.u32 {%0, %1}, [%2];"
+                                     : "=r"(a0), "=r"(a1)
+                                     : "r"(ring_k + fp8_tile_offset(tau, 32 * j + 8 * tig)));
+                        asm volatile("ld.shared.v2.u32 {%0, %1}, [%2];"
+                                     : "=r"(b0), "=r"(b1)
+                                     : "r"(ring_k + fp8_tile_offset(tau + 8, 32 * j + 8 * tig)));
+                        ka = e4m3x8_to_f16x8(a0, a1);
+                        kb = e4m3x8_to_f16x8(b0, b1);
+                    } else {
+                        const int c = 4 * j + tig;
+                        ka = lds128(kbase + tile_offset(tau, c));
+                        kb = lds128(kbase + tile_offset(tau + 8, c));
+                    }
+                    mma_16816<FP8>(sacc, ka.x, kb.x, ka.y, kb.y, qf[2 * j][0], qf[2 * j][1]);
+                    mma_16816<FP8>(sacc, ka.z, kb.z, ka.w, kb.w, qf[2 * j + 1][0], qf[2 * j + 1][1]);
+                }
+                if constexpr (C::kDirectK) {
+                    // K and V have left the ring: hand the slot back to the producer.
+                    if (APPEND && i == i_new) fence_proxy_async_smem();
+                    __syncwarp();
+                    if (lane == 0) mbar_arrive(&empty[s]);
                 }
                 // sacc: (token tau, col 2t), (tau, 2t+1), (tau+8, 2t), (tau+8, 2t+1)
-                const float s0 = tau < valid ? sacc[0] * p.scale_log2 : -INFINITY;
-                const float s1 = tau < valid ? sacc[1] * p.scale_log2 : -INFINITY;
-                const float s2 = tau + 8 < valid ? sacc[2] * p.scale_log2 : -INFINITY;
-                const float s3 = tau + 8 < valid ? sacc[3] * p.scale_log2 : -INFINITY;
+                const float s0 = tau < valid ? sacc[0] * s_scale : -INFINITY;
+                const float s1 = tau < valid ? sacc[1] * s_scale : -INFINITY;
+                const float s2 = tau + 8 < valid ? sacc[2] * s_scale : -INFINITY;
+                const float s3 = tau + 8 < valid ? sacc[3] * s_scale : -INFINITY;
                 float mx0 = fmaxf(s0, s2), mx1 = fmaxf(s1, s3);
 #pragma unroll
                 for (int off = 4; off < 32; off <<= 1) {
@@ -363,10 +568,18 @@ __global__ void __launch_bounds__(kThreads) paged_decode_kernel(
                     }
                 }
                 // ---- P^T as B fragments: hi + lo bf16 parts ----
-                const uint32_t h01 = pack_bf16x2(p0, p1);
-                const uint32_t h23 = pack_bf16x2(p2, p3);
-                const uint32_t l01 = pack_bf16x2(p0 - bf16_lo_to_float(h01), p1 - bf16_hi_to_float(h01));
-                const uint32_t l23 = pack_bf16x2(p2 - bf16_lo_to_float(h23), p3 - bf16_hi_to_float(h23));
+                uint32_t h01, h23, l01, l23;
+                if constexpr (FP8) {
+                    h01 = pack_f16x2(p0, p1);
+                    h23 = pack_f16x2(p2, p3);
+                    l01 = pack_f16x2(p0 - f16_lo_to_float(h01), p1 - f16_hi_to_float(h01));
+                    l23 = pack_f16x2(p2 - f16_lo_to_float(h23), p3 - f16_hi_to_float(h23));
+                } else {
+                    h01 = pack_bf16x2(p0, p1);
+                    h23 = pack_bf16x2(p2, p3);
+                    l01 = pack_bf16x2(p0 - bf16_lo_to_float(h01), p1 - bf16_hi_to_float(h01));
+                    l23 = pack_bf16x2(p2 - bf16_lo_to_float(h23), p3 - bf16_hi_to_float(h23));
+                }
                 const uint32_t bh0 = movmatrix_trans(h01), bh1 = movmatrix_trans(h23);
                 const uint32_t bl0 = movmatrix_trans(l01), bl1 = movmatrix_trans(l23);
                 // ---- O^T += V^T P^T ----
@@ -374,14 +587,20 @@ __global__ void __launch_bounds__(kThreads) paged_decode_kernel(
                 for (int mt = 0; mt < HEAD_DIM / 16; ++mt) {
                     uint32_t a0r, a1r, a2r, a3r;
                     ldmatrix_x4_trans(vbase + tile_offset(v_row, 2 * mt + v_chunk_hi), a0r, a1r, a2r, a3r);
-                    mma_bf16_16816(o[mt], a0r, a1r, a2r, a3r, bh0, bh1);
-                    mma_bf16_16816(o[mt], a0r, a1r, a2r, a3r, bl0, bl1);
+                    mma_16816<FP8>(o[mt], a0r, a1r, a2r, a3r, bh0, bh1);
+                    mma_16816<FP8>(o[mt], a0r, a1r, a2r, a3r, bl0, bl1);
                 }
-                if (valid < kTileTokens || (APPEND && i == i_new)) fence_proxy_async_smem();
+                if (!FP8 && (valid < kTileTokens || (APPEND && i == i_new))) fence_proxy_async_smem();
+            } else if (FP8) {
+                __syncwarp();
+                if (lane == 0) mbar_arrive(&empty[s]);  // skipped tile: release it here
             }
-            __syncwarp();
-            if (lane == 0) mbar_arrive(&empty[s]);
+            if constexpr (!FP8) {
+                __syncwarp();
+                if (lane == 0) mbar_arrive(&empty[s]);
+            }
         }
+        if (APPEND && i_new >= 0) cp_async_wait_all();  // never leave copies in flight
         // Row sums over this warp's tokens (lanes with the same tig share a column).
 #pragma unroll
         for (int off = 4; off < 32; off <<= 1) {
@@ -431,6 +650,11 @@ __global__ void __launch_bounds__(kThreads) paged_decode_kernel(
             }
         }
         const int64_t row = (int64_t)b * p.num_q_heads + (int64_t)h * G + n;
+#if PA_FP8_BIT_EXPAND
+        if (FP8) num *= p.v_scale * 256.f;  // the expanded V tile holds E4M3_value * 2^-8
+#else
+        if (FP8) num *= p.v_scale;
+#endif
         if (SPLIT) {
             p.part_o[(row * p.num_parts + part) * HEAD_DIM + d] = num / den;
             if (d == 0) {
@@ -539,11 +763,14 @@ struct MapKey {
     uint64_t rows;
     int head_dim;
     int box_rows;
+    bool fp8;
     int device;
 };
 
 // Small cache of pool tensor maps: a decode step re-uses the same pools.
-bool pool_tensor_map(const void *pool, uint64_t rows, int head_dim, int box_rows, CUtensorMap *out) {
+// bf16 pools: 64-column boxes with the 128-byte swizzle; fp8 pools: one box
+// spanning the row, 128-byte swizzled for head_dim 128 and unswizzled for 64.
+bool pool_tensor_map(const void *pool, uint64_t rows, int head_dim, int box_rows, bool fp8, CUtensorMap *out) {
     static std::mutex mu;
     static MapKey keys[8];
     static CUtensorMap maps[8];
@@ -553,7 +780,7 @@ bool pool_tensor_map(const void *pool, uint64_t rows, int head_dim, int box_rows
     std::lock_guard<std::mutex> lock(mu);
     for (int i = 0; i < used; ++i) {
         if (keys[i].ptr == pool && keys[i].rows == rows && keys[i].head_dim == head_dim &&
-            keys[i].box_rows == box_rows && keys[i].device == dev) {
+            keys[i].box_rows == box_rows && keys[i].fp8 == fp8 && keys[i].device == dev) {
             *out = maps[i];
             return true;
         }
@@ -562,15 +789,16 @@ bool pool_tensor_map(const void *pool, uint64_t rows, int head_dim, int box_rows
     if (!enc) return false;
     CUtensorMap m;
     cuuint64_t dims[2] = {(cuuint64_t)head_dim, (cuuint64_t)rows};
-    cuuint64_t strides[1] = {(cuuint64_t)head_dim * 2};
-    cuuint32_t box[2] = {64, (cuuint32_t)box_rows};
+    cuuint64_t strides[1] = {(cuuint64_t)head_dim * (fp8 ? 1 : 2)};
+    cuuint32_t box[2] = {(cuuint32_t)(fp8 ? head_dim : 64), (cuuint32_t)box_rows};
     cuuint32_t estr[2] = {1, 1};
-    CUresult r = enc(&m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void *>(pool), dims, strides,
-                     box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+    CUresult r = enc(&m, fp8 ? CU_TENSOR_MAP_DATA_TYPE_UINT8 : CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2,
+                     const_cast<void *>(pool), dims, strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE,
+                     (fp8 && head_dim != 128) ? CU_TENSOR_MAP_SWIZZLE_NONE : CU_TENSOR_MAP_SWIZZLE_128B,
                      CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
     if (r != CUDA_SUCCESS) return false;
     const int slot = used < 8 ? used++ : (next++ & 7);
-    keys[slot] = MapKey{pool, rows, head_dim, box_rows, dev};
+    keys[slot] = MapKey{pool, rows, head_dim, box_rows, fp8, dev};
     maps[slot] = m;
     *out = m;
     return true;
@@ -595,11 +823,11 @@ int resolve_partition(int batch, int num_kv_heads, int block_size, int max_seq_l
     return kDefaultPartition;
 }
 
-template <int HEAD_DIM, bool SPLIT, bool APPEND>
+template <int HEAD_DIM, bool SPLIT, bool APPEND, bool FP8>
 int launch_decode(const CUtensorMap &km, const CUtensorMap &vm, const DecodeParams &p, int batch,
                   cudaStream_t stream) {
-    using C = Cfg<HEAD_DIM>;
-    auto kern = paged_decode_kernel<HEAD_DIM, SPLIT, APPEND>;
+    using C = Cfg<HEAD_DIM, FP8>;
+    auto kern = paged_decode_kernel<HEAD_DIM, SPLIT, APPEND, FP8>;
     static std::once_flag once;
     static cudaError_t attr_err = cudaSuccess;
     std::call_once(once, [&] {
@@ -650,13 +878,24 @@ int builtin_scratch_address(void **out) {
     return PA_OK;
 }
 
-// Shared body of pa_decode and pa_decode_append (k_new == nullptr: no cache write).
+template <bool SPLIT, bool APPEND, bool FP8>
+int launch_decode_d(int head_dim, const CUtensorMap &km, const CUtensorMap &vm, const DecodeParams &p, int batch,
+                    cudaStream_t s) {
+    return head_dim == 128 ? launch_decode<128, SPLIT, APPEND, FP8>(km, vm, p, batch, s)
+                           : launch_decode<64, SPLIT, APPEND, FP8>(km, vm, p, batch, s);
+}
+
+// Shared body of every decode entry point (k_new == nullptr: no cache write;
+// fp8: E4M3 pools dequantised with k_scale / v_scale).
 int decode_impl(float *out, const void *q, const void *k_new, const void *v_new, const void *k_cache,
                 const void *v_cache, const int32_t *block_tables, int max_blocks_per_seq,
                 const int32_t *seq_lens, int batch, int max_seq_len, int num_q_heads, int num_kv_heads,
                 int head_dim, int block_size, int64_t num_blocks, float scale, int partition_tokens,
-                void *workspace, size_t workspace_bytes, int32_t *err_flag, void *stream) {
+                void *workspace, size_t workspace_bytes, int32_t *err_flag, void *stream, bool fp8,
+                float k_scale, float v_scale) {
     const bool append = k_new != nullptr;
+    if (fp8 && !(k_scale > 0.f && v_scale > 0.f && k_scale < 3.0e38f && v_scale < 3.0e38f))
+        return PA_ERR_INVALID_ARG;
     if (batch < 0 || max_seq_len < 0 || num_blocks <= 0 || max_blocks_per_seq < 0)
         return PA_ERR_INVALID_ARG;
     if (!supported_shape(num_q_heads, num_kv_heads, head_dim, block_size)) return PA_ERR_UNSUPPORTED;
@@ -688,6 +927,10 @@ int decode_impl(float *out, const void *q, const void *k_new, const void *v_new,
     p.v_new = static_cast<const uint16_t *>(v_new);
     p.k_pool = static_cast<uint16_t *>(const_cast<void *>(k_cache));
     p.v_pool = static_cast<uint16_t *>(const_cast<void *>(v_cache));
+    p.k_scale = fp8 ? k_scale : 1.f;
+    p.v_scale = fp8 ? v_scale : 1.f;
+    p.k_inv_scale = fp8 ? 1.0f / k_scale : 1.f;
+    p.v_inv_scale = fp8 ? 1.0f / v_scale : 1.f;
 
     const int pt = max_seq_len > 0
                        ? resolve_partition(batch, num_kv_heads, block_size, max_seq_len, partition_tokens)
@@ -711,22 +954,22 @@ int decode_impl(float *out, const void *q, const void *k_new, const void *v_new,
 
     CUtensorMap km, vm;
     const int box_rows = block_size < kTileTokens ? block_size : kTileTokens;
-    if (!pool_tensor_map(k_cache, rows, head_dim, box_rows, &km) ||
-        !pool_tensor_map(v_cache, rows, head_dim, box_rows, &vm))
+    if (!pool_tensor_map(k_cache, rows, head_dim, box_rows, fp8, &km) ||
+        !pool_tensor_map(v_cache, rows, head_dim, box_rows, fp8, &vm))
         return PA_ERR_CUDA;
     cudaStream_t s = static_cast<cudaStream_t>(stream);
-    if (head_dim == 128) {
+    if (fp8) {
         if (append)
-            return split ? launch_decode<128, true, true>(km, vm, p, batch, s)
-                         : launch_decode<128, false, true>(km, vm, p, batch, s);
-        return split ? launch_decode<128, true, false>(km, vm, p, batch, s)
-                     : launch_decode<128, false, false>(km, vm, p, batch, s);
+            return split ? launch_decode_d<true, true, true>(head_dim, km, vm, p, batch, s)
+                         : launch_decode_d<false, true, true>(head_dim, km, vm, p, batch, s);
+        return split ? launch_decode_d<true, false, true>(head_dim, km, vm, p, batch, s)
+                     : launch_decode_d<false, false, true>(head_dim, km, vm, p, batch, s);
     }
     if (append)
-        return split ? launch_decode<64, true, true>(km, vm, p, batch, s)
-                     : launch_decode<64, false, true>(km, vm, p, batch, s);
-    return split ? launch_decode<64, true, false>(km, vm, p, batch, s)
-                 : launch_decode<64, false, false>(km, vm, p, batch, s);
+        return split ? launch_decode_d<true, true, false>(head_dim, km, vm, p, batch, s)
+                     : launch_decode_d<false, true, false>(head_dim, km, vm, p, batch, s);
+    return split ? launch_decode_d<true, false, false>(head_dim, km, vm, p, batch, s)
+                 : launch_decode_d<false, false, false>(head_dim, km, vm, p, batch, s);
 }
 
 }  // namespace pa
@@ -759,7 +1002,8 @@ int pa_decode(float *out, const void *q, const void *k_cache, const void *v_cach
               void *workspace, size_t workspace_bytes, int32_t *err_flag, void *stream) {
     return pa::decode_impl(out, q, nullptr, nullptr, k_cache, v_cache, block_tables, max_blocks_per_seq,
                            seq_lens, batch, max_seq_len, num_q_heads, num_kv_heads, head_dim, block_size,
-                           num_blocks, scale, partition_tokens, workspace, workspace_bytes, err_flag, stream);
+                           num_blocks, scale, partition_tokens, workspace, workspace_bytes, err_flag, stream,
+                           false, 1.f, 1.f);
 }
 
 int pa_decode_append(float *out, const void *q, const void *k_new, const void *v_new, void *k_cache,
@@ -771,7 +1015,32 @@ int pa_decode_append(float *out, const void *q, const void *k_new, const void *v
     if (batch > 0 && (!k_new || !v_new)) return PA_ERR_INVALID_ARG;
     return pa::decode_impl(out, q, k_new, v_new, k_cache, v_cache, block_tables, max_blocks_per_seq,
                            seq_lens, batch, max_seq_len, num_q_heads, num_kv_heads, head_dim, block_size,
-                           num_blocks, scale, partition_tokens, workspace, workspace_bytes, err_flag, stream);
+                           num_blocks, scale, partition_tokens, workspace, workspace_bytes, err_flag, stream,
+                           false, 1.f, 1.f);
+}
+
+int pa_decode_fp8(float *out, const void *q, const void *k_cache, const void *v_cache,
+                  const int32_t *block_tables, int max_blocks_per_seq, const int32_t *seq_lens, int batch,
+                  int max_seq_len, int num_q_heads, int num_kv_heads, int head_dim, int block_size,
+                  int64_t num_blocks, float scale, float k_scale, float v_scale, int partition_tokens,
+                  void *workspace, size_t workspace_bytes, int32_t *err_flag, void *stream) {
+    return pa::decode_impl(out, q, nullptr, nullptr, k_cache, v_cache, block_tables, max_blocks_per_seq,
+                           seq_lens, batch, max_seq_len, num_q_heads, num_kv_heads, head_dim, block_size,
+                           num_blocks, scale, partition_tokens, workspace, workspace_bytes, err_flag, stream,
+                           true, k_scale, v_scale);
+}
+
+int pa_decode_append_fp8(float *out, const void *q, const void *k_new, const void *v_new, void *k_cache,
+                         void *v_cache, const int32_t *block_tables, int max_blocks_per_seq,
+                         const int32_t *seq_lens, int batch, int max_seq_len, int num_q_heads,
+                         int num_kv_heads, int head_dim, int block_size, int64_t num_blocks, float scale,
+                         float k_scale, float v_scale, int partition_tokens, void *workspace,
+                         size_t workspace_bytes, int32_t *err_flag, void *stream) {
+    if (batch > 0 && (!k_new || !v_new)) return PA_ERR_INVALID_ARG;
+    return pa::decode_impl(out, q, k_new, v_new, k_cache, v_cache, block_tables, max_blocks_per_seq,
+                           seq_lens, batch, max_seq_len, num_q_heads, num_kv_heads, head_dim, block_size,
+                           num_blocks, scale, partition_tokens, workspace, workspace_bytes, err_flag, stream,
+                           true, k_scale, v_scale);
 }
 
 int pa_decode_builtin_scratch(float *out, const void *q, const void *k_cache, const void *v_cache,

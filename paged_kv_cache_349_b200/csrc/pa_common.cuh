@@ -5,6 +5,8 @@
 
 #include <cuda.h>
 #include <cuda_bf16.h>
+#include <cuda_fp16.h>
+#include <cuda_fp8.h>
 #include <cuda_runtime.h>
 #include <stdint.h>
 
@@ -28,7 +30,8 @@ int decode_impl(float *out, const void *q, const void *k_new, const void *v_new,
                 const void *v_cache, const int32_t *block_tables, int max_blocks_per_seq,
                 const int32_t *seq_lens, int batch, int max_seq_len, int num_q_heads, int num_kv_heads,
                 int head_dim, int block_size, int64_t num_blocks, float scale, int partition_tokens,
-                void *workspace, size_t workspace_bytes, int32_t *err_flag, void *stream);
+                void *workspace, size_t workspace_bytes, int32_t *err_flag, void *stream, bool fp8,
+                float k_scale, float v_scale);
 
 inline bool supported_shape(int num_q_heads, int num_kv_heads, int head_dim, int block_size) {
     if (num_kv_heads <= 0 || num_q_heads <= 0 || num_q_heads % num_kv_heads) return false;
@@ -153,6 +156,16 @@ __device__ __forceinline__ uint64_t l2_policy_evict_first() {
     return p;
 }
 
+// Asynchronous global -> shared copies (no register staging); wait with cp_async_wait_all.
+__device__ __forceinline__ void cp_async16(uint32_t smem_dst, const void *gmem_src) {
+    asm volatile("cp.async.ca.shared.global [%0], [%1], 16;" ::"r"(smem_dst), "l"(gmem_src) : "memory");
+}
+__device__ __forceinline__ void cp_async4(uint32_t smem_dst, const void *gmem_src) {
+    asm volatile("cp.async.ca.shared.global [%0], [%1], 4;" ::"r"(smem_dst), "l"(gmem_src) : "memory");
+}
+__device__ __forceinline__ void cp_async_commit() { asm volatile("cp.async.commit_group;" ::: "memory"); }
+__device__ __forceinline__ void cp_async_wait_all() { asm volatile("cp.async.wait_all;" ::: "memory"); }
+
 __device__ __forceinline__ uint4 lds128(uint32_t addr) {
     uint4 v;
     asm volatile("ld.shared.v4.u32 {%0, %1, %2, %3}, [%4];"
@@ -183,6 +196,73 @@ __device__ __forceinline__ void mma_bf16_16816(float (&d)[4], uint32_t a0, uint3
         "{%8, %9}, {%0, %1, %2, %3};"
         : "+f"(d[0]), "+f"(d[1]), "+f"(d[2]), "+f"(d[3])
         : "r"(a0), "r"(a1), "r"(a2), "r"(a3), "r"(b0), "r"(b1));
+}
+
+// D = A(16x16, row) * B(16x8, col) + D, f16 inputs, fp32 accumulate.
+__device__ __forceinline__ void mma_f16_16816(float (&d)[4], uint32_t a0, uint32_t a1, uint32_t a2,
+                                              uint32_t a3, uint32_t b0, uint32_t b1) {
+    asm volatile(
+        "mma.sync.aligned.m16n8k16.row.col.f32.f16.f16.f32 {%0, %1, %2, %3}, {%4, %5, %6, %7}, "
+        "{%8, %9}, {%0, %1, %2, %3};"
+        : "+f"(d[0]), "+f"(d[1]), "+f"(d[2]), "+f"(d[3])
+        : "r"(a0), "r"(a1), "r"(a2), "r"(a3), "r"(b0), "r"(b1));
+}
+
+// Four E4M3 codes (byte 0 first) -> two f16x2 words (exact conversions).
+__device__ __forceinline__ void e4m3x4_to_f16x4(uint32_t four_codes, uint32_t &f01, uint32_t &f23) {
+    asm("{\n\t.reg .b16 lo, hi;\n\t"
+        "mov.b32 {lo, hi}, %2;\n\t"
+        "cvt.rn.f16x2.e4m3x2 %0, lo;\n\t"
+        "cvt.rn.f16x2.e4m3x2 %1, hi;\n\t}"
+        : "=r"(f01), "=r"(f23)
+        : "r"(four_codes));
+}
+
+// Two E4M3 codes (low byte first) -> two f16 values (exact), as one 32-bit word.
+__device__ __forceinline__ uint32_t e4m3x2_to_f16x2(uint32_t two_codes) {
+    uint32_t f01, f23;
+    e4m3x4_to_f16x4(two_codes, f01, f23);
+    return f01;
+}
+
+// Codes in bytes `sel` of w -> f16x2 whose values are exactly E4M3_value * 2^-8.
+// The E4M3 exponent and mantissa (7 bits) drop into the low bits of the f16
+// exponent and the top of its mantissa; the exponent bias difference (15 - 7)
+// is the 2^-8, and E4M3 subnormals land on f16 subnormals with the same factor.
+// NaN codes are not handled (the library never writes them).  Byte selectors:
+// 0x1404 = codes 0,1; 0x3424 = codes 2,3.
+template <unsigned SEL>
+__device__ __forceinline__ uint32_t e4m3x2_to_f16x2_scaled(uint32_t w) {
+    const uint32_t t = __byte_perm(w, 0u, SEL);  // [0, c_lo, 0, c_hi]: each code in the top byte of a half
+    return (t & 0x80008000u) | ((t >> 1) & 0x3F803F80u);
+}
+
+// Eight bf16 values -> eight E4M3 codes: code = E4M3(x * inv_scale), the product
+// in fp32, rounded to nearest even and saturated to the largest finite value.
+__device__ __forceinline__ uint2 bf16x8_to_e4m3x8(uint4 v, float inv_scale) {
+    const uint32_t w[4] = {v.x, v.y, v.z, v.w};
+    uint32_t out[2] = {0u, 0u};
+#pragma unroll
+    for (int k = 0; k < 4; ++k) {
+        const float lo = __fmul_rn(__uint_as_float(w[k] << 16), inv_scale);
+        const float hi = __fmul_rn(__uint_as_float(w[k] & 0xffff0000u), inv_scale);
+        const uint32_t pair = (uint32_t)__nv_cvt_float2_to_fp8x2(make_float2(lo, hi), __NV_SATFINITE, __NV_E4M3);
+        out[k >> 1] |= pair << ((k & 1) * 16);
+    }
+    return make_uint2(out[0], out[1]);
+}
+
+// Pack two floats as f16x2 (round to nearest even); `lo` lands in bits 0..15.
+__device__ __forceinline__ uint32_t pack_f16x2(float lo, float hi) {
+    const __half2 v = __floats2half2_rn(lo, hi);
+    return *reinterpret_cast<const uint32_t *>(&v);
+}
+
+__device__ __forceinline__ float f16_lo_to_float(uint32_t v) {
+    return __half2float(__ushort_as_half((unsigned short)(v & 0xffffu)));
+}
+__device__ __forceinline__ float f16_hi_to_float(uint32_t v) {
+    return __half2float(__ushort_as_half((unsigned short)(v >> 16)));
 }
 
 __device__ __forceinline__ float fast_exp2(float x) {

@@ -102,7 +102,8 @@ int pa_decode_step_host(float *out_host, const void *q_host, const void *k_new_h
                          reinterpret_cast<const int32_t *>(st + l.tables), max_blocks_per_seq,
                          reinterpret_cast<const int32_t *>(st + l.lens), batch, max_seq_len, num_q_heads,
                          num_kv_heads, head_dim, block_size, num_blocks, scale, partition_tokens,
-                         l.workspace_bytes ? st + l.workspace : nullptr, l.workspace_bytes, err_flag, stream);
+                         l.workspace_bytes ? st + l.workspace : nullptr, l.workspace_bytes, err_flag, stream,
+                         false, 1.f, 1.f);
     if (rc != PA_OK) return rc;
     if (cudaMemcpyAsync(out_host, out_dev, (size_t)batch * num_q_heads * head_dim * 4, cudaMemcpyDeviceToHost,
                         s) != cudaSuccess)

@@ -429,8 +429,10 @@ def split_last_tokens(case: DecodeCase):
 
 
 def algorithmic_decode_bytes(case_or_lens, *, num_q_heads=None, num_kv_heads=None,
-                             head_dim=None, block_size=None) -> int:
-    """Bytes a decode call must move at minimum: K+V rows once, q, fp32 out, table entries, lengths."""
+                             head_dim=None, block_size=None, kv_elem_bytes: int = 2) -> int:
+    """Bytes a decode call must move at minimum: K+V rows once, q, fp32 out, table entries, lengths.
+
+    ``kv_elem_bytes`` is 2 for bf16 pools and 1 for fp8 pools."""
     if isinstance(case_or_lens, DecodeCase):
         c = case_or_lens
         lens, Hq, Hkv, d, bs = c.seq_lens, c.num_q_heads, c.num_kv_heads, c.head_dim, c.block_size
@@ -438,7 +440,7 @@ def algorithmic_decode_bytes(case_or_lens, *, num_q_heads=None, num_kv_heads=Non
         lens, Hq, Hkv, d, bs = case_or_lens, num_q_heads, num_kv_heads, head_dim, block_size
     lens = np.asarray(lens, dtype=np.int64)
     B = lens.size
-    kv = int(lens.sum()) * Hkv * d * 2 * 2
+    kv = int(lens.sum()) * Hkv * d * kv_elem_bytes * 2
     qb = B * Hq * d * 2
     ob = B * Hq * d * 4
     tb = int((-(-lens // bs)).sum()) * 4
