@@ -510,7 +510,8 @@ def run_e2e(args, case, pa, stream, world, k_pool, v_pool):
         raise SystemExit("--unfused applies to the device-resident step only")
     run = pa.DecodeStepHost(out_host=h_out, q_host=h_q, k_new_host=h_k, v_new_host=h_v, tables_host=h_tables,
                             lens_host=h_lens, pairs_host=h_pairs, k_cache=k_pool, v_cache=v_pool,
-                            scale=float(case.scale), partition_tokens=case.partition_tokens, staging=staging,
+                            scale=float(case.scale), partition_tokens=case.partition_tokens,
+                            num_chunks=args.step_chunks, staging=staging,
                             err_flag=flag, stream=stream)
     acc = {"h2d": 0, "d2h": 0, "alg": 0, "tokens": 0}
 
@@ -546,6 +547,7 @@ def run_e2e(args, case, pa, stream, world, k_pool, v_pool):
             "ms_per_step": round(dt * 1e3 / steps, 4),
             "h2d_bytes_per_step": acc["h2d"] // steps, "d2h_bytes_per_step": acc["d2h"] // steps,
             "kv_tokens_per_s": round(_sum_over_ranks(float(acc["tokens"]), world) / dt, 1),
+            "step_chunks": args.step_chunks or "auto",
             "includes": "host allocator batched append + table export into pinned memory, then one "
                         "pa_decode_step_host call: H2D of q/k_new/v_new/tables/lens/copy pairs, block copies, "
                         "fused cache write + decode, D2H of out; timed until out is on the host"}
@@ -606,6 +608,8 @@ def main():
     ap.add_argument("--config", type=int, default=2, choices=[1, 2, 3, 4, 5])
     ap.add_argument("--impl", choices=["native", "reference"], default="native")
     ap.add_argument("--no-e2e", action="store_true")
+    ap.add_argument("--step-chunks", type=int, default=0,
+                    help="e2e: chunks of sequences pa_decode_step_host pipelines (0 = the library's choice)")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--cpu-budget", type=float, default=12.0, help="seconds of oracle time")
     ap.add_argument("--kv-dtype", choices=["bf16", "fp8"], default="bf16",

@@ -132,6 +132,9 @@ int pa_copy_blocks(void *k_cache, void *v_cache, const int32_t *pairs, int num_p
  * host -> device.  Both sides use the pool layout above with the same
  * num_kv_heads, block_size and head_dim; they may differ in block count.
  * pairs: int32 [num_pairs, 2] = (src block, dst block), device-addressable.
+ * Every pointer is checked with cudaPointerGetAttributes before the launch:
+ * one the device cannot reach (pageable host memory, another GPU's memory,
+ * an address CUDA does not know) gives PA_ERR_INVALID_ARG and nothing runs.
  * Destinations must be distinct.  Ids out of range set PA_FLAG_BAD_PAIR and
  * the pair is skipped.  Bandwidth is that of the slower side (PCIe or
  * NVLink-C2C for host memory).
@@ -208,17 +211,37 @@ int pa_decode_append(float *out, const void *q, const void *k_new, const void *v
                      void *stream);
 
 /* ------------------------------------------------------------------------
- * One decode step from host buffers.  Enqueues on `stream`, in order:
- *   1. host-to-device copies of q, k_new, v_new, the block tables, the
- *      sequence lengths and the copy pairs into `staging` (one
- *      cudaMemcpyAsync per input),
+ * One decode step from host buffers.  Enqueues, in order:
+ *   1. host-to-device copies of the copy pairs, the block tables, the
+ *      sequence lengths, q, k_new and v_new into `staging`,
  *   2. pa_copy_blocks of the copy pairs (if any),
  *   3. pa_decode_append (cache write of each sequence's new token + decode),
- *   4. a device-to-host copy of the fp32 output into out_host.
- * The call returns once everything is enqueued; synchronise the stream
- * before reading out_host.  Host buffers should be page-locked (pinned)
- * for the copies to be asynchronous, and must stay valid and unchanged
- * until the stream has passed them.
+ *   4. the fp32 output into out_host.  When out_host is page-locked host
+ *      memory the device can address (checked with cudaPointerGetAttributes),
+ *      the decode kernels store the output into it directly, so the transfer
+ *      overlaps the decode; otherwise the output is staged on the device and
+ *      copied back with cudaMemcpyAsync.
+ * The call returns once everything is enqueued; synchronise `stream` before
+ * reading out_host.  Host buffers should be page-locked (pinned) for the
+ * copies to be asynchronous, and must stay valid and unchanged until the
+ * stream has passed them.
+ *
+ * num_chunks: 1 runs the four steps on `stream` alone.  n in 2..8 cuts the
+ * batch into n chunks of consecutive sequences (the first about half the
+ * size of the others) and pipelines them: chunk uploads and downloads run on library-owned
+ * copy streams and chunk decodes alternate between `stream` and a
+ * library-owned compute stream, so transfers of one chunk overlap the decode
+ * of another.  All of them start after the work already enqueued on `stream`
+ * and are joined back into `stream` before the call returns (on error paths
+ * too), so synchronising `stream` covers the whole step.  0 picks the count
+ * from the bytes crossing the host link: one chunk per MiB, at most 4, at
+ * most one per sequence.  The output, the pools and the error flag do not
+ * depend on the chunk count: the partitioning is resolved once for the whole
+ * batch (as pa_decode_partition_tokens reports it) and each chunk decodes
+ * its sequences exactly as an unchunked call would.  The side streams and
+ * events of a device are created by its first chunked call and kept until
+ * the process exits; calls on one device serialise their enqueueing on a
+ * lock.  num_chunks < 0 or > 8: PA_ERR_INVALID_ARG.
  *
  * Host inputs: q_host bf16 [batch, Hq, d]; k_new_host, v_new_host bf16
  * [batch, Hkv, d] (the token at position seq_lens[b]-1); block_tables_host
@@ -228,7 +251,9 @@ int pa_decode_append(float *out, const void *q, const void *k_new, const void *v
  * staging: device memory of at least pa_decode_step_staging_size(...) bytes
  * (computed with the same batch, max_blocks_per_seq, max_copy_pairs and
  * shapes, and a max_seq_len at least this call's), 256-byte aligned; it
- * holds the uploaded inputs, the device output and the decode workspace.
+ * holds the uploaded inputs, the device output and the decode workspace
+ * (with room for one slice per chunk).  A staging buffer may be reused by
+ * the next call on the same stream.
  * Other arguments, layouts and errors: as pa_decode_append.
  * ---------------------------------------------------------------------- */
 size_t pa_decode_step_staging_size(int batch, int max_blocks_per_seq, int max_copy_pairs, int num_q_heads,
@@ -240,7 +265,7 @@ int pa_decode_step_host(float *out_host, const void *q_host, const void *k_new_h
                         const int32_t *copy_pairs_host, int num_pairs, int max_copy_pairs, void *k_cache,
                         void *v_cache, int batch, int max_seq_len, int num_q_heads, int num_kv_heads,
                         int head_dim, int block_size, int64_t num_blocks, float scale, int partition_tokens,
-                        void *staging, size_t staging_bytes, int32_t *err_flag, void *stream);
+                        int num_chunks, void *staging, size_t staging_bytes, int32_t *err_flag, void *stream);
 
 /* ------------------------------------------------------------------------
  * Decode with library-owned scratch (no workspace argument).

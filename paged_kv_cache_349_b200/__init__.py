@@ -230,12 +230,13 @@ class DecodeStepHost:
     Holds the argument tuple for a fixed set of pinned host buffers, pools and
     staging, so each step only marshals what changes (max_seq_len, the number of
     copy pairs).  Host arrays are torch CPU tensors (pinned); pools and staging are
-    CUDA tensors.
+    CUDA tensors.  ``num_chunks``: 0 lets the library pick how many chunks of
+    sequences to pipeline, 1 disables pipelining, 2..8 forces that many.
     """
 
     def __init__(self, *, out_host, q_host, k_new_host, v_new_host, tables_host, lens_host, pairs_host,
-                 k_cache, v_cache, scale: float, partition_tokens: int = 0, staging=None, err_flag=None,
-                 stream=None):
+                 k_cache, v_cache, scale: float, partition_tokens: int = 0, num_chunks: int = 0, staging=None,
+                 err_flag=None, stream=None):
         torch = _torch()
         B, Hq, d = q_host.shape
         NB, Hkv, bs, d2 = k_cache.shape
@@ -256,7 +257,7 @@ class DecodeStepHost:
                       ctypes.c_void_p(lens_host.data_ptr()), ctypes.c_void_p(pairs_host.data_ptr()))
         self._kv = (self.max_pairs, _dev(k_cache, torch.bfloat16, "k_cache"), _dev(v_cache, torch.bfloat16, "v_cache"),
                     B)
-        self._shape = (Hq, Hkv, d, bs, NB, float(scale), int(partition_tokens))
+        self._shape = (Hq, Hkv, d, bs, NB, float(scale), int(partition_tokens), int(num_chunks))
         self._tail = (ctypes.c_void_p(staging.data_ptr()), staging.numel() * staging.element_size(),
                       _opt_flag(err_flag), _stream(stream))
 

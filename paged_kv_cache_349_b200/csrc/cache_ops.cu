@@ -179,9 +179,19 @@ int pa_swap_blocks(void *dst_k_cache, void *dst_v_cache, int64_t dst_num_blocks,
     if (!pa::aligned16(dst_k_cache) || !pa::aligned16(dst_v_cache) || !pa::aligned16(src_k_cache) ||
         !pa::aligned16(src_v_cache))
         return PA_ERR_INVALID_ARG;
-    return pa::launch_block_copy(dst_k_cache, dst_v_cache, src_k_cache, src_v_cache, pairs, num_pairs,
-                                 src_num_blocks, dst_num_blocks, num_kv_heads, block_size, head_dim, 2,
-                                 PA_FLAG_BAD_PAIR, err_flag, stream);
+    // Each side must be reachable from the device: device memory, or host memory
+    // that is page-locked (pageable host memory is an argument error, not a fault).
+    void *dk = nullptr, *dv = nullptr, *sk = nullptr, *sv = nullptr;
+    int rc = pa::device_address(dst_k_cache, &dk);
+    if (rc == PA_OK) rc = pa::device_address(dst_v_cache, &dv);
+    if (rc == PA_OK) rc = pa::device_address(src_k_cache, &sk);
+    if (rc == PA_OK) rc = pa::device_address(src_v_cache, &sv);
+    void *pp = nullptr;
+    if (rc == PA_OK) rc = pa::device_address(pairs, &pp);
+    if (rc != PA_OK) return rc;
+    return pa::launch_block_copy(dk, dv, sk, sv, static_cast<const int32_t *>(pp), num_pairs, src_num_blocks,
+                                 dst_num_blocks, num_kv_heads, block_size, head_dim, 2, PA_FLAG_BAD_PAIR,
+                                 err_flag, stream);
 }
 
 int pa_reshape_and_cache_fp8(const void *k_new, const void *v_new, void *k_cache, void *v_cache,
@@ -244,9 +254,19 @@ int pa_swap_blocks_fp8(void *dst_k_cache, void *dst_v_cache, int64_t dst_num_blo
     if (!pa::aligned16(dst_k_cache) || !pa::aligned16(dst_v_cache) || !pa::aligned16(src_k_cache) ||
         !pa::aligned16(src_v_cache))
         return PA_ERR_INVALID_ARG;
-    return pa::launch_block_copy(dst_k_cache, dst_v_cache, src_k_cache, src_v_cache, pairs, num_pairs,
-                                 src_num_blocks, dst_num_blocks, num_kv_heads, block_size, head_dim, 1,
-                                 PA_FLAG_BAD_PAIR, err_flag, stream);
+    // Each side must be reachable from the device: device memory, or host memory
+    // that is page-locked (pageable host memory is an argument error, not a fault).
+    void *dk = nullptr, *dv = nullptr, *sk = nullptr, *sv = nullptr;
+    int rc = pa::device_address(dst_k_cache, &dk);
+    if (rc == PA_OK) rc = pa::device_address(dst_v_cache, &dv);
+    if (rc == PA_OK) rc = pa::device_address(src_k_cache, &sk);
+    if (rc == PA_OK) rc = pa::device_address(src_v_cache, &sv);
+    void *pp = nullptr;
+    if (rc == PA_OK) rc = pa::device_address(pairs, &pp);
+    if (rc != PA_OK) return rc;
+    return pa::launch_block_copy(dk, dv, sk, sv, static_cast<const int32_t *>(pp), num_pairs, src_num_blocks,
+                                 dst_num_blocks, num_kv_heads, block_size, head_dim, 1, PA_FLAG_BAD_PAIR,
+                                 err_flag, stream);
 }
 
 }  // extern "C"

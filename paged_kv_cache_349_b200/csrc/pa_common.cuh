@@ -22,6 +22,11 @@ void count_launch();
 int device_sm_count();
 // Maps the last CUDA error after a launch to a status.
 int launch_status();
+// The address a kernel on the current device uses for `p`: device or managed
+// memory as is, page-locked host memory through its device mapping.  Host
+// memory that is not page-locked (or a pointer CUDA does not know) gives
+// PA_ERR_INVALID_ARG, so no kernel is ever handed an address it cannot reach.
+int device_address(const void *p, void **dev_ptr);
 
 inline bool aligned16(const void *p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
 

@@ -27,6 +27,35 @@ int device_sm_count() {
 
 int launch_status() { return cudaGetLastError() == cudaSuccess ? PA_OK : PA_ERR_CUDA; }
 
+int device_address(const void *p, void **dev_ptr) {
+    *dev_ptr = nullptr;
+    if (!p) return PA_ERR_INVALID_ARG;
+    cudaPointerAttributes a{};
+    if (cudaPointerGetAttributes(&a, p) != cudaSuccess) {
+        cudaGetLastError();  // clear the (non-sticky) error so the next launch check does not report it
+        return PA_ERR_INVALID_ARG;
+    }
+    int dev = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess) return PA_ERR_CUDA;
+    switch (a.type) {
+    case cudaMemoryTypeDevice:
+        if (a.device != dev) return PA_ERR_INVALID_ARG;  // another GPU's memory: not this library's to reach
+        *dev_ptr = const_cast<void *>(p);
+        return PA_OK;
+    case cudaMemoryTypeManaged:
+        *dev_ptr = const_cast<void *>(p);
+        return PA_OK;
+    case cudaMemoryTypeHost:
+        if (!a.devicePointer) return PA_ERR_INVALID_ARG;
+        // the mapping of the allocation's base, offset to p
+        *dev_ptr = static_cast<char *>(a.devicePointer) +
+                   (static_cast<const char *>(p) - static_cast<const char *>(a.hostPointer));
+        return PA_OK;
+    default:
+        return PA_ERR_INVALID_ARG;
+    }
+}
+
 }  // namespace pa
 
 extern "C" {

@@ -1,16 +1,34 @@
 // One decode step from host buffers: upload the step's inputs, apply the
 // copy-on-write block copies, run the fused cache write + decode, and copy
-// the output back -- all enqueued on one stream by one call.
+// the output back -- all enqueued by one call.
+//
+// A page-locked output buffer is written by the kernels directly; any other
+// is staged on the device and copied back.  A large step is cut into chunks
+// of whole sequences and pipelined over streams owned by the library: while
+// chunk c decodes, chunk c+1 is uploaded (and, for a staged output, chunk c-1
+// downloaded).  Chunk decodes alternate between the caller's stream and a
+// second compute stream, so one chunk's last wave of CTAs overlaps the next
+// chunk's first.  Every side stream is joined back
+// into the caller's stream before the call returns, so synchronising that
+// stream covers the whole step.
+#include <mutex>
+
 #include "pa_common.cuh"
 
 namespace pa {
 namespace {
 
 constexpr size_t kAlign = 256;
+constexpr int kMaxChunks = 8;
+constexpr int kMaxDevices = 64;
+// Auto chunking: one chunk per this many bytes crossing the host link, at most 4.
+constexpr size_t kAutoChunkBytes = (size_t)1 << 20;
+constexpr int kAutoMaxChunks = 4;
 
 inline size_t round_up(size_t x) { return (x + kAlign - 1) / kAlign * kAlign; }
 
-// Device staging of one step, each section 256-byte aligned.
+// Device staging of one step, each section 256-byte aligned.  The workspace
+// section leaves room for every chunk to have a 256-byte aligned slice of its own.
 struct StagingLayout {
     size_t q, k_new, v_new, tables, lens, pairs, out, workspace, workspace_bytes, total;
 };
@@ -37,6 +55,7 @@ StagingLayout staging_layout(int batch, int max_blocks_per_seq, int max_copy_pai
     l.workspace = off;
     l.workspace_bytes = pa_decode_workspace_size(batch, num_q_heads, num_kv_heads, head_dim, block_size,
                                                  max_seq_len, partition_tokens);
+    if (l.workspace_bytes) l.workspace_bytes += 2 * kAlign * kMaxChunks;
     off += round_up(l.workspace_bytes);
     l.total = off;
     return l;
@@ -45,6 +64,51 @@ StagingLayout staging_layout(int batch, int max_blocks_per_seq, int max_copy_pai
 int h2d(void *dst, const void *src, size_t bytes, cudaStream_t s) {
     if (bytes == 0) return PA_OK;
     return cudaMemcpyAsync(dst, src, bytes, cudaMemcpyHostToDevice, s) == cudaSuccess ? PA_OK : PA_ERR_CUDA;
+}
+
+int d2h(void *dst, const void *src, size_t bytes, cudaStream_t s) {
+    if (bytes == 0) return PA_OK;
+    return cudaMemcpyAsync(dst, src, bytes, cudaMemcpyDeviceToHost, s) == cudaSuccess ? PA_OK : PA_ERR_CUDA;
+}
+
+// Side streams and events of one device, created on first use.  The events are
+// reused by every call, so one call's enqueue sequence holds `mu` throughout.
+struct Pipes {
+    std::mutex mu;
+    bool ready = false;
+    cudaStream_t up = nullptr, down = nullptr, comp = nullptr;
+    cudaEvent_t start = nullptr, copied = nullptr, up_done = nullptr, comp_done = nullptr, down_done = nullptr;
+    cudaEvent_t in[kMaxChunks] = {}, dec[kMaxChunks] = {};
+};
+
+Pipes g_pipes[kMaxDevices];
+
+bool make_pipes(Pipes &p) {
+    if (p.ready) return true;
+    const unsigned sf = cudaStreamNonBlocking;
+    const unsigned ef = cudaEventDisableTiming;
+    bool ok = cudaStreamCreateWithFlags(&p.up, sf) == cudaSuccess &&
+              cudaStreamCreateWithFlags(&p.down, sf) == cudaSuccess &&
+              cudaStreamCreateWithFlags(&p.comp, sf) == cudaSuccess;
+    for (cudaEvent_t *e : {&p.start, &p.copied, &p.up_done, &p.comp_done, &p.down_done})
+        ok = ok && cudaEventCreateWithFlags(e, ef) == cudaSuccess;
+    for (int c = 0; c < kMaxChunks; ++c)
+        ok = ok && cudaEventCreateWithFlags(&p.in[c], ef) == cudaSuccess &&
+             cudaEventCreateWithFlags(&p.dec[c], ef) == cudaSuccess;
+    p.ready = ok;  // on failure the handles made so far are kept and reused by the next attempt
+    return ok;
+}
+
+// Makes `waiter` wait for everything enqueued on `s` so far.
+int after(cudaStream_t waiter, cudaStream_t s, cudaEvent_t e) {
+    if (cudaEventRecord(e, s) != cudaSuccess) return PA_ERR_CUDA;
+    return cudaStreamWaitEvent(waiter, e, 0) == cudaSuccess ? PA_OK : PA_ERR_CUDA;
+}
+
+int auto_chunks(int batch, size_t link_bytes) {
+    const size_t n = link_bytes / kAutoChunkBytes;
+    int c = n < 1 ? 1 : (n > (size_t)kAutoMaxChunks ? kAutoMaxChunks : (int)n);
+    return c > batch ? batch : c;
 }
 
 }  // namespace
@@ -67,8 +131,9 @@ int pa_decode_step_host(float *out_host, const void *q_host, const void *k_new_h
                         const int32_t *copy_pairs_host, int num_pairs, int max_copy_pairs, void *k_cache,
                         void *v_cache, int batch, int max_seq_len, int num_q_heads, int num_kv_heads,
                         int head_dim, int block_size, int64_t num_blocks, float scale, int partition_tokens,
-                        void *staging, size_t staging_bytes, int32_t *err_flag, void *stream) {
-    if (batch < 0 || num_pairs < 0 || max_copy_pairs < 0 || max_blocks_per_seq < 0 || max_seq_len < 0)
+                        int num_chunks, void *staging, size_t staging_bytes, int32_t *err_flag, void *stream) {
+    if (batch < 0 || num_pairs < 0 || max_copy_pairs < 0 || max_blocks_per_seq < 0 || max_seq_len < 0 ||
+        num_chunks < 0 || num_chunks > pa::kMaxChunks)
         return PA_ERR_INVALID_ARG;
     if (!pa::supported_shape(num_q_heads, num_kv_heads, head_dim, block_size)) return PA_ERR_UNSUPPORTED;
     if (batch == 0) return PA_OK;
@@ -81,34 +146,131 @@ int pa_decode_step_host(float *out_host, const void *q_host, const void *k_new_h
                                                    partition_tokens);
     if (staging_bytes < l.total || (reinterpret_cast<uintptr_t>(staging) & (pa::kAlign - 1)))
         return PA_ERR_INVALID_ARG;
+    // Resolve the partitioning once for the whole batch, so that every chunk
+    // splits its sequences exactly as an unchunked call would.
+    const int pt = pa_decode_partition_tokens(batch, num_q_heads, num_kv_heads, head_dim, block_size, max_seq_len,
+                                              partition_tokens);
     char *st = static_cast<char *>(staging);
     cudaStream_t s = static_cast<cudaStream_t>(stream);
-    const size_t q_bytes = (size_t)batch * num_q_heads * head_dim * 2;
-    const size_t kv_bytes = (size_t)batch * num_kv_heads * head_dim * 2;
-    int rc = pa::h2d(st + l.q, q_host, q_bytes, s);
-    if (rc == PA_OK) rc = pa::h2d(st + l.k_new, k_new_host, kv_bytes, s);
-    if (rc == PA_OK) rc = pa::h2d(st + l.v_new, v_new_host, kv_bytes, s);
-    if (rc == PA_OK) rc = pa::h2d(st + l.tables, block_tables_host, (size_t)batch * max_blocks_per_seq * 4, s);
-    if (rc == PA_OK) rc = pa::h2d(st + l.lens, seq_lens_host, (size_t)batch * 4, s);
-    if (rc == PA_OK) rc = pa::h2d(st + l.pairs, copy_pairs_host, (size_t)num_pairs * 8, s);
-    if (rc != PA_OK) return rc;
-    if (num_pairs > 0) {
-        rc = pa_copy_blocks(k_cache, v_cache, reinterpret_cast<const int32_t *>(st + l.pairs), num_pairs,
-                            num_blocks, num_kv_heads, block_size, head_dim, err_flag, stream);
-        if (rc != PA_OK) return rc;
+    // bytes per sequence of each input and of the output
+    const size_t q_row = (size_t)num_q_heads * head_dim * 2;
+    const size_t kv_row = (size_t)num_kv_heads * head_dim * 2;
+    const size_t tab_row = (size_t)max_blocks_per_seq * 4;
+    const size_t out_row = (size_t)num_q_heads * head_dim * 4;
+    const size_t link_bytes = (size_t)batch * (q_row + 2 * kv_row + tab_row + 4 + out_row) + (size_t)num_pairs * 8;
+    const int chunks = num_chunks ? (num_chunks > batch ? batch : num_chunks) : pa::auto_chunks(batch, link_bytes);
+
+    // The output goes straight into out_host when the device can address it
+    // (page-locked host memory): the kernels' stores cross the host link while
+    // the decode runs, and no copy stage follows.  Otherwise it is staged on the
+    // device and copied back.
+    void *out_mapped = nullptr;
+    const bool direct = pa::device_address(out_host, &out_mapped) == PA_OK;
+    char *out_base = direct ? static_cast<char *>(out_mapped) : st + l.out;
+
+    // decode of sequences [b0, b0 + nb) with inputs in staging, on stream cs, workspace slice ws
+    auto decode_rows = [&](int b0, int nb, char *ws, size_t ws_bytes, cudaStream_t cs) {
+        return pa::decode_impl(reinterpret_cast<float *>(out_base + b0 * out_row), st + l.q + b0 * q_row,
+                               st + l.k_new + b0 * kv_row, st + l.v_new + b0 * kv_row, k_cache, v_cache,
+                               reinterpret_cast<const int32_t *>(st + l.tables + b0 * tab_row), max_blocks_per_seq,
+                               reinterpret_cast<const int32_t *>(st + l.lens) + b0, nb, max_seq_len, num_q_heads,
+                               num_kv_heads, head_dim, block_size, num_blocks, scale, pt, ws, ws_bytes, err_flag,
+                               cs, false, 1.f, 1.f);
+    };
+    // q, k_new and v_new of sequences [b0, b0 + nb)
+    auto upload_rows = [&](int b0, int nb, cudaStream_t cs) {
+        int rc = pa::h2d(st + l.q + b0 * q_row, static_cast<const char *>(q_host) + b0 * q_row, nb * q_row, cs);
+        if (rc == PA_OK)
+            rc = pa::h2d(st + l.k_new + b0 * kv_row, static_cast<const char *>(k_new_host) + b0 * kv_row,
+                         nb * kv_row, cs);
+        if (rc == PA_OK)
+            rc = pa::h2d(st + l.v_new + b0 * kv_row, static_cast<const char *>(v_new_host) + b0 * kv_row,
+                         nb * kv_row, cs);
+        return rc;
+    };
+    // copy pairs, block tables and lengths of the whole batch
+    auto upload_meta = [&](cudaStream_t cs) {
+        int rc = pa::h2d(st + l.pairs, copy_pairs_host, (size_t)num_pairs * 8, cs);
+        if (rc == PA_OK) rc = pa::h2d(st + l.tables, block_tables_host, batch * tab_row, cs);
+        if (rc == PA_OK) rc = pa::h2d(st + l.lens, seq_lens_host, (size_t)batch * 4, cs);
+        return rc;
+    };
+    auto copy_pairs = [&](cudaStream_t cs) {
+        if (num_pairs == 0) return (int)PA_OK;
+        return pa_copy_blocks(k_cache, v_cache, reinterpret_cast<const int32_t *>(st + l.pairs), num_pairs,
+                              num_blocks, num_kv_heads, block_size, head_dim, err_flag, cs);
+    };
+
+    if (chunks <= 1) {
+        int rc = upload_meta(s);
+        if (rc == PA_OK) rc = upload_rows(0, batch, s);
+        if (rc == PA_OK) rc = copy_pairs(s);
+        if (rc == PA_OK)
+            rc = decode_rows(0, batch, l.workspace_bytes ? st + l.workspace : nullptr, l.workspace_bytes, s);
+        if (rc == PA_OK && !direct) rc = pa::d2h(out_host, st + l.out, batch * out_row, s);
+        return rc;
     }
-    float *out_dev = reinterpret_cast<float *>(st + l.out);
-    rc = pa::decode_impl(out_dev, st + l.q, st + l.k_new, st + l.v_new, k_cache, v_cache,
-                         reinterpret_cast<const int32_t *>(st + l.tables), max_blocks_per_seq,
-                         reinterpret_cast<const int32_t *>(st + l.lens), batch, max_seq_len, num_q_heads,
-                         num_kv_heads, head_dim, block_size, num_blocks, scale, partition_tokens,
-                         l.workspace_bytes ? st + l.workspace : nullptr, l.workspace_bytes, err_flag, stream,
-                         false, 1.f, 1.f);
-    if (rc != PA_OK) return rc;
-    if (cudaMemcpyAsync(out_host, out_dev, (size_t)batch * num_q_heads * head_dim * 4, cudaMemcpyDeviceToHost,
-                        s) != cudaSuccess)
-        return PA_ERR_CUDA;
-    return PA_OK;
+
+    int dev = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= pa::kMaxDevices) return PA_ERR_CUDA;
+    pa::Pipes &p = pa::g_pipes[dev];
+    std::lock_guard<std::mutex> lock(p.mu);
+    if (!pa::make_pipes(p)) return PA_ERR_CUDA;
+
+    // Fork: the side streams start after everything already on the caller's stream
+    // (the previous step, which may still read this staging).
+    if (cudaEventRecord(p.start, s) != cudaSuccess) return PA_ERR_CUDA;
+    for (cudaStream_t side : {p.up, p.down, p.comp})
+        if (cudaStreamWaitEvent(side, p.start, 0) != cudaSuccess) return PA_ERR_CUDA;
+
+    // Block copies first, on the caller's stream; every chunk's decode comes after them.
+    int rc = upload_meta(p.up);
+    if (rc == PA_OK && num_pairs > 0) {
+        rc = pa::after(s, p.up, p.copied);
+        if (rc == PA_OK) rc = copy_pairs(s);
+        if (rc == PA_OK) rc = pa::after(p.comp, s, p.copied);
+    }
+    char *ws = l.workspace_bytes ? st + l.workspace : nullptr;
+    size_t ws_left = l.workspace_bytes;
+    // Chunk 0 has half the weight of the others: the first decode waits for its
+    // upload alone, while every later upload runs ahead of the decodes (the link
+    // delivers inputs faster than decode consumes them).
+    const int64_t units = 2LL * chunks - 1;
+    auto chunk_start = [&](int c) {  // at least one sequence per chunk (chunks <= batch)
+        const int b = c == 0 ? 0 : (int)((int64_t)batch * (2LL * c - 1) / units);
+        return b > c ? b : c;
+    };
+    for (int c = 0; c < chunks && rc == PA_OK; ++c) {
+        const int b0 = chunk_start(c);
+        const int nb = (c + 1 < chunks ? chunk_start(c + 1) : batch) - b0;
+        if (nb == 0) continue;
+        cudaStream_t cs = (c & 1) ? p.comp : s;
+        rc = upload_rows(b0, nb, p.up);
+        if (rc == PA_OK) rc = pa::after(cs, p.up, p.in[c]);
+        size_t ws_bytes = 0;
+        if (rc == PA_OK && ws) {
+            ws_bytes = pa_decode_workspace_size(nb, num_q_heads, num_kv_heads, head_dim, block_size, max_seq_len,
+                                                pt);
+            if (pa::round_up(ws_bytes) > ws_left) rc = PA_ERR_INVALID_ARG;
+        }
+        if (rc == PA_OK) rc = decode_rows(b0, nb, ws_bytes ? ws : nullptr, ws_bytes, cs);
+        if (rc == PA_OK && ws_bytes) {
+            ws += pa::round_up(ws_bytes);
+            ws_left -= pa::round_up(ws_bytes);
+        }
+        if (rc == PA_OK && !direct) {
+            rc = pa::after(p.down, cs, p.dec[c]);
+            if (rc == PA_OK)
+                rc = pa::d2h(reinterpret_cast<char *>(out_host) + b0 * out_row,
+                             st + l.out + b0 * out_row, nb * out_row, p.down);
+        }
+    }
+    // Join every side stream back into the caller's stream, on error paths too.
+    const int jc = pa::after(s, p.up, p.up_done);
+    const int jp = pa::after(s, p.comp, p.comp_done);
+    const int jd = pa::after(s, p.down, p.down_done);
+    if (rc == PA_OK) rc = jc != PA_OK ? jc : (jp != PA_OK ? jp : jd);
+    return rc;
 }
 
 }  // extern "C"

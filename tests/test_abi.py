@@ -94,3 +94,23 @@ def test_workspace_size_explicit_partitions(pt, maxlen, parts):
         o_bytes = -(-rows * d * 4 // 256) * 256
         assert size == o_bytes + rows * 8
         assert pa.pa_decode_partition_tokens(B, Hq, Hkv, d, 16, maxlen, pt) == pt
+
+
+def test_host_step_argument_errors_need_no_gpu():
+    f = lib.pa_decode_step_host
+    base = [_fake(), _fake(), _fake(), _fake(), _fake(), 4, _fake(), None, 0, 0, _fake(), _fake(), 2, 64, 8, 2,
+            128, 16, 64, 0.1, -1, 0, _fake(0x100000), 1 << 20, None, None]
+
+    def call(**kw):
+        a = list(base)
+        for i, v in kw.items():
+            a[int(i[1:])] = v
+        return f(*a)
+
+    assert call(a12=0) == pa.PA_OK                        # empty batch
+    assert call(a21=-1) == pa.PA_ERR_INVALID_ARG          # num_chunks < 0
+    assert call(a21=9) == pa.PA_ERR_INVALID_ARG           # more chunks than the library pipelines
+    assert call(a16=96) == pa.PA_ERR_UNSUPPORTED          # head_dim
+    assert call(a8=1) == pa.PA_ERR_INVALID_ARG            # pairs beyond max_copy_pairs
+    assert call(a23=16) == pa.PA_ERR_INVALID_ARG          # staging too small
+    assert call(a22=_fake(0x100010)) == pa.PA_ERR_INVALID_ARG  # staging not 256-byte aligned

@@ -62,13 +62,22 @@ def test_full_size_llama2_7b_sampled_rows():
     assert_close(got[rows[:, 0], rows[:, 1]], want, "cfg2 full fused")
 
 
-@pytest.mark.parametrize("cfg,kw", [
-    (2, dict(batch=6, max_len=300, num_blocks=256)),
-    (4, dict(batch=9, max_len=1500, num_blocks=512)),
-    (5, dict(batch=2, max_len=2048, num_blocks=640, num_copy_pairs=40)),
+@pytest.mark.parametrize("cfg,kw,chunks,pinned_out", [
+    (2, dict(batch=6, max_len=300, num_blocks=256), 1, True),
+    (2, dict(batch=6, max_len=300, num_blocks=256), 8, True),        # one sequence per chunk (8 clamps to 6)
+    (2, dict(batch=64, max_len=300, num_blocks=2048), 0, True),      # auto: ~2.6 MB over the link -> 2 chunks
+    (2, dict(batch=67, max_len=300, num_blocks=2048), 5, True),      # ragged chunk sizes
+    (2, dict(batch=67, max_len=300, num_blocks=2048), 5, False),     # pageable output: staged + copied back
+    (4, dict(batch=9, max_len=1500, num_blocks=512), 1, True),
+    (4, dict(batch=9, max_len=1500, num_blocks=512), 1, False),
+    (4, dict(batch=9, max_len=1500, num_blocks=512), 4, True),       # split decode: a workspace slice per chunk
+    (5, dict(batch=2, max_len=2048, num_blocks=640, num_copy_pairs=40), 1, True),
+    (5, dict(batch=3, max_len=2048, num_blocks=960, num_copy_pairs=40), 3, True),  # copies before every chunk
 ])
-def test_host_step_matches_device_path(cfg, kw):
-    """pa_decode_step_host (uploads, copies, fused decode, download) == the device-resident path."""
+def test_host_step_matches_device_path(cfg, kw, chunks, pinned_out):
+    """pa_decode_step_host (uploads, copies, fused decode, output to the host) == the device-resident
+    path, bit for bit, whether or not the step is cut into pipelined chunks and whether the output
+    buffer is page-locked (written by the kernels) or pageable (staged and copied back)."""
     import torch
     import paged_kv_cache_349_b200 as pa
     case = W.make_case(cfg, **kw)
@@ -82,7 +91,9 @@ def test_host_step_matches_device_path(cfg, kw):
         t = torch.from_numpy(np.ascontiguousarray(a))
         return (t.view(dtype) if dtype is torch.bfloat16 else t.to(dtype)).pin_memory()
 
-    out_h = torch.full(case.q.shape, float("nan"), dtype=torch.float32).pin_memory()
+    out_h = torch.full(case.q.shape, float("nan"), dtype=torch.float32)
+    if pinned_out:
+        out_h = out_h.pin_memory()
     pairs = case.copy_pairs.reshape(-1, 2)
     max_pairs = max(1, pairs.shape[0])
     pairs_h = torch.zeros((max_pairs, 2), dtype=torch.int32)
@@ -98,7 +109,8 @@ def test_host_step_matches_device_path(cfg, kw):
                              tables_host=pinned(case.block_tables, torch.int32),
                              lens_host=pinned(case.seq_lens, torch.int32), pairs_host=pairs_h,
                              k_cache=dc.k, v_cache=dc.v, scale=float(case.scale),
-                             partition_tokens=case.partition_tokens, staging=staging, err_flag=dc.flag)
+                             partition_tokens=case.partition_tokens, num_chunks=chunks, staging=staging,
+                             err_flag=dc.flag)
     step(case.max_seq_len, pairs.shape[0])
     torch.cuda.synchronize()
     got = out_h.numpy().astype(np.float64)

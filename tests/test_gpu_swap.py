@@ -59,3 +59,33 @@ def test_swap_bad_pair_flagged(torch_cuda):
     torch.cuda.synchronize()
     assert int(flag.item()) == pa.PA_FLAG_BAD_PAIR
     assert float(k[3].float().sum()) == 16 * 64 and float(k[0].float().sum()) == 0
+
+
+def test_swap_rejects_pageable_host_memory(torch_cuda):
+    """A host pool the device cannot address (pageable memory) is an argument error caught before any
+    launch: nothing is copied and the flag stays clear."""
+    import ctypes
+    torch = torch_cuda
+    import paged_kv_cache_349_b200 as pa
+    from paged_kv_cache_349_b200._lib import lib
+    k = torch.ones((4, 1, 16, 64), dtype=torch.bfloat16, device="cuda")
+    pageable = np.zeros((4, 1, 16, 64), np.uint16)           # plain numpy memory, never registered with CUDA
+    pairs = i32_dev(np.array([[0, 1]], np.int32))
+    flag = torch.zeros(1, dtype=torch.int32, device="cuda")
+    hp = ctypes.c_void_p(pageable.ctypes.data)
+    dp = ctypes.c_void_p(k.data_ptr())
+    before = pa.launch_count()
+    rc = lib.pa_swap_blocks(hp, hp, 4, dp, dp, 4, ctypes.c_void_p(pairs.data_ptr()), 1, 1, 16, 64,
+                            ctypes.c_void_p(flag.data_ptr()), None)
+    assert rc == pa.PA_ERR_INVALID_ARG
+    rc = lib.pa_swap_blocks(dp, dp, 4, hp, hp, 4, ctypes.c_void_p(pairs.data_ptr()), 1, 1, 16, 64,
+                            ctypes.c_void_p(flag.data_ptr()), None)
+    assert rc == pa.PA_ERR_INVALID_ARG
+    # pairs in pageable host memory too
+    hpairs = np.array([[0, 1]], np.int32)
+    rc = lib.pa_swap_blocks(dp, dp, 4, dp, dp, 4, ctypes.c_void_p(hpairs.ctypes.data), 1, 1, 16, 64,
+                            ctypes.c_void_p(flag.data_ptr()), None)
+    assert rc == pa.PA_ERR_INVALID_ARG
+    torch.cuda.synchronize()
+    assert pa.launch_count() == before
+    assert int(flag.item()) == 0 and not pageable.any() and float(k.float().sum()) == 4 * 16 * 64
