@@ -476,10 +476,11 @@ def run_e2e(args, case, pa, stream, world, k_pool, v_pool):
     """The same step through the public API with host buffers (pinned), timed end to end.
 
     Every step: the host allocator appends one token per sequence (and reports
-    copy-on-write pairs), exports the tables into pinned memory, and one
-    ``pa_decode_step_host`` call uploads the step's inputs, applies the copies,
-    runs the fused cache write + decode and copies the output back; the step
-    ends when the output is on the host.
+    copy-on-write pairs) and exports the tables into pinned memory (one
+    ``pa_alloc_step`` call); one ``pa_decode_step_host`` call then uploads the
+    step's inputs, applies the copies and runs the fused cache write + decode,
+    whose output lands in pinned host memory; the step ends when the output is
+    on the host.
     """
     import torch
     bs = case.block_size
@@ -515,13 +516,10 @@ def run_e2e(args, case, pa, stream, world, k_pool, v_pool):
                             err_flag=flag, stream=stream)
     acc = {"h2d": 0, "d2h": 0, "alg": 0, "tokens": 0}
 
+    host_step = alloc.step_fn(sids, tables_np, lens_np, pairs_np)
+
     def e2e_step(count):
-        _, pairs = alloc.append_batch(sids)
-        alloc.export(sids, max_blocks, tables=tables_np, lens=lens_np)
-        n_pairs = pairs.shape[0]
-        if n_pairs:
-            pairs_np[:n_pairs] = pairs
-        max_len = int(lens_np.max())
+        n_pairs, max_len = host_step()  # append one token per sequence, export tables + lengths
         run(max_len, n_pairs)
         stream.synchronize()  # the step's output is on the host
         if count:
@@ -548,7 +546,7 @@ def run_e2e(args, case, pa, stream, world, k_pool, v_pool):
             "h2d_bytes_per_step": acc["h2d"] // steps, "d2h_bytes_per_step": acc["d2h"] // steps,
             "kv_tokens_per_s": round(_sum_over_ranks(float(acc["tokens"]), world) / dt, 1),
             "step_chunks": args.step_chunks or "auto",
-            "includes": "host allocator batched append + table export into pinned memory, then one "
+            "includes": "host allocator step (pa_alloc_step: batched append + table export into pinned memory), then one "
                         "pa_decode_step_host call: H2D of q/k_new/v_new/tables/lens/copy pairs, block copies, "
                         "fused cache write + decode, D2H of out; timed until out is on the host"}
 

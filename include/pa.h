@@ -212,8 +212,11 @@ int pa_decode_append(float *out, const void *q, const void *k_new, const void *v
 
 /* ------------------------------------------------------------------------
  * One decode step from host buffers.  Enqueues, in order:
- *   1. host-to-device copies of the copy pairs, the block tables, the
- *      sequence lengths, q, k_new and v_new into `staging`,
+ *   1. the upload of the copy pairs, the block tables, the sequence
+ *      lengths, q, k_new and v_new into `staging`: one kernel reads every
+ *      input that is page-locked and 16-byte aligned straight from host
+ *      memory through its device mapping; any other input is copied with
+ *      cudaMemcpyAsync,
  *   2. pa_copy_blocks of the copy pairs (if any),
  *   3. pa_decode_append (cache write of each sequence's new token + decode),
  *   4. the fp32 output into out_host.  When out_host is page-locked host
@@ -409,6 +412,17 @@ int pa_seq_block_table(const pa_allocator *alloc, int seq_id, int32_t *out, int 
  * (unused entries = pad) plus int32 seq_lens[n]; host memory. */
 int pa_alloc_export(const pa_allocator *alloc, const int32_t *seq_ids, int n, int32_t *tables,
                     int max_blocks, int32_t pad, int32_t *seq_lens);
+/* The host side of one decode step in one call: pa_seq_append_batch on
+ * seq_ids[0..n) (slots are not reported: the fused decode derives each new
+ * token's slot from the table), then pa_alloc_export of the same sequences
+ * into tables [n, max_blocks] / seq_lens [n].  cow_pairs_out (capacity n
+ * pairs) receives the copies to apply before the decode, *n_cow their count,
+ * *max_seq_len the longest length after the append.  All-or-nothing: on
+ * PA_ERR_OOM, or PA_ERR_INVALID_ARG because a table would outgrow
+ * max_blocks, the allocator is unchanged (the output arrays may have been
+ * written).  Host memory throughout. */
+int pa_alloc_step(pa_allocator *alloc, const int32_t *seq_ids, int n, int32_t *tables, int max_blocks,
+                  int32_t pad, int32_t *seq_lens, int32_t *cow_pairs_out, int *n_cow, int *max_seq_len);
 int pa_alloc_num_free(const pa_allocator *alloc);
 /* Reference count of a block (0 = free), or -1 for an id out of range. */
 int pa_block_refcount(const pa_allocator *alloc, int32_t block);

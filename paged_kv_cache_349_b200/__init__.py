@@ -458,6 +458,34 @@ class Allocator:
                                    _np_ptr(lens)), "pa_alloc_export")
         return tables, lens
 
+    def step_fn(self, seq_ids, tables: np.ndarray, lens: np.ndarray, pairs: np.ndarray, pad: int = -1):
+        """A callable for the host side of repeated decode steps on fixed buffers (``pa_alloc_step``).
+
+        Each call appends one token to every sequence of ``seq_ids``, writes their padded tables into
+        ``tables`` (int32 [n, max_blocks]) and lengths into ``lens`` (int32 [n]), and the copy-on-write
+        pairs into ``pairs`` (int32 [>= n, 2]); it returns ``(num_pairs, max_seq_len)``.  The arrays
+        may be numpy views of pinned buffers; their pointers are taken once, here.
+        """
+        ids = np.ascontiguousarray(seq_ids, dtype=np.int32)
+        n = ids.size
+        for a, shape, name in ((tables, None, "tables"), (lens, (n,), "lens"), (pairs, None, "pairs")):
+            if a.dtype != np.int32 or not a.flags.c_contiguous:
+                raise ValueError(f"{name} must be a contiguous int32 array")
+        if tables.ndim != 2 or tables.shape[0] != n or lens.shape != (n,) or pairs.ndim != 2 or \
+                pairs.shape[1] != 2 or pairs.shape[0] < n:
+            raise ValueError("tables [n, max_blocks], lens [n], pairs [>= n, 2] expected")
+        n_cow, max_len = ctypes.c_int(), ctypes.c_int()
+        args = (self._h, _np_ptr(ids), n, _np_ptr(tables), int(tables.shape[1]), int(pad), _np_ptr(lens),
+                _np_ptr(pairs), ctypes.byref(n_cow), ctypes.byref(max_len))
+        fn = lib.pa_alloc_step
+
+        def step():
+            _check(fn(*args), "pa_alloc_step")
+            return n_cow.value, max_len.value
+
+        step.ids = ids  # keeps the id array alive with the callable
+        return step
+
     def num_free(self) -> int:
         return int(lib.pa_alloc_num_free(self._h))
 

@@ -96,6 +96,42 @@ struct pa_allocator {
     }
 };
 
+namespace {
+
+// Appends one token to each of ids[0..n) in order, all or nothing: on any
+// failure (out of blocks, or a table growing past max_blocks) every append
+// of the call is reverted.  Copy-on-write pairs go to pairs[2k], pairs[2k+1];
+// slots (optional) receive each new token's slot.
+int append_all(pa_allocator *a, const int32_t *ids, int n, int32_t *slots, int32_t *pairs, int *ncow,
+               int64_t max_blocks) {
+    std::vector<Undo> log;
+    log.reserve((size_t)n);
+    int count = 0;
+    int st = PA_OK;
+    for (int i = 0; i < n && st == PA_OK; ++i) {
+        int32_t slot, src, dst;
+        Undo u;
+        st = a->append(ids[i], &slot, &src, &dst, &u);
+        if (st != PA_OK) break;
+        log.push_back(u);
+        if (slots) slots[i] = slot;
+        if (src >= 0) {
+            pairs[2 * count] = src;
+            pairs[2 * count + 1] = dst;
+            ++count;
+        }
+        if ((int64_t)a->seqs[ids[i]].blocks.size() > max_blocks) st = PA_ERR_INVALID_ARG;
+    }
+    if (st != PA_OK) {
+        for (auto it = log.rbegin(); it != log.rend(); ++it) a->revert(*it);
+        return st;
+    }
+    *ncow = count;
+    return PA_OK;
+}
+
+}  // namespace
+
 extern "C" {
 
 int pa_alloc_create_ordered(int num_blocks, int block_size, const int32_t *order,
@@ -163,25 +199,30 @@ int pa_seq_append_batch(pa_allocator *alloc, const int32_t *seq_ids, int n, int3
         return PA_ERR_INVALID_ARG;
     for (int i = 0; i < n; ++i)
         if (!alloc->valid_seq(seq_ids[i])) return PA_ERR_BAD_INDEX;
-    std::vector<Undo> log;
-    log.reserve((size_t)n);
+    return append_all(alloc, seq_ids, n, slots_out, cow_pairs_out, n_cow, INT64_MAX);
+}
+
+int pa_alloc_step(pa_allocator *alloc, const int32_t *seq_ids, int n, int32_t *tables, int max_blocks,
+                  int32_t pad, int32_t *seq_lens, int32_t *cow_pairs_out, int *n_cow, int *max_seq_len) {
+    if (!alloc || n < 0 || max_blocks < 0 || !n_cow || !max_seq_len) return PA_ERR_INVALID_ARG;
+    if (n > 0 && (!seq_ids || !tables || !seq_lens || !cow_pairs_out)) return PA_ERR_INVALID_ARG;
+    for (int i = 0; i < n; ++i)
+        if (!alloc->valid_seq(seq_ids[i])) return PA_ERR_BAD_INDEX;
     int ncow = 0;
+    const int st = append_all(alloc, seq_ids, n, nullptr, cow_pairs_out, &ncow, max_blocks);
+    if (st != PA_OK) return st;
+    int64_t longest = 0;
     for (int i = 0; i < n; ++i) {
-        int32_t s, d;
-        Undo u;
-        const int st = alloc->append(seq_ids[i], &slots_out[i], &s, &d, &u);
-        if (st != PA_OK) {
-            for (auto it = log.rbegin(); it != log.rend(); ++it) alloc->revert(*it);
-            return st;
-        }
-        log.push_back(u);
-        if (s >= 0) {
-            cow_pairs_out[2 * ncow] = s;
-            cow_pairs_out[2 * ncow + 1] = d;
-            ++ncow;
-        }
+        const Seq &s = alloc->seqs[seq_ids[i]];
+        int32_t *row = tables + (size_t)i * (size_t)max_blocks;
+        const size_t nb = s.blocks.size();
+        if (nb) std::memcpy(row, s.blocks.data(), nb * sizeof(int32_t));
+        for (size_t j = nb; j < (size_t)max_blocks; ++j) row[j] = pad;
+        seq_lens[i] = (int32_t)s.tokens;
+        if (s.tokens > longest) longest = s.tokens;
     }
     *n_cow = ncow;
+    *max_seq_len = (int)longest;
     return PA_OK;
 }
 

@@ -66,6 +66,126 @@ int h2d(void *dst, const void *src, size_t bytes, cudaStream_t s) {
     return cudaMemcpyAsync(dst, src, bytes, cudaMemcpyHostToDevice, s) == cudaSuccess ? PA_OK : PA_ERR_CUDA;
 }
 
+// ---------------------------------------------------------------------------
+// Upload of a step's inputs by the SMs.  A copy engine pays a fixed latency of
+// several microseconds per copy and moves the step's sub-megabyte inputs far
+// below the link rate; SM loads from page-locked host memory (through its
+// device mapping), four 16-byte loads in flight per thread, fill the link with
+// one launch for all of them.
+// ---------------------------------------------------------------------------
+constexpr int kMaxSegs = 6;
+constexpr int kUploadThreads = 256;
+constexpr int kUploadInFlight = 4;
+
+struct UploadSeg {
+    const uint4 *src;          // device address of page-locked host memory, 16-byte aligned
+    uint4 *dst;                // device memory, 16-byte aligned
+    unsigned long long n16;    // whole 16-byte units
+    unsigned long long tail;   // bytes after them (< 16)
+};
+
+struct UploadArgs {
+    UploadSeg seg[kMaxSegs];
+    int n;
+};
+
+__global__ void __launch_bounds__(kUploadThreads) upload_kernel(const __grid_constant__ UploadArgs a) {
+    // end[i]: units of segments 0..i together
+    unsigned long long end[kMaxSegs];
+    unsigned long long total = 0;
+#pragma unroll
+    for (int i = 0; i < kMaxSegs; ++i) {
+        total += i < a.n ? a.seg[i].n16 : 0ull;
+        end[i] = total;
+    }
+    const unsigned long long stride = (unsigned long long)gridDim.x * blockDim.x;
+    for (unsigned long long x0 = (unsigned long long)blockIdx.x * blockDim.x + threadIdx.x; x0 < total;
+         x0 += kUploadInFlight * stride) {
+        uint4 v[kUploadInFlight];
+        uint4 *d[kUploadInFlight];
+#pragma unroll
+        for (int j = 0; j < kUploadInFlight; ++j) {
+            const unsigned long long x = x0 + j * stride;
+            d[j] = nullptr;
+            if (x < total) {
+                const uint4 *src = a.seg[0].src;
+                uint4 *dst = a.seg[0].dst;
+                unsigned long long base = 0;
+#pragma unroll
+                for (int i = 1; i < kMaxSegs; ++i)
+                    if (i < a.n && x >= end[i - 1]) {
+                        src = a.seg[i].src;
+                        dst = a.seg[i].dst;
+                        base = end[i - 1];
+                    }
+                v[j] = src[x - base];
+                d[j] = dst + (x - base);
+            }
+        }
+#pragma unroll
+        for (int j = 0; j < kUploadInFlight; ++j)
+            if (d[j]) *d[j] = v[j];
+    }
+    if (blockIdx.x == 0) {
+#pragma unroll
+        for (int i = 0; i < kMaxSegs; ++i)
+            if (i < a.n && threadIdx.x == (unsigned)i && a.seg[i].tail) {
+                const unsigned char *s8 = reinterpret_cast<const unsigned char *>(a.seg[i].src + a.seg[i].n16);
+                unsigned char *d8 = reinterpret_cast<unsigned char *>(a.seg[i].dst + a.seg[i].n16);
+                for (unsigned long long k = 0; k < a.seg[i].tail; ++k) d8[k] = s8[k];
+            }
+    }
+}
+
+// A host buffer as the device sees it: `mapped` is its device address when it is
+// page-locked and 16-byte aligned (the upload kernel reads it), else null (it
+// is copied with cudaMemcpyAsync).
+struct HostSrc {
+    const char *host = nullptr;
+    const char *mapped = nullptr;
+};
+
+HostSrc host_src(const void *p) {
+    HostSrc h;
+    h.host = static_cast<const char *>(p);
+    void *m = nullptr;
+    if (p && device_address(p, &m) == PA_OK && aligned16(m)) h.mapped = static_cast<const char *>(m);
+    return h;
+}
+
+// Collects the segments of one upload; copies what the kernel cannot read at once.
+struct Upload {
+    UploadArgs args{};
+
+    int add(void *dst, const HostSrc &src, size_t offset, size_t bytes, cudaStream_t s) {
+        if (bytes == 0) return PA_OK;
+        if (!src.mapped || !aligned16(static_cast<char *>(dst)) || !aligned16(src.mapped + offset) ||
+            args.n == kMaxSegs)
+            return h2d(dst, src.host + offset, bytes, s);
+        UploadSeg &g = args.seg[args.n++];
+        g.src = reinterpret_cast<const uint4 *>(src.mapped + offset);
+        g.dst = static_cast<uint4 *>(dst);
+        g.n16 = bytes / 16;
+        g.tail = bytes % 16;
+        return PA_OK;
+    }
+
+    int launch(cudaStream_t s) {
+        if (args.n == 0) return PA_OK;
+        unsigned long long units = 0;
+        for (int i = 0; i < args.n; ++i) units += args.seg[i].n16;
+        const unsigned long long per_cta = (unsigned long long)kUploadThreads * kUploadInFlight;
+        unsigned long long grid = (units + per_cta - 1) / per_cta;
+        const unsigned long long cap = 2ull * device_sm_count();
+        if (grid > cap) grid = cap;
+        if (grid == 0) grid = 1;  // tails only
+        upload_kernel<<<(unsigned)grid, kUploadThreads, 0, s>>>(args);
+        count_launch();
+        args.n = 0;
+        return launch_status();
+    }
+};
+
 int d2h(void *dst, const void *src, size_t bytes, cudaStream_t s) {
     if (bytes == 0) return PA_OK;
     return cudaMemcpyAsync(dst, src, bytes, cudaMemcpyDeviceToHost, s) == cudaSuccess ? PA_OK : PA_ERR_CUDA;
@@ -177,22 +297,24 @@ int pa_decode_step_host(float *out_host, const void *q_host, const void *k_new_h
                                num_kv_heads, head_dim, block_size, num_blocks, scale, pt, ws, ws_bytes, err_flag,
                                cs, false, 1.f, 1.f);
     };
-    // q, k_new and v_new of sequences [b0, b0 + nb)
-    auto upload_rows = [&](int b0, int nb, cudaStream_t cs) {
-        int rc = pa::h2d(st + l.q + b0 * q_row, static_cast<const char *>(q_host) + b0 * q_row, nb * q_row, cs);
-        if (rc == PA_OK)
-            rc = pa::h2d(st + l.k_new + b0 * kv_row, static_cast<const char *>(k_new_host) + b0 * kv_row,
-                         nb * kv_row, cs);
-        if (rc == PA_OK)
-            rc = pa::h2d(st + l.v_new + b0 * kv_row, static_cast<const char *>(v_new_host) + b0 * kv_row,
-                         nb * kv_row, cs);
-        return rc;
-    };
-    // copy pairs, block tables and lengths of the whole batch
-    auto upload_meta = [&](cudaStream_t cs) {
-        int rc = pa::h2d(st + l.pairs, copy_pairs_host, (size_t)num_pairs * 8, cs);
-        if (rc == PA_OK) rc = pa::h2d(st + l.tables, block_tables_host, batch * tab_row, cs);
-        if (rc == PA_OK) rc = pa::h2d(st + l.lens, seq_lens_host, (size_t)batch * 4, cs);
+    // Host inputs as the device sees them (resolved once per call).
+    const pa::HostSrc hq = pa::host_src(q_host), hk = pa::host_src(k_new_host), hv = pa::host_src(v_new_host);
+    const pa::HostSrc ht = pa::host_src(block_tables_host), hl = pa::host_src(seq_lens_host);
+    const pa::HostSrc hp = pa::host_src(num_pairs ? copy_pairs_host : nullptr);
+    // q, k_new and v_new of sequences [b0, b0 + nb); with `meta`, also the copy
+    // pairs, block tables and lengths of the whole batch.  One kernel launch.
+    auto upload = [&](int b0, int nb, bool meta, cudaStream_t cs) {
+        pa::Upload up;
+        int rc = PA_OK;
+        if (meta) {
+            rc = up.add(st + l.pairs, hp, 0, (size_t)num_pairs * 8, cs);
+            if (rc == PA_OK) rc = up.add(st + l.tables, ht, 0, batch * tab_row, cs);
+            if (rc == PA_OK) rc = up.add(st + l.lens, hl, 0, (size_t)batch * 4, cs);
+        }
+        if (rc == PA_OK) rc = up.add(st + l.q + b0 * q_row, hq, b0 * q_row, nb * q_row, cs);
+        if (rc == PA_OK) rc = up.add(st + l.k_new + b0 * kv_row, hk, b0 * kv_row, nb * kv_row, cs);
+        if (rc == PA_OK) rc = up.add(st + l.v_new + b0 * kv_row, hv, b0 * kv_row, nb * kv_row, cs);
+        if (rc == PA_OK) rc = up.launch(cs);
         return rc;
     };
     auto copy_pairs = [&](cudaStream_t cs) {
@@ -202,8 +324,7 @@ int pa_decode_step_host(float *out_host, const void *q_host, const void *k_new_h
     };
 
     if (chunks <= 1) {
-        int rc = upload_meta(s);
-        if (rc == PA_OK) rc = upload_rows(0, batch, s);
+        int rc = upload(0, batch, true, s);
         if (rc == PA_OK) rc = copy_pairs(s);
         if (rc == PA_OK)
             rc = decode_rows(0, batch, l.workspace_bytes ? st + l.workspace : nullptr, l.workspace_bytes, s);
@@ -224,9 +345,10 @@ int pa_decode_step_host(float *out_host, const void *q_host, const void *k_new_h
         if (cudaStreamWaitEvent(side, p.start, 0) != cudaSuccess) return PA_ERR_CUDA;
 
     // Block copies first, on the caller's stream; every chunk's decode comes after them.
-    int rc = upload_meta(p.up);
-    if (rc == PA_OK && num_pairs > 0) {
-        rc = pa::after(s, p.up, p.copied);
+    int rc = PA_OK;
+    if (num_pairs > 0) {
+        rc = upload(0, 0, true, p.up);
+        if (rc == PA_OK) rc = pa::after(s, p.up, p.copied);
         if (rc == PA_OK) rc = copy_pairs(s);
         if (rc == PA_OK) rc = pa::after(p.comp, s, p.copied);
     }
@@ -245,7 +367,7 @@ int pa_decode_step_host(float *out_host, const void *q_host, const void *k_new_h
         const int nb = (c + 1 < chunks ? chunk_start(c + 1) : batch) - b0;
         if (nb == 0) continue;
         cudaStream_t cs = (c & 1) ? p.comp : s;
-        rc = upload_rows(b0, nb, p.up);
+        rc = upload(b0, nb, c == 0 && num_pairs == 0, p.up);
         if (rc == PA_OK) rc = pa::after(cs, p.up, p.in[c]);
         size_t ws_bytes = 0;
         if (rc == PA_OK && ws) {

@@ -215,3 +215,84 @@ def test_replays_generator_placement():
     for b, L in enumerate(case.seq_lens):
         n = -(-int(L) // case.block_size)
         assert np.array_equal(t[b, :n], case.block_tables[b, :n])
+
+
+def _twin_allocators(seed):
+    """Two allocators in the same state: sequences with random lengths, some forked (shared blocks)."""
+    rng = np.random.default_rng(seed)
+    twins = [pa.Allocator(600, 16), pa.Allocator(600, 16)]
+    ids = []
+    for a in twins:
+        r = np.random.default_rng(seed)
+        got = []
+        for _ in range(6):
+            s = a.create()
+            for _ in range(int(r.integers(0, 70))):
+                a.append(s)
+            got.append(s)
+            if r.random() < 0.5:
+                got.append(a.fork(s))
+        ids.append(np.array(got, np.int32))
+    assert np.array_equal(ids[0], ids[1])
+    return twins, ids[0], rng
+
+
+@pytest.mark.parametrize("seed", [0, 1, 2])
+def test_alloc_step_equals_append_batch_then_export(seed):
+    """pa_alloc_step == pa_seq_append_batch followed by pa_alloc_export, step after step, forks and
+    copies on write included."""
+    (a, b), ids, _ = _twin_allocators(seed)
+    n, max_blocks = ids.size, 12
+    tables = np.zeros((n, max_blocks), np.int32)
+    lens = np.zeros(n, np.int32)
+    pairs = np.zeros((n, 2), np.int32)
+    step = a.step_fn(ids, tables, lens, pairs)
+    saw_copy = False
+    for _ in range(40):
+        n_cow, max_len = step()
+        _, want_pairs = b.append_batch(ids)
+        want_t, want_l = b.export(ids, max_blocks)
+        assert np.array_equal(tables, want_t) and np.array_equal(lens, want_l)
+        assert n_cow == want_pairs.shape[0] and np.array_equal(pairs[:n_cow], want_pairs)
+        assert max_len == int(want_l.max())
+        assert a.num_free() == b.num_free()
+        saw_copy |= n_cow > 0
+    assert saw_copy  # the forks made some appends copy
+    a.close(), b.close()
+
+
+def test_alloc_step_all_or_nothing():
+    """A table that would outgrow max_blocks, or a pool that runs dry, leaves the allocator as it was."""
+    a = pa.Allocator(5, 16)
+    s1, s2 = a.create(), a.create()
+    for _ in range(32):
+        a.append(s1)                        # 2 full blocks: the next append needs a third
+    a.append(s2)
+    ids = np.array([s2, s1], np.int32)
+    tables = np.zeros((2, 2), np.int32)
+    lens = np.zeros(2, np.int32)
+    pairs = np.zeros((2, 2), np.int32)
+    before = (a.num_free(), a.block_table(s1), a.block_table(s2))
+    with pytest.raises(RuntimeError, match="PA_ERR_INVALID_ARG"):
+        a.step_fn(ids, tables, lens, pairs)()
+    after = (a.num_free(), a.block_table(s1), a.block_table(s2))
+    assert before[0] == after[0] and all(np.array_equal(x[0], y[0]) and x[1] == y[1]
+                                         for x, y in zip(before[1:], after[1:]))
+    # pool of 5: s1 holds 2, s2 holds 1; a fork of s1 then 3 appends each need fresh blocks
+    c = a.fork(s1)
+    ids = np.array([s1, c, s2], np.int32)
+    tables = np.zeros((3, 8), np.int32)
+    lens = np.zeros(3, np.int32)
+    pairs = np.zeros((3, 2), np.int32)
+    step = a.step_fn(ids, tables, lens, pairs)
+    step()                                  # s1 -> new block 3, c -> new block 4: pool empty
+    free = a.num_free()
+    assert free == 0
+    snap = [a.block_table(x) for x in (s1, c, s2)]
+    for _ in range(14):
+        step()                              # s2 fills its block (16 tokens); s1, c write in place
+    with pytest.raises(RuntimeError, match="PA_ERR_OOM"):
+        step()                              # s1 and c append in place, then s2 needs a block: none left
+    assert a.num_free() == 0
+    assert [a.block_table(x)[1] for x in (s1, c, s2)] == [snap[0][1] + 14, snap[1][1] + 14, snap[2][1] + 14]
+    a.close()

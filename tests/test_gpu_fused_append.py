@@ -62,22 +62,26 @@ def test_full_size_llama2_7b_sampled_rows():
     assert_close(got[rows[:, 0], rows[:, 1]], want, "cfg2 full fused")
 
 
-@pytest.mark.parametrize("cfg,kw,chunks,pinned_out", [
-    (2, dict(batch=6, max_len=300, num_blocks=256), 1, True),
-    (2, dict(batch=6, max_len=300, num_blocks=256), 8, True),        # one sequence per chunk (8 clamps to 6)
-    (2, dict(batch=64, max_len=300, num_blocks=2048), 0, True),      # auto: ~2.6 MB over the link -> 2 chunks
-    (2, dict(batch=67, max_len=300, num_blocks=2048), 5, True),      # ragged chunk sizes
-    (2, dict(batch=67, max_len=300, num_blocks=2048), 5, False),     # pageable output: staged + copied back
-    (4, dict(batch=9, max_len=1500, num_blocks=512), 1, True),
-    (4, dict(batch=9, max_len=1500, num_blocks=512), 1, False),
-    (4, dict(batch=9, max_len=1500, num_blocks=512), 4, True),       # split decode: a workspace slice per chunk
-    (5, dict(batch=2, max_len=2048, num_blocks=640, num_copy_pairs=40), 1, True),
-    (5, dict(batch=3, max_len=2048, num_blocks=960, num_copy_pairs=40), 3, True),  # copies before every chunk
+@pytest.mark.parametrize("cfg,kw,chunks,pinned_out,inputs", [
+    (2, dict(batch=6, max_len=300, num_blocks=256), 1, True, "pinned"),
+    (2, dict(batch=6, max_len=300, num_blocks=256), 8, True, "pinned"),      # one sequence per chunk
+    (2, dict(batch=64, max_len=300, num_blocks=2048), 0, True, "pinned"),    # auto: ~2.6 MB over the link
+    (2, dict(batch=67, max_len=300, num_blocks=2048), 5, True, "pinned"),    # ragged chunk sizes
+    (2, dict(batch=67, max_len=300, num_blocks=2048), 5, False, "pinned"),   # pageable output: staged
+    (2, dict(batch=67, max_len=300, num_blocks=2048), 5, True, "pageable"),  # inputs copied, not read
+    (4, dict(batch=9, max_len=1500, num_blocks=512), 1, True, "pinned"),
+    (4, dict(batch=9, max_len=1500, num_blocks=512), 1, False, "misaligned"),  # 8-byte aligned inputs
+    (4, dict(batch=9, max_len=1500, num_blocks=512), 4, True, "pinned"),     # split: a workspace slice per chunk
+    (5, dict(batch=2, max_len=2048, num_blocks=640, num_copy_pairs=40), 1, True, "pinned"),
+    (5, dict(batch=3, max_len=2048, num_blocks=960, num_copy_pairs=40), 3, True, "pinned"),  # copies first
+    (5, dict(batch=3, max_len=2048, num_blocks=960, num_copy_pairs=40), 3, True, "misaligned"),
 ])
-def test_host_step_matches_device_path(cfg, kw, chunks, pinned_out):
+def test_host_step_matches_device_path(cfg, kw, chunks, pinned_out, inputs):
     """pa_decode_step_host (uploads, copies, fused decode, output to the host) == the device-resident
-    path, bit for bit, whether or not the step is cut into pipelined chunks and whether the output
-    buffer is page-locked (written by the kernels) or pageable (staged and copied back)."""
+    path, bit for bit, whether or not the step is cut into pipelined chunks, whether the output buffer
+    is page-locked (written by the kernels) or pageable (staged and copied back), and whether the
+    inputs are read by the upload kernel (page-locked, 16-byte aligned) or copied (pageable, or only
+    8-byte aligned)."""
     import torch
     import paged_kv_cache_349_b200 as pa
     case = W.make_case(cfg, **kw)
@@ -89,16 +93,26 @@ def test_host_step_matches_device_path(cfg, kw, chunks, pinned_out):
 
     def pinned(a, dtype):
         t = torch.from_numpy(np.ascontiguousarray(a))
-        return (t.view(dtype) if dtype is torch.bfloat16 else t.to(dtype)).pin_memory()
+        t = t.view(dtype) if dtype is torch.bfloat16 else t.to(dtype)
+        if inputs == "pageable":
+            return t
+        if inputs == "misaligned":      # a contiguous view 8 bytes into a page-locked buffer
+            esz = t.element_size()
+            buf = torch.empty(t.numel() + 8 // esz, dtype=dtype).pin_memory()
+            v = buf[8 // esz:].view(t.shape)
+            v.copy_(t)
+            assert v.data_ptr() % 16 == 8
+            return v
+        return t.pin_memory()
 
     out_h = torch.full(case.q.shape, float("nan"), dtype=torch.float32)
     if pinned_out:
         out_h = out_h.pin_memory()
     pairs = case.copy_pairs.reshape(-1, 2)
     max_pairs = max(1, pairs.shape[0])
-    pairs_h = torch.zeros((max_pairs, 2), dtype=torch.int32)
-    pairs_h[:pairs.shape[0]] = torch.from_numpy(pairs)
-    pairs_h = pairs_h.pin_memory()
+    pairs_np = np.zeros((max_pairs, 2), np.int32)
+    pairs_np[:pairs.shape[0]] = pairs
+    pairs_h = pinned(pairs_np, torch.int32)
     size = pa.pa_decode_step_staging_size(case.batch, case.max_blocks_per_seq, max_pairs, case.num_q_heads,
                                           case.num_kv_heads, case.head_dim, case.block_size, case.max_seq_len,
                                           case.partition_tokens)
