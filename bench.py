@@ -67,20 +67,21 @@ def _measured_peak():
         return FALLBACK_HBM_GBS, "fallback"
 
 
-def _decode_traffic_record():
-    """ncu DRAM traffic of the decode kernel for this workload, if taken on the current source."""
+def _decode_traffic_record(cfg: int, kv_dtype: str):
+    """ncu DRAM traffic of the decode kernel for this workload and KV dtype, if taken on the current source."""
     path = os.path.join(ROOT, "profiles", "decode_traffic.json")
     try:
         with open(path) as f:
-            rec = json.load(f)
+            recs = json.load(f)["records"]
     except Exception:
         return None
     src = os.path.join(ROOT, "paged_kv_cache_349_b200", "csrc", "decode.cu")
     with open(src, "rb") as f:
         digest = hashlib.sha256(f.read()).hexdigest()
-    if rec.get("decode_cu_sha256") != digest:
-        return None
-    return rec
+    for rec in recs:
+        if rec.get("decode_cu_sha256") == digest and rec.get("config") == cfg and rec.get("kv_dtype") == kv_dtype:
+            return rec
+    return None
 
 
 def step_bytes(case, kv_elem_bytes: int = 2):
@@ -374,10 +375,8 @@ def run_native(args):
 
     e2e = run_e2e(args, case, pa, stream, world, k, v) if not (args.no_e2e or args.unfused or fp8) else None
 
-    traffic = None
-    rec = _decode_traffic_record()
-    if rec and rec.get("config") == cfg:
-        traffic = rec.get("traffic_bytes_per_launch")
+    rec = _decode_traffic_record(cfg, "fp8" if fp8 else "bf16")
+    traffic = rec.get("traffic_bytes_per_launch") if rec else None
 
     line = {
         "metric": METRIC,
