@@ -41,10 +41,6 @@ namespace {
 #define PA_DECODE_PRODUCER_LANES 8
 #endif
 // fp8 tiles: 1 = expand E4M3 with integer bit moves (value * 2^-8), 0 = hardware cvt.
-#ifndef PA_FP8_BIT_EXPAND
-#define PA_FP8_BIT_EXPAND 0
-#endif
-
 constexpr int kTileTokens = 16;
 constexpr int kConsumerWarps = PA_DECODE_CONSUMER_WARPS;
 constexpr int kThreads = (kConsumerWarps + 1) * 32;
@@ -131,15 +127,10 @@ __device__ __forceinline__ uint32_t fp8_tile_offset(int r, int byte) {
 
 // Eight E4M3 codes -> four f16x2 words (codes 0,1 | 2,3 | 4,5 | 6,7).
 __device__ __forceinline__ uint4 e4m3x8_to_f16x8(uint32_t lo, uint32_t hi) {
-#if PA_FP8_BIT_EXPAND
-    return make_uint4(e4m3x2_to_f16x2_scaled<0x1404u>(lo), e4m3x2_to_f16x2_scaled<0x3424u>(lo),
-                      e4m3x2_to_f16x2_scaled<0x1404u>(hi), e4m3x2_to_f16x2_scaled<0x3424u>(hi));
-#else
     uint4 r;
     e4m3x4_to_f16x4(lo, r.x, r.y);
     e4m3x4_to_f16x4(hi, r.z, r.w);
     return r;
-#endif
 }
 
 template <bool FP8>
@@ -343,9 +334,6 @@ __global__ void __launch_bounds__(kThreads, FP8 ? PA_DECODE_MIN_CTAS_FP8 : PA_DE
                 qf[k][1] = pack_f16x2(bf16_lo_to_float(qf[k][1]) * up, bf16_hi_to_float(qf[k][1]) * up);
             }
             s_scale = p.scale_log2 * p.k_scale * down;
-#if PA_FP8_BIT_EXPAND
-            s_scale *= 256.f;  // the expanded K tile holds E4M3_value * 2^-8
-#endif
         }
         // Token row of mma row gid (gid+8 -> +8): this order keeps both the K
         // fragment loads and the V ldmatrix reads free of bank conflicts.
@@ -650,11 +638,7 @@ __global__ void __launch_bounds__(kThreads, FP8 ? PA_DECODE_MIN_CTAS_FP8 : PA_DE
             }
         }
         const int64_t row = (int64_t)b * p.num_q_heads + (int64_t)h * G + n;
-#if PA_FP8_BIT_EXPAND
-        if (FP8) num *= p.v_scale * 256.f;  // the expanded V tile holds E4M3_value * 2^-8
-#else
         if (FP8) num *= p.v_scale;
-#endif
         if (SPLIT) {
             p.part_o[(row * p.num_parts + part) * HEAD_DIM + d] = num / den;
             if (d == 0) {

@@ -230,18 +230,6 @@ __device__ __forceinline__ uint32_t e4m3x2_to_f16x2(uint32_t two_codes) {
     return f01;
 }
 
-// Codes in bytes `sel` of w -> f16x2 whose values are exactly E4M3_value * 2^-8.
-// The E4M3 exponent and mantissa (7 bits) drop into the low bits of the f16
-// exponent and the top of its mantissa; the exponent bias difference (15 - 7)
-// is the 2^-8, and E4M3 subnormals land on f16 subnormals with the same factor.
-// NaN codes are not handled (the library never writes them).  Byte selectors:
-// 0x1404 = codes 0,1; 0x3424 = codes 2,3.
-template <unsigned SEL>
-__device__ __forceinline__ uint32_t e4m3x2_to_f16x2_scaled(uint32_t w) {
-    const uint32_t t = __byte_perm(w, 0u, SEL);  // [0, c_lo, 0, c_hi]: each code in the top byte of a half
-    return (t & 0x80008000u) | ((t >> 1) & 0x3F803F80u);
-}
-
 // Eight bf16 values -> eight E4M3 codes: code = E4M3(x * inv_scale), the product
 // in fp32, rounded to nearest even and saturated to the largest finite value.
 __device__ __forceinline__ uint2 bf16x8_to_e4m3x8(uint4 v, float inv_scale) {
