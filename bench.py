@@ -68,20 +68,27 @@ def _measured_peak():
 
 
 def _decode_traffic_record(cfg: int, kv_dtype: str):
-    """ncu DRAM traffic of the decode kernel for this workload and KV dtype, if taken on the current source."""
+    """ncu DRAM traffic of the decode call for this workload and KV dtype, if taken on the current device code."""
     path = os.path.join(ROOT, "profiles", "decode_traffic.json")
     try:
         with open(path) as f:
             recs = json.load(f)["records"]
     except Exception:
         return None
-    src = os.path.join(ROOT, "paged_kv_cache_349_b200", "csrc", "decode.cu")
-    with open(src, "rb") as f:
-        digest = hashlib.sha256(f.read()).hexdigest()
+    digest = kernel_src_sha256()
     for rec in recs:
-        if rec.get("decode_cu_sha256") == digest and rec.get("config") == cfg and rec.get("kv_dtype") == kv_dtype:
+        if rec.get("kernel_src_sha256") == digest and rec.get("config") == cfg and rec.get("kv_dtype") == kv_dtype:
             return rec
     return None
+
+
+def kernel_src_sha256() -> str:
+    """Hash of the decode's device sources (kernel header + device helpers), in that order."""
+    h = hashlib.sha256()
+    for name in ("decode_kernels.cuh", "pa_common.cuh"):
+        with open(os.path.join(ROOT, "paged_kv_cache_349_b200", "csrc", name), "rb") as f:
+            h.update(f.read())
+    return h.hexdigest()
 
 
 def step_bytes(case, kv_elem_bytes: int = 2):

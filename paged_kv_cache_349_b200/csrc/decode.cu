@@ -1,726 +1,12 @@
-// Paged decode attention for sm_100a.
-//
-// What it computes ("Walk through paged attention end to end", attention
-// step): for each sequence b and query head g, softmax(scale * q K^T) V over
-// the sequence's L tokens, where token p lives in block
-// block_tables[b][p / bs] at row p % bs of the pool ("What is PagedAttention
-// and how does it manage KV cache", How PagedAttention works: two-level
-// indirection, tokens contiguous inside a block).
-//
-// How it runs on B200:
-//  * One CTA per (kv head h, sequence b[, sequence partition]) serves all G
-//    query heads of the group, so each K/V byte leaves HBM once.
-//  * The sequence is cut into 16-token tiles.  A producer warp dereferences
-//    the block table and stages each tile's K and V (16 rows x head_dim
-//    bf16, contiguous in the pool) into shared memory with TMA tile loads
-//    (128-byte swizzle, no multicast) through an 8-deep mbarrier ring.
-//  * Four consumer warps take tiles round-robin.  Per tile a warp computes
-//    S^T = K_tile Q^T with bf16 mma.sync (M = 16 tokens, N = 8 query-head
-//    columns, K = head_dim), runs an online softmax in fp32 (log2 domain),
-//    and accumulates O^T += V_tile^T P^T with a second mma (M = 16 dims,
-//    N = 8 heads, K = 16 tokens).  P is split into bf16 hi + lo parts so the
-//    PV product keeps ~16 mantissa bits.
-//  * Warps merge their (max, sum, O) states through shared memory.  In the
-//    split variant each CTA writes its partition's state to the workspace
-//    and a log-sum-exp reduce kernel combines the partitions.
+// Host side of the paged decode: tensor maps of the pools, the choice of
+// partitioning, the launches of the decode and reduce kernels (the device
+// code is in decode_kernels.cuh) and the C entry points.
 #include <mutex>
 
-#include "pa_common.cuh"
+#include "decode_kernels.cuh"
 
 namespace pa {
 namespace {
-
-// Compile-time shape of the decode CTA (overridable for tuning builds).
-#ifndef PA_DECODE_CONSUMER_WARPS
-#define PA_DECODE_CONSUMER_WARPS 4
-#endif
-#ifndef PA_DECODE_STAGES
-#define PA_DECODE_STAGES 8
-#endif
-#ifndef PA_DECODE_PRODUCER_LANES
-#define PA_DECODE_PRODUCER_LANES 8
-#endif
-// fp8 tiles: 1 = expand E4M3 with integer bit moves (value * 2^-8), 0 = hardware cvt.
-constexpr int kTileTokens = 16;
-constexpr int kConsumerWarps = PA_DECODE_CONSUMER_WARPS;
-constexpr int kThreads = (kConsumerWarps + 1) * 32;
-constexpr int kStages = PA_DECODE_STAGES;
-// Producer lanes issue tiles round-robin; lane k owns ring slots k, k+P, ...
-constexpr int kProducerLanes = PA_DECODE_PRODUCER_LANES;
-static_assert(kStages % kProducerLanes == 0, "each producer lane owns whole ring slots");
-static_assert(kProducerLanes >= 1 && kProducerLanes <= 8, "window indexing assumes <= 8 lanes");
-// A 16-bit tile (bf16, or f16 expanded from fp8) is stored as HEAD_DIM/64
-// boxes of 16 rows x 128 bytes with the TMA 128-byte swizzle.
-constexpr int kBox16Bytes = kTileTokens * 128;
-constexpr float kLog2e = 1.4426950408889634f;
-
-template <int HEAD_DIM, bool FP8>
-struct Cfg {
-    // What TMA lands in the ring: bf16 tiles in 64-column swizzled boxes, or
-    // fp8 tiles as one unswizzled box of 16 rows x HEAD_DIM bytes.
-    static constexpr int kBoxes = FP8 ? 1 : HEAD_DIM / 64;
-    static constexpr int kBoxCols = FP8 ? HEAD_DIM : 64;
-    static constexpr int kBoxRowBytes = FP8 ? HEAD_DIM : 128;
-    static constexpr int kBoxBytes = kTileTokens * kBoxRowBytes;
-    static constexpr int kTileBytes = kBoxes * kBoxBytes;  // K or V of one tile
-    static constexpr int kStageBytes = 2 * kTileBytes;
-    static constexpr int kRingBytes = kStages * kStageBytes;
-    // fp8, head_dim 128: the ring tile carries the 128-byte swizzle; K fragments
-    // are built straight from it and only V is expanded to a 16-bit tile.
-    // fp8, head_dim 64: the ring tile is unswizzled and both K and V are expanded.
-    static constexpr bool kDirectK = FP8 && HEAD_DIM == 128;
-    static constexpr int kTile16Bytes = (HEAD_DIM / 64) * kBox16Bytes;
-    static constexpr int kStagingBytes = FP8 ? kConsumerWarps * (kDirectK ? 1 : 2) * kTile16Bytes : 0;
-    static constexpr int kDataBytes = kRingBytes + kStagingBytes;
-    static constexpr int kMergeStride = HEAD_DIM + 4;  // padded row: conflict-free merge stores
-    static constexpr int kMergeBytes = kConsumerWarps * 8 * (kMergeStride + 2) * 4;
-    static_assert(kMergeBytes <= kDataBytes, "merge area reuses the ring");
-    // + barriers, tile flags, the fused write's row (32 x 16 bytes) and its block id
-    static constexpr int kSmemBytes =
-        1024 /*align slack*/ + kDataBytes + kStages * 8 * 2 + kStages * 4 + 32 * 16 + 16;
-};
-
-struct DecodeParams {
-    float *out;                 // [B, Hq, d]            (single pass)
-    float *part_o;              // [B, Hq, P, d]         (split)
-    float *part_ml;             // [B, Hq, P, 2]         (split)
-    const uint16_t *q;          // [B, Hq, d] bf16
-    const int32_t *block_tables;
-    const int32_t *seq_lens;
-    int32_t *err_flag;
-    const uint16_t *k_new;      // [B, Hkv, d] bf16 (fused cache write only)
-    const uint16_t *v_new;
-    uint16_t *k_pool;           // pools, written by the fused cache write
-    uint16_t *v_pool;
-    int64_t num_blocks;
-    int max_blocks;
-    int max_seq_len;
-    int num_q_heads;
-    int num_kv_heads;
-    int group;
-    int block_size;
-    int part_tokens;            // tokens per CTA along the sequence
-    int num_parts;
-    float scale_log2;           // softmax scale * log2(e)
-    float k_scale;              // fp8 pools: dequantisation multipliers
-    float v_scale;
-    float k_inv_scale;          // fp8 pools: 1 / scale, for the fused cache write
-    float v_inv_scale;
-};
-
-// Sequence length as every kernel of one call sees it: out-of-contract values
-// are clamped (and reported once by the caller of this helper).
-__device__ __forceinline__ int clamp_len(int L, const DecodeParams &p) {
-    const int cap = min(p.max_seq_len, p.max_blocks * p.block_size);
-    return L < 0 ? 0 : (L > cap ? cap : L);
-}
-
-// Byte offset of 16-byte chunk c of token row r inside one swizzled 16-bit tile.
-__device__ __forceinline__ uint32_t tile_offset(int r, int c) {
-    return (uint32_t)((c >> 3) * kBox16Bytes + r * 128 + (((c & 7) ^ (r & 7)) << 4));
-}
-
-// Byte offset of byte `byte` of row r in a 128-byte-swizzled fp8 tile (128-byte rows).
-__device__ __forceinline__ uint32_t fp8_tile_offset(int r, int byte) {
-    return (uint32_t)(r * 128 + ((((byte >> 4) ^ (r & 7))) << 4) + (byte & 15));
-}
-
-// Eight E4M3 codes -> four f16x2 words (codes 0,1 | 2,3 | 4,5 | 6,7).
-__device__ __forceinline__ uint4 e4m3x8_to_f16x8(uint32_t lo, uint32_t hi) {
-    uint4 r;
-    e4m3x4_to_f16x4(lo, r.x, r.y);
-    e4m3x4_to_f16x4(hi, r.z, r.w);
-    return r;
-}
-
-template <bool FP8>
-__device__ __forceinline__ void mma_16816(float (&d)[4], uint32_t a0, uint32_t a1, uint32_t a2, uint32_t a3,
-                                          uint32_t b0, uint32_t b1) {
-    if constexpr (FP8)
-        mma_f16_16816(d, a0, a1, a2, a3, b0, b1);
-    else
-        mma_bf16_16816(d, a0, a1, a2, a3, b0, b1);
-}
-
-// CTAs per SM the register allocation must allow (bf16 is limited to 3 by shared memory).
-#ifndef PA_DECODE_MIN_CTAS_FP8
-#define PA_DECODE_MIN_CTAS_FP8 3
-#endif
-#ifndef PA_DECODE_MIN_CTAS_BF16
-#define PA_DECODE_MIN_CTAS_BF16 3
-#endif
-
-template <int HEAD_DIM, bool SPLIT, bool APPEND, bool FP8>
-__global__ void __launch_bounds__(kThreads, FP8 ? PA_DECODE_MIN_CTAS_FP8 : PA_DECODE_MIN_CTAS_BF16) paged_decode_kernel(
-    const __grid_constant__ CUtensorMap k_map, const __grid_constant__ CUtensorMap v_map,
-    const DecodeParams p) {
-    using C = Cfg<HEAD_DIM, FP8>;
-    extern __shared__ uint8_t smem_raw[];
-    uint8_t *smem = reinterpret_cast<uint8_t *>(
-        (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~static_cast<uintptr_t>(1023));
-    uint64_t *full = reinterpret_cast<uint64_t *>(smem + C::kDataBytes);
-    uint64_t *empty = full + kStages;
-    int *tile_ok = reinterpret_cast<int *>(empty + kStages);
-    // Fused write: the new token's bf16 K/V row (16 bytes per lane) and its block id,
-    // fetched asynchronously so no registers are held until the tile is reached.
-    uint4 *append_row = reinterpret_cast<uint4 *>(tile_ok + kStages);
-    int *append_phys = reinterpret_cast<int *>(append_row + 32);
-
-    const int part = blockIdx.x;
-    const int h = blockIdx.y;
-    const int b = blockIdx.z;
-    const int warp = threadIdx.x >> 5;
-    const int lane = threadIdx.x & 31;
-
-    const int L_raw = __ldg(p.seq_lens + b);
-    const int L = clamp_len(L_raw, p);
-    const int tok_begin = part * p.part_tokens;
-    const int tok_end = min(L, tok_begin + p.part_tokens);
-    const int n_tiles = tok_end > tok_begin ? (tok_end - tok_begin + kTileTokens - 1) / kTileTokens : 0;
-    // Let the log-sum-exp reduce (launched as a programmatic dependent) get
-    // scheduled while this grid's last wave runs; it waits for our results.
-    if (SPLIT) asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
-    if (SPLIT && n_tiles == 0) return;  // empty partition: the reduce skips it
-    if (threadIdx.x == 0 && part == 0 && h == 0 && L != L_raw) raise_flag(p.err_flag, PA_FLAG_BAD_LEN);
-
-    if (threadIdx.x == 0) {
-        for (int s = 0; s < kStages; ++s) {
-            mbar_init(&full[s], 1);
-            mbar_init(&empty[s], 1);
-        }
-        fence_mbar_init();
-    }
-    __syncthreads();
-
-    // Per consumer thread: softmax state of query-head columns 2t, 2t+1.
-    const int gid = lane >> 2;  // mma group id
-    const int tig = lane & 3;   // thread in group
-    float m_run[2] = {-INFINITY, -INFINITY};
-    float l_run[2] = {0.f, 0.f};
-    float o[HEAD_DIM / 16][4];
-#pragma unroll
-    for (int mt = 0; mt < HEAD_DIM / 16; ++mt) o[mt][0] = o[mt][1] = o[mt][2] = o[mt][3] = 0.f;
-
-    if (warp == kConsumerWarps) {
-        // ---------------- producer: block-table dereference + TMA ----------------
-        // The whole warp walks the tiles so that block-table entries arrive 32 at a
-        // time (one coalesced load per window, the next window loaded ahead).
-        // kProducerLanes lanes wait on the ring and issue copies in parallel:
-        // lane k handles tiles k, k+P, k+2P, ... and therefore ring slots k, k+P, ...
-        const int32_t *table = p.block_tables + (int64_t)b * p.max_blocks;
-        const int j_end = (tok_end + p.block_size - 1) / p.block_size;  // blocks this CTA reads
-        int win = tok_begin / p.block_size;                             // first entry of the window
-        int32_t cur = win + lane < j_end ? __ldg(table + win + lane) : -1;
-        int32_t nxt = win + 32 + lane < j_end ? __ldg(table + win + 32 + lane) : -1;
-        uint64_t policy = 0;
-        if (lane < kProducerLanes) {
-            if (lane == 0) {
-                prefetch_tensormap(&k_map);
-                prefetch_tensormap(&v_map);
-            }
-            policy = l2_policy_evict_first();
-        }
-        int issued = 0;  // tiles issued by this lane's rounds (max over lanes below)
-        bool stop = false;
-        for (int i0 = 0; i0 < n_tiles; i0 += kProducerLanes) {
-            const int j0 = (tok_begin + i0 * kTileTokens) / p.block_size;
-            if (j0 >= win + 32) {  // warp-uniform: slide the window
-                win += 32;
-                cur = nxt;
-                nxt = win + 32 + lane < j_end ? __ldg(table + win + 32 + lane) : -1;
-            }
-            const int i = i0 + lane;
-            const bool mine = lane < kProducerLanes && i < n_tiles;
-            const int tok0 = tok_begin + i * kTileTokens;
-            const int j = mine ? tok0 / p.block_size : win;
-            const int row = tok0 - j * p.block_size;
-            // A tile is one slice of a block, or two whole 8-token blocks.
-            const int idx = j - win;  // in [0, 32 + 2 * kProducerLanes)
-            const int32_t a_cur = __shfl_sync(0xffffffffu, cur, idx & 31);
-            const int32_t a_nxt = __shfl_sync(0xffffffffu, nxt, idx & 31);
-            const int32_t b_cur = __shfl_sync(0xffffffffu, cur, (idx + 1) & 31);
-            const int32_t b_nxt = __shfl_sync(0xffffffffu, nxt, (idx + 1) & 31);
-            const int64_t phys = idx < 32 ? a_cur : a_nxt;
-            const int64_t phys2 = idx + 1 < 32 ? b_cur : b_nxt;
-            const bool two_blocks = p.block_size < kTileTokens;
-            const bool second = two_blocks && tok0 + p.block_size < tok_end;
-            if (mine) {
-                const int s = i % kStages;
-                if (i >= kStages && !mbar_wait_bounded(&empty[s], ((i / kStages) - 1) & 1, p.err_flag)) {
-                    stop = true;
-                } else {
-                    issued = i + 1;
-                    if (phys < 0 || phys >= p.num_blocks || (second && (phys2 < 0 || phys2 >= p.num_blocks))) {
-                        raise_flag(p.err_flag, PA_FLAG_BAD_BLOCK);
-                        tile_ok[s] = 0;
-                        mbar_arrive(&full[s]);
-                    } else {
-                        tile_ok[s] = 1;
-                        const int y = (int)((phys * p.num_kv_heads + h) * p.block_size + row);
-                        uint8_t *dst = smem + s * C::kStageBytes;
-                        mbar_arrive_expect_tx(&full[s], two_blocks && !second ? C::kStageBytes / 2 : C::kStageBytes);
-#pragma unroll
-                        for (int bx = 0; bx < C::kBoxes; ++bx)
-                            tma_load_2d(dst + bx * C::kBoxBytes, &k_map, bx * C::kBoxCols, y, &full[s], policy);
-#pragma unroll
-                        for (int bx = 0; bx < C::kBoxes; ++bx)
-                            tma_load_2d(dst + C::kTileBytes + bx * C::kBoxBytes, &v_map, bx * C::kBoxCols, y,
-                                        &full[s], policy);
-                        if (second) {  // rows 8..15 of the tile come from the next 8-token block
-                            const int y2 = (int)((phys2 * p.num_kv_heads + h) * p.block_size);
-#pragma unroll
-                            for (int bx = 0; bx < C::kBoxes; ++bx)
-                                tma_load_2d(dst + bx * C::kBoxBytes + C::kBoxBytes / 2, &k_map, bx * C::kBoxCols, y2,
-                                            &full[s], policy);
-#pragma unroll
-                            for (int bx = 0; bx < C::kBoxes; ++bx)
-                                tma_load_2d(dst + C::kTileBytes + bx * C::kBoxBytes + C::kBoxBytes / 2, &v_map,
-                                            bx * C::kBoxCols, y2, &full[s], policy);
-                        }
-                    }
-                }
-            }
-            if (__any_sync(0xffffffffu, stop)) break;
-        }
-        // Drain: every issued tile has landed before the ring is reused or the CTA exits.
-        // A tile is the last user of its slot when no tile kStages later was issued.
-        const int issued_all = __reduce_max_sync(0xffffffffu, issued);
-        if (lane < kProducerLanes) {
-            for (int i = lane; i < issued_all; i += kProducerLanes)
-                if (i + kStages >= issued_all && i < issued)
-                    if (!mbar_wait_bounded(&full[i % kStages], (i / kStages) & 1, p.err_flag)) break;
-        }
-    } else {
-        // ---------------- consumers ----------------
-        const int G = p.group;
-        // Q^T as mma B fragments (k = head dim, permuted; n = query head column gid).
-        uint32_t qf[HEAD_DIM / 16][2];
-        if (gid < G) {
-            const uint4 *qrow = reinterpret_cast<const uint4 *>(
-                p.q + ((int64_t)b * p.num_q_heads + (int64_t)h * G + gid) * HEAD_DIM);
-#pragma unroll
-            for (int j = 0; j < HEAD_DIM / 32; ++j) {
-                const uint4 v = __ldg(qrow + 4 * j + tig);
-                qf[2 * j][0] = v.x;
-                qf[2 * j][1] = v.y;
-                qf[2 * j + 1][0] = v.z;
-                qf[2 * j + 1][1] = v.w;
-            }
-        } else {
-#pragma unroll
-            for (int k = 0; k < HEAD_DIM / 16; ++k) qf[k][0] = qf[k][1] = 0u;
-        }
-        // fp8 pools run the mma in f16: q is scaled by a power of two 2^qexp so its
-        // largest entry lands just below 2^14 (exact, well inside the f16 range);
-        // 2^-qexp and the K dequantisation scale fold into the softmax scale.
-        float s_scale = p.scale_log2;
-        if constexpr (FP8) {
-            float amax = 0.f;
-#pragma unroll
-            for (int k = 0; k < HEAD_DIM / 16; ++k) {
-                amax = fmaxf(amax, fmaxf(fabsf(bf16_lo_to_float(qf[k][0])), fabsf(bf16_hi_to_float(qf[k][0]))));
-                amax = fmaxf(amax, fmaxf(fabsf(bf16_lo_to_float(qf[k][1])), fabsf(bf16_hi_to_float(qf[k][1]))));
-            }
-#pragma unroll
-            for (int off = 16; off; off >>= 1) amax = fmaxf(amax, __shfl_xor_sync(0xffffffffu, amax, off));
-            // amax in [2^e, 2^(e+1)) -> qexp = 13 - e; amax == 0 -> qexp = 0
-            const int e = amax > 0.f ? (int)((__float_as_uint(amax) >> 23) & 0xff) - 127 : 13;
-            const int qexp = max(-100, min(100, 13 - e));
-            const float up = __uint_as_float((uint32_t)(127 + qexp) << 23);
-            const float down = __uint_as_float((uint32_t)(127 - qexp) << 23);
-#pragma unroll
-            for (int k = 0; k < HEAD_DIM / 16; ++k) {
-                qf[k][0] = pack_f16x2(bf16_lo_to_float(qf[k][0]) * up, bf16_hi_to_float(qf[k][0]) * up);
-                qf[k][1] = pack_f16x2(bf16_lo_to_float(qf[k][1]) * up, bf16_hi_to_float(qf[k][1]) * up);
-            }
-            s_scale = p.scale_log2 * p.k_scale * down;
-        }
-        // Token row of mma row gid (gid+8 -> +8): this order keeps both the K
-        // fragment loads and the V ldmatrix reads free of bank conflicts.
-        // (fp8 with K read straight from the swizzled fp8 tile uses 0,2,4,6,1,3,5,7.)
-        auto token_of = [](int g) { return C::kDirectK ? ((g & 3) << 1) | (g >> 2) : (g >> 1) | ((g & 1) << 2); };
-        const int tau = token_of(gid);
-        // ldmatrix row address pattern for V: matrix (lane>>3), row (lane&7).
-        const int v_row = token_of(lane & 7) + (((lane >> 4) & 1) << 3);
-        const int v_chunk_hi = (lane >> 3) & 1;
-
-        // Fused cache write ("append, then attend"): the warp that owns the tile
-        // holding position L-1 fetches the new token's K row (lanes 0..15) and
-        // V row (lanes 16..31) up front, stores them to the pool, and patches
-        // them into its staged tile before computing.  The block receiving the
-        // token is owned by this sequence alone (copy-on-write), so no other
-        // CTA reads that row.
-        int i_new = -1;
-        if (APPEND && L == L_raw && L > 0 && L - 1 >= tok_begin && L - 1 < tok_end) {
-            const int it = (L - 1 - tok_begin) / kTileTokens;
-            if (it % kConsumerWarps == warp) {
-                i_new = it;
-                const int c = lane & 15;
-                if (c < HEAD_DIM / 8) {
-                    const uint16_t *src = (lane < 16 ? p.k_new : p.v_new) +
-                                          ((int64_t)b * p.num_kv_heads + h) * HEAD_DIM + c * 8;
-                    cp_async16(smem_addr(append_row + lane), src);
-                }
-                if (lane == 0)
-                    cp_async4(smem_addr(append_phys),
-                              p.block_tables + (int64_t)b * p.max_blocks + (L - 1) / p.block_size);
-                cp_async_commit();
-            }
-        }
-        // This lane's share of the fused write at the tile that holds L-1: returns the
-        // bf16 row chunk and the pool index of its 8 values (-1 if the block id is bad).
-        auto append_fetch = [&](uint4 &row) -> int64_t {
-            cp_async_wait_all();
-            __syncwarp();
-            const int64_t phys = *reinterpret_cast<volatile int *>(append_phys);
-            row = append_row[lane];
-            if (phys < 0 || phys >= p.num_blocks) return -1;
-            return ((phys * p.num_kv_heads + h) * p.block_size + (L - 1) % p.block_size) * (HEAD_DIM / 8) +
-                   (lane & 15);
-        };
-
-        for (int i = warp; i < n_tiles; i += kConsumerWarps) {
-            const int s = i % kStages;
-            const bool got = mbar_wait_bounded(&full[s], (i / kStages) & 1, p.err_flag);
-            if (!__all_sync(0xffffffffu, got)) break;
-            const int valid = min(kTileTokens, tok_end - (tok_begin + i * kTileTokens));
-            if (tile_ok[s]) {
-                uint32_t kbase = smem_addr(smem + s * C::kStageBytes);
-                uint32_t vbase = kbase + C::kTileBytes;
-                uint32_t ring_k = kbase;  // fp8 direct-K: K stays in the ring until QK is done
-                if constexpr (C::kDirectK) {
-                    // The fused cache write lands in the (swizzled) fp8 tile first, and in the pool.
-                    if (APPEND && i == i_new) {
-                        const int r = (L - 1 - tok_begin) - i_new * kTileTokens;
-                        const int c = lane & 15;  // 8-byte piece of the 128-byte row
-                        uint4 row;
-                        const int64_t dst = append_fetch(row);
-                        const uint2 q8 = bf16x8_to_e4m3x8(row, lane < 16 ? p.k_inv_scale : p.v_inv_scale);
-                        const uint32_t a = (lane < 16 ? kbase : vbase) + fp8_tile_offset(r, c * 8);
-                        asm volatile("st.shared.v2.u32 [%0], {%1, %2};" ::"r"(a), "r"(q8.x), "r"(q8.y) : "memory");
-                        if (dst >= 0) reinterpret_cast<uint2 *>(lane < 16 ? p.k_pool : p.v_pool)[dst] = q8;
-                        __syncwarp();
-                    }
-                    // Expand V into this warp's 16-bit tile.  Each group of 8 lanes takes rows
-                    // r and r^5 and four 16-byte chunks of one column box, so both the swizzled
-                    // fp8 reads and the swizzled 16-bit writes hit 8 distinct bank groups.
-                    const uint32_t stg_v = smem_addr(smem + C::kRingBytes + warp * C::kTile16Bytes);
-#pragma unroll
-                    for (int x = lane; x < kTileTokens * (HEAD_DIM / 16); x += 32) {
-                        const int grp = x >> 3, pair = grp >> 1, box = grp & 1;
-                        const int r0 = ((pair & 1) << 1) | (((pair >> 1) & 1) << 3) | (pair >> 2);
-                        const int r = (x & 4) ? (r0 ^ 5) : r0;
-                        const int c16 = box * 4 + (x & 3);
-                        const uint4 w = lds128(vbase + fp8_tile_offset(r, c16 * 16));
-                        const uint4 lo = e4m3x8_to_f16x8(w.x, w.y);
-                        const uint4 hi = e4m3x8_to_f16x8(w.z, w.w);
-                        asm volatile("st.shared.v4.u32 [%0], {%1, %2, %3, %4};" ::"r"(stg_v + tile_offset(r, 2 * c16)),
-                                     "r"(lo.x), "r"(lo.y), "r"(lo.z), "r"(lo.w)
-                                     : "memory");
-                        asm volatile("st.shared.v4.u32 [%0], {%1, %2, %3, %4};" ::"r"(stg_v + tile_offset(r, 2 * c16 + 1)),
-                                     "r"(hi.x), "r"(hi.y), "r"(hi.z), "r"(hi.w)
-                                     : "memory");
-                    }
-                    __syncwarp();
-                    vbase = stg_v;
-                } else if constexpr (FP8) {
-                    // head_dim 64: the fused write lands in the unswizzled fp8 tile first.
-                    if (APPEND && i == i_new) {
-                        const int r = (L - 1 - tok_begin) - i_new * kTileTokens;
-                        const int c = lane & 15;
-                        uint4 row;
-                        const int64_t dst = append_fetch(row);
-                        if (c < HEAD_DIM / 8) {
-                            const uint2 q8 = bf16x8_to_e4m3x8(row, lane < 16 ? p.k_inv_scale : p.v_inv_scale);
-                            const uint32_t a = (lane < 16 ? kbase : vbase) + r * HEAD_DIM + c * 8;
-                            asm volatile("st.shared.v2.u32 [%0], {%1, %2};" ::"r"(a), "r"(q8.x), "r"(q8.y)
-                                         : "memory");
-                            if (dst >= 0) reinterpret_cast<uint2 *>(lane < 16 ? p.k_pool : p.v_pool)[dst] = q8;
-                        }
-                        __syncwarp();
-                    }
-                    // Expand K and V into this warp's 16-bit tiles (E4M3 -> f16 is exact),
-                    // laid out like a TMA-swizzled bf16 tile so the code below is shared.
-                    const uint32_t stg_k = smem_addr(smem + C::kRingBytes + warp * 2 * C::kTile16Bytes);
-                    const uint32_t stg_v = stg_k + C::kTile16Bytes;
-                    constexpr int kChunksPerRow = HEAD_DIM / 16;  // 16 fp8 values per 16-byte chunk
-#pragma unroll
-                    for (int x = lane; x < kTileTokens * kChunksPerRow; x += 32) {
-                        const int r = x / kChunksPerRow;
-                        const int c16 = x - r * kChunksPerRow;
-#pragma unroll
-                        for (int kv = 0; kv < 2; ++kv) {
-                            const uint4 w = lds128((kv ? vbase : kbase) + x * 16);
-                            const uint32_t dst = kv ? stg_v : stg_k;
-                            const uint4 lo = e4m3x8_to_f16x8(w.x, w.y);
-                            const uint4 hi = e4m3x8_to_f16x8(w.z, w.w);
-                            asm volatile("st.shared.v4.u32 [%0], {%1, %2, %3, %4};" ::"r"(dst + tile_offset(r, 2 * c16)),
-                                         "r"(lo.x), "r"(lo.y), "r"(lo.z), "r"(lo.w)
-                                         : "memory");
-                            asm volatile("st.shared.v4.u32 [%0], {%1, %2, %3, %4};" ::"r"(dst + tile_offset(r, 2 * c16 + 1)),
-                                         "r"(hi.x), "r"(hi.y), "r"(hi.z), "r"(hi.w)
-                                         : "memory");
-                        }
-                    }
-                    if (APPEND && i == i_new) fence_proxy_async_smem();
-                    __syncwarp();
-                    if (lane == 0) mbar_arrive(&empty[s]);  // the ring slot is free again
-                    kbase = stg_k;
-                    vbase = stg_v;
-                }
-                if (valid < kTileTokens) {
-                    // Rows past the sequence end hold stale data: zero them so
-                    // that P = 0 times V cannot produce NaN.
-                    constexpr int kBoxes16 = HEAD_DIM / 64;  // boxes of the 16-bit tile
-                    const int lines = (kTileTokens - valid) * kBoxes16;
-                    for (int x = lane; x < lines * 8; x += 32) {
-                        const int line = x >> 3;
-                        const int r = valid + line / kBoxes16;
-                        const int bx = line % kBoxes16;
-                        const uint32_t a = vbase + bx * kBox16Bytes + r * 128 + ((x & 7) << 4);
-                        asm volatile("st.shared.v4.u32 [%0], {%1, %1, %1, %1};" ::"r"(a), "r"(0u)
-                                     : "memory");
-                    }
-                    __syncwarp();
-                }
-                if (APPEND && !FP8 && i == i_new) {
-                    const int r = (L - 1 - tok_begin) - i_new * kTileTokens;  // row of L-1 in this tile
-                    const int c = lane & 15;
-                    uint4 row;
-                    const int64_t dst = append_fetch(row);
-                    if (c < HEAD_DIM / 8) {
-                        const uint32_t a = (lane < 16 ? kbase : vbase) + tile_offset(r, c);
-                        asm volatile("st.shared.v4.u32 [%0], {%1, %2, %3, %4};" ::"r"(a), "r"(row.x), "r"(row.y),
-                                     "r"(row.z), "r"(row.w)
-                                     : "memory");
-                        if (dst >= 0) reinterpret_cast<uint4 *>(lane < 16 ? p.k_pool : p.v_pool)[dst] = row;
-                    }
-                    __syncwarp();
-                }
-                // ---- S^T = K Q^T ----
-                float sacc[4] = {0.f, 0.f, 0.f, 0.f};
-#pragma unroll
-                for (int j = 0; j < HEAD_DIM / 32; ++j) {
-                    uint4 ka, kb;
-                    if constexpr (C::kDirectK) {
-                        // 8 fp8 codes (dims 32j+8t .. +7) of rows tau and tau+8, expanded in registers
-                        uint32_t a0, a1, b0, b1;
-                        asm volatile("ld.shared.v2.u32 {%0, %1}, [%2];"
-                                     : "=r"(a0), "=r"(a1)
-                                     : "r"(ring_k + fp8_tile_offset(tau, 32 * j + 8 * tig)));
-                        asm volatile("ld.shared.v2.u32 {%0, %1}, [%2];"
-                                     : "=r"(b0), "=r"(b1)
-                                     : "r"(ring_k + fp8_tile_offset(tau + 8, 32 * j + 8 * tig)));
-                        ka = e4m3x8_to_f16x8(a0, a1);
-                        kb = e4m3x8_to_f16x8(b0, b1);
-                    } else {
-                        const int c = 4 * j + tig;
-                        ka = lds128(kbase + tile_offset(tau, c));
-                        kb = lds128(kbase + tile_offset(tau + 8, c));
-                    }
-                    mma_16816<FP8>(sacc, ka.x, kb.x, ka.y, kb.y, qf[2 * j][0], qf[2 * j][1]);
-                    mma_16816<FP8>(sacc, ka.z, kb.z, ka.w, kb.w, qf[2 * j + 1][0], qf[2 * j + 1][1]);
-                }
-                if constexpr (C::kDirectK) {
-                    // K and V have left the ring: hand the slot back to the producer.
-                    if (APPEND && i == i_new) fence_proxy_async_smem();
-                    __syncwarp();
-                    if (lane == 0) mbar_arrive(&empty[s]);
-                }
-                // sacc: (token tau, col 2t), (tau, 2t+1), (tau+8, 2t), (tau+8, 2t+1)
-                const float s0 = tau < valid ? sacc[0] * s_scale : -INFINITY;
-                const float s1 = tau < valid ? sacc[1] * s_scale : -INFINITY;
-                const float s2 = tau + 8 < valid ? sacc[2] * s_scale : -INFINITY;
-                const float s3 = tau + 8 < valid ? sacc[3] * s_scale : -INFINITY;
-                float mx0 = fmaxf(s0, s2), mx1 = fmaxf(s1, s3);
-#pragma unroll
-                for (int off = 4; off < 32; off <<= 1) {
-                    mx0 = fmaxf(mx0, __shfl_xor_sync(0xffffffffu, mx0, off));
-                    mx1 = fmaxf(mx1, __shfl_xor_sync(0xffffffffu, mx1, off));
-                }
-                const float mn0 = fmaxf(m_run[0], mx0), mn1 = fmaxf(m_run[1], mx1);
-                const float a0 = fast_exp2(m_run[0] - mn0), a1 = fast_exp2(m_run[1] - mn1);
-                m_run[0] = mn0;
-                m_run[1] = mn1;
-                const float p0 = fast_exp2(s0 - mn0), p1 = fast_exp2(s1 - mn1);
-                const float p2 = fast_exp2(s2 - mn0), p3 = fast_exp2(s3 - mn1);
-                l_run[0] = l_run[0] * a0 + (p0 + p2);
-                l_run[1] = l_run[1] * a1 + (p1 + p3);
-                if (__any_sync(0xffffffffu, a0 != 1.f || a1 != 1.f)) {
-#pragma unroll
-                    for (int mt = 0; mt < HEAD_DIM / 16; ++mt) {
-                        o[mt][0] *= a0;
-                        o[mt][1] *= a1;
-                        o[mt][2] *= a0;
-                        o[mt][3] *= a1;
-                    }
-                }
-                // ---- P^T as B fragments: hi + lo bf16 parts ----
-                uint32_t h01, h23, l01, l23;
-                if constexpr (FP8) {
-                    h01 = pack_f16x2(p0, p1);
-                    h23 = pack_f16x2(p2, p3);
-                    l01 = pack_f16x2(p0 - f16_lo_to_float(h01), p1 - f16_hi_to_float(h01));
-                    l23 = pack_f16x2(p2 - f16_lo_to_float(h23), p3 - f16_hi_to_float(h23));
-                } else {
-                    h01 = pack_bf16x2(p0, p1);
-                    h23 = pack_bf16x2(p2, p3);
-                    l01 = pack_bf16x2(p0 - bf16_lo_to_float(h01), p1 - bf16_hi_to_float(h01));
-                    l23 = pack_bf16x2(p2 - bf16_lo_to_float(h23), p3 - bf16_hi_to_float(h23));
-                }
-                const uint32_t bh0 = movmatrix_trans(h01), bh1 = movmatrix_trans(h23);
-                const uint32_t bl0 = movmatrix_trans(l01), bl1 = movmatrix_trans(l23);
-                // ---- O^T += V^T P^T ----
-#pragma unroll
-                for (int mt = 0; mt < HEAD_DIM / 16; ++mt) {
-                    uint32_t a0r, a1r, a2r, a3r;
-                    ldmatrix_x4_trans(vbase + tile_offset(v_row, 2 * mt + v_chunk_hi), a0r, a1r, a2r, a3r);
-                    mma_16816<FP8>(o[mt], a0r, a1r, a2r, a3r, bh0, bh1);
-                    mma_16816<FP8>(o[mt], a0r, a1r, a2r, a3r, bl0, bl1);
-                }
-                if (!FP8 && (valid < kTileTokens || (APPEND && i == i_new))) fence_proxy_async_smem();
-            } else if (FP8) {
-                __syncwarp();
-                if (lane == 0) mbar_arrive(&empty[s]);  // skipped tile: release it here
-            }
-            if constexpr (!FP8) {
-                __syncwarp();
-                if (lane == 0) mbar_arrive(&empty[s]);
-            }
-        }
-        if (APPEND && i_new >= 0) cp_async_wait_all();  // never leave copies in flight
-        // Row sums over this warp's tokens (lanes with the same tig share a column).
-#pragma unroll
-        for (int off = 4; off < 32; off <<= 1) {
-            l_run[0] += __shfl_xor_sync(0xffffffffu, l_run[0], off);
-            l_run[1] += __shfl_xor_sync(0xffffffffu, l_run[1], off);
-        }
-    }
-
-    // ---------------- merge the warps' states (ring memory is free now) ----------------
-    __syncthreads();
-    float *mo = reinterpret_cast<float *>(smem);                      // [W][8][kMergeStride]
-    float *mm = mo + kConsumerWarps * 8 * C::kMergeStride;            // [W][8]
-    float *ml = mm + kConsumerWarps * 8;                              // [W][8]
-    if (warp < kConsumerWarps) {
-        const int gid = lane >> 2, tig = lane & 3;
-        float *w0 = mo + (warp * 8 + 2 * tig) * C::kMergeStride;
-        float *w1 = w0 + C::kMergeStride;
-#pragma unroll
-        for (int mt = 0; mt < HEAD_DIM / 16; ++mt) {
-            w0[16 * mt + gid] = o[mt][0];
-            w1[16 * mt + gid] = o[mt][1];
-            w0[16 * mt + gid + 8] = o[mt][2];
-            w1[16 * mt + gid + 8] = o[mt][3];
-        }
-        if (gid == 0) {
-            mm[warp * 8 + 2 * tig] = m_run[0];
-            mm[warp * 8 + 2 * tig + 1] = m_run[1];
-            ml[warp * 8 + 2 * tig] = l_run[0];
-            ml[warp * 8 + 2 * tig + 1] = l_run[1];
-        }
-    }
-    __syncthreads();
-    const int G = p.group;
-    for (int x = threadIdx.x; x < G * HEAD_DIM; x += kThreads) {
-        const int n = x / HEAD_DIM;
-        const int d = x - n * HEAD_DIM;
-        float M = -INFINITY;
-#pragma unroll
-        for (int w = 0; w < kConsumerWarps; ++w) M = fmaxf(M, mm[w * 8 + n]);
-        float num = 0.f, den = 0.f;
-        if (M != -INFINITY) {
-#pragma unroll
-            for (int w = 0; w < kConsumerWarps; ++w) {
-                const float f = fast_exp2(mm[w * 8 + n] - M);
-                num += f * mo[(w * 8 + n) * C::kMergeStride + d];
-                den += f * ml[w * 8 + n];
-            }
-        }
-        const int64_t row = (int64_t)b * p.num_q_heads + (int64_t)h * G + n;
-        if (FP8) num *= p.v_scale;
-        if (SPLIT) {
-            p.part_o[(row * p.num_parts + part) * HEAD_DIM + d] = num / den;
-            if (d == 0) {
-                p.part_ml[(row * p.num_parts + part) * 2] = M;
-                p.part_ml[(row * p.num_parts + part) * 2 + 1] = den;
-            }
-        } else {
-            p.out[row * HEAD_DIM + d] = den > 0.f ? num / den : 0.f;
-        }
-    }
-}
-
-// Log-sum-exp merge of the partitions of one (sequence, query head):
-//   out = sum_p 2^(m_p - M) l_p o_p / sum_p 2^(m_p - M) l_p,  M = max_p m_p.
-// Four warps split the partitions; each lane owns HEAD_DIM/32 output dims.
-constexpr int kReduceThreads = 128;
-
-template <int HEAD_DIM>
-__global__ void __launch_bounds__(kReduceThreads) lse_reduce_kernel(const DecodeParams p) {
-    // Launched as a programmatic dependent of the decode grid: wait for its results.
-    asm volatile("griddepcontrol.wait;" ::: "memory");
-    constexpr int kWarps = kReduceThreads / 32;
-    constexpr int V = HEAD_DIM / 32;  // dims per lane: 4 or 2
-    __shared__ float s_max[kWarps];
-    __shared__ float s_den[kWarps];
-    __shared__ float s_acc[kWarps][HEAD_DIM];
-    const int hq = blockIdx.x;
-    const int b = blockIdx.y;
-    const int warp = threadIdx.x >> 5;
-    const int lane = threadIdx.x & 31;
-    const int L = clamp_len(__ldg(p.seq_lens + b), p);
-    const int n = (L + p.part_tokens - 1) / p.part_tokens;
-    const int64_t row = (int64_t)b * p.num_q_heads + hq;
-    const float2 *ml = reinterpret_cast<const float2 *>(p.part_ml + row * p.num_parts * 2);
-    const float *po = p.part_o + row * p.num_parts * HEAD_DIM + lane * V;
-
-    float M = -INFINITY;
-    for (int i = threadIdx.x; i < n; i += kReduceThreads) M = fmaxf(M, __ldg(&ml[i].x));
-#pragma unroll
-    for (int off = 16; off; off >>= 1) M = fmaxf(M, __shfl_xor_sync(0xffffffffu, M, off));
-    if (lane == 0) s_max[warp] = M;
-    __syncthreads();
-#pragma unroll
-    for (int w = 0; w < kWarps; ++w) M = fmaxf(M, s_max[w]);
-
-    float acc[V];
-#pragma unroll
-    for (int k = 0; k < V; ++k) acc[k] = 0.f;
-    float den = 0.f;
-    if (M != -INFINITY) {
-#pragma unroll 4
-        for (int i = warp; i < n; i += kWarps) {
-            const float2 mlv = __ldg(&ml[i]);
-            const float w = fast_exp2(mlv.x - M) * mlv.y;
-            if constexpr (V == 4) {
-                const float4 v = __ldg(reinterpret_cast<const float4 *>(po + (int64_t)i * HEAD_DIM));
-                acc[0] += w * v.x;
-                acc[1] += w * v.y;
-                acc[2] += w * v.z;
-                acc[3] += w * v.w;
-            } else {
-                const float2 v = __ldg(reinterpret_cast<const float2 *>(po + (int64_t)i * HEAD_DIM));
-                acc[0] += w * v.x;
-                acc[1] += w * v.y;
-            }
-            den += w;
-        }
-    }
-#pragma unroll
-    for (int k = 0; k < V; ++k) s_acc[warp][lane * V + k] = acc[k];
-    if (lane == 0) s_den[warp] = den;
-    __syncthreads();
-    for (int x = threadIdx.x; x < HEAD_DIM; x += kReduceThreads) {
-        float num = 0.f, dd = 0.f;
-#pragma unroll
-        for (int w = 0; w < kWarps; ++w) {
-            num += s_acc[w][x];
-            dd += s_den[w];
-        }
-        p.out[row * HEAD_DIM + x] = dd > 0.f ? num / dd : 0.f;
-    }
-}
 
 // ---------------------------------------------------------------------------
 // Host helpers
@@ -812,12 +98,21 @@ int launch_decode(const CUtensorMap &km, const CUtensorMap &vm, const DecodePara
                   cudaStream_t stream) {
     using C = Cfg<HEAD_DIM, FP8>;
     auto kern = paged_decode_kernel<HEAD_DIM, SPLIT, APPEND, FP8>;
-    static std::once_flag once;
-    static cudaError_t attr_err = cudaSuccess;
-    std::call_once(once, [&] {
-        attr_err = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, C::kSmemBytes);
-    });
-    if (attr_err != cudaSuccess) return PA_ERR_CUDA;
+    {
+        // The shared-memory opt-in belongs to the kernel as loaded on one device:
+        // set it once per device.
+        static std::mutex mu;
+        static bool done[64] = {};
+        int dev = 0;
+        if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) return PA_ERR_CUDA;
+        std::lock_guard<std::mutex> lock(mu);
+        if (!done[dev]) {
+            if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, C::kSmemBytes) !=
+                cudaSuccess)
+                return PA_ERR_CUDA;
+            done[dev] = true;
+        }
+    }
     dim3 grid((unsigned)p.num_parts, (unsigned)p.num_kv_heads, (unsigned)batch);
     kern<<<grid, kThreads, C::kSmemBytes, stream>>>(km, vm, p);
     count_launch();
