@@ -380,7 +380,9 @@ def run_native(args):
     peak, peak_kind = _measured_peak()
     achieved = dec_b / (dec_ms / 1e3) / 1e9
 
-    e2e = run_e2e(args, case, pa, stream, world, k, v) if not (args.no_e2e or args.unfused or fp8) else None
+    e2e = None
+    if not (args.no_e2e or args.unfused):
+        e2e = run_e2e(args, case, pa, stream, world, k, v, (k_scale, v_scale) if fp8 else None)
 
     rec = _decode_traffic_record(cfg, "fp8" if fp8 else "bf16")
     traffic = rec.get("traffic_bytes_per_launch") if rec else None
@@ -478,7 +480,7 @@ def replay_allocator(pa, case):
     return alloc, sids
 
 
-def run_e2e(args, case, pa, stream, world, k_pool, v_pool):
+def run_e2e(args, case, pa, stream, world, k_pool, v_pool, kv_scales=None):
     """The same step through the public API with host buffers (pinned), timed end to end.
 
     Every step: the host allocator appends one token per sequence (and reports
@@ -486,7 +488,7 @@ def run_e2e(args, case, pa, stream, world, k_pool, v_pool):
     ``pa_alloc_step`` call); one ``pa_decode_step_host`` call then uploads the
     step's inputs, applies the copies and runs the fused cache write + decode,
     whose output lands in pinned host memory; the step ends when the output is
-    on the host.
+    on the host.  ``kv_scales`` = (k_scale, v_scale) for fp8 pools.
     """
     import torch
     bs = case.block_size
@@ -519,7 +521,9 @@ def run_e2e(args, case, pa, stream, world, k_pool, v_pool):
                             lens_host=h_lens, pairs_host=h_pairs, k_cache=k_pool, v_cache=v_pool,
                             scale=float(case.scale), partition_tokens=case.partition_tokens,
                             num_chunks=args.step_chunks, staging=staging,
-                            err_flag=flag, stream=stream)
+                            err_flag=flag, stream=stream,
+                            k_scale=kv_scales[0] if kv_scales else None, v_scale=kv_scales[1] if kv_scales else None)
+    elem = 1 if kv_scales else 2
     acc = {"h2d": 0, "d2h": 0, "alg": 0, "tokens": 0}
 
     host_step = alloc.step_fn(sids, tables_np, lens_np, pairs_np)
@@ -532,7 +536,7 @@ def run_e2e(args, case, pa, stream, world, k_pool, v_pool):
             acc["h2d"] += sum(t.numel() * t.element_size() for t in (h_q, h_k, h_v, h_tables, h_lens)) + n_pairs * 8
             acc["d2h"] += h_out.numel() * 4
             acc["tokens"] += int(lens_np.sum())
-            c, w, d = step_bytes_from(case, lens_np, n_pairs)
+            c, w, d = step_bytes_from(case, lens_np, n_pairs, elem)
             acc["alg"] += c + w + d
 
     for _ in range(warm):
@@ -553,17 +557,19 @@ def run_e2e(args, case, pa, stream, world, k_pool, v_pool):
             "kv_tokens_per_s": round(_sum_over_ranks(float(acc["tokens"]), world) / dt, 1),
             "step_chunks": args.step_chunks or "auto",
             "includes": "host allocator step (pa_alloc_step: batched append + table export into pinned memory), then one "
-                        "pa_decode_step_host call: H2D of q/k_new/v_new/tables/lens/copy pairs, block copies, "
-                        "fused cache write + decode, D2H of out; timed until out is on the host"}
+                        + ("pa_decode_step_host_fp8" if kv_scales else "pa_decode_step_host")
+                        + " call: upload of q/k_new/v_new/tables/lens/copy pairs, block copies, fused cache write "
+                          "+ decode, out stored into pinned host memory; timed until out is on the host"}
 
 
-def step_bytes_from(case, lens, n_pairs):
+def step_bytes_from(case, lens, n_pairs, kv_elem_bytes: int = 2):
+    """Algorithmic bytes of one e2e step (copy, write, decode) from its lengths and copy-pair count."""
     bs, d, Hkv = case.block_size, case.head_dim, case.num_kv_heads
-    copy = n_pairs * Hkv * bs * d * 2 * 2 * 2
+    copy = n_pairs * Hkv * bs * d * kv_elem_bytes * 2 * 2 + n_pairs * 8
     T = int(lens.size)
-    write = T * Hkv * d * 2 * 2 * 2 + T * 4
+    write = T * Hkv * d * (2 + kv_elem_bytes) * 2 + T * 4
     dec = W.algorithmic_decode_bytes(lens, num_q_heads=case.num_q_heads, num_kv_heads=Hkv, head_dim=d,
-                                     block_size=bs)
+                                     block_size=bs, kv_elem_bytes=kv_elem_bytes)
     return copy, write, dec
 
 
@@ -617,7 +623,7 @@ def main():
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--cpu-budget", type=float, default=12.0, help="seconds of oracle time")
     ap.add_argument("--kv-dtype", choices=["bf16", "fp8"], default="bf16",
-                    help="fp8: E4M3 pools quantised by the library (per-pool scales); e2e is bf16-only")
+                    help="fp8: E4M3 pools quantised by the library (per-pool scales)")
     ap.add_argument("--unfused", action="store_true",
                     help="time pa_reshape_and_cache + pa_decode instead of the fused pa_decode_append")
     ap.add_argument("--num-blocks", type=int, default=None,

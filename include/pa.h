@@ -270,6 +270,21 @@ int pa_decode_step_host(float *out_host, const void *q_host, const void *k_new_h
                         int head_dim, int block_size, int64_t num_blocks, float scale, int partition_tokens,
                         int num_chunks, void *staging, size_t staging_bytes, int32_t *err_flag, void *stream);
 
+/* The same step over fp8 (E4M3) pools (format and scales: see the fp8
+ * section below).  The new rows arrive in bf16 and are quantised by the
+ * fused write; copy pairs move E4M3 blocks (pa_copy_blocks_fp8); the decode
+ * is pa_decode_append_fp8.  Staging is sized by pa_decode_step_staging_size
+ * as for bf16 pools.  k_scale, v_scale not finite and > 0:
+ * PA_ERR_INVALID_ARG, nothing enqueued.  Everything else: as
+ * pa_decode_step_host. */
+int pa_decode_step_host_fp8(float *out_host, const void *q_host, const void *k_new_host, const void *v_new_host,
+                            const int32_t *block_tables_host, int max_blocks_per_seq, const int32_t *seq_lens_host,
+                            const int32_t *copy_pairs_host, int num_pairs, int max_copy_pairs, void *k_cache,
+                            void *v_cache, int batch, int max_seq_len, int num_q_heads, int num_kv_heads,
+                            int head_dim, int block_size, int64_t num_blocks, float scale, float k_scale,
+                            float v_scale, int partition_tokens, int num_chunks, void *staging,
+                            size_t staging_bytes, int32_t *err_flag, void *stream);
+
 /* ------------------------------------------------------------------------
  * Decode with library-owned scratch (no workspace argument).
  *

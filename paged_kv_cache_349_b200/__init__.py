@@ -5,11 +5,17 @@ host numpy arrays for the allocator) into the plain pointers and sizes of
 the C ABI declared in ``include/pa.h`` and raises ``PaError`` on a non-zero
 status.  All device work runs in the library's CUDA kernels.
 
-Device ops (names as in the C ABI):
-    pa_reshape_and_cache, pa_copy_blocks, pa_decode,
-    pa_decode_workspace_size, pa_decode_partition_tokens
+Device ops on bf16 pools (names as in the C ABI):
+    pa_reshape_and_cache, pa_copy_blocks, pa_swap_blocks, pa_decode,
+    pa_decode_append, pa_decode_builtin_scratch, pa_decode_workspace_size,
+    pa_decode_partition_tokens
+Device ops on fp8 (E4M3) pools:
+    pa_quantize_fp8, pa_reshape_and_cache_fp8, pa_copy_blocks_fp8,
+    pa_swap_blocks_fp8, pa_decode_fp8 (with k_new/v_new: the fused write)
+A whole decode step from pinned host buffers:
+    pa_decode_step_staging_size, DecodeStepHost (pa_decode_step_host[_fp8])
 Host allocator:
-    Allocator (pa_alloc_* / pa_seq_* / pa_block_refcount)
+    Allocator (pa_alloc_* / pa_seq_* / pa_block_refcount; step_fn = pa_alloc_step)
 """
 from __future__ import annotations
 
@@ -225,7 +231,8 @@ def pa_decode_step_staging_size(batch, max_blocks_per_seq, max_copy_pairs, num_q
 
 
 class DecodeStepHost:
-    """One decode step from host buffers through ``pa_decode_step_host``.
+    """One decode step from host buffers through ``pa_decode_step_host`` (bf16 pools) or
+    ``pa_decode_step_host_fp8`` (uint8 E4M3 pools, given ``k_scale`` and ``v_scale``).
 
     Holds the argument tuple for a fixed set of pinned host buffers, pools and
     staging, so each step only marshals what changes (max_seq_len, the number of
@@ -236,7 +243,7 @@ class DecodeStepHost:
 
     def __init__(self, *, out_host, q_host, k_new_host, v_new_host, tables_host, lens_host, pairs_host,
                  k_cache, v_cache, scale: float, partition_tokens: int = 0, num_chunks: int = 0, staging=None,
-                 err_flag=None, stream=None):
+                 err_flag=None, stream=None, k_scale: Optional[float] = None, v_scale: Optional[float] = None):
         torch = _torch()
         B, Hq, d = q_host.shape
         NB, Hkv, bs, d2 = k_cache.shape
@@ -248,6 +255,10 @@ class DecodeStepHost:
                             (pairs_host, torch.int32, "pairs_host")):
             if t.is_cuda or t.dtype != dt or not t.is_contiguous():
                 raise TypeError(f"{name} must be a contiguous host {dt} tensor")
+        self.fp8 = k_cache.dtype == torch.uint8
+        if self.fp8 != (k_scale is not None and v_scale is not None):
+            raise ValueError("uint8 (E4M3) pools need k_scale and v_scale; bf16 pools take neither")
+        pool_dt = torch.uint8 if self.fp8 else torch.bfloat16
         self.max_blocks = int(tables_host.shape[1])
         self.max_pairs = int(pairs_host.shape[0])
         self.staging = staging
@@ -255,15 +266,17 @@ class DecodeStepHost:
                       ctypes.c_void_p(k_new_host.data_ptr()), ctypes.c_void_p(v_new_host.data_ptr()),
                       ctypes.c_void_p(tables_host.data_ptr()), self.max_blocks,
                       ctypes.c_void_p(lens_host.data_ptr()), ctypes.c_void_p(pairs_host.data_ptr()))
-        self._kv = (self.max_pairs, _dev(k_cache, torch.bfloat16, "k_cache"), _dev(v_cache, torch.bfloat16, "v_cache"),
-                    B)
-        self._shape = (Hq, Hkv, d, bs, NB, float(scale), int(partition_tokens), int(num_chunks))
+        self._kv = (self.max_pairs, _dev(k_cache, pool_dt, "k_cache"), _dev(v_cache, pool_dt, "v_cache"), B)
+        scales = (float(k_scale), float(v_scale)) if self.fp8 else ()
+        self._shape = (Hq, Hkv, d, bs, NB, float(scale), *scales, int(partition_tokens), int(num_chunks))
         self._tail = (ctypes.c_void_p(staging.data_ptr()), staging.numel() * staging.element_size(),
                       _opt_flag(err_flag), _stream(stream))
+        self._fn = lib.pa_decode_step_host_fp8 if self.fp8 else lib.pa_decode_step_host
+        self._name = "pa_decode_step_host_fp8" if self.fp8 else "pa_decode_step_host"
 
     def __call__(self, max_seq_len: int, num_pairs: int = 0) -> None:
-        _check(lib.pa_decode_step_host(*self._head, int(num_pairs), *self._kv, int(max_seq_len), *self._shape,
-                                       *self._tail), "pa_decode_step_host")
+        _check(self._fn(*self._head, int(num_pairs), *self._kv, int(max_seq_len), *self._shape, *self._tail),
+               self._name)
 
 
 # ---------------------------------------------------------------------------

@@ -246,12 +246,16 @@ size_t pa_decode_step_staging_size(int batch, int max_blocks_per_seq, int max_co
         .total;
 }
 
-int pa_decode_step_host(float *out_host, const void *q_host, const void *k_new_host, const void *v_new_host,
-                        const int32_t *block_tables_host, int max_blocks_per_seq, const int32_t *seq_lens_host,
-                        const int32_t *copy_pairs_host, int num_pairs, int max_copy_pairs, void *k_cache,
-                        void *v_cache, int batch, int max_seq_len, int num_q_heads, int num_kv_heads,
-                        int head_dim, int block_size, int64_t num_blocks, float scale, int partition_tokens,
-                        int num_chunks, void *staging, size_t staging_bytes, int32_t *err_flag, void *stream) {
+// The host step for either pool type: bf16 pools, or E4M3 pools with their scales.
+static int step_host(float *out_host, const void *q_host, const void *k_new_host, const void *v_new_host,
+                     const int32_t *block_tables_host, int max_blocks_per_seq, const int32_t *seq_lens_host,
+                     const int32_t *copy_pairs_host, int num_pairs, int max_copy_pairs, void *k_cache,
+                     void *v_cache, int batch, int max_seq_len, int num_q_heads, int num_kv_heads, int head_dim,
+                     int block_size, int64_t num_blocks, float scale, int partition_tokens, int num_chunks,
+                     void *staging, size_t staging_bytes, int32_t *err_flag, void *stream, bool fp8,
+                     float k_scale, float v_scale) {
+    if (fp8 && !(k_scale > 0.f && v_scale > 0.f && k_scale < 3.0e38f && v_scale < 3.0e38f))
+        return PA_ERR_INVALID_ARG;
     if (batch < 0 || num_pairs < 0 || max_copy_pairs < 0 || max_blocks_per_seq < 0 || max_seq_len < 0 ||
         num_chunks < 0 || num_chunks > pa::kMaxChunks)
         return PA_ERR_INVALID_ARG;
@@ -295,7 +299,7 @@ int pa_decode_step_host(float *out_host, const void *q_host, const void *k_new_h
                                reinterpret_cast<const int32_t *>(st + l.tables + b0 * tab_row), max_blocks_per_seq,
                                reinterpret_cast<const int32_t *>(st + l.lens) + b0, nb, max_seq_len, num_q_heads,
                                num_kv_heads, head_dim, block_size, num_blocks, scale, pt, ws, ws_bytes, err_flag,
-                               cs, false, 1.f, 1.f);
+                               cs, fp8, k_scale, v_scale);
     };
     // Host inputs as the device sees them (resolved once per call).
     const pa::HostSrc hq = pa::host_src(q_host), hk = pa::host_src(k_new_host), hv = pa::host_src(v_new_host);
@@ -319,8 +323,11 @@ int pa_decode_step_host(float *out_host, const void *q_host, const void *k_new_h
     };
     auto copy_pairs = [&](cudaStream_t cs) {
         if (num_pairs == 0) return (int)PA_OK;
-        return pa_copy_blocks(k_cache, v_cache, reinterpret_cast<const int32_t *>(st + l.pairs), num_pairs,
-                              num_blocks, num_kv_heads, block_size, head_dim, err_flag, cs);
+        const int32_t *pairs = reinterpret_cast<const int32_t *>(st + l.pairs);
+        return fp8 ? pa_copy_blocks_fp8(k_cache, v_cache, pairs, num_pairs, num_blocks, num_kv_heads, block_size,
+                                        head_dim, err_flag, cs)
+                   : pa_copy_blocks(k_cache, v_cache, pairs, num_pairs, num_blocks, num_kv_heads, block_size,
+                                    head_dim, err_flag, cs);
     };
 
     if (chunks <= 1) {
@@ -393,6 +400,31 @@ int pa_decode_step_host(float *out_host, const void *q_host, const void *k_new_h
     const int jd = pa::after(s, p.down, p.down_done);
     if (rc == PA_OK) rc = jc != PA_OK ? jc : (jp != PA_OK ? jp : jd);
     return rc;
+}
+
+int pa_decode_step_host(float *out_host, const void *q_host, const void *k_new_host, const void *v_new_host,
+                        const int32_t *block_tables_host, int max_blocks_per_seq, const int32_t *seq_lens_host,
+                        const int32_t *copy_pairs_host, int num_pairs, int max_copy_pairs, void *k_cache,
+                        void *v_cache, int batch, int max_seq_len, int num_q_heads, int num_kv_heads,
+                        int head_dim, int block_size, int64_t num_blocks, float scale, int partition_tokens,
+                        int num_chunks, void *staging, size_t staging_bytes, int32_t *err_flag, void *stream) {
+    return step_host(out_host, q_host, k_new_host, v_new_host, block_tables_host, max_blocks_per_seq,
+                     seq_lens_host, copy_pairs_host, num_pairs, max_copy_pairs, k_cache, v_cache, batch,
+                     max_seq_len, num_q_heads, num_kv_heads, head_dim, block_size, num_blocks, scale,
+                     partition_tokens, num_chunks, staging, staging_bytes, err_flag, stream, false, 1.f, 1.f);
+}
+
+int pa_decode_step_host_fp8(float *out_host, const void *q_host, const void *k_new_host, const void *v_new_host,
+                            const int32_t *block_tables_host, int max_blocks_per_seq, const int32_t *seq_lens_host,
+                            const int32_t *copy_pairs_host, int num_pairs, int max_copy_pairs, void *k_cache,
+                            void *v_cache, int batch, int max_seq_len, int num_q_heads, int num_kv_heads,
+                            int head_dim, int block_size, int64_t num_blocks, float scale, float k_scale,
+                            float v_scale, int partition_tokens, int num_chunks, void *staging,
+                            size_t staging_bytes, int32_t *err_flag, void *stream) {
+    return step_host(out_host, q_host, k_new_host, v_new_host, block_tables_host, max_blocks_per_seq,
+                     seq_lens_host, copy_pairs_host, num_pairs, max_copy_pairs, k_cache, v_cache, batch,
+                     max_seq_len, num_q_heads, num_kv_heads, head_dim, block_size, num_blocks, scale,
+                     partition_tokens, num_chunks, staging, staging_bytes, err_flag, stream, true, k_scale, v_scale);
 }
 
 }  // extern "C"

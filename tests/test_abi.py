@@ -114,3 +114,12 @@ def test_host_step_argument_errors_need_no_gpu():
     assert call(a8=1) == pa.PA_ERR_INVALID_ARG            # pairs beyond max_copy_pairs
     assert call(a23=16) == pa.PA_ERR_INVALID_ARG          # staging too small
     assert call(a22=_fake(0x100010)) == pa.PA_ERR_INVALID_ARG  # staging not 256-byte aligned
+
+
+def test_fp8_host_step_rejects_bad_scales():
+    """Scales that are not finite and positive are refused before anything is enqueued."""
+    for ks, vs in ((0.0, 1.0), (1.0, -1.0), (float("inf"), 1.0), (1.0, float("nan"))):
+        rc = lib.pa_decode_step_host_fp8(_fake(), _fake(), _fake(), _fake(), _fake(), 4, _fake(), None, 0, 0,
+                                         _fake(), _fake(), 2, 64, 8, 2, 128, 16, 64, 0.1, ks, vs, -1, 0,
+                                         _fake(0x100000), 1 << 20, None, None)
+        assert rc == pa.PA_ERR_INVALID_ARG

@@ -180,3 +180,51 @@ def test_fp8_full_size_llama2_7b_sampled_rows(torch_cuda):
     got, gk, gv = _gpu_step_fp8(case, k8, v8, k_scale, v_scale, fused=True)
     assert np.array_equal(gk, k_ref) and np.array_equal(gv, v_ref)
     assert_close(got[rows[:, 0], rows[:, 1]], want, "fp8 cfg2 full")
+
+
+@pytest.mark.parametrize("cfg,kw,chunks", [
+    (2, dict(batch=64, max_len=300, num_blocks=2048), 0),
+    (2, dict(batch=6, max_len=300, num_blocks=256), 1),
+    (4, dict(batch=9, max_len=1500, num_blocks=512), 4),                              # split decode
+    (5, dict(batch=3, max_len=2048, num_blocks=960, num_copy_pairs=40), 3),           # E4M3 block copies
+])
+def test_fp8_host_step_matches_device_path(torch_cuda, cfg, kw, chunks):
+    """pa_decode_step_host_fp8 == fp8 block copies + fused fp8 write and decode on the device, bit for bit."""
+    torch = torch_cuda
+    import paged_kv_cache_349_b200 as pa
+    case = W.make_case(cfg, **kw)
+    k_last, v_last, other = W.split_last_tokens(case)
+    assert other.size == 0
+    k_scale, v_scale = amax_scale(case.k_cache), amax_scale(case.v_cache)
+    k8, v8 = _fp8_case(case, k_scale, v_scale)
+    want, want_k, want_v = _gpu_step_fp8(case, k8, v8, k_scale, v_scale, fused=True)
+
+    def pinned(a, dtype):
+        t = torch.from_numpy(np.ascontiguousarray(a))
+        return (t.view(dtype) if dtype is torch.bfloat16 else t.to(dtype)).pin_memory()
+
+    pairs = case.copy_pairs.reshape(-1, 2)
+    max_pairs = max(1, pairs.shape[0])
+    pairs_np = np.zeros((max_pairs, 2), np.int32)
+    pairs_np[:pairs.shape[0]] = pairs
+    out_h = torch.full(case.q.shape, float("nan"), dtype=torch.float32).pin_memory()
+    gk, gv = u8_dev(k8), u8_dev(v8)
+    flag = torch.zeros(1, dtype=torch.int32, device="cuda")
+    size = pa.pa_decode_step_staging_size(case.batch, case.max_blocks_per_seq, max_pairs, case.num_q_heads,
+                                          case.num_kv_heads, case.head_dim, case.block_size, case.max_seq_len,
+                                          case.partition_tokens)
+    staging = torch.empty(size, dtype=torch.uint8, device="cuda")
+    step = pa.DecodeStepHost(out_host=out_h, q_host=pinned(case.q.view(np.int16), torch.bfloat16),
+                             k_new_host=pinned(k_last.view(np.int16), torch.bfloat16),
+                             v_new_host=pinned(v_last.view(np.int16), torch.bfloat16),
+                             tables_host=pinned(case.block_tables, torch.int32),
+                             lens_host=pinned(case.seq_lens, torch.int32), pairs_host=pinned(pairs_np, torch.int32),
+                             k_cache=gk, v_cache=gv, scale=float(case.scale), k_scale=k_scale, v_scale=v_scale,
+                             partition_tokens=case.partition_tokens, num_chunks=chunks, staging=staging,
+                             err_flag=flag)
+    step(case.max_seq_len, pairs.shape[0])
+    torch.cuda.synchronize()
+    assert int(flag.item()) == 0
+    assert np.array_equal(out_h.numpy().astype(np.float64), want)
+    assert np.array_equal(u8_host(gk), want_k) and np.array_equal(u8_host(gv), want_v)
+
