@@ -365,7 +365,7 @@ def run_native(args):
     t1.record(stream)
     torch.cuda.synchronize()
     _barrier(world)
-    launches = pa.launch_count() - launches0
+    launches = int(_sum_over_ranks(float(pa.launch_count() - launches0), world))  # whole job, like value
     clocks = sampler.stop() if sampler else None
     ms_local = t0.elapsed_time(t1)
     ms = _max_over_ranks(ms_local, world)
