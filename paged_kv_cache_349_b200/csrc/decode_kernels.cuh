@@ -13,7 +13,8 @@
 //  * The sequence is cut into 16-token tiles.  A producer warp dereferences
 //    the block table and stages each tile's K and V (16 rows x head_dim
 //    bf16, contiguous in the pool) into shared memory with TMA tile loads
-//    (128-byte swizzle, no multicast) through an 8-deep mbarrier ring.
+//    (128-byte swizzle, no multicast) through an 8-deep mbarrier ring
+//    (16-deep for fp8 pools at head_dim 128, whose tiles are half the size).
 //  * Four consumer warps take tiles round-robin.  Per tile a warp computes
 //    S^T = K_tile Q^T with bf16 mma.sync (M = 16 tokens, N = 8 query-head
 //    columns, K = head_dim), runs an online softmax in fp32 (log2 domain),
@@ -45,14 +46,12 @@ namespace {
 #ifndef PA_DECODE_PRODUCER_LANES
 #define PA_DECODE_PRODUCER_LANES 8
 #endif
-// fp8 tiles: 1 = expand E4M3 with integer bit moves (value * 2^-8), 0 = hardware cvt.
 constexpr int kTileTokens = 16;
 constexpr int kConsumerWarps = PA_DECODE_CONSUMER_WARPS;
 constexpr int kThreads = (kConsumerWarps + 1) * 32;
-constexpr int kStages = PA_DECODE_STAGES;
+constexpr int kDefaultStages = PA_DECODE_STAGES;
 // Producer lanes issue tiles round-robin; lane k owns ring slots k, k+P, ...
 constexpr int kProducerLanes = PA_DECODE_PRODUCER_LANES;
-static_assert(kStages % kProducerLanes == 0, "each producer lane owns whole ring slots");
 static_assert(kProducerLanes >= 1 && kProducerLanes <= 8, "window indexing assumes <= 8 lanes");
 // A 16-bit tile (bf16, or f16 expanded from fp8) is stored as HEAD_DIM/64
 // boxes of 16 rows x 128 bytes with the TMA 128-byte swizzle.
@@ -69,13 +68,20 @@ struct Cfg {
     static constexpr int kBoxBytes = kTileTokens * kBoxRowBytes;
     static constexpr int kTileBytes = kBoxes * kBoxBytes;  // K or V of one tile
     static constexpr int kStageBytes = 2 * kTileBytes;
+    // fp8, head_dim 128: the ring tile carries the 128-byte swizzle; the K and V
+    // mma fragments are built straight from it, in registers.
+    // fp8, head_dim 64: the ring tile is unswizzled and both K and V are expanded
+    // to per-warp 16-bit tiles.
+    static constexpr bool kDirect = FP8 && HEAD_DIM == 128;
+    // Ring depth.  With K and V read from the ring, a slot stays busy until its
+    // tile has gone through PV, and fp8 tiles are half the size: twice the
+    // default depth keeps enough bytes in flight (measured on B200: 8-11 % less
+    // time per call than the default depth).
+    static constexpr int kStages = kDirect ? 2 * kDefaultStages : kDefaultStages;
+    static_assert(kStages % kProducerLanes == 0, "each producer lane owns whole ring slots");
     static constexpr int kRingBytes = kStages * kStageBytes;
-    // fp8, head_dim 128: the ring tile carries the 128-byte swizzle; K fragments
-    // are built straight from it and only V is expanded to a 16-bit tile.
-    // fp8, head_dim 64: the ring tile is unswizzled and both K and V are expanded.
-    static constexpr bool kDirectK = FP8 && HEAD_DIM == 128;
     static constexpr int kTile16Bytes = (HEAD_DIM / 64) * kBox16Bytes;
-    static constexpr int kStagingBytes = FP8 ? kConsumerWarps * (kDirectK ? 1 : 2) * kTile16Bytes : 0;
+    static constexpr int kStagingBytes = FP8 && !kDirect ? kConsumerWarps * 2 * kTile16Bytes : 0;
     static constexpr int kDataBytes = kRingBytes + kStagingBytes;
     static constexpr int kMergeStride = HEAD_DIM + 4;  // padded row: conflict-free merge stores
     static constexpr int kMergeBytes = kConsumerWarps * 8 * (kMergeStride + 2) * 4;
@@ -164,11 +170,11 @@ __global__ void __launch_bounds__(kThreads, FP8 ? PA_DECODE_MIN_CTAS_FP8 : PA_DE
     uint8_t *smem = reinterpret_cast<uint8_t *>(
         (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~static_cast<uintptr_t>(1023));
     uint64_t *full = reinterpret_cast<uint64_t *>(smem + C::kDataBytes);
-    uint64_t *empty = full + kStages;
-    int *tile_ok = reinterpret_cast<int *>(empty + kStages);
+    uint64_t *empty = full + C::kStages;
+    int *tile_ok = reinterpret_cast<int *>(empty + C::kStages);
     // Fused write: the new token's bf16 K/V row (16 bytes per lane) and its block id,
     // fetched asynchronously so no registers are held until the tile is reached.
-    uint4 *append_row = reinterpret_cast<uint4 *>(tile_ok + kStages);
+    uint4 *append_row = reinterpret_cast<uint4 *>(tile_ok + C::kStages);
     int *append_phys = reinterpret_cast<int *>(append_row + 32);
 
     const int part = blockIdx.x;
@@ -189,7 +195,7 @@ __global__ void __launch_bounds__(kThreads, FP8 ? PA_DECODE_MIN_CTAS_FP8 : PA_DE
     if (threadIdx.x == 0 && part == 0 && h == 0 && L != L_raw) raise_flag(p.err_flag, PA_FLAG_BAD_LEN);
 
     if (threadIdx.x == 0) {
-        for (int s = 0; s < kStages; ++s) {
+        for (int s = 0; s < C::kStages; ++s) {
             mbar_init(&full[s], 1);
             mbar_init(&empty[s], 1);
         }
@@ -250,8 +256,8 @@ __global__ void __launch_bounds__(kThreads, FP8 ? PA_DECODE_MIN_CTAS_FP8 : PA_DE
             const bool two_blocks = p.block_size < kTileTokens;
             const bool second = two_blocks && tok0 + p.block_size < tok_end;
             if (mine) {
-                const int s = i % kStages;
-                if (i >= kStages && !mbar_wait_bounded(&empty[s], ((i / kStages) - 1) & 1, p.err_flag)) {
+                const int s = i % C::kStages;
+                if (i >= C::kStages && !mbar_wait_bounded(&empty[s], ((i / C::kStages) - 1) & 1, p.err_flag)) {
                     stop = true;
                 } else {
                     issued = i + 1;
@@ -288,12 +294,12 @@ __global__ void __launch_bounds__(kThreads, FP8 ? PA_DECODE_MIN_CTAS_FP8 : PA_DE
             if (__any_sync(0xffffffffu, stop)) break;
         }
         // Drain: every issued tile has landed before the ring is reused or the CTA exits.
-        // A tile is the last user of its slot when no tile kStages later was issued.
+        // A tile is the last user of its slot when no tile one ring depth later was issued.
         const int issued_all = __reduce_max_sync(0xffffffffu, issued);
         if (lane < kProducerLanes) {
             for (int i = lane; i < issued_all; i += kProducerLanes)
-                if (i + kStages >= issued_all && i < issued)
-                    if (!mbar_wait_bounded(&full[i % kStages], (i / kStages) & 1, p.err_flag)) break;
+                if (i + C::kStages >= issued_all && i < issued)
+                    if (!mbar_wait_bounded(&full[i % C::kStages], (i / C::kStages) & 1, p.err_flag)) break;
         }
     } else {
         // ---------------- consumers ----------------
@@ -343,7 +349,7 @@ __global__ void __launch_bounds__(kThreads, FP8 ? PA_DECODE_MIN_CTAS_FP8 : PA_DE
         // Token row of mma row gid (gid+8 -> +8): this order keeps both the K
         // fragment loads and the V ldmatrix reads free of bank conflicts.
         // (fp8 with K read straight from the swizzled fp8 tile uses 0,2,4,6,1,3,5,7.)
-        auto token_of = [](int g) { return C::kDirectK ? ((g & 3) << 1) | (g >> 2) : (g >> 1) | ((g & 1) << 2); };
+        auto token_of = [](int g) { return C::kDirect ? ((g & 3) << 1) | (g >> 2) : (g >> 1) | ((g & 1) << 2); };
         const int tau = token_of(gid);
         // ldmatrix row address pattern for V: matrix (lane>>3), row (lane&7).
         const int v_row = token_of(lane & 7) + (((lane >> 4) & 1) << 3);
@@ -385,15 +391,15 @@ __global__ void __launch_bounds__(kThreads, FP8 ? PA_DECODE_MIN_CTAS_FP8 : PA_DE
         };
 
         for (int i = warp; i < n_tiles; i += kConsumerWarps) {
-            const int s = i % kStages;
-            const bool got = mbar_wait_bounded(&full[s], (i / kStages) & 1, p.err_flag);
+            const int s = i % C::kStages;
+            const bool got = mbar_wait_bounded(&full[s], (i / C::kStages) & 1, p.err_flag);
             if (!__all_sync(0xffffffffu, got)) break;
             const int valid = min(kTileTokens, tok_end - (tok_begin + i * kTileTokens));
             if (tile_ok[s]) {
                 uint32_t kbase = smem_addr(smem + s * C::kStageBytes);
                 uint32_t vbase = kbase + C::kTileBytes;
                 uint32_t ring_k = kbase;  // fp8 direct-K: K stays in the ring until QK is done
-                if constexpr (C::kDirectK) {
+                if constexpr (C::kDirect) {
                     // The fused cache write lands in the (swizzled) fp8 tile first, and in the pool.
                     if (APPEND && i == i_new) {
                         const int r = (L - 1 - tok_begin) - i_new * kTileTokens;
@@ -406,28 +412,6 @@ __global__ void __launch_bounds__(kThreads, FP8 ? PA_DECODE_MIN_CTAS_FP8 : PA_DE
                         if (dst >= 0) reinterpret_cast<uint2 *>(lane < 16 ? p.k_pool : p.v_pool)[dst] = q8;
                         __syncwarp();
                     }
-                    // Expand V into this warp's 16-bit tile.  Each group of 8 lanes takes rows
-                    // r and r^5 and four 16-byte chunks of one column box, so both the swizzled
-                    // fp8 reads and the swizzled 16-bit writes hit 8 distinct bank groups.
-                    const uint32_t stg_v = smem_addr(smem + C::kRingBytes + warp * C::kTile16Bytes);
-#pragma unroll
-                    for (int x = lane; x < kTileTokens * (HEAD_DIM / 16); x += 32) {
-                        const int grp = x >> 3, pair = grp >> 1, box = grp & 1;
-                        const int r0 = ((pair & 1) << 1) | (((pair >> 1) & 1) << 3) | (pair >> 2);
-                        const int r = (x & 4) ? (r0 ^ 5) : r0;
-                        const int c16 = box * 4 + (x & 3);
-                        const uint4 w = lds128(vbase + fp8_tile_offset(r, c16 * 16));
-                        const uint4 lo = e4m3x8_to_f16x8(w.x, w.y);
-                        const uint4 hi = e4m3x8_to_f16x8(w.z, w.w);
-                        asm volatile("st.shared.v4.u32 [%0], {%1, %2, %3, %4};" ::"r"(stg_v + tile_offset(r, 2 * c16)),
-                                     "r"(lo.x), "r"(lo.y), "r"(lo.z), "r"(lo.w)
-                                     : "memory");
-                        asm volatile("st.shared.v4.u32 [%0], {%1, %2, %3, %4};" ::"r"(stg_v + tile_offset(r, 2 * c16 + 1)),
-                                     "r"(hi.x), "r"(hi.y), "r"(hi.z), "r"(hi.w)
-                                     : "memory");
-                    }
-                    __syncwarp();
-                    vbase = stg_v;
                 } else if constexpr (FP8) {
                     // head_dim 64: the fused write lands in the unswizzled fp8 tile first.
                     if (APPEND && i == i_new) {
@@ -473,9 +457,10 @@ __global__ void __launch_bounds__(kThreads, FP8 ? PA_DECODE_MIN_CTAS_FP8 : PA_DE
                     kbase = stg_k;
                     vbase = stg_v;
                 }
-                if (valid < kTileTokens) {
+                if (!C::kDirect && valid < kTileTokens) {
                     // Rows past the sequence end hold stale data: zero them so
-                    // that P = 0 times V cannot produce NaN.
+                    // that P = 0 times V cannot produce NaN.  (fp8, head_dim 128
+                    // masks them in registers instead, below.)
                     constexpr int kBoxes16 = HEAD_DIM / 64;  // boxes of the 16-bit tile
                     const int lines = (kTileTokens - valid) * kBoxes16;
                     for (int x = lane; x < lines * 8; x += 32) {
@@ -507,7 +492,7 @@ __global__ void __launch_bounds__(kThreads, FP8 ? PA_DECODE_MIN_CTAS_FP8 : PA_DE
 #pragma unroll
                 for (int j = 0; j < HEAD_DIM / 32; ++j) {
                     uint4 ka, kb;
-                    if constexpr (C::kDirectK) {
+                    if constexpr (C::kDirect) {
                         // 8 fp8 codes (dims 32j+8t .. +7) of rows tau and tau+8, expanded in registers
                         uint32_t a0, a1, b0, b1;
                         asm volatile("ld.shared.v2.u32 {%0, %1}, [%2];"
@@ -525,12 +510,6 @@ __global__ void __launch_bounds__(kThreads, FP8 ? PA_DECODE_MIN_CTAS_FP8 : PA_DE
                     }
                     mma_16816<FP8>(sacc, ka.x, kb.x, ka.y, kb.y, qf[2 * j][0], qf[2 * j][1]);
                     mma_16816<FP8>(sacc, ka.z, kb.z, ka.w, kb.w, qf[2 * j + 1][0], qf[2 * j + 1][1]);
-                }
-                if constexpr (C::kDirectK) {
-                    // K and V have left the ring: hand the slot back to the producer.
-                    if (APPEND && i == i_new) fence_proxy_async_smem();
-                    __syncwarp();
-                    if (lane == 0) mbar_arrive(&empty[s]);
                 }
                 // sacc: (token tau, col 2t), (tau, 2t+1), (tau+8, 2t), (tau+8, 2t+1)
                 const float s0 = tau < valid ? sacc[0] * s_scale : -INFINITY;
@@ -576,12 +555,55 @@ __global__ void __launch_bounds__(kThreads, FP8 ? PA_DECODE_MIN_CTAS_FP8 : PA_DE
                 const uint32_t bh0 = movmatrix_trans(h01), bh1 = movmatrix_trans(h23);
                 const uint32_t bl0 = movmatrix_trans(l01), bl1 = movmatrix_trans(l23);
                 // ---- O^T += V^T P^T ----
+                if constexpr (C::kDirect) {
+                    // V^T fragments straight from the swizzled fp8 tile.  ldmatrix.trans on
+                    // 16-bit pairs hands each lane, per register, the codes of tokens
+                    // (k, k+1) for two neighbouring dims; split into an even-dim and an
+                    // odd-dim m-tile and widened to f16 they are the A fragments.  M-tile
+                    // 2c+e holds dims 32c + 2r + e (row r < 8) and 32c + 16 + 2(r-8) + e.
+                    // Matrices: rows tau (+8 for 1, 3) of byte columns 32c (+16 for 2, 3).
+                    const int mtx = lane >> 3;
+                    const uint32_t v_addr = vbase + fp8_tile_offset(token_of(lane & 7) + ((mtx & 1) << 3), (mtx >> 1) << 4);
+                    const bool partial = valid < kTileTokens;
+                    uint32_t keep_lo = 0xffffffffu, keep_hi = 0xffffffffu;  // tokens past the end read as 0
+                    if (partial) {
+                        const int k0 = token_of(2 * tig), k1 = token_of(2 * tig + 1);
+                        keep_lo = (k0 < valid ? 0x0000ffffu : 0u) | (k1 < valid ? 0xffff0000u : 0u);
+                        keep_hi = (k0 + 8 < valid ? 0x0000ffffu : 0u) | (k1 + 8 < valid ? 0xffff0000u : 0u);
+                    }
 #pragma unroll
-                for (int mt = 0; mt < HEAD_DIM / 16; ++mt) {
-                    uint32_t a0r, a1r, a2r, a3r;
-                    ldmatrix_x4_trans(vbase + tile_offset(v_row, 2 * mt + v_chunk_hi), a0r, a1r, a2r, a3r);
-                    mma_16816<FP8>(o[mt], a0r, a1r, a2r, a3r, bh0, bh1);
-                    mma_16816<FP8>(o[mt], a0r, a1r, a2r, a3r, bl0, bl1);
+                    for (int c = 0; c < HEAD_DIM / 32; ++c) {
+                        uint32_t r0, r1, r2, r3;
+                        // + 32c bytes: the swizzle only permutes 16-byte chunks within 128, so
+                        // chunk (2c + hi) ^ (row & 7) is reached by xor-ing 2c into the chunk bits
+                        ldmatrix_x4_trans(v_addr ^ ((uint32_t)(2 * c) << 4), r0, r1, r2, r3);
+                        const uint32_t m[4] = {r0, r2, r1, r3};  // a0: tokens k, rows < 8; a1: rows >= 8; a2, a3: +8 tokens
+                        uint32_t ev[4], od[4];
+#pragma unroll
+                        for (int q = 0; q < 4; ++q) {
+                            e4m3x4_to_f16x4(__byte_perm(m[q], 0u, 0x3120), ev[q], od[q]);
+                            if (partial) {
+                                ev[q] &= q < 2 ? keep_lo : keep_hi;
+                                od[q] &= q < 2 ? keep_lo : keep_hi;
+                            }
+                        }
+                        mma_16816<FP8>(o[2 * c], ev[0], ev[1], ev[2], ev[3], bh0, bh1);
+                        mma_16816<FP8>(o[2 * c], ev[0], ev[1], ev[2], ev[3], bl0, bl1);
+                        mma_16816<FP8>(o[2 * c + 1], od[0], od[1], od[2], od[3], bh0, bh1);
+                        mma_16816<FP8>(o[2 * c + 1], od[0], od[1], od[2], od[3], bl0, bl1);
+                    }
+                    // K and V have left the ring: hand the slot back to the producer.
+                    if (APPEND && i == i_new) fence_proxy_async_smem();
+                    __syncwarp();
+                    if (lane == 0) mbar_arrive(&empty[s]);
+                } else {
+#pragma unroll
+                    for (int mt = 0; mt < HEAD_DIM / 16; ++mt) {
+                        uint32_t a0r, a1r, a2r, a3r;
+                        ldmatrix_x4_trans(vbase + tile_offset(v_row, 2 * mt + v_chunk_hi), a0r, a1r, a2r, a3r);
+                        mma_16816<FP8>(o[mt], a0r, a1r, a2r, a3r, bh0, bh1);
+                        mma_16816<FP8>(o[mt], a0r, a1r, a2r, a3r, bl0, bl1);
+                    }
                 }
                 if (!FP8 && (valid < kTileTokens || (APPEND && i == i_new))) fence_proxy_async_smem();
             } else if (FP8) {
@@ -613,10 +635,13 @@ __global__ void __launch_bounds__(kThreads, FP8 ? PA_DECODE_MIN_CTAS_FP8 : PA_DE
         float *w1 = w0 + C::kMergeStride;
 #pragma unroll
         for (int mt = 0; mt < HEAD_DIM / 16; ++mt) {
-            w0[16 * mt + gid] = o[mt][0];
-            w1[16 * mt + gid] = o[mt][1];
-            w0[16 * mt + gid + 8] = o[mt][2];
-            w1[16 * mt + gid + 8] = o[mt][3];
+            // dims of rows gid and gid + 8 of m-tile mt (fp8 head_dim 128: even/odd-dim m-tiles)
+            const int d0 = C::kDirect ? 32 * (mt >> 1) + 2 * gid + (mt & 1) : 16 * mt + gid;
+            const int d1 = C::kDirect ? d0 + 16 : d0 + 8;
+            w0[d0] = o[mt][0];
+            w1[d0] = o[mt][1];
+            w0[d1] = o[mt][2];
+            w1[d1] = o[mt][3];
         }
         if (gid == 0) {
             mm[warp * 8 + 2 * tig] = m_run[0];
