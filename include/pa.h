@@ -9,8 +9,8 @@
  *   - the cache-append write through a slot mapping ("Walk through paged
  *     attention end to end" (zenaique.com), conceptual
  *     paged_attention_decode, append step),
- *   - single-query decode attention that dereferences the block table for
- *     every attended position (same page, attention step; "What is
+ *   - single-query decode attention that looks up each token's block
+ *     through the table (same page, attention step; "What is
  *     PagedAttention and how does it manage KV cache" (n4n.ai), section
  *     "How PagedAttention works": two-level indirection, tokens contiguous
  *     inside a block),
@@ -104,7 +104,7 @@ int pa_reshape_and_cache(const void *k_new, const void *v_new, void *k_cache, vo
 
 /* ------------------------------------------------------------------------
  * Copy-on-write block copy ("PagedAttention & vLLM", Copy-on-write sharing:
- * duplicate just that one block, then write).
+ * a sequence about to change a shared block first gets a private copy).
  *
  * For each pair i: block pairs[2i+1] of both pools becomes a bit copy of
  * block pairs[2i] (all heads, rows and dims).
@@ -120,9 +120,8 @@ int pa_copy_blocks(void *k_cache, void *v_cache, const int32_t *pairs, int num_p
 
 /* ------------------------------------------------------------------------
  * Block swap between two pools ("What is PagedAttention and how does it
- * manage KV cache", Swapping and preemption: blocks are evicted to CPU
- * memory when GPU memory runs short and fetched back when the request
- * resumes).
+ * manage KV cache", Swapping and preemption: under memory pressure a
+ * request's blocks move out to host memory and come back when it resumes).
  *
  * For each pair i: block pairs[2i+1] of the destination pools becomes a bit
  * copy of block pairs[2i] of the source pools (K and V, all heads, rows and

@@ -17,15 +17,17 @@
  *  - attend: textbook softmax attention of one query over the gathered rows,
  *    s_p = scale * sum_i q_i k_p,i ; w_p = exp(s_p - max s) ;
  *    out = sum_p w_p v_p / sum_p w_p   -- paging leaves this math unchanged
- *    ("Walk through paged attention end to end", red flags: "the math is
- *    identical to standard attention").  L = 0 gives a zero row.
+ *    ("Walk through paged attention end to end", red flags: paging moves
+ *    where K and V live, not what attention computes).  L = 0 gives a zero
+ *    row.
  *  - decode: for every requested (sequence b, query head g) the kv head is
  *    h = g / (Hq / Hkv) (grouped-query sharing), gather + attend.
  *  - reshape_and_cache: write new K/V rows at slot s, i.e. block s / bs,
  *    row s % bs ("Walk through paged attention end to end", append step:
  *    last_block, offset); slot -1 is skipped.
  *  - copy_blocks: copy whole blocks src -> dst, K and V ("PagedAttention &
- *    vLLM", Copy-on-write sharing: duplicate just that one block).
+ *    vLLM", Copy-on-write sharing: the writer gets a private copy of the
+ *    shared block).
  *  - swap_blocks: the same copy between two different pools (device pool
  *    and CPU-side pool), "What is PagedAttention and how does it manage KV
  *    cache", Swapping and preemption.
