@@ -631,6 +631,10 @@ def main():
     args = ap.parse_args()
     if args.warmup < 3:
         ap.error("--warmup must be at least 3")
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    if args.gpus != world:
+        print(f"bench.py: --gpus {args.gpus} but WORLD_SIZE={world}; launch N > 1 under torchrun "
+              f"(one rank per GPU). Measuring {world} rank(s).", file=sys.stderr)
     if args.impl == "reference":
         run_reference(args)
     else:
