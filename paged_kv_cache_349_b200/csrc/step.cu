@@ -265,6 +265,7 @@ static int step_host(float *out_host, const void *q_host, const void *k_new_host
         !k_cache || !v_cache)
         return PA_ERR_INVALID_ARG;
     if (num_pairs > max_copy_pairs || (num_pairs > 0 && !copy_pairs_host)) return PA_ERR_INVALID_ARG;
+    if (partition_tokens > 0 && partition_tokens % block_size) return PA_ERR_INVALID_ARG;  // as pa_decode
     const pa::StagingLayout l = pa::staging_layout(batch, max_blocks_per_seq, max_copy_pairs, num_q_heads,
                                                    num_kv_heads, head_dim, block_size, max_seq_len,
                                                    partition_tokens);

@@ -114,6 +114,7 @@ def test_host_step_argument_errors_need_no_gpu():
     assert call(a8=1) == pa.PA_ERR_INVALID_ARG            # pairs beyond max_copy_pairs
     assert call(a23=16) == pa.PA_ERR_INVALID_ARG          # staging too small
     assert call(a22=_fake(0x100010)) == pa.PA_ERR_INVALID_ARG  # staging not 256-byte aligned
+    assert call(a20=24) == pa.PA_ERR_INVALID_ARG          # partition not a multiple of block_size
 
 
 def test_fp8_host_step_rejects_bad_scales():
