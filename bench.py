@@ -103,7 +103,7 @@ def step_bytes(case, kv_elem_bytes: int = 2):
 
 
 class ClockSampler:
-    """nvidia-smi clocks and throttle reasons sampled every 200 ms in the background."""
+    """nvidia-smi clocks and throttle reasons sampled every 50 ms in the background."""
 
     FIELDS = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
               "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
@@ -119,7 +119,7 @@ class ClockSampler:
         try:
             self._proc = subprocess.Popen(
                 ["nvidia-smi", f"--id={self.device_index}", f"--query-gpu={self.FIELDS}",
-                 "--format=csv,noheader,nounits", "-lms", "200"],
+                 "--format=csv,noheader,nounits", "-lms", "50"],
                 stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
         except Exception:
             self._proc = None
@@ -353,7 +353,17 @@ def run_native(args):
     assert int(flag.item()) == 0, f"error flag {int(flag.item()):#x}"
 
     sampler = ClockSampler(torch.cuda.current_device()).start() if rank == 0 else None
-    time.sleep(0.3 if sampler else 0)
+    # The timed region lasts milliseconds, shorter than the sampling period: keep the
+    # GPU under the same (untimed, idempotent) step for ~0.4 s first, so the clock
+    # samples show the clocks under this load.
+    load_steps = 0
+    if sampler:
+        t_load = time.perf_counter() + 0.4
+        while time.perf_counter() < t_load:
+            for _ in range(10):
+                step()
+            load_steps += 10
+            torch.cuda.synchronize()
     _barrier(world)
     torch.cuda.synchronize()
     launches0 = pa.launch_count()
@@ -367,6 +377,8 @@ def run_native(args):
     _barrier(world)
     launches = int(_sum_over_ranks(float(pa.launch_count() - launches0), world))  # whole job, like value
     clocks = sampler.stop() if sampler else None
+    if clocks is not None:
+        clocks["untimed_load_steps_before_timing"] = load_steps
     ms_local = t0.elapsed_time(t1)
     ms = _max_over_ranks(ms_local, world)
     dec_ms = statistics.mean(a.elapsed_time(b) for a, b in dec_ev)
