@@ -438,6 +438,18 @@ int pa_alloc_export(const pa_allocator *alloc, const int32_t *seq_ids, int n, in
 int pa_alloc_step(pa_allocator *alloc, const int32_t *seq_ids, int n, int32_t *tables, int max_blocks,
                   int32_t pad, int32_t *seq_lens, int32_t *cow_pairs_out, int *n_cow, int *max_seq_len);
 int pa_alloc_num_free(const pa_allocator *alloc);
+/* Host-side check of decode inputs held in host memory, a debugging aid
+ * (the kernels bounds-check the same things and report them through
+ * err_flag).  For every sequence b: 0 <= seq_lens[b] <= max_blocks *
+ * block_size, and the first ceil(seq_lens[b] / block_size) entries of row b
+ * of tables [batch, max_blocks] are block ids in [0, num_blocks), none
+ * repeated within the row (rows may share blocks with each other: forks).
+ * Entries past those are not read.  Returns PA_OK with *bad_seq =
+ * *bad_entry = -1, or PA_ERR_BAD_INDEX with the first offending sequence in
+ * *bad_seq and table entry in *bad_entry (-1 when the length itself is out
+ * of range).  Bad arguments: PA_ERR_INVALID_ARG. */
+int pa_validate_tables(const int32_t *tables, int batch, int max_blocks, const int32_t *seq_lens,
+                       int64_t num_blocks, int block_size, int *bad_seq, int *bad_entry);
 /* Reference count of a block (0 = free), or -1 for an id out of range. */
 int pa_block_refcount(const pa_allocator *alloc, int32_t block);
 

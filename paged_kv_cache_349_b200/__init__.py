@@ -16,6 +16,7 @@ A whole decode step from pinned host buffers:
     pa_decode_step_staging_size, DecodeStepHost (pa_decode_step_host[_fp8])
 Host allocator:
     Allocator (pa_alloc_* / pa_seq_* / pa_block_refcount; step_fn = pa_alloc_step)
+    validate_tables (pa_validate_tables: host-side check of decode tables)
 """
 from __future__ import annotations
 
@@ -387,6 +388,27 @@ def pa_decode_builtin_scratch(out, q, k_cache, v_cache, block_tables, seq_lens, 
 
 def _np_ptr(a: np.ndarray):
     return a.ctypes.data_as(ctypes.c_void_p)
+
+
+def validate_tables(tables: np.ndarray, seq_lens: np.ndarray, num_blocks: int, block_size: int):
+    """Host-side check of decode tables (``pa_validate_tables``).
+
+    Returns None when every attended entry is a block id in range, unrepeated within its row,
+    and every length fits its row; otherwise (bad_seq, bad_entry) of the first offence
+    (bad_entry -1: the length itself).
+    """
+    t = np.ascontiguousarray(tables, dtype=np.int32)
+    lens = np.ascontiguousarray(seq_lens, dtype=np.int32)
+    if t.ndim != 2 or lens.shape != (t.shape[0],):
+        raise ValueError("tables [B, max_blocks] and seq_lens [B] expected")
+    bs_, be = ctypes.c_int(), ctypes.c_int()
+    st = lib.pa_validate_tables(_np_ptr(t), t.shape[0], t.shape[1], _np_ptr(lens), int(num_blocks), int(block_size),
+                                ctypes.byref(bs_), ctypes.byref(be))
+    if st == PA_OK:
+        return None
+    if st == PA_ERR_BAD_INDEX:
+        return bs_.value, be.value
+    _check(st, "pa_validate_tables")
 
 
 class Allocator:

@@ -56,6 +56,7 @@ SIGNATURES = {
     "pa_alloc_export": (_I, [_P, _P, _I, _P, _I, ctypes.c_int32, _P]),
     "pa_alloc_step": (_I, [_P, _P, _I, _P, _I, ctypes.c_int32, _P, _P, _PI, _PI]),
     "pa_alloc_num_free": (_I, [_P]),
+    "pa_validate_tables": (_I, [_P, _I, _I, _P, _I64, _I, _PI, _PI]),
     "pa_block_refcount": (_I, [_P, ctypes.c_int32]),
 }
 

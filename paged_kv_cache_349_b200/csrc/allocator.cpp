@@ -284,6 +284,42 @@ int pa_alloc_export(const pa_allocator *alloc, const int32_t *seq_ids, int n, in
     return PA_OK;
 }
 
+int pa_validate_tables(const int32_t *tables, int batch, int max_blocks, const int32_t *seq_lens,
+                       int64_t num_blocks, int block_size, int *bad_seq, int *bad_entry) {
+    if (batch < 0 || max_blocks < 0 || num_blocks <= 0 || block_size <= 0 || !bad_seq || !bad_entry)
+        return PA_ERR_INVALID_ARG;
+    *bad_seq = -1;
+    *bad_entry = -1;
+    if (batch == 0) return PA_OK;
+    if (!tables || !seq_lens) return PA_ERR_INVALID_ARG;
+    // seen[id] == b + 1: block id already used by row b (a repeat within a row)
+    std::vector<int32_t> seen;
+    try {
+        seen.assign((size_t)num_blocks, 0);
+    } catch (...) {
+        return PA_ERR_OOM;
+    }
+    for (int b = 0; b < batch; ++b) {
+        const int64_t L = seq_lens[b];
+        if (L < 0 || L > (int64_t)max_blocks * block_size) {
+            *bad_seq = b;
+            return PA_ERR_BAD_INDEX;
+        }
+        const int64_t used = (L + block_size - 1) / block_size;
+        const int32_t *row = tables + (size_t)b * (size_t)max_blocks;
+        for (int64_t j = 0; j < used; ++j) {
+            const int32_t id = row[j];
+            if (id < 0 || id >= num_blocks || seen[(size_t)id] == b + 1) {
+                *bad_seq = b;
+                *bad_entry = (int)j;
+                return PA_ERR_BAD_INDEX;
+            }
+            seen[(size_t)id] = b + 1;
+        }
+    }
+    return PA_OK;
+}
+
 int pa_alloc_num_free(const pa_allocator *alloc) {
     return alloc ? (int)alloc->free_stack.size() : -1;
 }

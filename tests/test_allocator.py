@@ -296,3 +296,29 @@ def test_alloc_step_all_or_nothing():
     assert a.num_free() == 0
     assert [a.block_table(x)[1] for x in (s1, c, s2)] == [snap[0][1] + 14, snap[1][1] + 14, snap[2][1] + 14]
     a.close()
+
+
+def test_validate_tables_accepts_workloads_and_locates_corruption():
+    case = W.make_case(2, batch=6, max_len=300, num_blocks=256)
+    t, L, NB, bs = case.block_tables, case.seq_lens, case.num_blocks, case.block_size
+    assert pa.validate_tables(t, L, NB, bs) is None
+    chat = W.make_case(3, batch=8, max_len=260, num_blocks=512)  # rows share prefix blocks: allowed
+    assert pa.validate_tables(chat.block_tables, chat.seq_lens, chat.num_blocks, chat.block_size) is None
+    used = (L + bs - 1) // bs
+    b = int(np.argmax(used >= 2))
+    bad = t.copy()
+    bad[b, used[b] - 1] = NB                      # id out of range in the last attended entry
+    assert pa.validate_tables(bad, L, NB, bs) == (b, int(used[b]) - 1)
+    bad = t.copy()
+    bad[b, 1] = bad[b, 0]                         # a block twice in one row
+    assert pa.validate_tables(bad, L, NB, bs) == (b, 1)
+    bad = t.copy()
+    bad[b, 0] = -1                                # padding value where a block is needed
+    assert pa.validate_tables(bad, L, NB, bs) == (b, 0)
+    long_l = L.copy()
+    long_l[4] = t.shape[1] * bs + 1               # longer than its row can hold
+    assert pa.validate_tables(t, long_l, NB, bs) == (4, -1)
+    pad = t.copy()
+    pad[0, used[0]:] = -7                         # entries past the attended ones are never read
+    assert pa.validate_tables(pad, L, NB, bs) is None
+    assert pa.validate_tables(np.zeros((0, 4), np.int32), np.zeros(0, np.int32), NB, bs) is None
