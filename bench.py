@@ -257,7 +257,8 @@ def run_native(args):
     world, rank, local = _dist_setup()
     torch.cuda.set_device(local)
     cfg = args.config
-    seed = 1000 + cfg + 7919 * rank  # weak scaling: every rank owns its own batch
+    base = 1000 + cfg if args.seed is None else args.seed
+    seed = base + 7919 * rank  # weak scaling: every rank owns its own batch
     case = W.make_case(cfg, seed=seed, fill=W.BF16_ZERO, num_blocks=args.num_blocks)
     fp8 = args.kv_dtype == "fp8"
     copy_b, write_b, dec_b = step_bytes(case, 1 if fp8 else 2)
@@ -416,6 +417,7 @@ def run_native(args):
         "config": {
             "workload": WORKLOAD_NAMES[cfg],
             "config_index": cfg,
+            "seed": seed,
             "batch_per_gpu": case.batch,
             "global_batch": case.batch * world,
             "kv_tokens_per_gpu": kv_tokens,
@@ -595,7 +597,7 @@ def run_reference(args):
     if rank != 0:
         return
     cfg = args.config
-    case = W.make_case(cfg, fill=W.BF16_ZERO)
+    case = W.make_case(cfg, seed=1000 + cfg if args.seed is None else args.seed, fill=W.BF16_ZERO)
     per_step = max(1.0, args.cpu_budget / max(1, args.steps + args.warmup))
     for _ in range(args.warmup):
         cpu_baseline(case, budget_s=per_step / 4)
@@ -638,6 +640,7 @@ def main():
                     help="fp8: E4M3 pools quantised by the library (per-pool scales)")
     ap.add_argument("--unfused", action="store_true",
                     help="time pa_reshape_and_cache + pa_decode instead of the fused pa_decode_append")
+    ap.add_argument("--seed", type=int, default=None, help="input seed (default 1000 + config; + 7919 per rank)")
     ap.add_argument("--num-blocks", type=int, default=None,
                     help="pool size override (same decode launch, smaller pool: for profiler captures)")
     args = ap.parse_args()
