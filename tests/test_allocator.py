@@ -322,3 +322,28 @@ def test_validate_tables_accepts_workloads_and_locates_corruption():
     pad[0, used[0]:] = -7                         # entries past the attended ones are never read
     assert pa.validate_tables(pad, L, NB, bs) is None
     assert pa.validate_tables(np.zeros((0, 4), np.int32), np.zeros(0, np.int32), NB, bs) is None
+
+
+@pytest.mark.parametrize("cfg,kw", [
+    (2, dict(batch=6, max_len=300, num_blocks=256)),
+    (3, dict(batch=8, max_len=260, num_blocks=512)),
+    (5, dict(batch=2, max_len=2048, num_blocks=640, num_copy_pairs=0)),
+])
+def test_bench_e2e_host_state_matches_workload(cfg, kw):
+    """The bench's e2e leg rebuilds the pre-append state with the allocator and runs pa_alloc_step:
+    the step's lengths are the workload's, every table it exports is valid, and max_seq_len is the
+    longest length.  (Placement may differ from the generator's for a token that opens a block:
+    the allocator deals that block at step time.)"""
+    import bench
+    case = W.make_case(cfg, **kw)
+    alloc, sids = bench.replay_allocator(pa, case)
+    B, mb = case.batch, case.block_tables.shape[1]
+    tables = np.zeros((B, mb), np.int32)
+    lens = np.zeros(B, np.int32)
+    pairs = np.zeros((B, 2), np.int32)
+    n_pairs, max_len = alloc.step_fn(sids, tables, lens, pairs)()
+    assert np.array_equal(lens, case.seq_lens)
+    assert max_len == int(case.seq_lens.max())
+    assert pa.validate_tables(tables, lens, case.num_blocks, case.block_size) is None
+    assert n_pairs == 0  # copy-on-write already happened while the state was rebuilt
+    alloc.close()
