@@ -124,3 +124,20 @@ def test_fp8_host_step_rejects_bad_scales():
                                          _fake(), _fake(), 2, 64, 8, 2, 128, 16, 64, 0.1, ks, vs, -1, 0,
                                          _fake(0x100000), 1 << 20, None, None)
         assert rc == pa.PA_ERR_INVALID_ARG
+
+
+def test_header_is_c99_and_links(tmp_path):
+    """include/pa.h is a C header: a C99 program using it compiles, links against libpa.so and runs
+    (the program only calls pa_version; its decode-step function shows one serving-loop step)."""
+    import shutil
+    import subprocess
+    from paged_kv_cache_349_b200 import build as B
+    cc = shutil.which("gcc") or shutil.which("cc")
+    if cc is None:
+        pytest.skip("no C compiler")
+    exe = tmp_path / "c_abi_example"
+    lib_dir = os.path.dirname(B.LIB)
+    subprocess.check_call([cc, "-std=c99", "-Wall", "-Werror", "-pedantic", "-I", os.path.join(ROOT, "include"),
+                           os.path.join(ROOT, "tests", "csrc", "c_abi_example.c"), "-L", lib_dir, "-lpa",
+                           f"-Wl,-rpath,{lib_dir}", "-o", str(exe)])
+    assert subprocess.run([str(exe)]).returncode == 0
