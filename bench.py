@@ -2,20 +2,26 @@
 
 A step is the whole hot path for one batch: copy-on-write block copies,
 the cache write of each sequence's new token, and paged decode attention.
-Default workload: Llama-2-7B-shaped single-layer decode (64 sequences,
-32 q / 32 kv heads, head_dim 128, block size 16, lengths U{128..2048},
-16384-block pool, placement by a seeded permutation).
+The headline workload is the largest single-GPU one, the Llama-2-13B-shaped
+chat mix (128 sequences in 32 groups of n=4 samples sharing a 512-token
+prompt prefix, 40 q / 40 kv heads, head_dim 128, block size 16, 24576-block
+pool); its decode reads each group's shared tiles once
+(pa_decode_shared_prefix).  The same line carries a ``per_config`` entry for
+each other workload whose K/V exceeds L2 (Llama-2-7B-shaped, Llama-3-8B GQA,
+long-context split), each timed the same way.
 
 Prints one JSON line.  ``value`` is the step's algorithmic HBM bytes per
 second (inputs resident in HBM, timed on the device with CUDA events, max
-over ranks); ``e2e`` is the same metric measured through the public API
-with pinned host buffers (host allocator append, host->device copies of
-the step's inputs, the three launches, device->host read of the output).
+over ranks); the chat mix counts each shared K/V row once (the DRAM
+minimum), its logical bytes (every sequence's whole history) are reported
+beside.  ``e2e`` is the same metric measured through the public API with
+pinned host buffers (host allocator append, host->device upload of the
+step's inputs, copies, fused write + decode, output into host memory).
 ``roofline`` reports the decode call against the measured HBM copy peak;
-``cpu_baseline`` is the fp64 oracle timed on this host's cores on a
-bounded sample of the same workload.
+``cpu_baseline`` is the fp64 oracle timed on this host's cores on a bounded
+sample of the headline workload.
 
-    python bench.py [--gpus N] [--steps K] [--warmup W] [--config 1..5]
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--config 1..5] [--per-config 2,4,5]
     python bench.py --impl reference ...   (the oracle arm)
 """
 from __future__ import annotations
@@ -67,8 +73,9 @@ def _measured_peak():
         return FALLBACK_HBM_GBS, "fallback"
 
 
-def _decode_traffic_record(cfg: int, kv_dtype: str):
-    """ncu DRAM traffic of the decode call for this workload and KV dtype, if taken on the current device code."""
+def _decode_traffic_record(cfg: int, kv_dtype: str, kernel: str):
+    """ncu DRAM traffic of the decode call for this workload, KV dtype and entry point, if taken on the
+    current device code."""
     path = os.path.join(ROOT, "profiles", "decode_traffic.json")
     try:
         with open(path) as f:
@@ -77,7 +84,8 @@ def _decode_traffic_record(cfg: int, kv_dtype: str):
         return None
     digest = kernel_src_sha256()
     for rec in recs:
-        if rec.get("kernel_src_sha256") == digest and rec.get("config") == cfg and rec.get("kv_dtype") == kv_dtype:
+        if (rec.get("kernel_src_sha256") == digest and rec.get("config") == cfg and rec.get("kv_dtype") == kv_dtype
+                and rec.get("kernel", "").startswith(kernel)):
             return rec
     return None
 
@@ -249,19 +257,46 @@ def cpu_baseline(case, budget_s: float = 12.0):
 # native arm
 # ---------------------------------------------------------------------------
 
-def run_native(args):
+def unique_kv_rows(case) -> int:
+    """K/V rows (per kv head) a decode must read from DRAM at least: each physical block's rows
+    counted once, as many as the furthest-reaching sequence reads from it."""
+    bs = case.block_size
+    rows = {}
+    for b, L in enumerate(case.seq_lens):
+        L = int(L)
+        for j in range(-(-L // bs)):
+            blk = int(case.block_tables[b, j])
+            rows[blk] = max(rows.get(blk, 0), min(bs, L - j * bs))
+    return sum(rows.values())
+
+
+def decode_bytes(case, kv_elem_bytes: int, unique: bool) -> int:
+    """Algorithmic decode bytes; with ``unique`` the K/V part counts each shared row once."""
+    logical = W.algorithmic_decode_bytes(case, kv_elem_bytes=kv_elem_bytes)
+    if not unique:
+        return logical
+    kv_row = case.num_kv_heads * case.head_dim * kv_elem_bytes * 2
+    return logical - int(case.seq_lens.sum()) * kv_row + unique_kv_rows(case) * kv_row
+
+
+def measure_workload(cfg, args, world, rank, pa, headline):
+    """Time one workload's step (device-resident) and, unless disabled, its e2e step.
+
+    Returns the fields of one bench entry (the headline line or a per_config entry)."""
     import torch
 
-    import paged_kv_cache_349_b200 as pa
-
-    world, rank, local = _dist_setup()
-    torch.cuda.set_device(local)
-    cfg = args.config
     base = 1000 + cfg if args.seed is None else args.seed
     seed = base + 7919 * rank  # weak scaling: every rank owns its own batch
     case = W.make_case(cfg, seed=seed, fill=W.BF16_ZERO, num_blocks=args.num_blocks)
     fp8 = args.kv_dtype == "fp8"
-    copy_b, write_b, dec_b = step_bytes(case, 1 if fp8 else 2)
+    elem = 1 if fp8 else 2
+    # Shared-prefix groups (the n=4 chat mix): their shared tiles are read once per group.
+    prefix = case.groups is not None and args.decode != "plain" and not fp8 and not args.unfused
+    group_size = 4
+    copy_b, write_b, _ = step_bytes(case, elem)
+    shared_rows = case.groups is not None
+    dec_b = decode_bytes(case, elem, unique=shared_rows)
+    dec_logical = decode_bytes(case, elem, unique=False)
     total_b = copy_b + write_b + dec_b
     kv_tokens = int(case.seq_lens.sum())
 
@@ -301,52 +336,58 @@ def run_native(args):
     pt = case.partition_tokens
     resolved_pt = pa.pa_decode_partition_tokens(case.batch, case.num_q_heads, case.num_kv_heads,
                                                 case.head_dim, case.block_size, case.max_seq_len, pt)
-    ws_bytes = pa.pa_decode_workspace_size(case.batch, case.num_q_heads, case.num_kv_heads, case.head_dim,
+    ws_plain = pa.pa_decode_workspace_size(case.batch, case.num_q_heads, case.num_kv_heads, case.head_dim,
                                            case.block_size, case.max_seq_len, pt)
+    ws_bytes = ws_plain
+    prefix_lens = None
+    if prefix:
+        prefix_lens = i32(case.shared_tokens[::group_size])
+        ws_bytes = max(ws_bytes, pa.pa_decode_shared_prefix_workspace_size(
+            case.batch, group_size, case.num_q_heads, case.num_kv_heads, case.head_dim, case.block_size,
+            case.max_seq_len, pt))
     ws = torch.empty(max(ws_bytes, 16), dtype=torch.uint8, device="cuda")
     stream = torch.cuda.current_stream()
 
     dec_ev = []
 
-    def step_fp8(record):
-        if case.copy_pairs.shape[0]:
-            pa.pa_copy_blocks_fp8(k, v, pairs, err_flag=flag, stream=stream)
-        if other.size:
-            pa.pa_reshape_and_cache_fp8(k_other, v_other, k, v, slots_other, k_scale=k_scale, v_scale=v_scale,
-                                        err_flag=flag, stream=stream)
-        if record:
-            e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-            e0.record(stream)
-        pa.pa_decode_fp8(out, q, k, v, tables, lens, max_seq_len=case.max_seq_len, scale=float(case.scale),
-                         k_scale=k_scale, v_scale=v_scale, partition_tokens=pt, workspace=ws, err_flag=flag,
-                         stream=stream, k_new=k_last, v_new=v_last)
-        if record:
-            e1.record(stream)
-            dec_ev.append((e0, e1))
-
-    def step(record=False):
+    def decode_call(kind):
         if fp8:
-            return step_fp8(record)
-        if case.copy_pairs.shape[0]:
-            pa.pa_copy_blocks(k, v, pairs, err_flag=flag, stream=stream)
-        if fused:
-            if other.size:
-                pa.pa_reshape_and_cache(k_other, v_other, k, v, slots_other, err_flag=flag, stream=stream)
-        else:
-            pa.pa_reshape_and_cache(k_new, v_new, k, v, slots, err_flag=flag, stream=stream)
-        if record:
-            e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-            e0.record(stream)
-        if fused:
+            pa.pa_decode_fp8(out, q, k, v, tables, lens, max_seq_len=case.max_seq_len, scale=float(case.scale),
+                             k_scale=k_scale, v_scale=v_scale, partition_tokens=pt, workspace=ws, err_flag=flag,
+                             stream=stream, k_new=k_last, v_new=v_last)
+        elif kind == "shared-prefix":
+            pa.pa_decode_shared_prefix(out, q, k, v, tables, lens, prefix_lens, group_size=group_size,
+                                       max_seq_len=case.max_seq_len, scale=float(case.scale), partition_tokens=pt,
+                                       workspace=ws, err_flag=flag, stream=stream, k_new=k_last, v_new=v_last)
+        elif fused:
             pa.pa_decode_append(out, q, k_last, v_last, k, v, tables, lens, max_seq_len=case.max_seq_len,
                                 scale=float(case.scale), partition_tokens=pt, workspace=ws, err_flag=flag,
                                 stream=stream)
         else:
             pa.pa_decode(out, q, k, v, tables, lens, max_seq_len=case.max_seq_len, scale=float(case.scale),
                          partition_tokens=pt, workspace=ws, err_flag=flag, stream=stream)
+
+    kind_main = "shared-prefix" if prefix else "plain"
+
+    def step(record=False, kind=kind_main, evs=dec_ev):
+        if case.copy_pairs.shape[0]:
+            (pa.pa_copy_blocks_fp8 if fp8 else pa.pa_copy_blocks)(k, v, pairs, err_flag=flag, stream=stream)
+        if fused:
+            if other.size:
+                if fp8:
+                    pa.pa_reshape_and_cache_fp8(k_other, v_other, k, v, slots_other, k_scale=k_scale,
+                                                v_scale=v_scale, err_flag=flag, stream=stream)
+                else:
+                    pa.pa_reshape_and_cache(k_other, v_other, k, v, slots_other, err_flag=flag, stream=stream)
+        else:
+            pa.pa_reshape_and_cache(k_new, v_new, k, v, slots, err_flag=flag, stream=stream)
+        if record:
+            e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+            e0.record(stream)
+        decode_call(kind)
         if record:
             e1.record(stream)
-            dec_ev.append((e0, e1))
+            evs.append((e0, e1))
 
     for _ in range(args.warmup):
         step()
@@ -382,9 +423,21 @@ def run_native(args):
         clocks["untimed_load_steps_before_timing"] = load_steps
     ms_local = t0.elapsed_time(t1)
     ms = _max_over_ranks(ms_local, world)
-    dec_ms = statistics.mean(a.elapsed_time(b) for a, b in dec_ev)
-    dec_ms = _max_over_ranks(dec_ms, world)
+    dec_ms = _max_over_ranks(statistics.mean(a.elapsed_time(b) for a, b in dec_ev), world)
     assert int(flag.item()) == 0, f"error flag {int(flag.item()):#x}"
+
+    # The same step with the plain decode, for comparison (the chat mix only).
+    alt_ms = None
+    if prefix:
+        alt_ev = []
+        for _ in range(args.warmup):
+            step(kind="plain")
+        torch.cuda.synchronize()
+        for _ in range(args.steps):
+            step(record=True, kind="plain", evs=alt_ev)
+        torch.cuda.synchronize()
+        alt_ms = _max_over_ranks(statistics.mean(a.elapsed_time(b) for a, b in alt_ev), world)
+        assert int(flag.item()) == 0, f"error flag {int(flag.item()):#x}"
 
     all_bytes = _sum_over_ranks(float(total_b), world)
     all_tokens = _sum_over_ranks(float(kv_tokens), world)
@@ -397,35 +450,52 @@ def run_native(args):
     if not (args.no_e2e or args.unfused):
         e2e = run_e2e(args, case, pa, stream, world, k, v, (k_scale, v_scale) if fp8 else None)
 
-    rec = _decode_traffic_record(cfg, "fp8" if fp8 else "bf16")
+    kernel = ("pa_decode_append_fp8" if fp8 else "pa_decode_shared_prefix (fused write)" if prefix else
+              "pa_decode_append" if fused else "pa_decode")
+    rec = _decode_traffic_record(cfg, "fp8" if fp8 else "bf16", kernel)
     traffic = rec.get("traffic_bytes_per_launch") if rec else None
+    split = prefix or resolved_pt > 0
+    roof = {
+        "kernel": kernel + (" (split, merged in-kernel)" if split else " (single pass)"),
+        "bound": "hbm",
+        "achieved": round(achieved, 1),
+        "peak": peak,
+        "peak_kind": f"{peak_kind} (HBM copy)",
+        "unit": "GB/s",
+        "frac": round(achieved / peak, 4),
+        "traffic": traffic,
+        "algorithmic_bytes_per_launch": dec_b,
+        "launch_ms": round(dec_ms, 5),
+    }
+    if shared_rows:
+        roof["algorithmic_bytes_note"] = ("each shared K/V row counted once (DRAM minimum); logical bytes count "
+                                          "it once per sequence")
+        roof["logical_bytes_per_launch"] = dec_logical
+        roof["logical_gbps"] = round(dec_logical / (dec_ms / 1e3) / 1e9, 1)
+        if traffic:
+            roof["traffic_vs_unique"] = round(traffic / dec_b, 4)
+            roof["traffic_vs_logical"] = round(traffic / dec_logical, 4)
+    if alt_ms is not None:
+        roof["plain_decode_launch_ms"] = round(alt_ms, 5)
+        roof["plain_decode_achieved"] = round(dec_b / (alt_ms / 1e3) / 1e9, 1)
 
-    line = {
-        "metric": METRIC,
+    entry = {
         "value": round(value, 1),
         "unit": "GB/s",
-        "n_gpus": world,
-        "steps": args.steps,
-        "warmup": args.warmup,
         "ms_per_step": round(ms / args.steps, 4),
-        "higher_is_better": True,
-        "scaling": "weak",
-        "vs_baseline": None,
-        "dtype": "bf16" if not fp8 else "e4m3 K/V (f16 mma), bf16 q",
-        "accumulate": "fp32",
-        "data": "synthetic (seeded bf16 N(0,1) K/V/q, seeded placement)",
         "config": {
             "workload": WORKLOAD_NAMES[cfg],
             "config_index": cfg,
-            "seed": seed,
+            "seed": base,
             "batch_per_gpu": case.batch,
             "global_batch": case.batch * world,
-            "kv_tokens_per_gpu": kv_tokens,
-            "partition_tokens": resolved_pt,
+            "partition_tokens": case.partition_tokens,
             "parallelism": f"dp{world} (independent sequences per GPU, no collective)",
             "l2": f"inputs larger than L2: {dec_b / 1e9:.2f} GB of K/V per step vs 126 MB L2; no flush",
             "step": ("block copies, then pa_decode_append_fp8 (the write quantises to E4M3 and is fused into decode)"
                      if fp8 else
+                     "block copies, cache write of copy-on-write rows, then pa_decode_shared_prefix (each group's "
+                     "shared tiles read once; cache write of each sequence's new token fused)" if prefix else
                      "block copies, then pa_decode_append (cache write fused into decode)" if fused else
                      "block copies, pa_reshape_and_cache, pa_decode"),
         },
@@ -433,30 +503,56 @@ def run_native(args):
                         f"{peak_kind}_{peak:.0f}GBps": round(100 * value / peak, 1)},
         "kv_tokens_per_s": round(all_tokens / step_s, 1),
         "kv_head_tokens_per_s": round(all_tokens * case.num_kv_heads / step_s, 1),
+        "kv_tokens_per_gpu": kv_tokens,
+        "decode_partition_tokens": resolved_pt,
         "step_bytes": {"copy": copy_b, "write": write_b, "decode": dec_b},
         "gpu_launches": launches,
-        "roofline": {
-            "kernel": ("pa_decode_append_fp8" if fp8 else "pa_decode_append" if fused else "pa_decode") +
-                      (" (split kernel + LSE reduce)" if resolved_pt > 0 else " (single pass)"),
-            "bound": "hbm",
-            "achieved": round(achieved, 1),
-            "peak": peak,
-            "peak_kind": f"{peak_kind} (HBM copy)",
-            "unit": "GB/s",
-            "frac": round(achieved / peak, 4),
-            "traffic": traffic,
-            "algorithmic_bytes_per_launch": dec_b,
-            "launch_ms": round(dec_ms, 5),
-        },
+        "roofline": roof,
         "e2e": e2e,
         "clocks": clocks,
     }
     if fp8:
-        line["config"]["kv_scales"] = {"k": k_scale, "v": v_scale}
-    if rank == 0 and world == 1 and not args.no_cpu_baseline and not fp8:
+        entry["config"]["kv_scales"] = {"k": k_scale, "v": v_scale}
+    cpu = None
+    if headline and rank == 0 and world == 1 and not args.no_cpu_baseline and not fp8:
         gbs, cores, sample, _, _ = cpu_baseline(case, budget_s=args.cpu_budget)
-        line["cpu_baseline"] = {"value": round(gbs, 4), "unit": "GB/s", "cores": cores, "kind": "oracle",
-                                "sample": sample}
+        cpu = {"value": round(gbs, 4), "unit": "GB/s", "cores": cores, "kind": "oracle", "sample": sample}
+    del k, v, q, ws
+    torch.cuda.synchronize()
+    torch.cuda.empty_cache()
+    return entry, cpu
+
+
+def run_native(args):
+    import paged_kv_cache_349_b200 as pa
+
+    world, rank, local = _dist_setup()
+    head, cpu = measure_workload(args.config, args, world, rank, pa, headline=True)
+    per = {}
+    for cfg in args.per_config:
+        if cfg != args.config:
+            e, _ = measure_workload(cfg, args, world, rank, pa, headline=False)
+            per[str(cfg)] = e
+    line = {
+        "metric": METRIC,
+        "value": head["value"],
+        "unit": "GB/s",
+        "n_gpus": world,
+        "steps": args.steps,
+        "warmup": args.warmup,
+        "ms_per_step": head["ms_per_step"],
+        "higher_is_better": True,
+        "scaling": "weak",
+        "vs_baseline": None,
+        "dtype": "bf16" if args.kv_dtype == "bf16" else "e4m3 K/V (f16 mma), bf16 q",
+        "accumulate": "fp32",
+        "data": "synthetic (seeded bf16 N(0,1) K/V/q, seeded placement)",
+    }
+    line.update({k: v for k, v in head.items() if k not in ("value", "unit", "ms_per_step")})
+    if cpu is not None:
+        line["cpu_baseline"] = cpu
+    if per:
+        line["per_config"] = per
     if rank == 0:
         print(json.dumps(line), flush=True)
     if world > 1:
@@ -591,13 +687,33 @@ def step_bytes_from(case, lens, n_pairs, kv_elem_bytes: int = 2):
 # reference arm: the fp64 oracle on the host cores
 # ---------------------------------------------------------------------------
 
+def reference_config(case, cfg, base, world):
+    """The reference arm's ``config``: the same keys and values as the native arm's headline."""
+    prefix = case.groups is not None
+    dec_b = decode_bytes(case, 2, unique=prefix)
+    return {
+        "workload": WORKLOAD_NAMES[cfg],
+        "config_index": cfg,
+        "seed": base,
+        "batch_per_gpu": case.batch,
+        "global_batch": case.batch * world,
+        "partition_tokens": case.partition_tokens,
+        "parallelism": f"dp{world} (independent sequences per GPU, no collective)",
+        "l2": f"inputs larger than L2: {dec_b / 1e9:.2f} GB of K/V per step vs 126 MB L2; no flush",
+        "step": ("block copies, cache write of copy-on-write rows, then pa_decode_shared_prefix (each group's "
+                 "shared tiles read once; cache write of each sequence's new token fused)" if prefix else
+                 "block copies, then pa_decode_append (cache write fused into decode)"),
+    }
+
+
 def run_reference(args):
     world = int(os.environ.get("WORLD_SIZE", "1"))
     rank = int(os.environ.get("RANK", "0"))
     if rank != 0:
         return
     cfg = args.config
-    case = W.make_case(cfg, seed=1000 + cfg if args.seed is None else args.seed, fill=W.BF16_ZERO)
+    base = 1000 + cfg if args.seed is None else args.seed
+    case = W.make_case(cfg, seed=base, fill=W.BF16_ZERO)
     per_step = max(1.0, args.cpu_budget / max(1, args.steps + args.warmup))
     for _ in range(args.warmup):
         cpu_baseline(case, budget_s=per_step / 4)
@@ -615,7 +731,7 @@ def run_reference(args):
         "steps": args.steps, "warmup": args.warmup, "ms_per_step": round(secs * 1e3 / args.steps, 2),
         "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64",
         "data": "synthetic (seeded bf16 N(0,1) K/V/q, seeded placement)",
-        "config": {"workload": WORKLOAD_NAMES[cfg], "config_index": cfg, "batch_per_gpu": case.batch},
+        "config": reference_config(case, cfg, base, world),
         "impl": "reference",
         "cpu_baseline": {"value": round(value, 4), "unit": "GB/s", "cores": cores, "kind": "oracle",
                          "sample": "per step: " + sample},
@@ -629,7 +745,13 @@ def main():
     ap.add_argument("--gpus", type=int, default=1)
     ap.add_argument("--steps", type=int, default=20)
     ap.add_argument("--warmup", type=int, default=5)
-    ap.add_argument("--config", type=int, default=2, choices=[1, 2, 3, 4, 5])
+    ap.add_argument("--config", type=int, default=3, choices=[1, 2, 3, 4, 5],
+                    help="headline workload (default 3, the chat mix: the largest single-GPU workload)")
+    ap.add_argument("--per-config", type=str, default=None,
+                    help="comma-separated workloads timed after the headline into per_config "
+                         "(default: 2,4,5 when --config is left at its default, none otherwise)")
+    ap.add_argument("--decode", choices=["auto", "plain"], default="auto",
+                    help="plain: the chat mix decodes with pa_decode_append instead of the shared-prefix decode")
     ap.add_argument("--impl", choices=["native", "reference"], default="native")
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--step-chunks", type=int, default=0,
@@ -644,6 +766,11 @@ def main():
     ap.add_argument("--num-blocks", type=int, default=None,
                     help="pool size override (same decode launch, smaller pool: for profiler captures)")
     args = ap.parse_args()
+    explicit = any(a == "--config" or a.startswith("--config=") for a in sys.argv[1:])
+    if args.per_config is None:
+        args.per_config = [] if explicit else [2, 4, 5]
+    else:
+        args.per_config = [int(x) for x in args.per_config.split(",") if x.strip()]
     if args.warmup < 3:
         ap.error("--warmup must be at least 3")
     world = int(os.environ.get("WORLD_SIZE", "1"))

@@ -164,13 +164,25 @@ int pa_swap_blocks(void *dst_k_cache, void *dst_v_cache, int64_t dst_num_blocks,
  * scale         : softmax scale (usually 1/sqrt(head_dim))
  * partition_tokens : 0 = library default for this shape, -1 = one pass per
  *                 (sequence, kv head), > 0 = split each sequence into
- *                 partitions of this many tokens (a multiple of block_size)
- *                 whose partial softmax states are merged by a second
- *                 log-sum-exp reduce kernel.
+ *                 partitions of this many tokens (a multiple of block_size).
+ *                 Each partition stores its partial softmax state (max, sum,
+ *                 normalised output) in the workspace; the CTA whose
+ *                 partition of a (sequence, kv head) finishes last merges
+ *                 them (log-sum-exp) and writes the output, inside the same
+ *                 launch.  A sequence that fits one partition is written
+ *                 directly.
  * workspace     : device scratch of at least pa_decode_workspace_size(...)
  *                 bytes, 16-byte aligned (may be NULL if that size is 0).
+ *                 Its contents need no initialisation: the arrival counters
+ *                 it holds carry a per-call tag, so whatever an earlier call
+ *                 (or uninitialised memory) left there reads as zero.  Calls
+ *                 that run at the same time need separate workspaces.
  * Each (sequence, kv head) is processed by one CTA (per partition) that
  * serves all query heads of the group, so every K/V byte is read once.
+ * Launches exactly one kernel (none when batch == 0).  Shared-prefix
+ * locality: the grid runs the kv heads and partitions of a sequence next to
+ * each other with the sequence index slowest, so sequences that follow each
+ * other in the batch and share blocks (forks) re-read those blocks from L2.
  * ---------------------------------------------------------------------- */
 size_t pa_decode_workspace_size(int batch, int num_q_heads, int num_kv_heads, int head_dim,
                                 int block_size, int max_seq_len, int partition_tokens);
@@ -208,6 +220,55 @@ int pa_decode_append(float *out, const void *q, const void *k_new, const void *v
                      int num_kv_heads, int head_dim, int block_size, int64_t num_blocks, float scale,
                      int partition_tokens, void *workspace, size_t workspace_bytes, int32_t *err_flag,
                      void *stream);
+
+/* ------------------------------------------------------------------------
+ * Shared-prefix decode.  "PagedAttention & vLLM", Copy-on-write sharing:
+ * n samples of one prompt keep the prompt's KV in one set of physical
+ * blocks ("one copy, not four"); "What is PagedAttention and how does it
+ * manage KV cache", Concrete example: requests sharing a system prompt
+ * allocate its blocks once.  This call turns that shared storage into shared
+ * reads: the shared tokens of a group are read from HBM once per kv head for
+ * all of its members, instead of once per member.
+ *
+ * Computes exactly what pa_decode computes (pa_decode_append when k_new and
+ * v_new are given), for batches laid out in groups: sequences
+ * [g*group_size, (g+1)*group_size) form group g (the last group may be
+ * shorter), and for every member b of group g the K/V rows of positions
+ * p < prefix_lens[g] must equal those of the group's first member (the same
+ * physical blocks, as after pa_seq_fork, or copies of them, as after a
+ * copy-on-write).  Per group, the shared range actually used is
+ *     S_g = min(prefix_lens[g], L_b - 1 over members b), rounded down to a
+ *           multiple of 16 tokens (0 for groups of one sequence),
+ * so the token appended in this step is never read through another member's
+ * table.  The rows of [0, S_g) are read once per kv head through the first
+ * member's block table and combined with each member's query heads (up to
+ * 8 / (num_q_heads / num_kv_heads) members per read); each member's own
+ * rows [S_g, L_b) are read through its own table, and the two partial
+ * softmax states are merged as in the split decode.  prefix_lens[g] = 0
+ * means group g shares nothing; prefix_lens[g] < 0 sets PA_FLAG_BAD_LEN and
+ * is read as 0.
+ *
+ * prefix_lens : device int32 [ceil(batch / group_size)]
+ * group_size  : 1 .. 64
+ * k_new, v_new: both NULL (no cache write) or both device bf16
+ *               [batch, num_kv_heads, head_dim] as in pa_decode_append.
+ * partition_tokens: as pa_decode, except that -1 (and a default that would
+ *               not split) means one work item for the shared range and one
+ *               for each member's own range.
+ * workspace   : at least pa_decode_shared_prefix_workspace_size(...) bytes,
+ *               16-byte aligned, no initialisation needed (as pa_decode).
+ * Other arguments, layouts and errors: as pa_decode / pa_decode_append.
+ * ---------------------------------------------------------------------- */
+size_t pa_decode_shared_prefix_workspace_size(int batch, int group_size, int num_q_heads, int num_kv_heads,
+                                              int head_dim, int block_size, int max_seq_len,
+                                              int partition_tokens);
+
+int pa_decode_shared_prefix(float *out, const void *q, const void *k_new, const void *v_new, void *k_cache,
+                            void *v_cache, const int32_t *block_tables, int max_blocks_per_seq,
+                            const int32_t *seq_lens, const int32_t *prefix_lens, int group_size, int batch,
+                            int max_seq_len, int num_q_heads, int num_kv_heads, int head_dim, int block_size,
+                            int64_t num_blocks, float scale, int partition_tokens, void *workspace,
+                            size_t workspace_bytes, int32_t *err_flag, void *stream);
 
 /* ------------------------------------------------------------------------
  * One decode step from host buffers.  Enqueues, in order:
@@ -300,20 +361,26 @@ int pa_decode_step_host_fp8(float *out_host, const void *q_host, const void *k_n
  * device array owned by the library instead of a caller workspace.
  *
  *  - The array is a file-scope device variable of
- *    PA_DECODE_BUILTIN_SCRATCH_BYTES bytes.  Every GPU on which the library
- *    is loaded holds it until the process exits.
- *  - The first call on each device looks up the array's device address
- *    (cudaGetSymbolAddress) with that device current.  Make that first call
- *    before any stream capture.
+ *    PA_DECODE_BUILTIN_SCRATCH_BYTES bytes.  The CUDA driver reserves it
+ *    when the library's decode module is loaded on a device, which (with
+ *    lazy module loading, the CUDA 12 default) may be this entry point's
+ *    first call there; if that reservation fails the call returns
+ *    PA_ERR_CUDA.  The device then holds the array until the process exits.
+ *  - Every call looks up the array's device address (cudaGetSymbolAddress)
+ *    with the current device, so a context that was reset and rebuilt gets
+ *    the new address.  Make the first call on a device before any stream
+ *    capture, since it may load the module.
  *  - If the split this call would use needs more scratch than
  *    PA_DECODE_BUILTIN_SCRATCH_BYTES (see pa_decode_workspace_size), the
  *    call returns PA_ERR_UNSUPPORTED and launches nothing.
  *  - No cudaMalloc, cudaFree or other allocating routine is called.
  *  - All calls share the one array, and it keeps whatever the last call
  *    wrote.  Nothing in it has to start at zero: each partition's state is
- *    written before it is read within the same call.  Calls whose kernels
- *    can overlap on the GPU (different streams, or several host threads)
- *    race on the array; issue them on one stream.
+ *    written before it is read within the same call, and the arrival
+ *    counters carry a per-call tag.  Calls queued one after another on one
+ *    stream are safe.  Calls whose kernels can overlap on the GPU (different
+ *    streams, or several host threads) race on the array; issue them on one
+ *    stream.
  * Other arguments, layouts and errors: as pa_decode.
  * ---------------------------------------------------------------------- */
 #define PA_DECODE_BUILTIN_SCRATCH_BYTES ((size_t)32 << 20)
@@ -396,7 +463,10 @@ int pa_decode_append_fp8(float *out, const void *q, const void *k_new, const voi
  * ---------------------------------------------------------------------- */
 typedef struct pa_allocator pa_allocator;
 
-/* Pool of num_blocks blocks handed out in id order 0, 1, 2, ... */
+/* Pool of num_blocks blocks handed out in id order 0, 1, 2, ...
+ * block_size must be one the kernels address (8, 16, 32 or 64; else
+ * PA_ERR_UNSUPPORTED), and every slot id must fit int32:
+ * num_blocks * block_size <= INT32_MAX (else PA_ERR_INVALID_ARG). */
 int pa_alloc_create(int num_blocks, int block_size, pa_allocator **out);
 /* Same, but fresh blocks are handed out in the order order[0], order[1], ...
  * (order must be a permutation of 0..num_blocks-1; host memory, copied). */

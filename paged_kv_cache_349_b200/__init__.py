@@ -7,7 +7,8 @@ status.  All device work runs in the library's CUDA kernels.
 
 Device ops on bf16 pools (names as in the C ABI):
     pa_reshape_and_cache, pa_copy_blocks, pa_swap_blocks, pa_decode,
-    pa_decode_append, pa_decode_builtin_scratch, pa_decode_workspace_size,
+    pa_decode_append, pa_decode_shared_prefix, pa_decode_builtin_scratch,
+    pa_decode_workspace_size, pa_decode_shared_prefix_workspace_size,
     pa_decode_partition_tokens
 Device ops on fp8 (E4M3) pools:
     pa_quantize_fp8, pa_reshape_and_cache_fp8, pa_copy_blocks_fp8,
@@ -223,6 +224,48 @@ def pa_decode_append(out, q, k_new, v_new, k_cache, v_cache, block_tables, seq_l
         _dev(seq_lens, torch.int32, "seq_lens"), B, int(max_seq_len), Hq, Hkv, d, bs, NB,
         float(scale), int(partition_tokens), ws_ptr, ws_bytes, _opt_flag(err_flag),
         _stream(stream)), "pa_decode_append")
+
+
+def pa_decode_shared_prefix_workspace_size(batch, group_size, num_q_heads, num_kv_heads, head_dim, block_size,
+                                           max_seq_len, partition_tokens=0) -> int:
+    return int(lib.pa_decode_shared_prefix_workspace_size(batch, group_size, num_q_heads, num_kv_heads, head_dim,
+                                                          block_size, max_seq_len, partition_tokens))
+
+
+def pa_decode_shared_prefix(out, q, k_cache, v_cache, block_tables, seq_lens, prefix_lens, *, group_size: int,
+                            max_seq_len: int, scale: float, partition_tokens: int = 0, workspace=None,
+                            err_flag=None, stream=None, k_new=None, v_new=None) -> None:
+    """Decode of a batch laid out in groups of ``group_size`` sequences whose first
+    ``prefix_lens[g]`` tokens (int32 device tensor, one entry per group) hold the same
+    K/V: the shared tiles are read once per group and kv head.  With k_new/v_new
+    (bf16 [B, Hkv, d]) each sequence's new token is written first, as pa_decode_append."""
+    torch = _torch()
+    B, Hq, d = q.shape
+    NB, Hkv, bs, d2 = k_cache.shape
+    if d2 != d or out.shape != q.shape or v_cache.shape != k_cache.shape:
+        raise ValueError("shape mismatch")
+    if block_tables.dim() != 2 or block_tables.shape[0] != B or seq_lens.numel() != B:
+        raise ValueError("block_tables must be [B, max_blocks] and seq_lens [B]")
+    if group_size < 1 or prefix_lens.numel() != -(-B // group_size):
+        raise ValueError("prefix_lens must hold one entry per group of group_size sequences")
+    if (k_new is None) != (v_new is None):
+        raise ValueError("pass both k_new and v_new, or neither")
+    new = (None, None)
+    if k_new is not None:
+        if tuple(k_new.shape) != (B, Hkv, d) or v_new.shape != k_new.shape:
+            raise ValueError("k_new/v_new must be [B, Hkv, d]")
+        new = (_dev(k_new, torch.bfloat16, "k_new"), _dev(v_new, torch.bfloat16, "v_new"))
+    ws_ptr, ws_bytes = None, 0
+    if workspace is not None:
+        ws_ptr = _dev(workspace, workspace.dtype, "workspace")
+        ws_bytes = workspace.numel() * workspace.element_size()
+    _check(lib.pa_decode_shared_prefix(
+        _dev(out, torch.float32, "out"), _dev(q, torch.bfloat16, "q"), *new,
+        _dev(k_cache, torch.bfloat16, "k_cache"), _dev(v_cache, torch.bfloat16, "v_cache"),
+        _dev(block_tables, torch.int32, "block_tables"), block_tables.shape[1],
+        _dev(seq_lens, torch.int32, "seq_lens"), _dev(prefix_lens, torch.int32, "prefix_lens"), int(group_size),
+        B, int(max_seq_len), Hq, Hkv, d, bs, NB, float(scale), int(partition_tokens), ws_ptr, ws_bytes,
+        _opt_flag(err_flag), _stream(stream)), "pa_decode_shared_prefix")
 
 
 def pa_decode_step_staging_size(batch, max_blocks_per_seq, max_copy_pairs, num_q_heads, num_kv_heads, head_dim,

@@ -35,6 +35,9 @@ SIGNATURES = {
                                  _I, _I, _P, _SZ, _P, _P]),
     "pa_decode_step_host_fp8": (_I, [_P, _P, _P, _P, _P, _I, _P, _P, _I, _I, _P, _P, _I, _I, _I, _I, _I, _I, _I64,
                                      _F, _F, _F, _I, _I, _P, _SZ, _P, _P]),
+    "pa_decode_shared_prefix_workspace_size": (_SZ, [_I, _I, _I, _I, _I, _I, _I, _I]),
+    "pa_decode_shared_prefix": (_I, [_P, _P, _P, _P, _P, _P, _P, _I, _P, _P, _I, _I, _I, _I, _I, _I, _I, _I64, _F,
+                                     _I, _P, _SZ, _P, _P]),
     "pa_decode_builtin_scratch": (_I, [_P, _P, _P, _P, _P, _I, _P, _I, _I, _I, _I, _I, _I, _I64, _F, _I, _P, _P]),
     "pa_quantize_fp8": (_I, [_P, _P, _I64, _F, _P]),
     "pa_reshape_and_cache_fp8": (_I, [_P, _P, _P, _P, _P, _I, _I64, _I, _I, _I, _F, _F, _P, _P]),

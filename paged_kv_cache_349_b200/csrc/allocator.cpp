@@ -138,6 +138,10 @@ int pa_alloc_create_ordered(int num_blocks, int block_size, const int32_t *order
                             pa_allocator **out) {
     if (!out || num_blocks <= 0 || block_size <= 0) return PA_ERR_INVALID_ARG;
     *out = nullptr;
+    // Block sizes the kernels address (8, 16, 32, 64 tokens).
+    if (block_size != 8 && block_size != 16 && block_size != 32 && block_size != 64) return PA_ERR_UNSUPPORTED;
+    // A slot is block * block_size + row in int32: every slot of the pool must fit.
+    if ((int64_t)num_blocks * block_size > (int64_t)INT32_MAX) return PA_ERR_INVALID_ARG;
     pa_allocator *a = new (std::nothrow) pa_allocator();
     if (!a) return PA_ERR_OOM;
     a->num_blocks = num_blocks;

@@ -1,7 +1,10 @@
 // Host side of the paged decode: tensor maps of the pools, the choice of
-// partitioning, the launches of the decode and reduce kernels (the device
+// partitioning, the split workspace layout, the decode launches (the device
 // code is in decode_kernels.cuh) and the C entry points.
+#include <atomic>
+#include <chrono>
 #include <mutex>
+#include <random>
 
 #include "decode_kernels.cuh"
 
@@ -93,11 +96,11 @@ int resolve_partition(int batch, int num_kv_heads, int block_size, int max_seq_l
     return kDefaultPartition;
 }
 
-template <int HEAD_DIM, bool SPLIT, bool APPEND, bool FP8>
-int launch_decode(const CUtensorMap &km, const CUtensorMap &vm, const DecodeParams &p, int batch,
+template <int HEAD_DIM, bool SPLIT, bool APPEND, bool FP8, bool PREFIX>
+int launch_decode(const CUtensorMap &km, const CUtensorMap &vm, const DecodeParams &p, int grid_z,
                   cudaStream_t stream) {
     using C = Cfg<HEAD_DIM, FP8>;
-    auto kern = paged_decode_kernel<HEAD_DIM, SPLIT, APPEND, FP8>;
+    auto kern = paged_decode_kernel<HEAD_DIM, SPLIT, APPEND, FP8, PREFIX>;
     {
         // The shared-memory opt-in belongs to the kernel as loaded on one device:
         // set it once per device.
@@ -113,24 +116,53 @@ int launch_decode(const CUtensorMap &km, const CUtensorMap &vm, const DecodePara
             done[dev] = true;
         }
     }
-    dim3 grid((unsigned)p.num_parts, (unsigned)p.num_kv_heads, (unsigned)batch);
+    // B (or the item index) is the slowest grid dimension: the kv heads and
+    // partitions of one sequence -- and with prefix groups the shared items and
+    // then the members of a group -- are launched next to each other, so rows
+    // several CTAs read (shared prefix blocks) are still in L2 when the later
+    // ones reach them.
+    dim3 grid((unsigned)p.num_parts, (unsigned)p.num_kv_heads, (unsigned)grid_z);
     kern<<<grid, kThreads, C::kSmemBytes, stream>>>(km, vm, p);
     count_launch();
-    int st = launch_status();
-    if (st != PA_OK || !SPLIT) return st;
-    cudaLaunchConfig_t cfg = {};
-    cfg.gridDim = dim3((unsigned)p.num_q_heads, (unsigned)batch);
-    cfg.blockDim = dim3(kReduceThreads);
-    cfg.dynamicSmemBytes = 0;
-    cfg.stream = stream;
-    cudaLaunchAttribute attr[1];
-    attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
-    attr[0].val.programmaticStreamSerializationAllowed = 1;
-    cfg.attrs = attr;
-    cfg.numAttrs = 1;
-    const cudaError_t e = cudaLaunchKernelEx(&cfg, lse_reduce_kernel<HEAD_DIM>, p);
-    count_launch();
-    return e == cudaSuccess ? launch_status() : PA_ERR_CUDA;
+    return launch_status();
+}
+
+// Tag of one split call in the arrival tickets: a process-wide counter that
+// starts at a random value (so a workspace left over by another process does
+// not share tags with this one) and skips 0.
+unsigned int next_epoch() {
+    static std::atomic<unsigned int> ctr{[] {
+        std::random_device rd;
+        return (unsigned int)rd() ^ (unsigned int)std::chrono::steady_clock::now().time_since_epoch().count();
+    }()};
+    unsigned int e = ctr.fetch_add(1u);
+    while (e == 0u) e = ctr.fetch_add(1u);
+    return e;
+}
+
+// Split workspace: partial states part_o [B, Hq, slots, d] and part_ml
+// [B, Hq, slots, 2] (fp32), then the tickets [B, Hkv] (uint64); each section
+// 256-byte aligned.
+struct SplitLayout {
+    size_t o, ml, tickets, total;
+};
+
+SplitLayout split_layout(int64_t batch, int num_q_heads, int num_kv_heads, int head_dim, int64_t slots) {
+    auto up = [](int64_t x) { return (size_t)((x + 255) / 256 * 256); };
+    const int64_t rows = batch * num_q_heads * slots;
+    SplitLayout l{};
+    l.o = 0;
+    l.ml = up(rows * head_dim * 4);
+    l.tickets = l.ml + up(rows * 2 * 4);
+    l.total = l.tickets + (size_t)(batch * num_kv_heads * 8);
+    return l;
+}
+
+// Partial-state slots per row: one per partition, twice that with prefix groups
+// (the shared items' partitions, then the sequence's own).  pt = -1: one each.
+int64_t split_slots(int max_seq_len, int pt, bool prefix) {
+    const int64_t parts = pt > 0 ? ((int64_t)max_seq_len + pt - 1) / pt : 1;
+    return prefix ? 2 * parts : parts;
 }
 
 }  // namespace
@@ -140,43 +172,39 @@ int launch_decode(const CUtensorMap &km, const CUtensorMap &vm, const DecodePara
 // device address that cudaGetSymbolAddress returns for the current device.
 static __device__ __align__(256) unsigned char g_builtin_scratch[PA_DECODE_BUILTIN_SCRATCH_BYTES];
 
-// Device address of the scratch array on the current device, looked up once
-// per device (the first call on a device does the lookup).
+// Device address of the scratch array in the current device's context.  It is
+// looked up on every call (a host-side lookup once the module is loaded), so a
+// context that was torn down and rebuilt never gets a stale address.
 int builtin_scratch_address(void **out) {
-    static std::mutex mu;
-    static void *addr[64] = {};
-    int dev = 0;
-    if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) return PA_ERR_CUDA;
-    std::lock_guard<std::mutex> lock(mu);
-    if (!addr[dev]) {
-        void *p = nullptr;
-        if (cudaGetSymbolAddress(&p, g_builtin_scratch) != cudaSuccess || p == nullptr) return PA_ERR_CUDA;
-        addr[dev] = p;
-    }
-    *out = addr[dev];
+    void *p = nullptr;
+    if (cudaGetSymbolAddress(&p, g_builtin_scratch) != cudaSuccess || p == nullptr) return PA_ERR_CUDA;
+    *out = p;
     return PA_OK;
 }
 
-template <bool SPLIT, bool APPEND, bool FP8>
-int launch_decode_d(int head_dim, const CUtensorMap &km, const CUtensorMap &vm, const DecodeParams &p, int batch,
+template <bool SPLIT, bool APPEND, bool FP8, bool PREFIX = false>
+int launch_decode_d(int head_dim, const CUtensorMap &km, const CUtensorMap &vm, const DecodeParams &p, int grid_z,
                     cudaStream_t s) {
-    return head_dim == 128 ? launch_decode<128, SPLIT, APPEND, FP8>(km, vm, p, batch, s)
-                           : launch_decode<64, SPLIT, APPEND, FP8>(km, vm, p, batch, s);
+    return head_dim == 128 ? launch_decode<128, SPLIT, APPEND, FP8, PREFIX>(km, vm, p, grid_z, s)
+                           : launch_decode<64, SPLIT, APPEND, FP8, PREFIX>(km, vm, p, grid_z, s);
 }
 
 // Shared body of every decode entry point (k_new == nullptr: no cache write;
-// fp8: E4M3 pools dequantised with k_scale / v_scale).
+// fp8: E4M3 pools dequantised with k_scale / v_scale; prefix_lens != nullptr:
+// groups of group_size sequences read their shared prefix once).
 int decode_impl(float *out, const void *q, const void *k_new, const void *v_new, const void *k_cache,
                 const void *v_cache, const int32_t *block_tables, int max_blocks_per_seq,
                 const int32_t *seq_lens, int batch, int max_seq_len, int num_q_heads, int num_kv_heads,
                 int head_dim, int block_size, int64_t num_blocks, float scale, int partition_tokens,
                 void *workspace, size_t workspace_bytes, int32_t *err_flag, void *stream, bool fp8,
-                float k_scale, float v_scale) {
+                float k_scale, float v_scale, const int32_t *prefix_lens, int group_size) {
     const bool append = k_new != nullptr;
+    const bool prefix = prefix_lens != nullptr;
     if (fp8 && !(k_scale > 0.f && v_scale > 0.f && k_scale < 3.0e38f && v_scale < 3.0e38f))
         return PA_ERR_INVALID_ARG;
     if (batch < 0 || max_seq_len < 0 || num_blocks <= 0 || max_blocks_per_seq < 0)
         return PA_ERR_INVALID_ARG;
+    if (prefix && (group_size < 1 || group_size > kMaxGroupSize)) return PA_ERR_INVALID_ARG;
     if (!supported_shape(num_q_heads, num_kv_heads, head_dim, block_size)) return PA_ERR_UNSUPPORTED;
     if (batch == 0) return PA_OK;
     if (!out || !q || !k_cache || !v_cache || !block_tables || !seq_lens) return PA_ERR_INVALID_ARG;
@@ -210,25 +238,48 @@ int decode_impl(float *out, const void *q, const void *k_new, const void *v_new,
     p.v_scale = fp8 ? v_scale : 1.f;
     p.k_inv_scale = fp8 ? 1.0f / k_scale : 1.f;
     p.v_inv_scale = fp8 ? 1.0f / v_scale : 1.f;
+    p.batch = batch;
 
-    const int pt = max_seq_len > 0
-                       ? resolve_partition(batch, num_kv_heads, block_size, max_seq_len, partition_tokens)
-                       : -1;
+    int pt = max_seq_len > 0
+                 ? resolve_partition(batch, num_kv_heads, block_size, max_seq_len, partition_tokens)
+                 : -1;
+    // With prefix groups every call merges partial states (the shared items'
+    // and each sequence's own); "one pass" then means one item of each kind.
+    if (prefix && max_seq_len > 0 && pt <= 0) pt = max_seq_len;
     const bool split = pt > 0;
+    int grid_z = batch;
     if (split) {
-        const size_t need = pa_decode_workspace_size(batch, num_q_heads, num_kv_heads, head_dim,
-                                                     block_size, max_seq_len, partition_tokens);
+        const size_t need = prefix ? pa_decode_shared_prefix_workspace_size(batch, group_size, num_q_heads,
+                                                                            num_kv_heads, head_dim, block_size,
+                                                                            max_seq_len, partition_tokens)
+                                   : pa_decode_workspace_size(batch, num_q_heads, num_kv_heads, head_dim,
+                                                              block_size, max_seq_len, partition_tokens);
         if (!workspace || workspace_bytes < need || !aligned16(workspace)) return PA_ERR_INVALID_ARG;
         p.part_tokens = pt;
         p.num_parts = (max_seq_len + pt - 1) / pt;
-        const int64_t prow = (int64_t)batch * num_q_heads * p.num_parts;
-        p.part_o = static_cast<float *>(workspace);
-        p.part_ml = reinterpret_cast<float *>(static_cast<char *>(workspace) +
-                                              ((prow * head_dim * 4) + 255) / 256 * 256);
         if (p.num_parts > 65535) return PA_ERR_UNSUPPORTED;
+        const int64_t slots = split_slots(max_seq_len, pt, prefix);
+        p.num_slots = (int)slots;
+        const SplitLayout l = split_layout(batch, num_q_heads, num_kv_heads, head_dim, slots);
+        char *ws = static_cast<char *>(workspace);
+        p.part_o = reinterpret_cast<float *>(ws + l.o);
+        p.part_ml = reinterpret_cast<float *>(ws + l.ml);
+        p.tickets = reinterpret_cast<unsigned long long *>(ws + l.tickets);
+        p.epoch = next_epoch();
+        if (prefix) {
+            p.prefix_lens = prefix_lens;
+            p.group_size = group_size;
+            p.num_groups = (batch + group_size - 1) / group_size;
+            p.members_per_item = 8 / p.group;
+            p.items_per_group = (group_size + p.members_per_item - 1) / p.members_per_item;
+            const int64_t z = (int64_t)p.num_groups * p.items_per_group + batch;
+            if (z > 65535) return PA_ERR_UNSUPPORTED;
+            grid_z = (int)z;
+        }
     } else {
         p.part_tokens = max_seq_len > 0 ? max_seq_len : 1;
         p.num_parts = 1;
+        p.num_slots = 1;
     }
 
     CUtensorMap km, vm;
@@ -237,18 +288,25 @@ int decode_impl(float *out, const void *q, const void *k_new, const void *v_new,
         !pool_tensor_map(v_cache, rows, head_dim, box_rows, fp8, &vm))
         return PA_ERR_CUDA;
     cudaStream_t s = static_cast<cudaStream_t>(stream);
+    if (prefix && split) {
+        if (fp8)
+            return append ? launch_decode_d<true, true, true, true>(head_dim, km, vm, p, grid_z, s)
+                          : launch_decode_d<true, false, true, true>(head_dim, km, vm, p, grid_z, s);
+        return append ? launch_decode_d<true, true, false, true>(head_dim, km, vm, p, grid_z, s)
+                      : launch_decode_d<true, false, false, true>(head_dim, km, vm, p, grid_z, s);
+    }
     if (fp8) {
         if (append)
-            return split ? launch_decode_d<true, true, true>(head_dim, km, vm, p, batch, s)
-                         : launch_decode_d<false, true, true>(head_dim, km, vm, p, batch, s);
-        return split ? launch_decode_d<true, false, true>(head_dim, km, vm, p, batch, s)
-                     : launch_decode_d<false, false, true>(head_dim, km, vm, p, batch, s);
+            return split ? launch_decode_d<true, true, true>(head_dim, km, vm, p, grid_z, s)
+                         : launch_decode_d<false, true, true>(head_dim, km, vm, p, grid_z, s);
+        return split ? launch_decode_d<true, false, true>(head_dim, km, vm, p, grid_z, s)
+                     : launch_decode_d<false, false, true>(head_dim, km, vm, p, grid_z, s);
     }
     if (append)
-        return split ? launch_decode_d<true, true, false>(head_dim, km, vm, p, batch, s)
-                     : launch_decode_d<false, true, false>(head_dim, km, vm, p, batch, s);
-    return split ? launch_decode_d<true, false, false>(head_dim, km, vm, p, batch, s)
-                 : launch_decode_d<false, false, false>(head_dim, km, vm, p, batch, s);
+        return split ? launch_decode_d<true, true, false>(head_dim, km, vm, p, grid_z, s)
+                     : launch_decode_d<false, true, false>(head_dim, km, vm, p, grid_z, s);
+    return split ? launch_decode_d<true, false, false>(head_dim, km, vm, p, grid_z, s)
+                 : launch_decode_d<false, false, false>(head_dim, km, vm, p, grid_z, s);
 }
 
 }  // namespace pa
@@ -268,10 +326,18 @@ size_t pa_decode_workspace_size(int batch, int num_q_heads, int num_kv_heads, in
     if (batch <= 0 || num_q_heads <= 0 || num_kv_heads <= 0 || max_seq_len <= 0) return 0;
     const int pt = pa::resolve_partition(batch, num_kv_heads, block_size, max_seq_len, partition_tokens);
     if (pt <= 0) return 0;
-    const int64_t parts = ((int64_t)max_seq_len + pt - 1) / pt;
-    const int64_t rows = (int64_t)batch * num_q_heads * parts;
-    const int64_t o_bytes = ((rows * head_dim * 4) + 255) / 256 * 256;
-    return (size_t)(o_bytes + rows * 2 * 4);
+    return pa::split_layout(batch, num_q_heads, num_kv_heads, head_dim, pa::split_slots(max_seq_len, pt, false))
+        .total;
+}
+
+size_t pa_decode_shared_prefix_workspace_size(int batch, int group_size, int num_q_heads, int num_kv_heads,
+                                              int head_dim, int block_size, int max_seq_len,
+                                              int partition_tokens) {
+    if (batch <= 0 || group_size <= 0 || num_q_heads <= 0 || num_kv_heads <= 0 || max_seq_len <= 0) return 0;
+    int pt = pa::resolve_partition(batch, num_kv_heads, block_size, max_seq_len, partition_tokens);
+    if (pt <= 0) pt = max_seq_len;
+    return pa::split_layout(batch, num_q_heads, num_kv_heads, head_dim, pa::split_slots(max_seq_len, pt, true))
+        .total;
 }
 
 int pa_decode(float *out, const void *q, const void *k_cache, const void *v_cache,
@@ -282,7 +348,7 @@ int pa_decode(float *out, const void *q, const void *k_cache, const void *v_cach
     return pa::decode_impl(out, q, nullptr, nullptr, k_cache, v_cache, block_tables, max_blocks_per_seq,
                            seq_lens, batch, max_seq_len, num_q_heads, num_kv_heads, head_dim, block_size,
                            num_blocks, scale, partition_tokens, workspace, workspace_bytes, err_flag, stream,
-                           false, 1.f, 1.f);
+                           false, 1.f, 1.f, nullptr, 0);
 }
 
 int pa_decode_append(float *out, const void *q, const void *k_new, const void *v_new, void *k_cache,
@@ -295,7 +361,7 @@ int pa_decode_append(float *out, const void *q, const void *k_new, const void *v
     return pa::decode_impl(out, q, k_new, v_new, k_cache, v_cache, block_tables, max_blocks_per_seq,
                            seq_lens, batch, max_seq_len, num_q_heads, num_kv_heads, head_dim, block_size,
                            num_blocks, scale, partition_tokens, workspace, workspace_bytes, err_flag, stream,
-                           false, 1.f, 1.f);
+                           false, 1.f, 1.f, nullptr, 0);
 }
 
 int pa_decode_fp8(float *out, const void *q, const void *k_cache, const void *v_cache,
@@ -306,7 +372,7 @@ int pa_decode_fp8(float *out, const void *q, const void *k_cache, const void *v_
     return pa::decode_impl(out, q, nullptr, nullptr, k_cache, v_cache, block_tables, max_blocks_per_seq,
                            seq_lens, batch, max_seq_len, num_q_heads, num_kv_heads, head_dim, block_size,
                            num_blocks, scale, partition_tokens, workspace, workspace_bytes, err_flag, stream,
-                           true, k_scale, v_scale);
+                           true, k_scale, v_scale, nullptr, 0);
 }
 
 int pa_decode_append_fp8(float *out, const void *q, const void *k_new, const void *v_new, void *k_cache,
@@ -319,7 +385,21 @@ int pa_decode_append_fp8(float *out, const void *q, const void *k_new, const voi
     return pa::decode_impl(out, q, k_new, v_new, k_cache, v_cache, block_tables, max_blocks_per_seq,
                            seq_lens, batch, max_seq_len, num_q_heads, num_kv_heads, head_dim, block_size,
                            num_blocks, scale, partition_tokens, workspace, workspace_bytes, err_flag, stream,
-                           true, k_scale, v_scale);
+                           true, k_scale, v_scale, nullptr, 0);
+}
+
+int pa_decode_shared_prefix(float *out, const void *q, const void *k_new, const void *v_new, void *k_cache,
+                            void *v_cache, const int32_t *block_tables, int max_blocks_per_seq,
+                            const int32_t *seq_lens, const int32_t *prefix_lens, int group_size, int batch,
+                            int max_seq_len, int num_q_heads, int num_kv_heads, int head_dim, int block_size,
+                            int64_t num_blocks, float scale, int partition_tokens, void *workspace,
+                            size_t workspace_bytes, int32_t *err_flag, void *stream) {
+    if (batch > 0 && (!prefix_lens || (k_new == nullptr) != (v_new == nullptr))) return PA_ERR_INVALID_ARG;
+    if (batch > 0 && max_seq_len > 0 && !prefix_lens) return PA_ERR_INVALID_ARG;
+    return pa::decode_impl(out, q, k_new, v_new, k_cache, v_cache, block_tables, max_blocks_per_seq, seq_lens,
+                           batch, max_seq_len, num_q_heads, num_kv_heads, head_dim, block_size, num_blocks, scale,
+                           partition_tokens, workspace, workspace_bytes, err_flag, stream, false, 1.f, 1.f,
+                           batch > 0 ? prefix_lens : nullptr, group_size);
 }
 
 int pa_decode_builtin_scratch(float *out, const void *q, const void *k_cache, const void *v_cache,

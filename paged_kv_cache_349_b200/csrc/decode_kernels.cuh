@@ -22,11 +22,18 @@
 //    N = 8 heads, K = 16 tokens).  P is split into bf16 hi + lo parts so the
 //    PV product keeps ~16 mantissa bits.
 //  * Warps merge their (max, sum, O) states through shared memory.  In the
-//    split variant each CTA writes its partition's state to the workspace
-//    and a log-sum-exp reduce kernel combines the partitions.
+//    split variant each CTA writes its partition's state to the workspace,
+//    then takes a ticket on its (sequence, kv head); the CTA that arrives
+//    last merges every partition of that pair (log-sum-exp) and writes the
+//    output, so no second kernel runs.
+//  * Shared-prefix variant: sequences that share their first tokens (n-way
+//    sampling of one prompt) get one extra work item per group and kv head
+//    that reads the shared tiles once and serves every member's query heads
+//    as extra mma columns; each member's own work items start after the
+//    shared tiles, and the ticket merge combines both.
 //
-// This header holds the device code (the decode kernel, the log-sum-exp
-// reduce, their shared-memory layout and parameters).  decode.cu includes it
+// This header holds the device code (the decode kernel with its split
+// merge, its shared-memory layout and parameters).  decode.cu includes it
 // and holds the host side, so a change there leaves the device code -- and
 // any profile taken of it -- untouched.
 #pragma once
@@ -117,6 +124,17 @@ struct DecodeParams {
     float v_scale;
     float k_inv_scale;          // fp8 pools: 1 / scale, for the fused cache write
     float v_inv_scale;
+    int batch;
+    // Split: partial states per (sequence, query head) and the arrival tickets.
+    int num_slots;              // partial-state slots per row: num_parts (x2 with prefix groups)
+    unsigned long long *tickets;  // [B, Hkv]: (epoch << 32) | partitions arrived
+    unsigned int epoch;         // this call's tag in the tickets (never 0)
+    // Shared-prefix groups: sequences [g*group_size, (g+1)*group_size) share prefix_lens[g] tokens.
+    const int32_t *prefix_lens; // [num_groups]
+    int group_size;
+    int num_groups;
+    int members_per_item;       // members one prefix item serves: 8 / G (the mma N columns)
+    int items_per_group;        // ceil(group_size / members_per_item)
 };
 
 // Sequence length as every kernel of one call sees it: out-of-contract values
@@ -124,6 +142,53 @@ struct DecodeParams {
 __device__ __forceinline__ int clamp_len(int L, const DecodeParams &p) {
     const int cap = min(p.max_seq_len, p.max_blocks * p.block_size);
     return L < 0 ? 0 : (L > cap ? cap : L);
+}
+
+// Partitions of `tokens` tokens at `part_tokens` per partition.
+__device__ __forceinline__ int parts_of(int tokens, int part_tokens) {
+    return tokens > 0 ? (tokens + part_tokens - 1) / part_tokens : 0;
+}
+
+// Tokens at the start of group g's sequences that are read once for the whole
+// group: the group's prefix_lens entry, cut to every member's length minus one
+// (the token appended in this step is never shared) and rounded down to whole
+// 16-token tiles, so each member's own tiles start tile-aligned.  0 for groups
+// of one sequence.
+// Every lane of a warp loads members in parallel, so call it from whole warps.
+__device__ __forceinline__ int group_shared_tokens(const DecodeParams &p, int g) {
+    const int m0 = g * p.group_size;
+    const int m1 = min(m0 + p.group_size, p.batch);
+    if (m1 - m0 < 2) return 0;
+    int s = __ldg(p.prefix_lens + g);
+    for (int m = m0 + (int)(threadIdx.x & 31); m < m1; m += 32) s = min(s, clamp_len(__ldg(p.seq_lens + m), p) - 1);
+#pragma unroll
+    for (int off = 16; off; off >>= 1) s = min(s, __shfl_xor_sync(0xffffffffu, s, off));
+    return s > 0 ? s / kTileTokens * kTileTokens : 0;
+}
+
+// Arrival ticket of one partition on (sequence, kv head): returns true for the
+// last of the `expected` partitions of this call.  A ticket word holds
+// (epoch << 32) | count; a word tagged with another epoch (an earlier call, or
+// uninitialised memory) counts as zero, so the workspace needs no clearing.
+// The last arrival resets the word to 0, which keeps a replayed call (same
+// epoch) correct.  The CAS loop only retries when another partition arrived
+// in between; it is bounded all the same.
+__device__ __forceinline__ bool take_ticket(unsigned long long *t, unsigned int epoch, int expected,
+                                            int32_t *flag) {
+    unsigned long long old = *reinterpret_cast<volatile unsigned long long *>(t);
+    for (int it = 0; it < (1 << 20); ++it) {
+        const unsigned int cnt = (unsigned int)(old >> 32) == epoch ? (unsigned int)old : 0u;
+        const unsigned long long want = ((unsigned long long)epoch << 32) | (cnt + 1u);
+        const unsigned long long seen = atomicCAS(t, old, want);
+        if (seen == old) {
+            if ((int)(cnt + 1u) < expected) return false;
+            atomicExch(t, 0ull);
+            return true;
+        }
+        old = seen;
+    }
+    raise_flag(flag, PA_FLAG_TIMEOUT);
+    return false;
 }
 
 // Byte offset of 16-byte chunk c of token row r inside one swizzled 16-bit tile.
@@ -161,12 +226,54 @@ __device__ __forceinline__ void mma_16816(float (&d)[4], uint32_t a0, uint32_t a
 #define PA_DECODE_MIN_CTAS_BF16 3
 #endif
 
-template <int HEAD_DIM, bool SPLIT, bool APPEND, bool FP8>
+// Log-sum-exp merge of every partial state of (sequence b, kv head h), run by
+// the CTA whose partition arrived last:
+//   out = sum_p 2^(m_p - M) l_p o_p / sum_p 2^(m_p - M) l_p,  M = max_p m_p,
+// over the shared-prefix slots [0, n_pre) and the sequence's own slots
+// [s0, s0 + n_own).  Partials written by other CTAs are read through L2.
+template <int HEAD_DIM>
+__device__ __forceinline__ void merge_partials(const DecodeParams &p, int b, int h, int n_pre, int s0, int n_own) {
+    constexpr int kCols = HEAD_DIM / 4;  // float4 columns of a row
+    const int G = p.group;
+    for (int x = threadIdx.x; x < G * kCols; x += kThreads) {
+        const int g = x / kCols;
+        const int c4 = x - g * kCols;
+        const int64_t row = (int64_t)b * p.num_q_heads + (int64_t)h * G + g;
+        const float2 *ml = reinterpret_cast<const float2 *>(p.part_ml) + row * p.num_slots;
+        const float4 *po = reinterpret_cast<const float4 *>(p.part_o + row * p.num_slots * HEAD_DIM) + c4;
+        const int n = n_pre + n_own;
+        float M = -INFINITY;
+        for (int k = 0; k < n; ++k) M = fmaxf(M, __ldcg(ml + (k < n_pre ? k : s0 + k - n_pre)).x);
+        float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
+        float den = 0.f;
+        if (M != -INFINITY) {
+#pragma unroll 4
+            for (int k = 0; k < n; ++k) {
+                const int s = k < n_pre ? k : s0 + k - n_pre;
+                const float2 mlv = __ldcg(ml + s);
+                const float w = fast_exp2(mlv.x - M) * mlv.y;
+                const float4 o = __ldcg(po + (int64_t)s * kCols);
+                acc.x += w * o.x;
+                acc.y += w * o.y;
+                acc.z += w * o.z;
+                acc.w += w * o.w;
+                den += w;
+            }
+        }
+        const float r = den > 0.f ? 1.f / den : 0.f;
+        reinterpret_cast<float4 *>(p.out + row * HEAD_DIM)[c4] =
+            make_float4(acc.x * r, acc.y * r, acc.z * r, acc.w * r);
+    }
+}
+
+template <int HEAD_DIM, bool SPLIT, bool APPEND, bool FP8, bool PREFIX>
 __global__ void __launch_bounds__(kThreads, FP8 ? PA_DECODE_MIN_CTAS_FP8 : PA_DECODE_MIN_CTAS_BF16) paged_decode_kernel(
     const __grid_constant__ CUtensorMap k_map, const __grid_constant__ CUtensorMap v_map,
     const DecodeParams p) {
+    static_assert(SPLIT || !PREFIX, "shared-prefix items always merge through the split path");
     using C = Cfg<HEAD_DIM, FP8>;
     extern __shared__ uint8_t smem_raw[];
+    __shared__ unsigned int s_last;  // split: members whose merge falls to this CTA (bit mask)
     uint8_t *smem = reinterpret_cast<uint8_t *>(
         (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~static_cast<uintptr_t>(1023));
     uint64_t *full = reinterpret_cast<uint64_t *>(smem + C::kDataBytes);
@@ -179,20 +286,58 @@ __global__ void __launch_bounds__(kThreads, FP8 ? PA_DECODE_MIN_CTAS_FP8 : PA_DE
 
     const int part = blockIdx.x;
     const int h = blockIdx.y;
-    const int b = blockIdx.z;
     const int warp = threadIdx.x >> 5;
     const int lane = threadIdx.x & 31;
 
+    // ---- the work item ----
+    // Normal item: sequence b = blockIdx.z, tokens [part * pt, ...) of it.
+    // With prefix groups, z < num_groups * items_per_group names a prefix item
+    // (group, member chunk): tokens [part * pt, ...) of the group's shared
+    // range, read through the first member's table, for up to 8 / G members;
+    // any other z names sequence b's own item: tokens from its group's shared
+    // length on.
+    bool pre = false;
+    int b = blockIdx.z;  // the first member served
+    int tb = b;          // the sequence whose block table is read
+    int nmem = 1;        // members served (their query heads are the mma columns)
+    int shared = 0;      // tokens of b's group read by the prefix items
+    if constexpr (PREFIX) {
+        const int n_pre_items = p.num_groups * p.items_per_group;
+        if (b < n_pre_items) {
+            pre = true;
+            const int g = b / p.items_per_group;
+            const int chunk = b - g * p.items_per_group;
+            const int m_end = min((g + 1) * p.group_size, p.batch);
+            tb = g * p.group_size;  // every member chunk reads the first member's blocks
+            b = tb + chunk * p.members_per_item;
+            nmem = min(p.members_per_item, m_end - b);
+            if (nmem <= 0) return;  // member chunk past a short last group
+            if (threadIdx.x == 0 && chunk == 0 && part == 0 && h == 0 && __ldg(p.prefix_lens + g) < 0)
+                raise_flag(p.err_flag, PA_FLAG_BAD_LEN);
+            shared = group_shared_tokens(p, g);
+        } else {
+            b -= n_pre_items;
+            tb = b;
+            shared = group_shared_tokens(p, b / p.group_size);
+        }
+    }
     const int L_raw = __ldg(p.seq_lens + b);
     const int L = clamp_len(L_raw, p);
-    const int tok_begin = part * p.part_tokens;
-    const int tok_end = min(L, tok_begin + p.part_tokens);
+    const int tok_begin = (pre ? 0 : shared) + part * p.part_tokens;
+    const int tok_end = min(pre ? shared : L, tok_begin + p.part_tokens);
     const int n_tiles = tok_end > tok_begin ? (tok_end - tok_begin + kTileTokens - 1) / kTileTokens : 0;
-    // Let the log-sum-exp reduce (launched as a programmatic dependent) get
-    // scheduled while this grid's last wave runs; it waits for our results.
-    if (SPLIT) asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
-    if (SPLIT && n_tiles == 0) return;  // empty partition: the reduce skips it
-    if (threadIdx.x == 0 && part == 0 && h == 0 && L != L_raw) raise_flag(p.err_flag, PA_FLAG_BAD_LEN);
+    if (!pre && threadIdx.x == 0 && part == 0 && h == 0 && L != L_raw) raise_flag(p.err_flag, PA_FLAG_BAD_LEN);
+    // Split: a sequence whose own tokens fit one partition (and share none) has
+    // a single partial state -- that CTA writes the output itself.
+    const bool direct = SPLIT && !pre && shared == 0 && L <= p.part_tokens;
+    if (SPLIT && n_tiles == 0) {
+        // Nothing to read.  An empty sequence has no partial states at all, so
+        // its partition-0 CTA writes its zero rows; other empty partitions just end.
+        if (!pre && part == 0 && L == 0)
+            for (int x = threadIdx.x; x < p.group * HEAD_DIM; x += kThreads)
+                p.out[((int64_t)b * p.num_q_heads + (int64_t)h * p.group) * HEAD_DIM + x] = 0.f;
+        return;
+    }
 
     if (threadIdx.x == 0) {
         for (int s = 0; s < C::kStages; ++s) {
@@ -218,7 +363,7 @@ __global__ void __launch_bounds__(kThreads, FP8 ? PA_DECODE_MIN_CTAS_FP8 : PA_DE
         // time (one coalesced load per window, the next window loaded ahead).
         // kProducerLanes lanes wait on the ring and issue copies in parallel:
         // lane k handles tiles k, k+P, k+2P, ... and therefore ring slots k, k+P, ...
-        const int32_t *table = p.block_tables + (int64_t)b * p.max_blocks;
+        const int32_t *table = p.block_tables + (int64_t)tb * p.max_blocks;
         const int j_end = (tok_end + p.block_size - 1) / p.block_size;  // blocks this CTA reads
         int win = tok_begin / p.block_size;                             // first entry of the window
         int32_t cur = win + lane < j_end ? __ldg(table + win + lane) : -1;
@@ -305,10 +450,11 @@ __global__ void __launch_bounds__(kThreads, FP8 ? PA_DECODE_MIN_CTAS_FP8 : PA_DE
         // ---------------- consumers ----------------
         const int G = p.group;
         // Q^T as mma B fragments (k = head dim, permuted; n = query head column gid).
+        // Column gid is query head gid % G of member b + gid / G.
         uint32_t qf[HEAD_DIM / 16][2];
-        if (gid < G) {
+        if (gid < nmem * G) {
             const uint4 *qrow = reinterpret_cast<const uint4 *>(
-                p.q + ((int64_t)b * p.num_q_heads + (int64_t)h * G + gid) * HEAD_DIM);
+                p.q + ((int64_t)(b + gid / G) * p.num_q_heads + (int64_t)h * G + gid % G) * HEAD_DIM);
 #pragma unroll
             for (int j = 0; j < HEAD_DIM / 32; ++j) {
                 const uint4 v = __ldg(qrow + 4 * j + tig);
@@ -362,7 +508,7 @@ __global__ void __launch_bounds__(kThreads, FP8 ? PA_DECODE_MIN_CTAS_FP8 : PA_DE
         // token is owned by this sequence alone (copy-on-write), so no other
         // CTA reads that row.
         int i_new = -1;
-        if (APPEND && L == L_raw && L > 0 && L - 1 >= tok_begin && L - 1 < tok_end) {
+        if (APPEND && !pre && L == L_raw && L > 0 && L - 1 >= tok_begin && L - 1 < tok_end) {
             const int it = (L - 1 - tok_begin) / kTileTokens;
             if (it % kConsumerWarps == warp) {
                 i_new = it;
@@ -652,7 +798,10 @@ __global__ void __launch_bounds__(kThreads, FP8 ? PA_DECODE_MIN_CTAS_FP8 : PA_DE
     }
     __syncthreads();
     const int G = p.group;
-    for (int x = threadIdx.x; x < G * HEAD_DIM; x += kThreads) {
+    // Column n is query head n % G of member b + n / G; in the split variant
+    // its partial state goes to slot `slot` of that row.
+    const int slot = PREFIX && !pre ? p.num_parts + part : part;
+    for (int x = threadIdx.x; x < nmem * G * HEAD_DIM; x += kThreads) {
         const int n = x / HEAD_DIM;
         const int d = x - n * HEAD_DIM;
         float M = -INFINITY;
@@ -667,88 +816,45 @@ __global__ void __launch_bounds__(kThreads, FP8 ? PA_DECODE_MIN_CTAS_FP8 : PA_DE
                 den += f * ml[w * 8 + n];
             }
         }
-        const int64_t row = (int64_t)b * p.num_q_heads + (int64_t)h * G + n;
+        const int64_t row = (int64_t)(b + n / G) * p.num_q_heads + (int64_t)h * G + n % G;
         if (FP8) num *= p.v_scale;
-        if (SPLIT) {
-            p.part_o[(row * p.num_parts + part) * HEAD_DIM + d] = num / den;
+        if (SPLIT && !direct) {
+            p.part_o[(row * p.num_slots + slot) * HEAD_DIM + d] = den > 0.f ? num / den : 0.f;
             if (d == 0) {
-                p.part_ml[(row * p.num_parts + part) * 2] = M;
-                p.part_ml[(row * p.num_parts + part) * 2 + 1] = den;
+                p.part_ml[(row * p.num_slots + slot) * 2] = M;
+                p.part_ml[(row * p.num_slots + slot) * 2 + 1] = den;
             }
         } else {
             p.out[row * HEAD_DIM + d] = den > 0.f ? num / den : 0.f;
         }
     }
-}
-
-// Log-sum-exp merge of the partitions of one (sequence, query head):
-//   out = sum_p 2^(m_p - M) l_p o_p / sum_p 2^(m_p - M) l_p,  M = max_p m_p.
-// Four warps split the partitions; each lane owns HEAD_DIM/32 output dims.
-constexpr int kReduceThreads = 128;
-
-template <int HEAD_DIM>
-__global__ void __launch_bounds__(kReduceThreads) lse_reduce_kernel(const DecodeParams p) {
-    // Launched as a programmatic dependent of the decode grid: wait for its results.
-    asm volatile("griddepcontrol.wait;" ::: "memory");
-    constexpr int kWarps = kReduceThreads / 32;
-    constexpr int V = HEAD_DIM / 32;  // dims per lane: 4 or 2
-    __shared__ float s_max[kWarps];
-    __shared__ float s_den[kWarps];
-    __shared__ float s_acc[kWarps][HEAD_DIM];
-    const int hq = blockIdx.x;
-    const int b = blockIdx.y;
-    const int warp = threadIdx.x >> 5;
-    const int lane = threadIdx.x & 31;
-    const int L = clamp_len(__ldg(p.seq_lens + b), p);
-    const int n = (L + p.part_tokens - 1) / p.part_tokens;
-    const int64_t row = (int64_t)b * p.num_q_heads + hq;
-    const float2 *ml = reinterpret_cast<const float2 *>(p.part_ml + row * p.num_parts * 2);
-    const float *po = p.part_o + row * p.num_parts * HEAD_DIM + lane * V;
-
-    float M = -INFINITY;
-    for (int i = threadIdx.x; i < n; i += kReduceThreads) M = fmaxf(M, __ldg(&ml[i].x));
-#pragma unroll
-    for (int off = 16; off; off >>= 1) M = fmaxf(M, __shfl_xor_sync(0xffffffffu, M, off));
-    if (lane == 0) s_max[warp] = M;
-    __syncthreads();
-#pragma unroll
-    for (int w = 0; w < kWarps; ++w) M = fmaxf(M, s_max[w]);
-
-    float acc[V];
-#pragma unroll
-    for (int k = 0; k < V; ++k) acc[k] = 0.f;
-    float den = 0.f;
-    if (M != -INFINITY) {
-#pragma unroll 4
-        for (int i = warp; i < n; i += kWarps) {
-            const float2 mlv = __ldg(&ml[i]);
-            const float w = fast_exp2(mlv.x - M) * mlv.y;
-            if constexpr (V == 4) {
-                const float4 v = __ldg(reinterpret_cast<const float4 *>(po + (int64_t)i * HEAD_DIM));
-                acc[0] += w * v.x;
-                acc[1] += w * v.y;
-                acc[2] += w * v.z;
-                acc[3] += w * v.w;
-            } else {
-                const float2 v = __ldg(reinterpret_cast<const float2 *>(po + (int64_t)i * HEAD_DIM));
-                acc[0] += w * v.x;
-                acc[1] += w * v.y;
+    if constexpr (SPLIT) {
+        if (direct) return;
+        // Ticket: this partition's state is stored.  The CTA whose ticket is the
+        // last of a (member, kv head) merges that pair's partitions.
+        __threadfence();  // every thread's partial stores, visible GPU-wide before the ticket
+        __syncthreads();
+        if (threadIdx.x == 0) {
+            unsigned int mask = 0;
+            for (int m = 0; m < nmem; ++m) {
+                const int bm = b + m;
+                const int Lm = pre ? clamp_len(__ldg(p.seq_lens + bm), p) : L;
+                const int expected = parts_of(shared, p.part_tokens) + parts_of(Lm - shared, p.part_tokens);
+                if (take_ticket(p.tickets + (int64_t)bm * p.num_kv_heads + h, p.epoch, expected, p.err_flag))
+                    mask |= 1u << m;
             }
-            den += w;
+            if (mask) __threadfence();  // the other partitions' states, seen before they are read
+            s_last = mask;
         }
-    }
-#pragma unroll
-    for (int k = 0; k < V; ++k) s_acc[warp][lane * V + k] = acc[k];
-    if (lane == 0) s_den[warp] = den;
-    __syncthreads();
-    for (int x = threadIdx.x; x < HEAD_DIM; x += kReduceThreads) {
-        float num = 0.f, dd = 0.f;
-#pragma unroll
-        for (int w = 0; w < kWarps; ++w) {
-            num += s_acc[w][x];
-            dd += s_den[w];
+        __syncthreads();
+        const unsigned int mask = s_last;
+        for (int m = 0; m < nmem; ++m) {
+            if (!(mask & (1u << m))) continue;
+            const int bm = b + m;
+            const int Lm = pre ? clamp_len(__ldg(p.seq_lens + bm), p) : L;
+            merge_partials<HEAD_DIM>(p, bm, h, parts_of(shared, p.part_tokens), PREFIX ? p.num_parts : 0,
+                                     parts_of(Lm - shared, p.part_tokens));
         }
-        p.out[row * HEAD_DIM + x] = dd > 0.f ? num / dd : 0.f;
     }
 }
 

@@ -30,13 +30,17 @@ int device_address(const void *p, void **dev_ptr);
 
 inline bool aligned16(const void *p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
 
-// Shared body of pa_decode / pa_decode_append (k_new == nullptr: no cache write).
+// Largest sequence group of the shared-prefix decode.
+constexpr int kMaxGroupSize = 64;
+
+// Shared body of every decode entry point (k_new == nullptr: no cache write;
+// prefix_lens != nullptr: groups of group_size sequences share a prefix).
 int decode_impl(float *out, const void *q, const void *k_new, const void *v_new, const void *k_cache,
                 const void *v_cache, const int32_t *block_tables, int max_blocks_per_seq,
                 const int32_t *seq_lens, int batch, int max_seq_len, int num_q_heads, int num_kv_heads,
                 int head_dim, int block_size, int64_t num_blocks, float scale, int partition_tokens,
                 void *workspace, size_t workspace_bytes, int32_t *err_flag, void *stream, bool fp8,
-                float k_scale, float v_scale);
+                float k_scale, float v_scale, const int32_t *prefix_lens, int group_size);
 
 inline bool supported_shape(int num_q_heads, int num_kv_heads, int head_dim, int block_size) {
     if (num_kv_heads <= 0 || num_q_heads <= 0 || num_q_heads % num_kv_heads) return false;

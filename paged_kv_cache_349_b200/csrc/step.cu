@@ -55,7 +55,9 @@ StagingLayout staging_layout(int batch, int max_blocks_per_seq, int max_copy_pai
     l.workspace = off;
     l.workspace_bytes = pa_decode_workspace_size(batch, num_q_heads, num_kv_heads, head_dim, block_size,
                                                  max_seq_len, partition_tokens);
-    if (l.workspace_bytes) l.workspace_bytes += 2 * kAlign * kMaxChunks;
+    // Each chunk's slice rounds its three sections (partial states, their
+    // maxima and sums, the tickets) and itself up to kAlign.
+    if (l.workspace_bytes) l.workspace_bytes += 4 * kAlign * kMaxChunks;
     off += round_up(l.workspace_bytes);
     l.total = off;
     return l;
@@ -300,7 +302,7 @@ static int step_host(float *out_host, const void *q_host, const void *k_new_host
                                reinterpret_cast<const int32_t *>(st + l.tables + b0 * tab_row), max_blocks_per_seq,
                                reinterpret_cast<const int32_t *>(st + l.lens) + b0, nb, max_seq_len, num_q_heads,
                                num_kv_heads, head_dim, block_size, num_blocks, scale, pt, ws, ws_bytes, err_flag,
-                               cs, fp8, k_scale, v_scale);
+                               cs, fp8, k_scale, v_scale, nullptr, 0);
     };
     // Host inputs as the device sees them (resolved once per call).
     const pa::HostSrc hq = pa::host_src(q_host), hk = pa::host_src(k_new_host), hv = pa::host_src(v_new_host);

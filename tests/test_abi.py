@@ -90,10 +90,45 @@ def test_workspace_size_explicit_partitions(pt, maxlen, parts):
         assert size == 0
         assert pa.pa_decode_partition_tokens(B, Hq, Hkv, d, 16, maxlen, pt) == -1
     else:
+        # partial outputs, then (max, sum) pairs, each 256-byte aligned, then one
+        # 8-byte arrival ticket per (sequence, kv head)
         rows = B * Hq * parts
         o_bytes = -(-rows * d * 4 // 256) * 256
-        assert size == o_bytes + rows * 8
+        ml_bytes = -(-rows * 8 // 256) * 256
+        assert size == o_bytes + ml_bytes + B * Hkv * 8
         assert pa.pa_decode_partition_tokens(B, Hq, Hkv, d, 16, maxlen, pt) == pt
+
+
+@pytest.mark.parametrize("pt,maxlen,parts", [(512, 32768, 64), (-1, 4096, 1), (0, 2500, 1), (16, 40, 3)])
+def test_shared_prefix_workspace_size(pt, maxlen, parts):
+    """Two slots per partition (the shared items', then the sequence's own); a call that would
+    not split still has one of each."""
+    B, n, Hq, Hkv, d = 128, 4, 40, 40, 128
+    size = pa.pa_decode_shared_prefix_workspace_size(B, n, Hq, Hkv, d, 16, maxlen, pt)
+    rows = B * Hq * 2 * parts
+    assert size == -(-rows * d * 4 // 256) * 256 + -(-rows * 8 // 256) * 256 + B * Hkv * 8
+    assert pa.pa_decode_shared_prefix_workspace_size(0, n, Hq, Hkv, d, 16, maxlen, pt) == 0
+
+
+def test_shared_prefix_argument_errors_need_no_gpu():
+    f = lib.pa_decode_shared_prefix
+    base = [_fake(), _fake(), None, None, _fake(), _fake(), _fake(), 4, _fake(), _fake(), 4, 8, 64, 8, 8, 128,
+            16, 64, 0.1, -1, _fake(0x100000), 1 << 20, None, None]
+
+    def call(**kw):
+        a = list(base)
+        for i, v in kw.items():
+            a[int(i[1:])] = v
+        return f(*a)
+
+    assert call(a11=0) == pa.PA_OK                        # empty batch
+    assert call(a9=None) == pa.PA_ERR_INVALID_ARG         # prefix_lens missing
+    assert call(a10=0) == pa.PA_ERR_INVALID_ARG           # group size 0
+    assert call(a10=65) == pa.PA_ERR_INVALID_ARG          # group size above 64
+    assert call(a2=_fake()) == pa.PA_ERR_INVALID_ARG      # k_new without v_new
+    assert call(a15=96) == pa.PA_ERR_UNSUPPORTED          # head_dim
+    assert call(a20=None) == pa.PA_ERR_INVALID_ARG        # always merges: needs a workspace
+    assert call(a21=16) == pa.PA_ERR_INVALID_ARG          # workspace too small
 
 
 def test_host_step_argument_errors_need_no_gpu():

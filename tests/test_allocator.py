@@ -74,11 +74,11 @@ def test_oom_leaves_state_unchanged():
     assert e.value.status == pa.PA_ERR_OOM
     assert a.block_table(s)[1] == 32
     # batched append is all-or-nothing
-    b = pa.Allocator(3, 4)
+    b = pa.Allocator(3, 8)
     x, y = b.create(), b.create()
-    for _ in range(4):
+    for _ in range(8):
         b.append(x)
-    for _ in range(3):
+    for _ in range(7):
         b.append(y)
     before = (b.block_table(x), b.block_table(y), b.num_free())
     b.append(y)                     # y fills its block
@@ -87,7 +87,7 @@ def test_oom_leaves_state_unchanged():
     with pytest.raises(pa.PaError):
         b.append_batch([x, y, z, y])  # needs 1 (x new) + 1 (y new) + 1 (z new) + ... > free
     assert b.num_free() == free_before
-    assert b.block_table(x)[1] == 4 and b.block_table(y)[1] == 4 and b.block_table(z)[1] == 4
+    assert b.block_table(x)[1] == 8 and b.block_table(y)[1] == 8 and b.block_table(z)[1] == 8
     del before
 
 
@@ -119,7 +119,7 @@ def test_export_pads_tables():
 def test_random_ops_match_model(seed):
     """Random create/append/batch-append/fork/free on the C++ allocator and the model."""
     rng = np.random.default_rng(seed)
-    bs, NB = 4, 40
+    bs, NB = 8, 40
     a = pa.Allocator(NB, bs)
     m = oracle.AllocModel(NB, bs)
     ids = {}                 # product id -> model id
@@ -347,3 +347,18 @@ def test_bench_e2e_host_state_matches_workload(cfg, kw):
     assert pa.validate_tables(tables, lens, case.num_blocks, case.block_size) is None
     assert n_pairs == 0  # copy-on-write already happened while the state was rebuilt
     alloc.close()
+
+
+def test_create_rejects_sizes_the_kernels_cannot_address():
+    """Slot ids are int32 (block * block_size + row): a pool whose slots overflow int32 is refused,
+    and so is a block size the kernels do not support; neither creates an allocator."""
+    for nb, bs in ((1 << 27, 16), ((1 << 31) // 16 + 1, 16), (8, 4), (8, 12), (8, 128)):
+        with pytest.raises(pa.PaError) as e:
+            pa.Allocator(nb, bs)
+        assert e.value.status in (pa.PA_ERR_INVALID_ARG, pa.PA_ERR_UNSUPPORTED)
+    # the largest pool whose slots still fit int32
+    a = pa.Allocator((1 << 31) // 64 - 1, 64)
+    s = a.create()
+    slot, _ = a.append(s)
+    assert 0 <= slot < (1 << 31)
+    a.close()

@@ -158,12 +158,123 @@ def test_error_flags_and_skipped_accesses():
                  scale=float(case.scale), partition_tokens=-1, err_flag=dc.flag)
     torch.cuda.synchronize()
     assert int(dc.flag.item()) & pa.PA_FLAG_BAD_BLOCK
-    # a sequence longer than max_seq_len
+    # a sequence longer than max_seq_len (split modes: test_bad_lengths_flagged_in_every_mode)
     dc.flag.zero_()
     pa.pa_decode(dc.out, dc.q, dc.k, dc.v, dc.tables, dc.lens, max_seq_len=20,
                  scale=float(case.scale), partition_tokens=-1, err_flag=dc.flag)
     torch.cuda.synchronize()
     assert int(dc.flag.item()) & pa.PA_FLAG_BAD_LEN
+
+
+@pytest.mark.parametrize("pt", [-1, 16, 0])
+def test_bad_lengths_flagged_in_every_mode(pt):
+    """A negative length reads nothing and gives zero rows; a length past max_seq_len is cut to it.
+    Both raise PA_FLAG_BAD_LEN, single pass, 16-token partitions and the default split alike."""
+    import torch
+    import paged_kv_cache_349_b200 as pa
+    case = W.make_custom_case([20, 33, 700, 1500], num_q_heads=8, num_kv_heads=2, head_dim=128, block_size=16,
+                              seed=13)
+    dc = DeviceCase(case)
+    # the default of this shape splits (4 sequences x 2 kv heads, up to 1500 tokens)
+    assert pt != 0 or pa.pa_decode_partition_tokens(4, 8, 2, 128, 16, case.max_seq_len, 0) > 0
+    for lens, max_len in (([-5, 33, 700, 1500], case.max_seq_len), ([20, 33, 700, 1500], 1000)):
+        bad = np.array(lens, np.int32)
+        ws_bytes = pa.pa_decode_workspace_size(case.batch, 8, 2, 128, 16, max_len, pt)
+        ws = torch.empty(max(ws_bytes, 16), dtype=torch.uint8, device="cuda")
+        dc.flag.zero_()
+        dc.out.fill_(float("nan"))
+        pa.pa_decode(dc.out, dc.q, dc.k, dc.v, dc.tables, i32_dev(bad), max_seq_len=max_len,
+                     scale=float(case.scale), partition_tokens=pt, workspace=ws, err_flag=dc.flag)
+        torch.cuda.synchronize()
+        assert int(dc.flag.item()) == pa.PA_FLAG_BAD_LEN, (lens, max_len, pt)
+        got = dc.out.cpu().numpy().astype(np.float64)
+        clamped = np.clip(bad, 0, max_len)
+        want = oracle.decode(case.q, case.k_cache, case.v_cache, case.block_tables, clamped,
+                             num_kv_heads=2, block_size=16, scale=case.scale)
+        assert_close(got, want, f"lens {lens} max {max_len} pt {pt}")
+        if lens[0] < 0:
+            assert np.all(got[0] == 0)
+
+
+def test_split_workspace_needs_no_clearing():
+    """The split merge's arrival tickets carry a per-call tag: a workspace full of zeros, of
+    random bytes or of all-ones bytes gives bit-identical outputs, and a call queued right
+    behind another on the same workspace (different inputs, no synchronisation) does too.
+    Every ticket a merged pair used is back at zero after the call."""
+    import torch
+    import paged_kv_cache_349_b200 as pa
+    case = W.make_case(5, batch=3, max_len=3000, num_blocks=800, num_copy_pairs=0, partition_tokens=256,
+                       fill=W.BF16_ZERO)
+    dc = DeviceCase(case)
+    need = pa.pa_decode_workspace_size(case.batch, case.num_q_heads, case.num_kv_heads, case.head_dim,
+                                       case.block_size, case.max_seq_len, 256)
+    outs = []
+    for fill in ("zero", "random", "ones"):
+        ws = torch.zeros(need, dtype=torch.uint8, device="cuda")
+        if fill == "random":
+            ws = torch.randint(0, 256, (need,), dtype=torch.uint8, device="cuda")
+        elif fill == "ones":
+            ws.fill_(255)
+        out = torch.empty_like(dc.out)
+        pa.pa_decode(out, dc.q, dc.k, dc.v, dc.tables, dc.lens, max_seq_len=case.max_seq_len,
+                     scale=float(case.scale), partition_tokens=256, workspace=ws, err_flag=dc.flag)
+        torch.cuda.synchronize()
+        outs.append(out)
+        if fill == "zero":
+            tickets = ws[need - case.batch * case.num_kv_heads * 8:]
+            assert int(tickets.count_nonzero()) == 0, "last arrivals reset their tickets"
+    assert int(dc.flag.item()) == 0
+    assert torch.equal(outs[0], outs[1]) and torch.equal(outs[0], outs[2])
+    want = oracle.decode(case.q, case.k_cache, case.v_cache, case.block_tables, case.seq_lens,
+                         num_kv_heads=case.num_kv_heads, block_size=16, scale=case.scale)
+    assert_close(outs[0].cpu().numpy(), want, "split 256")
+    # back to back on one workspace: q, then -q (a different softmax), no sync in between
+    ws = torch.randint(0, 256, (need,), dtype=torch.uint8, device="cuda")
+    q2 = (-dc.q.float()).to(torch.bfloat16)
+    a, b = torch.empty_like(dc.out), torch.empty_like(dc.out)
+    for qq, o in ((dc.q, a), (q2, b)):
+        pa.pa_decode(o, qq, dc.k, dc.v, dc.tables, dc.lens, max_seq_len=case.max_seq_len,
+                     scale=float(case.scale), partition_tokens=256, workspace=ws, err_flag=dc.flag)
+    torch.cuda.synchronize()
+    b_alone = torch.empty_like(dc.out)
+    pa.pa_decode(b_alone, q2, dc.k, dc.v, dc.tables, dc.lens, max_seq_len=case.max_seq_len,
+                 scale=float(case.scale), partition_tokens=256, workspace=torch.zeros_like(ws), err_flag=dc.flag)
+    torch.cuda.synchronize()
+    assert torch.equal(a, outs[0]) and torch.equal(b, b_alone)
+
+
+def test_split_decode_replays_in_a_cuda_graph():
+    """A captured split call replays with the same tag each time: correct because the last
+    arrival of every pair resets its ticket."""
+    import torch
+    import paged_kv_cache_349_b200 as pa
+    case = W.make_case(4, batch=6, max_len=2500, num_blocks=700, partition_tokens=512, fill=W.BF16_ZERO)
+    dc = DeviceCase(case)
+    need = pa.pa_decode_workspace_size(case.batch, case.num_q_heads, case.num_kv_heads, case.head_dim,
+                                       case.block_size, case.max_seq_len, 512)
+    ws = torch.zeros(need, dtype=torch.uint8, device="cuda")
+
+    def call():
+        pa.pa_decode(dc.out, dc.q, dc.k, dc.v, dc.tables, dc.lens, max_seq_len=case.max_seq_len,
+                     scale=float(case.scale), partition_tokens=512, workspace=ws, err_flag=dc.flag)
+
+    s = torch.cuda.Stream()
+    s.wait_stream(torch.cuda.current_stream())
+    with torch.cuda.stream(s):
+        call()  # warm-up outside the capture (kernel attributes, tensor maps)
+    torch.cuda.current_stream().wait_stream(s)
+    torch.cuda.synchronize()
+    eager = dc.out.clone()
+    g = torch.cuda.CUDAGraph()
+    with torch.cuda.graph(g):
+        call()
+    for _ in range(3):
+        dc.out.fill_(float("nan"))
+        g.replay()
+        torch.cuda.synchronize()
+        assert torch.equal(dc.out, eager)
+    assert int(dc.flag.item()) == 0
+    del g
 
 
 def test_kernels_are_native_launches():
