@@ -257,7 +257,6 @@ int decode_impl(float *out, const void *q, const void *k_new, const void *v_new,
         if (!workspace || workspace_bytes < need || !aligned16(workspace)) return PA_ERR_INVALID_ARG;
         p.part_tokens = pt;
         p.num_parts = (max_seq_len + pt - 1) / pt;
-        if (p.num_parts > 65535) return PA_ERR_UNSUPPORTED;
         const int64_t slots = split_slots(max_seq_len, pt, prefix);
         p.num_slots = (int)slots;
         const SplitLayout l = split_layout(batch, num_q_heads, num_kv_heads, head_dim, slots);
@@ -276,6 +275,7 @@ int decode_impl(float *out, const void *q, const void *k_new, const void *v_new,
             if (z > 65535) return PA_ERR_UNSUPPORTED;
             grid_z = (int)z;
         }
+        if (p.num_parts > 65535) return PA_ERR_UNSUPPORTED;
     } else {
         p.part_tokens = max_seq_len > 0 ? max_seq_len : 1;
         p.num_parts = 1;
@@ -295,18 +295,18 @@ int decode_impl(float *out, const void *q, const void *k_new, const void *v_new,
         return append ? launch_decode_d<true, true, false, true>(head_dim, km, vm, p, grid_z, s)
                       : launch_decode_d<true, false, false, true>(head_dim, km, vm, p, grid_z, s);
     }
-    if (fp8) {
-        if (append)
-            return split ? launch_decode_d<true, true, true>(head_dim, km, vm, p, grid_z, s)
-                         : launch_decode_d<false, true, true>(head_dim, km, vm, p, grid_z, s);
-        return split ? launch_decode_d<true, false, true>(head_dim, km, vm, p, grid_z, s)
-                     : launch_decode_d<false, false, true>(head_dim, km, vm, p, grid_z, s);
+    if (!split) {
+        if (fp8)
+            return append ? launch_decode_d<false, true, true>(head_dim, km, vm, p, grid_z, s)
+                          : launch_decode_d<false, false, true>(head_dim, km, vm, p, grid_z, s);
+        return append ? launch_decode_d<false, true, false>(head_dim, km, vm, p, grid_z, s)
+                      : launch_decode_d<false, false, false>(head_dim, km, vm, p, grid_z, s);
     }
-    if (append)
-        return split ? launch_decode_d<true, true, false>(head_dim, km, vm, p, grid_z, s)
-                     : launch_decode_d<false, true, false>(head_dim, km, vm, p, grid_z, s);
-    return split ? launch_decode_d<true, false, false>(head_dim, km, vm, p, grid_z, s)
-                 : launch_decode_d<false, false, false>(head_dim, km, vm, p, grid_z, s);
+    if (fp8)
+        return append ? launch_decode_d<true, true, true>(head_dim, km, vm, p, grid_z, s)
+                      : launch_decode_d<true, false, true>(head_dim, km, vm, p, grid_z, s);
+    return append ? launch_decode_d<true, true, false>(head_dim, km, vm, p, grid_z, s)
+                  : launch_decode_d<true, false, false>(head_dim, km, vm, p, grid_z, s);
 }
 
 }  // namespace pa

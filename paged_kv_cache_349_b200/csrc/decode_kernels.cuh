@@ -166,29 +166,42 @@ __device__ __forceinline__ int group_shared_tokens(const DecodeParams &p, int g)
     return s > 0 ? s / kTileTokens * kTileTokens : 0;
 }
 
-// Arrival ticket of one partition on (sequence, kv head): returns true for the
-// last of the `expected` partitions of this call.  A ticket word holds
+// Arrival ticket of `count` partitions on (sequence, kv head): returns true
+// for the CTA whose arrival completes the `expected` partitions of this call.  A ticket word holds
 // (epoch << 32) | count; a word tagged with another epoch (an earlier call, or
 // uninitialised memory) counts as zero, so the workspace needs no clearing.
-// The last arrival resets the word to 0, which keeps a replayed call (same
-// epoch) correct.  The CAS loop only retries when another partition arrived
-// in between; it is bounded all the same.
-__device__ __forceinline__ bool take_ticket(unsigned long long *t, unsigned int epoch, int expected,
+// All partitions of a pair tend to finish together, so the common path is one
+// atomicAdd: only a word still carrying a stale tag is claimed with a CAS, and
+// a CAS that loses to another arrival re-reads a word that now carries this
+// call's tag.  (The tag cannot change under an arrival that has not counted
+// yet: the count cannot reach `expected` without it.)  The last arrival resets
+// the word to 0, which keeps a replayed call (same epoch) correct.
+__device__ __forceinline__ bool take_ticket(unsigned long long *t, unsigned int epoch, int count, int expected,
                                             int32_t *flag) {
+    const unsigned long long tag = (unsigned long long)epoch << 32;
     unsigned long long old = *reinterpret_cast<volatile unsigned long long *>(t);
-    for (int it = 0; it < (1 << 20); ++it) {
-        const unsigned int cnt = (unsigned int)(old >> 32) == epoch ? (unsigned int)old : 0u;
-        const unsigned long long want = ((unsigned long long)epoch << 32) | (cnt + 1u);
-        const unsigned long long seen = atomicCAS(t, old, want);
-        if (seen == old) {
-            if ((int)(cnt + 1u) < expected) return false;
-            atomicExch(t, 0ull);
-            return true;
+    bool counted = false;
+    for (int it = 0; it < 64 && !counted; ++it) {
+        if ((old >> 32) == epoch) {
+            old = atomicAdd(t, (unsigned long long)count);
+            counted = true;
+        } else {
+            const unsigned long long seen = atomicCAS(t, old, tag | (unsigned long long)count);
+            if (seen == old) {
+                old = tag;
+                counted = true;
+            } else {
+                old = seen;
+            }
         }
-        old = seen;
     }
-    raise_flag(flag, PA_FLAG_TIMEOUT);
-    return false;
+    if (!counted) {
+        raise_flag(flag, PA_FLAG_TIMEOUT);
+        return false;
+    }
+    if ((int)((unsigned int)old + (unsigned int)count) < expected) return false;
+    atomicExch(t, 0ull);
+    return true;
 }
 
 // Byte offset of 16-byte chunk c of token row r inside one swizzled 16-bit tile.
@@ -231,39 +244,104 @@ __device__ __forceinline__ void mma_16816(float (&d)[4], uint32_t a0, uint32_t a
 //   out = sum_p 2^(m_p - M) l_p o_p / sum_p 2^(m_p - M) l_p,  M = max_p m_p,
 // over the shared-prefix slots [0, n_pre) and the sequence's own slots
 // [s0, s0 + n_own).  Partials written by other CTAs are read through L2.
+// All threads of the CTA take part: one warp per head finds M and writes the
+// weights of a chunk of slots to shared memory (`sm`, 16 + 8 * kMergeChunk
+// floats), and each thread sums up to two float4 output columns with eight
+// slot loads in flight.
+constexpr int kMergeChunk = 256;
+
 template <int HEAD_DIM>
-__device__ __forceinline__ void merge_partials(const DecodeParams &p, int b, int h, int n_pre, int s0, int n_own) {
+__device__ __forceinline__ void merge_partials(const DecodeParams &p, int b, int h, int n_pre, int s0, int n_own,
+                                               float *sm) {
     constexpr int kCols = HEAD_DIM / 4;  // float4 columns of a row
+    constexpr int kWarps = kThreads / 32;
     const int G = p.group;
-    for (int x = threadIdx.x; x < G * kCols; x += kThreads) {
-        const int g = x / kCols;
-        const int c4 = x - g * kCols;
-        const int64_t row = (int64_t)b * p.num_q_heads + (int64_t)h * G + g;
-        const float2 *ml = reinterpret_cast<const float2 *>(p.part_ml) + row * p.num_slots;
-        const float4 *po = reinterpret_cast<const float4 *>(p.part_o + row * p.num_slots * HEAD_DIM) + c4;
-        const int n = n_pre + n_own;
+    const int n = n_pre + n_own;
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    float *s_max = sm;       // [8]
+    float *s_w = sm + 16;    // [8][kMergeChunk]
+    const int64_t row0 = (int64_t)b * p.num_q_heads + (int64_t)h * G;
+    const float2 *ml0 = reinterpret_cast<const float2 *>(p.part_ml) + row0 * p.num_slots;
+    auto slot_of = [&](int k) { return k < n_pre ? k : s0 + k - n_pre; };
+    // One warp per head: the (max, sum) pairs of the first kMergeChunk slots are
+    // read once, kept in registers for the max and turned into weights in place.
+    constexpr int kPerLane = kMergeChunk / 32;
+    for (int g = warp; g < G; g += kWarps) {
+        const float2 *mlg = ml0 + (int64_t)g * p.num_slots;
+        float2 v[kPerLane];
         float M = -INFINITY;
-        for (int k = 0; k < n; ++k) M = fmaxf(M, __ldcg(ml + (k < n_pre ? k : s0 + k - n_pre)).x);
-        float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
-        float den = 0.f;
-        if (M != -INFINITY) {
-#pragma unroll 4
-            for (int k = 0; k < n; ++k) {
-                const int s = k < n_pre ? k : s0 + k - n_pre;
-                const float2 mlv = __ldcg(ml + s);
-                const float w = fast_exp2(mlv.x - M) * mlv.y;
-                const float4 o = __ldcg(po + (int64_t)s * kCols);
-                acc.x += w * o.x;
-                acc.y += w * o.y;
-                acc.z += w * o.z;
-                acc.w += w * o.w;
-                den += w;
+#pragma unroll
+        for (int i = 0; i < kPerLane; ++i) {
+            const int k = lane + 32 * i;
+            v[i] = k < n ? __ldcg(mlg + slot_of(k)) : make_float2(-INFINITY, 0.f);
+            M = fmaxf(M, v[i].x);
+        }
+        for (int k = kMergeChunk + lane; k < n; k += 32) M = fmaxf(M, __ldcg(mlg + slot_of(k)).x);
+#pragma unroll
+        for (int off = 16; off; off >>= 1) M = fmaxf(M, __shfl_xor_sync(0xffffffffu, M, off));
+        if (lane == 0) s_max[g] = M;
+#pragma unroll
+        for (int i = 0; i < kPerLane; ++i) {
+            const int k = lane + 32 * i;
+            if (k < n && k < kMergeChunk) s_w[g * kMergeChunk + k] = M == -INFINITY ? 0.f : fast_exp2(v[i].x - M) * v[i].y;
+        }
+    }
+    // Output columns of this thread: x and x + kThreads (G * kCols <= 256 <= 2 * kThreads).
+    int col[2], gcol[2];
+    const float4 *po[2];
+#pragma unroll
+    for (int i = 0; i < 2; ++i) {
+        col[i] = threadIdx.x + i * kThreads;
+        gcol[i] = col[i] / kCols;
+        po[i] = reinterpret_cast<const float4 *>(p.part_o + (row0 + gcol[i]) * p.num_slots * HEAD_DIM) +
+                (col[i] - gcol[i] * kCols);
+    }
+    const bool on0 = col[0] < G * kCols, on1 = col[1] < G * kCols;
+    float4 acc[2] = {make_float4(0.f, 0.f, 0.f, 0.f), make_float4(0.f, 0.f, 0.f, 0.f)};
+    float den[2] = {0.f, 0.f};
+    for (int c0 = 0; c0 < n; c0 += kMergeChunk) {
+        const int cn = min(kMergeChunk, n - c0);
+        __syncthreads();  // the first chunk's weights are written; a later chunk's predecessor is consumed
+        if (c0 > 0) {
+            for (int x = threadIdx.x; x < G * cn; x += kThreads) {
+                const int g = x / cn, k = x - g * cn;
+                const float M = s_max[g];
+                const float2 mlv = __ldcg(ml0 + (int64_t)g * p.num_slots + slot_of(c0 + k));
+                s_w[g * kMergeChunk + k] = M == -INFINITY ? 0.f : fast_exp2(mlv.x - M) * mlv.y;
+            }
+            __syncthreads();
+        }
+#pragma unroll 8
+        for (int k = 0; k < cn; ++k) {
+            const int64_t s = slot_of(c0 + k);
+            if (on0) {
+                const float w = s_w[gcol[0] * kMergeChunk + k];
+                const float4 o = __ldcg(po[0] + s * kCols);
+                acc[0].x += w * o.x;
+                acc[0].y += w * o.y;
+                acc[0].z += w * o.z;
+                acc[0].w += w * o.w;
+                den[0] += w;
+            }
+            if (on1) {
+                const float w = s_w[gcol[1] * kMergeChunk + k];
+                const float4 o = __ldcg(po[1] + s * kCols);
+                acc[1].x += w * o.x;
+                acc[1].y += w * o.y;
+                acc[1].z += w * o.z;
+                acc[1].w += w * o.w;
+                den[1] += w;
             }
         }
-        const float r = den > 0.f ? 1.f / den : 0.f;
-        reinterpret_cast<float4 *>(p.out + row * HEAD_DIM)[c4] =
-            make_float4(acc.x * r, acc.y * r, acc.z * r, acc.w * r);
     }
+#pragma unroll
+    for (int i = 0; i < 2; ++i) {
+        if (i == 0 ? !on0 : !on1) continue;
+        const float r = den[i] == 0.f ? 0.f : 1.f / den[i];  // no tokens: zeros; a NaN stays NaN
+        reinterpret_cast<float4 *>(p.out + row0 * HEAD_DIM)[col[i]] =
+            make_float4(acc[i].x * r, acc[i].y * r, acc[i].z * r, acc[i].w * r);
+    }
+    __syncthreads();  // the scratch is free for the next merge of this CTA
 }
 
 template <int HEAD_DIM, bool SPLIT, bool APPEND, bool FP8, bool PREFIX>
@@ -819,28 +897,32 @@ __global__ void __launch_bounds__(kThreads, FP8 ? PA_DECODE_MIN_CTAS_FP8 : PA_DE
         const int64_t row = (int64_t)(b + n / G) * p.num_q_heads + (int64_t)h * G + n % G;
         if (FP8) num *= p.v_scale;
         if (SPLIT && !direct) {
-            p.part_o[(row * p.num_slots + slot) * HEAD_DIM + d] = den > 0.f ? num / den : 0.f;
+            p.part_o[(row * p.num_slots + slot) * HEAD_DIM + d] = den == 0.f ? 0.f : num / den;
             if (d == 0) {
                 p.part_ml[(row * p.num_slots + slot) * 2] = M;
                 p.part_ml[(row * p.num_slots + slot) * 2 + 1] = den;
             }
         } else {
-            p.out[row * HEAD_DIM + d] = den > 0.f ? num / den : 0.f;
+            // No tokens: a zero row.  A NaN read from an attended row stays NaN.
+            p.out[row * HEAD_DIM + d] = den == 0.f ? 0.f : num / den;
         }
     }
     if constexpr (SPLIT) {
         if (direct) return;
         // Ticket: this partition's state is stored.  The CTA whose ticket is the
-        // last of a (member, kv head) merges that pair's partitions.
-        __threadfence();  // every thread's partial stores, visible GPU-wide before the ticket
+        // last of a (member, kv head) merges that pair's partitions.  The barrier
+        // orders every thread's partial stores before thread 0's device-scope
+        // fence, which publishes them before the ticket (and, for the last
+        // arrival, orders the other partitions' states before they are read).
         __syncthreads();
         if (threadIdx.x == 0) {
+            __threadfence();
             unsigned int mask = 0;
             for (int m = 0; m < nmem; ++m) {
                 const int bm = b + m;
                 const int Lm = pre ? clamp_len(__ldg(p.seq_lens + bm), p) : L;
                 const int expected = parts_of(shared, p.part_tokens) + parts_of(Lm - shared, p.part_tokens);
-                if (take_ticket(p.tickets + (int64_t)bm * p.num_kv_heads + h, p.epoch, expected, p.err_flag))
+                if (take_ticket(p.tickets + (int64_t)bm * p.num_kv_heads + h, p.epoch, 1, expected, p.err_flag))
                     mask |= 1u << m;
             }
             if (mask) __threadfence();  // the other partitions' states, seen before they are read
@@ -848,12 +930,13 @@ __global__ void __launch_bounds__(kThreads, FP8 ? PA_DECODE_MIN_CTAS_FP8 : PA_DE
         }
         __syncthreads();
         const unsigned int mask = s_last;
+        static_assert((16 + 8 * kMergeChunk) * 4 <= C::kRingBytes, "merge scratch reuses the ring");
         for (int m = 0; m < nmem; ++m) {
             if (!(mask & (1u << m))) continue;
             const int bm = b + m;
             const int Lm = pre ? clamp_len(__ldg(p.seq_lens + bm), p) : L;
             merge_partials<HEAD_DIM>(p, bm, h, parts_of(shared, p.part_tokens), PREFIX ? p.num_parts : 0,
-                                     parts_of(Lm - shared, p.part_tokens));
+                                     parts_of(Lm - shared, p.part_tokens), reinterpret_cast<float *>(smem));
         }
     }
 }

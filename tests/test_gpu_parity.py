@@ -177,6 +177,10 @@ def test_bad_lengths_flagged_in_every_mode(pt):
     dc = DeviceCase(case)
     # the default of this shape splits (4 sequences x 2 kv heads, up to 1500 tokens)
     assert pt != 0 or pa.pa_decode_partition_tokens(4, 8, 2, 128, 16, case.max_seq_len, 0) > 0
+    # complete the pools with the step's new tokens, on both sides
+    pa.pa_reshape_and_cache(dc.k_new, dc.v_new, dc.k, dc.v, dc.slots, err_flag=dc.flag)
+    k_ref, v_ref = case.k_cache.copy(), case.v_cache.copy()
+    assert oracle.reshape_and_cache(case.k_new, case.v_new, k_ref, v_ref, case.slot_mapping, 16) == 0
     for lens, max_len in (([-5, 33, 700, 1500], case.max_seq_len), ([20, 33, 700, 1500], 1000)):
         bad = np.array(lens, np.int32)
         ws_bytes = pa.pa_decode_workspace_size(case.batch, 8, 2, 128, 16, max_len, pt)
@@ -189,7 +193,7 @@ def test_bad_lengths_flagged_in_every_mode(pt):
         assert int(dc.flag.item()) == pa.PA_FLAG_BAD_LEN, (lens, max_len, pt)
         got = dc.out.cpu().numpy().astype(np.float64)
         clamped = np.clip(bad, 0, max_len)
-        want = oracle.decode(case.q, case.k_cache, case.v_cache, case.block_tables, clamped,
+        want = oracle.decode(case.q, k_ref, v_ref, case.block_tables, clamped,
                              num_kv_heads=2, block_size=16, scale=case.scale)
         assert_close(got, want, f"lens {lens} max {max_len} pt {pt}")
         if lens[0] < 0:
@@ -275,6 +279,34 @@ def test_split_decode_replays_in_a_cuda_graph():
         assert torch.equal(dc.out, eager)
     assert int(dc.flag.item()) == 0
     del g
+
+
+@pytest.mark.parametrize("pt", [-1, 16])
+def test_nan_in_an_attended_row_propagates(pt):
+    """A NaN in a row the decode attends gives NaN in that sequence's outputs, as in the oracle;
+    sequences that do not read the row are unaffected and empty ones stay zero."""
+    import torch
+    import paged_kv_cache_349_b200 as pa
+    case = W.make_custom_case([0, 40, 70], num_q_heads=4, num_kv_heads=2, head_dim=128, block_size=16, seed=17)
+    dc = DeviceCase(case)
+    pa.pa_reshape_and_cache(dc.k_new, dc.v_new, dc.k, dc.v, dc.slots, err_flag=dc.flag)
+    k_ref, v_ref = case.k_cache.copy(), case.v_cache.copy()
+    oracle.reshape_and_cache(case.k_new, case.v_new, k_ref, v_ref, case.slot_mapping, 16)
+    blk = int(case.block_tables[1, 1])  # token 20 of sequence 1, kv head 0
+    k_ref[blk, 0, 4, 7] = 0x7FC0
+    dc.k[blk, 0, 4, 7] = float("nan")
+    ws = torch.empty(max(pa.pa_decode_workspace_size(3, 4, 2, 128, 16, 70, pt), 16), dtype=torch.uint8,
+                     device="cuda")
+    pa.pa_decode(dc.out, dc.q, dc.k, dc.v, dc.tables, dc.lens, max_seq_len=70, scale=float(case.scale),
+                 partition_tokens=pt, workspace=ws, err_flag=dc.flag)
+    torch.cuda.synchronize()
+    got = dc.out.cpu().numpy().astype(np.float64)
+    want = oracle.decode(case.q, k_ref, v_ref, case.block_tables, case.seq_lens, num_kv_heads=2, block_size=16,
+                         scale=case.scale)
+    assert np.all(np.isnan(want[1, :2])) and np.all(np.isnan(got[1, :2]))
+    assert np.all(got[0] == 0)
+    assert_close(got[1, 2:], want[1, 2:], "other kv head")
+    assert_close(got[2], want[2], "other sequence")
 
 
 def test_kernels_are_native_launches():
