@@ -223,6 +223,9 @@ def cpu_baseline(case, budget_s: float = 12.0):
     workload until about ``budget_s`` seconds of oracle time have passed.
     Returns the oracle's throughput in the bench's unit (algorithmic GB/s),
     the threads it used, what the sample was, the seconds and bytes timed.
+    Bytes are counted as the GPU arm counts them: for a workload whose
+    sequences share blocks, the sample's logical bytes are scaled by the
+    workload's ratio of unique to logical decode bytes.
     """
     import oracle
     threads = len(os.sched_getaffinity(0))
@@ -246,11 +249,18 @@ def cpu_baseline(case, budget_s: float = 12.0):
         done_bytes += sum(int(case.seq_lens[b]) * case.head_dim * 4 + G * case.head_dim * 6 for b, _ in sel)
         if dt < budget_s / 20:
             chunk *= 2
-    gbs = done_bytes / elapsed / 1e9
+    scale = 1.0
+    if case.groups is not None:
+        scale = decode_bytes(case, 2, unique=True) / decode_bytes(case, 2, unique=False)
+    counted = done_bytes * scale
+    gbs = counted / elapsed / 1e9
     sample = (f"{done_units} (sequence, kv head) units ({done_units / len(units):.2f} passes over the "
               f"workload's {len(units)}), {done_units * G} query-head rows, {done_bytes / 1e9:.2f} GB of "
-              f"K/V/q/out, {elapsed:.1f} s of oracle time")
-    return gbs, threads, sample, elapsed, done_bytes
+              f"K/V/q/out read"
+              + (f", counted as {counted / 1e9:.2f} GB (x{scale:.3f}: shared rows once, as the GPU arm counts)"
+                 if scale != 1.0 else "")
+              + f", {elapsed:.1f} s of oracle time")
+    return gbs, threads, sample, elapsed, counted
 
 
 # ---------------------------------------------------------------------------
@@ -290,8 +300,12 @@ def measure_workload(cfg, args, world, rank, pa, headline):
     case = W.make_case(cfg, seed=seed, fill=W.BF16_ZERO, num_blocks=args.num_blocks)
     fp8 = args.kv_dtype == "fp8"
     elem = 1 if fp8 else 2
-    # Shared-prefix groups (the n=4 chat mix): their shared tiles are read once per group.
-    prefix = case.groups is not None and args.decode != "plain" and not fp8 and not args.unfused
+    # Shared-prefix groups (the n=4 chat mix): the step decodes with the plain fused decode
+    # (on B200 the 126 MB L2 already serves the repeated prefix reads of neighbouring CTAs);
+    # the shared-prefix decode, which reads each group's shared tiles once, is timed beside it,
+    # with L2 warm and with L2 flushed before each call.
+    has_groups = case.groups is not None and not fp8 and not args.unfused
+    prefix = has_groups and args.decode == "shared-prefix"
     group_size = 4
     copy_b, write_b, _ = step_bytes(case, elem)
     shared_rows = case.groups is not None
@@ -340,7 +354,7 @@ def measure_workload(cfg, args, world, rank, pa, headline):
                                            case.block_size, case.max_seq_len, pt)
     ws_bytes = ws_plain
     prefix_lens = None
-    if prefix:
+    if has_groups:
         prefix_lens = i32(case.shared_tokens[::group_size])
         ws_bytes = max(ws_bytes, pa.pa_decode_shared_prefix_workspace_size(
             case.batch, group_size, case.num_q_heads, case.num_kv_heads, case.head_dim, case.block_size,
@@ -426,17 +440,28 @@ def measure_workload(cfg, args, world, rank, pa, headline):
     dec_ms = _max_over_ranks(statistics.mean(a.elapsed_time(b) for a, b in dec_ev), world)
     assert int(flag.item()) == 0, f"error flag {int(flag.item()):#x}"
 
-    # The same step with the plain decode, for comparison (the chat mix only).
-    alt_ms = None
-    if prefix:
-        alt_ev = []
-        for _ in range(args.warmup):
-            step(kind="plain")
-        torch.cuda.synchronize()
-        for _ in range(args.steps):
-            step(record=True, kind="plain", evs=alt_ev)
-        torch.cuda.synchronize()
-        alt_ms = _max_over_ranks(statistics.mean(a.elapsed_time(b) for a, b in alt_ev), world)
+    # The chat mix: the other decode of the same step, and both with L2 flushed before each call.
+    alt_ms, cold = None, None
+    if has_groups:
+        kind_alt = "plain" if prefix else "shared-prefix"
+
+        def decode_ms(kind, flush=None):
+            evs = []
+            for _ in range(args.warmup):
+                step(kind=kind)
+            torch.cuda.synchronize()
+            for _ in range(args.steps):
+                if flush is not None:
+                    flush.fill_(1)
+                step(record=True, kind=kind, evs=evs)
+            torch.cuda.synchronize()
+            return _max_over_ranks(statistics.mean(a.elapsed_time(b) for a, b in evs), world)
+
+        alt_ms = decode_ms(kind_alt)
+        l2 = torch.cuda.get_device_properties(torch.cuda.current_device()).L2_cache_size
+        flush = torch.empty(2 * l2, dtype=torch.uint8, device="cuda")
+        cold = {kind: round(decode_ms(kind, flush), 5) for kind in ("plain", "shared-prefix")}
+        del flush
         assert int(flag.item()) == 0, f"error flag {int(flag.item()):#x}"
 
     all_bytes = _sum_over_ranks(float(total_b), world)
@@ -476,8 +501,13 @@ def measure_workload(cfg, args, world, rank, pa, headline):
             roof["traffic_vs_unique"] = round(traffic / dec_b, 4)
             roof["traffic_vs_logical"] = round(traffic / dec_logical, 4)
     if alt_ms is not None:
-        roof["plain_decode_launch_ms"] = round(alt_ms, 5)
-        roof["plain_decode_achieved"] = round(dec_b / (alt_ms / 1e3) / 1e9, 1)
+        alt_name = "plain_decode" if prefix else "shared_prefix_decode"
+        roof[f"{alt_name}_launch_ms"] = round(alt_ms, 5)
+        roof[f"{alt_name}_achieved"] = round(dec_b / (alt_ms / 1e3) / 1e9, 1)
+        roof["l2_flushed_launch_ms"] = cold
+        roof["l2_flushed_note"] = (f"decode call with a {2 * l2 >> 20} MiB buffer written before each call: "
+                                   "the shared-prefix decode reads each group's shared tiles once, the plain "
+                                   "decode relies on L2 for the repeats")
 
     entry = {
         "value": round(value, 1),
@@ -492,12 +522,7 @@ def measure_workload(cfg, args, world, rank, pa, headline):
             "partition_tokens": case.partition_tokens,
             "parallelism": f"dp{world} (independent sequences per GPU, no collective)",
             "l2": f"inputs larger than L2: {dec_b / 1e9:.2f} GB of K/V per step vs 126 MB L2; no flush",
-            "step": ("block copies, then pa_decode_append_fp8 (the write quantises to E4M3 and is fused into decode)"
-                     if fp8 else
-                     "block copies, cache write of copy-on-write rows, then pa_decode_shared_prefix (each group's "
-                     "shared tiles read once; cache write of each sequence's new token fused)" if prefix else
-                     "block copies, then pa_decode_append (cache write fused into decode)" if fused else
-                     "block copies, pa_reshape_and_cache, pa_decode"),
+            "step": step_description(case, fp8, prefix, fused),
         },
         "pct_of_peak": {"nominal_8TBps": round(100 * value / NOMINAL_HBM_GBS, 1),
                         f"{peak_kind}_{peak:.0f}GBps": round(100 * value / peak, 1)},
@@ -687,6 +712,21 @@ def step_bytes_from(case, lens, n_pairs, kv_elem_bytes: int = 2):
 # reference arm: the fp64 oracle on the host cores
 # ---------------------------------------------------------------------------
 
+def step_description(case, fp8: bool, prefix: bool, fused: bool) -> str:
+    """What one timed step runs, in order."""
+    copies = "block copies, " if case.copy_pairs.shape[0] else ""
+    _, _, other = W.split_last_tokens(case)
+    cow = "cache write of the copy-on-write rows, " if other.size else ""
+    if fp8:
+        return copies + cow + "pa_decode_append_fp8 (each new token quantised to E4M3 and written by the decode)"
+    if prefix:
+        return (copies + cow + "pa_decode_shared_prefix (each group's shared tiles read once; each new token "
+                "written by the decode)")
+    if fused:
+        return copies + cow + "pa_decode_append (each sequence's new token written by the decode launch)"
+    return copies + "pa_reshape_and_cache, pa_decode"
+
+
 def reference_config(case, cfg, base, world):
     """The reference arm's ``config``: the same keys and values as the native arm's headline."""
     prefix = case.groups is not None
@@ -700,9 +740,7 @@ def reference_config(case, cfg, base, world):
         "partition_tokens": case.partition_tokens,
         "parallelism": f"dp{world} (independent sequences per GPU, no collective)",
         "l2": f"inputs larger than L2: {dec_b / 1e9:.2f} GB of K/V per step vs 126 MB L2; no flush",
-        "step": ("block copies, cache write of copy-on-write rows, then pa_decode_shared_prefix (each group's "
-                 "shared tiles read once; cache write of each sequence's new token fused)" if prefix else
-                 "block copies, then pa_decode_append (cache write fused into decode)"),
+        "step": step_description(case, False, False, True),
     }
 
 
@@ -750,8 +788,9 @@ def main():
     ap.add_argument("--per-config", type=str, default=None,
                     help="comma-separated workloads timed after the headline into per_config "
                          "(default: 2,4,5 when --config is left at its default, none otherwise)")
-    ap.add_argument("--decode", choices=["auto", "plain"], default="auto",
-                    help="plain: the chat mix decodes with pa_decode_append instead of the shared-prefix decode")
+    ap.add_argument("--decode", choices=["plain", "shared-prefix"], default="plain",
+                    help="the chat mix's step: pa_decode_append (plain) or pa_decode_shared_prefix; the other "
+                         "is timed beside it")
     ap.add_argument("--impl", choices=["native", "reference"], default="native")
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--step-chunks", type=int, default=0,

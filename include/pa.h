@@ -166,20 +166,18 @@ int pa_swap_blocks(void *dst_k_cache, void *dst_v_cache, int64_t dst_num_blocks,
  *                 (sequence, kv head), > 0 = split each sequence into
  *                 partitions of this many tokens (a multiple of block_size).
  *                 Each partition stores its partial softmax state (max, sum,
- *                 normalised output) in the workspace; the CTA whose
- *                 partition of a (sequence, kv head) finishes last merges
- *                 them (log-sum-exp) and writes the output, inside the same
- *                 launch.  A sequence that fits one partition is written
- *                 directly.
+ *                 normalised output) in the workspace, and a second kernel,
+ *                 launched as a programmatic dependent, merges them
+ *                 (log-sum-exp).  A sequence that fits one partition is
+ *                 written by the decode directly.
  * workspace     : device scratch of at least pa_decode_workspace_size(...)
  *                 bytes, 16-byte aligned (may be NULL if that size is 0).
- *                 Its contents need no initialisation: the arrival counters
- *                 it holds carry a per-call tag, so whatever an earlier call
- *                 (or uninitialised memory) left there reads as zero.  Calls
+ *                 Its contents need no initialisation: every partial state
+ *                 the merge reads is written earlier in the same call.  Calls
  *                 that run at the same time need separate workspaces.
  * Each (sequence, kv head) is processed by one CTA (per partition) that
  * serves all query heads of the group, so every K/V byte is read once.
- * Launches exactly one kernel (none when batch == 0).  Shared-prefix
+ * Launches one kernel, two when it splits (none when batch == 0).  Shared-prefix
  * locality: the grid runs the kv heads and partitions of a sequence next to
  * each other with the sequence index slowest, so sequences that follow each
  * other in the batch and share blocks (forks) re-read those blocks from L2.
@@ -376,9 +374,8 @@ int pa_decode_step_host_fp8(float *out_host, const void *q_host, const void *k_n
  *  - No cudaMalloc, cudaFree or other allocating routine is called.
  *  - All calls share the one array, and it keeps whatever the last call
  *    wrote.  Nothing in it has to start at zero: each partition's state is
- *    written before it is read within the same call, and the arrival
- *    counters carry a per-call tag.  Calls queued one after another on one
- *    stream are safe.  Calls whose kernels can overlap on the GPU (different
+ *    written before it is read within the same call.  Calls queued one
+ *    after another on one stream are safe.  Calls whose kernels can overlap on the GPU (different
  *    streams, or several host threads) race on the array; issue them on one
  *    stream.
  * Other arguments, layouts and errors: as pa_decode.

@@ -1,10 +1,7 @@
 // Host side of the paged decode: tensor maps of the pools, the choice of
 // partitioning, the split workspace layout, the decode launches (the device
 // code is in decode_kernels.cuh) and the C entry points.
-#include <atomic>
-#include <chrono>
 #include <mutex>
-#include <random>
 
 #include "decode_kernels.cuh"
 
@@ -124,37 +121,38 @@ int launch_decode(const CUtensorMap &km, const CUtensorMap &vm, const DecodePara
     dim3 grid((unsigned)p.num_parts, (unsigned)p.num_kv_heads, (unsigned)grid_z);
     kern<<<grid, kThreads, C::kSmemBytes, stream>>>(km, vm, p);
     count_launch();
-    return launch_status();
+    int st = launch_status();
+    if (st != PA_OK || !SPLIT) return st;
+    // The reduce, one CTA per (query head, sequence), launched as a programmatic
+    // dependent: it is scheduled while the decode's last wave runs and waits
+    // (griddepcontrol.wait) for the decode grid's results.
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = dim3((unsigned)p.num_q_heads, (unsigned)p.batch);
+    cfg.blockDim = dim3(kReduceThreads);
+    cfg.dynamicSmemBytes = 0;
+    cfg.stream = stream;
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    attr[0].val.programmaticStreamSerializationAllowed = 1;
+    cfg.attrs = attr;
+    cfg.numAttrs = 1;
+    const cudaError_t e = cudaLaunchKernelEx(&cfg, lse_reduce_kernel<HEAD_DIM, PREFIX>, p);
+    count_launch();
+    return e == cudaSuccess ? launch_status() : PA_ERR_CUDA;
 }
 
-// Tag of one split call in the arrival tickets: a process-wide counter that
-// starts at a random value (so a workspace left over by another process does
-// not share tags with this one) and skips 0.
-unsigned int next_epoch() {
-    static std::atomic<unsigned int> ctr{[] {
-        std::random_device rd;
-        return (unsigned int)rd() ^ (unsigned int)std::chrono::steady_clock::now().time_since_epoch().count();
-    }()};
-    unsigned int e = ctr.fetch_add(1u);
-    while (e == 0u) e = ctr.fetch_add(1u);
-    return e;
-}
-
-// Split workspace: partial states part_o [B, Hq, slots, d] and part_ml
-// [B, Hq, slots, 2] (fp32), then the tickets [B, Hkv] (uint64); each section
-// 256-byte aligned.
+// Split workspace: partial states part_o [B, Hq, slots, d], then part_ml
+// [B, Hq, slots, 2] (fp32) 256-byte aligned.
 struct SplitLayout {
-    size_t o, ml, tickets, total;
+    size_t o, ml, total;
 };
 
-SplitLayout split_layout(int64_t batch, int num_q_heads, int num_kv_heads, int head_dim, int64_t slots) {
-    auto up = [](int64_t x) { return (size_t)((x + 255) / 256 * 256); };
+SplitLayout split_layout(int64_t batch, int num_q_heads, int head_dim, int64_t slots) {
     const int64_t rows = batch * num_q_heads * slots;
     SplitLayout l{};
     l.o = 0;
-    l.ml = up(rows * head_dim * 4);
-    l.tickets = l.ml + up(rows * 2 * 4);
-    l.total = l.tickets + (size_t)(batch * num_kv_heads * 8);
+    l.ml = (size_t)((rows * head_dim * 4 + 255) / 256 * 256);
+    l.total = l.ml + (size_t)(rows * 2 * 4);
     return l;
 }
 
@@ -259,12 +257,10 @@ int decode_impl(float *out, const void *q, const void *k_new, const void *v_new,
         p.num_parts = (max_seq_len + pt - 1) / pt;
         const int64_t slots = split_slots(max_seq_len, pt, prefix);
         p.num_slots = (int)slots;
-        const SplitLayout l = split_layout(batch, num_q_heads, num_kv_heads, head_dim, slots);
+        const SplitLayout l = split_layout(batch, num_q_heads, head_dim, slots);
         char *ws = static_cast<char *>(workspace);
         p.part_o = reinterpret_cast<float *>(ws + l.o);
         p.part_ml = reinterpret_cast<float *>(ws + l.ml);
-        p.tickets = reinterpret_cast<unsigned long long *>(ws + l.tickets);
-        p.epoch = next_epoch();
         if (prefix) {
             p.prefix_lens = prefix_lens;
             p.group_size = group_size;
@@ -326,8 +322,7 @@ size_t pa_decode_workspace_size(int batch, int num_q_heads, int num_kv_heads, in
     if (batch <= 0 || num_q_heads <= 0 || num_kv_heads <= 0 || max_seq_len <= 0) return 0;
     const int pt = pa::resolve_partition(batch, num_kv_heads, block_size, max_seq_len, partition_tokens);
     if (pt <= 0) return 0;
-    return pa::split_layout(batch, num_q_heads, num_kv_heads, head_dim, pa::split_slots(max_seq_len, pt, false))
-        .total;
+    return pa::split_layout(batch, num_q_heads, head_dim, pa::split_slots(max_seq_len, pt, false)).total;
 }
 
 size_t pa_decode_shared_prefix_workspace_size(int batch, int group_size, int num_q_heads, int num_kv_heads,
@@ -336,8 +331,7 @@ size_t pa_decode_shared_prefix_workspace_size(int batch, int group_size, int num
     if (batch <= 0 || group_size <= 0 || num_q_heads <= 0 || num_kv_heads <= 0 || max_seq_len <= 0) return 0;
     int pt = pa::resolve_partition(batch, num_kv_heads, block_size, max_seq_len, partition_tokens);
     if (pt <= 0) pt = max_seq_len;
-    return pa::split_layout(batch, num_q_heads, num_kv_heads, head_dim, pa::split_slots(max_seq_len, pt, true))
-        .total;
+    return pa::split_layout(batch, num_q_heads, head_dim, pa::split_slots(max_seq_len, pt, true)).total;
 }
 
 int pa_decode(float *out, const void *q, const void *k_cache, const void *v_cache,

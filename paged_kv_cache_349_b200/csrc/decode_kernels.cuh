@@ -22,18 +22,17 @@
 //    N = 8 heads, K = 16 tokens).  P is split into bf16 hi + lo parts so the
 //    PV product keeps ~16 mantissa bits.
 //  * Warps merge their (max, sum, O) states through shared memory.  In the
-//    split variant each CTA writes its partition's state to the workspace,
-//    then takes a ticket on its (sequence, kv head); the CTA that arrives
-//    last merges every partition of that pair (log-sum-exp) and writes the
-//    output, so no second kernel runs.
+//    split variant each CTA writes its partition's state to the workspace
+//    and a log-sum-exp reduce kernel, launched as a programmatic dependent,
+//    combines the partitions.
 //  * Shared-prefix variant: sequences that share their first tokens (n-way
 //    sampling of one prompt) get one extra work item per group and kv head
 //    that reads the shared tiles once and serves every member's query heads
 //    as extra mma columns; each member's own work items start after the
-//    shared tiles, and the ticket merge combines both.
+//    shared tiles, and the reduce combines both.
 //
-// This header holds the device code (the decode kernel with its split
-// merge, its shared-memory layout and parameters).  decode.cu includes it
+// This header holds the device code (the decode kernel, the log-sum-exp
+// reduce, their shared-memory layout and parameters).  decode.cu includes it
 // and holds the host side, so a change there leaves the device code -- and
 // any profile taken of it -- untouched.
 #pragma once
@@ -125,10 +124,7 @@ struct DecodeParams {
     float k_inv_scale;          // fp8 pools: 1 / scale, for the fused cache write
     float v_inv_scale;
     int batch;
-    // Split: partial states per (sequence, query head) and the arrival tickets.
-    int num_slots;              // partial-state slots per row: num_parts (x2 with prefix groups)
-    unsigned long long *tickets;  // [B, Hkv]: (epoch << 32) | partitions arrived
-    unsigned int epoch;         // this call's tag in the tickets (never 0)
+    int num_slots;              // split: partial-state slots per row: num_parts (x2 with prefix groups)
     // Shared-prefix groups: sequences [g*group_size, (g+1)*group_size) share prefix_lens[g] tokens.
     const int32_t *prefix_lens; // [num_groups]
     int group_size;
@@ -166,44 +162,6 @@ __device__ __forceinline__ int group_shared_tokens(const DecodeParams &p, int g)
     return s > 0 ? s / kTileTokens * kTileTokens : 0;
 }
 
-// Arrival ticket of `count` partitions on (sequence, kv head): returns true
-// for the CTA whose arrival completes the `expected` partitions of this call.  A ticket word holds
-// (epoch << 32) | count; a word tagged with another epoch (an earlier call, or
-// uninitialised memory) counts as zero, so the workspace needs no clearing.
-// All partitions of a pair tend to finish together, so the common path is one
-// atomicAdd: only a word still carrying a stale tag is claimed with a CAS, and
-// a CAS that loses to another arrival re-reads a word that now carries this
-// call's tag.  (The tag cannot change under an arrival that has not counted
-// yet: the count cannot reach `expected` without it.)  The last arrival resets
-// the word to 0, which keeps a replayed call (same epoch) correct.
-__device__ __forceinline__ bool take_ticket(unsigned long long *t, unsigned int epoch, int count, int expected,
-                                            int32_t *flag) {
-    const unsigned long long tag = (unsigned long long)epoch << 32;
-    unsigned long long old = *reinterpret_cast<volatile unsigned long long *>(t);
-    bool counted = false;
-    for (int it = 0; it < 64 && !counted; ++it) {
-        if ((old >> 32) == epoch) {
-            old = atomicAdd(t, (unsigned long long)count);
-            counted = true;
-        } else {
-            const unsigned long long seen = atomicCAS(t, old, tag | (unsigned long long)count);
-            if (seen == old) {
-                old = tag;
-                counted = true;
-            } else {
-                old = seen;
-            }
-        }
-    }
-    if (!counted) {
-        raise_flag(flag, PA_FLAG_TIMEOUT);
-        return false;
-    }
-    if ((int)((unsigned int)old + (unsigned int)count) < expected) return false;
-    atomicExch(t, 0ull);
-    return true;
-}
-
 // Byte offset of 16-byte chunk c of token row r inside one swizzled 16-bit tile.
 __device__ __forceinline__ uint32_t tile_offset(int r, int c) {
     return (uint32_t)((c >> 3) * kBox16Bytes + r * 128 + (((c & 7) ^ (r & 7)) << 4));
@@ -239,111 +197,6 @@ __device__ __forceinline__ void mma_16816(float (&d)[4], uint32_t a0, uint32_t a
 #define PA_DECODE_MIN_CTAS_BF16 3
 #endif
 
-// Log-sum-exp merge of every partial state of (sequence b, kv head h), run by
-// the CTA whose partition arrived last:
-//   out = sum_p 2^(m_p - M) l_p o_p / sum_p 2^(m_p - M) l_p,  M = max_p m_p,
-// over the shared-prefix slots [0, n_pre) and the sequence's own slots
-// [s0, s0 + n_own).  Partials written by other CTAs are read through L2.
-// All threads of the CTA take part: one warp per head finds M and writes the
-// weights of a chunk of slots to shared memory (`sm`, 16 + 8 * kMergeChunk
-// floats), and each thread sums up to two float4 output columns with eight
-// slot loads in flight.
-constexpr int kMergeChunk = 256;
-
-template <int HEAD_DIM>
-__device__ __forceinline__ void merge_partials(const DecodeParams &p, int b, int h, int n_pre, int s0, int n_own,
-                                               float *sm) {
-    constexpr int kCols = HEAD_DIM / 4;  // float4 columns of a row
-    constexpr int kWarps = kThreads / 32;
-    const int G = p.group;
-    const int n = n_pre + n_own;
-    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-    float *s_max = sm;       // [8]
-    float *s_w = sm + 16;    // [8][kMergeChunk]
-    const int64_t row0 = (int64_t)b * p.num_q_heads + (int64_t)h * G;
-    const float2 *ml0 = reinterpret_cast<const float2 *>(p.part_ml) + row0 * p.num_slots;
-    auto slot_of = [&](int k) { return k < n_pre ? k : s0 + k - n_pre; };
-    // One warp per head: the (max, sum) pairs of the first kMergeChunk slots are
-    // read once, kept in registers for the max and turned into weights in place.
-    constexpr int kPerLane = kMergeChunk / 32;
-    for (int g = warp; g < G; g += kWarps) {
-        const float2 *mlg = ml0 + (int64_t)g * p.num_slots;
-        float2 v[kPerLane];
-        float M = -INFINITY;
-#pragma unroll
-        for (int i = 0; i < kPerLane; ++i) {
-            const int k = lane + 32 * i;
-            v[i] = k < n ? __ldcg(mlg + slot_of(k)) : make_float2(-INFINITY, 0.f);
-            M = fmaxf(M, v[i].x);
-        }
-        for (int k = kMergeChunk + lane; k < n; k += 32) M = fmaxf(M, __ldcg(mlg + slot_of(k)).x);
-#pragma unroll
-        for (int off = 16; off; off >>= 1) M = fmaxf(M, __shfl_xor_sync(0xffffffffu, M, off));
-        if (lane == 0) s_max[g] = M;
-#pragma unroll
-        for (int i = 0; i < kPerLane; ++i) {
-            const int k = lane + 32 * i;
-            if (k < n && k < kMergeChunk) s_w[g * kMergeChunk + k] = M == -INFINITY ? 0.f : fast_exp2(v[i].x - M) * v[i].y;
-        }
-    }
-    // Output columns of this thread: x and x + kThreads (G * kCols <= 256 <= 2 * kThreads).
-    int col[2], gcol[2];
-    const float4 *po[2];
-#pragma unroll
-    for (int i = 0; i < 2; ++i) {
-        col[i] = threadIdx.x + i * kThreads;
-        gcol[i] = col[i] / kCols;
-        po[i] = reinterpret_cast<const float4 *>(p.part_o + (row0 + gcol[i]) * p.num_slots * HEAD_DIM) +
-                (col[i] - gcol[i] * kCols);
-    }
-    const bool on0 = col[0] < G * kCols, on1 = col[1] < G * kCols;
-    float4 acc[2] = {make_float4(0.f, 0.f, 0.f, 0.f), make_float4(0.f, 0.f, 0.f, 0.f)};
-    float den[2] = {0.f, 0.f};
-    for (int c0 = 0; c0 < n; c0 += kMergeChunk) {
-        const int cn = min(kMergeChunk, n - c0);
-        __syncthreads();  // the first chunk's weights are written; a later chunk's predecessor is consumed
-        if (c0 > 0) {
-            for (int x = threadIdx.x; x < G * cn; x += kThreads) {
-                const int g = x / cn, k = x - g * cn;
-                const float M = s_max[g];
-                const float2 mlv = __ldcg(ml0 + (int64_t)g * p.num_slots + slot_of(c0 + k));
-                s_w[g * kMergeChunk + k] = M == -INFINITY ? 0.f : fast_exp2(mlv.x - M) * mlv.y;
-            }
-            __syncthreads();
-        }
-#pragma unroll 8
-        for (int k = 0; k < cn; ++k) {
-            const int64_t s = slot_of(c0 + k);
-            if (on0) {
-                const float w = s_w[gcol[0] * kMergeChunk + k];
-                const float4 o = __ldcg(po[0] + s * kCols);
-                acc[0].x += w * o.x;
-                acc[0].y += w * o.y;
-                acc[0].z += w * o.z;
-                acc[0].w += w * o.w;
-                den[0] += w;
-            }
-            if (on1) {
-                const float w = s_w[gcol[1] * kMergeChunk + k];
-                const float4 o = __ldcg(po[1] + s * kCols);
-                acc[1].x += w * o.x;
-                acc[1].y += w * o.y;
-                acc[1].z += w * o.z;
-                acc[1].w += w * o.w;
-                den[1] += w;
-            }
-        }
-    }
-#pragma unroll
-    for (int i = 0; i < 2; ++i) {
-        if (i == 0 ? !on0 : !on1) continue;
-        const float r = den[i] == 0.f ? 0.f : 1.f / den[i];  // no tokens: zeros; a NaN stays NaN
-        reinterpret_cast<float4 *>(p.out + row0 * HEAD_DIM)[col[i]] =
-            make_float4(acc[i].x * r, acc[i].y * r, acc[i].z * r, acc[i].w * r);
-    }
-    __syncthreads();  // the scratch is free for the next merge of this CTA
-}
-
 template <int HEAD_DIM, bool SPLIT, bool APPEND, bool FP8, bool PREFIX>
 __global__ void __launch_bounds__(kThreads, FP8 ? PA_DECODE_MIN_CTAS_FP8 : PA_DECODE_MIN_CTAS_BF16) paged_decode_kernel(
     const __grid_constant__ CUtensorMap k_map, const __grid_constant__ CUtensorMap v_map,
@@ -351,7 +204,6 @@ __global__ void __launch_bounds__(kThreads, FP8 ? PA_DECODE_MIN_CTAS_FP8 : PA_DE
     static_assert(SPLIT || !PREFIX, "shared-prefix items always merge through the split path");
     using C = Cfg<HEAD_DIM, FP8>;
     extern __shared__ uint8_t smem_raw[];
-    __shared__ unsigned int s_last;  // split: members whose merge falls to this CTA (bit mask)
     uint8_t *smem = reinterpret_cast<uint8_t *>(
         (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~static_cast<uintptr_t>(1023));
     uint64_t *full = reinterpret_cast<uint64_t *>(smem + C::kDataBytes);
@@ -405,8 +257,12 @@ __global__ void __launch_bounds__(kThreads, FP8 ? PA_DECODE_MIN_CTAS_FP8 : PA_DE
     const int tok_end = min(pre ? shared : L, tok_begin + p.part_tokens);
     const int n_tiles = tok_end > tok_begin ? (tok_end - tok_begin + kTileTokens - 1) / kTileTokens : 0;
     if (!pre && threadIdx.x == 0 && part == 0 && h == 0 && L != L_raw) raise_flag(p.err_flag, PA_FLAG_BAD_LEN);
+    // Let the log-sum-exp reduce (launched as a programmatic dependent) get
+    // scheduled while this grid's last wave runs; it waits for our results.
+    if (SPLIT) asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
     // Split: a sequence whose own tokens fit one partition (and share none) has
-    // a single partial state -- that CTA writes the output itself.
+    // a single partial state -- that CTA writes the output itself, and the
+    // reduce skips it.
     const bool direct = SPLIT && !pre && shared == 0 && L <= p.part_tokens;
     if (SPLIT && n_tiles == 0) {
         // Nothing to read.  An empty sequence has no partial states at all, so
@@ -532,7 +388,9 @@ __global__ void __launch_bounds__(kThreads, FP8 ? PA_DECODE_MIN_CTAS_FP8 : PA_DE
         uint32_t qf[HEAD_DIM / 16][2];
         if (gid < nmem * G) {
             const uint4 *qrow = reinterpret_cast<const uint4 *>(
-                p.q + ((int64_t)(b + gid / G) * p.num_q_heads + (int64_t)h * G + gid % G) * HEAD_DIM);
+                p.q + ((PREFIX ? (int64_t)(b + gid / G) * p.num_q_heads + (int64_t)h * G + gid % G
+                               : (int64_t)b * p.num_q_heads + (int64_t)h * G + gid) *
+                       HEAD_DIM));
 #pragma unroll
             for (int j = 0; j < HEAD_DIM / 32; ++j) {
                 const uint4 v = __ldg(qrow + 4 * j + tig);
@@ -879,7 +737,7 @@ __global__ void __launch_bounds__(kThreads, FP8 ? PA_DECODE_MIN_CTAS_FP8 : PA_DE
     // Column n is query head n % G of member b + n / G; in the split variant
     // its partial state goes to slot `slot` of that row.
     const int slot = PREFIX && !pre ? p.num_parts + part : part;
-    for (int x = threadIdx.x; x < nmem * G * HEAD_DIM; x += kThreads) {
+    for (int x = threadIdx.x; x < (PREFIX ? nmem : 1) * G * HEAD_DIM; x += kThreads) {
         const int n = x / HEAD_DIM;
         const int d = x - n * HEAD_DIM;
         float M = -INFINITY;
@@ -894,7 +752,8 @@ __global__ void __launch_bounds__(kThreads, FP8 ? PA_DECODE_MIN_CTAS_FP8 : PA_DE
                 den += f * ml[w * 8 + n];
             }
         }
-        const int64_t row = (int64_t)(b + n / G) * p.num_q_heads + (int64_t)h * G + n % G;
+        const int64_t row = PREFIX ? (int64_t)(b + n / G) * p.num_q_heads + (int64_t)h * G + n % G
+                                   : (int64_t)b * p.num_q_heads + (int64_t)h * G + n;
         if (FP8) num *= p.v_scale;
         if (SPLIT && !direct) {
             p.part_o[(row * p.num_slots + slot) * HEAD_DIM + d] = den == 0.f ? 0.f : num / den;
@@ -907,37 +766,86 @@ __global__ void __launch_bounds__(kThreads, FP8 ? PA_DECODE_MIN_CTAS_FP8 : PA_DE
             p.out[row * HEAD_DIM + d] = den == 0.f ? 0.f : num / den;
         }
     }
-    if constexpr (SPLIT) {
-        if (direct) return;
-        // Ticket: this partition's state is stored.  The CTA whose ticket is the
-        // last of a (member, kv head) merges that pair's partitions.  The barrier
-        // orders every thread's partial stores before thread 0's device-scope
-        // fence, which publishes them before the ticket (and, for the last
-        // arrival, orders the other partitions' states before they are read).
-        __syncthreads();
-        if (threadIdx.x == 0) {
-            __threadfence();
-            unsigned int mask = 0;
-            for (int m = 0; m < nmem; ++m) {
-                const int bm = b + m;
-                const int Lm = pre ? clamp_len(__ldg(p.seq_lens + bm), p) : L;
-                const int expected = parts_of(shared, p.part_tokens) + parts_of(Lm - shared, p.part_tokens);
-                if (take_ticket(p.tickets + (int64_t)bm * p.num_kv_heads + h, p.epoch, 1, expected, p.err_flag))
-                    mask |= 1u << m;
+}
+
+// Log-sum-exp merge of the partial states of one (sequence, query head):
+//   out = sum_p 2^(m_p - M) l_p o_p / sum_p 2^(m_p - M) l_p,  M = max_p m_p,
+// over the shared-prefix slots [0, n_pre) and the sequence's own slots
+// [s0, s0 + n_own).  Rows with a single partial state were written by the
+// decode itself and are skipped.  Four warps split the slots; each lane owns
+// HEAD_DIM/32 output dims.
+constexpr int kReduceThreads = 128;
+
+template <int HEAD_DIM, bool PREFIX>
+__global__ void __launch_bounds__(kReduceThreads) lse_reduce_kernel(const DecodeParams p) {
+    // Launched as a programmatic dependent of the decode grid: wait for its results.
+    asm volatile("griddepcontrol.wait;" ::: "memory");
+    constexpr int kWarps = kReduceThreads / 32;
+    constexpr int V = HEAD_DIM / 32;  // dims per lane: 4 or 2
+    __shared__ float s_max[kWarps];
+    __shared__ float s_den[kWarps];
+    __shared__ float s_acc[kWarps][HEAD_DIM];
+    const int hq = blockIdx.x;
+    const int b = blockIdx.y;
+    const int warp = threadIdx.x >> 5;
+    const int lane = threadIdx.x & 31;
+    const int shared = PREFIX ? group_shared_tokens(p, b / p.group_size) : 0;
+    const int L = clamp_len(__ldg(p.seq_lens + b), p);
+    const int n_pre = parts_of(shared, p.part_tokens);
+    const int n_own = parts_of(L - shared, p.part_tokens);
+    const int n = n_pre + n_own;
+    if (n_pre == 0 && n_own <= 1) return;  // written by the decode
+    const int s0 = PREFIX ? p.num_parts : 0;
+    auto slot_of = [&](int k) { return k < n_pre ? k : s0 + k - n_pre; };
+    const int64_t row = (int64_t)b * p.num_q_heads + hq;
+    const float2 *ml = reinterpret_cast<const float2 *>(p.part_ml) + row * p.num_slots;
+    const float *po = p.part_o + row * p.num_slots * HEAD_DIM + lane * V;
+
+    float M = -INFINITY;
+    for (int i = threadIdx.x; i < n; i += kReduceThreads) M = fmaxf(M, __ldg(&ml[slot_of(i)].x));
+#pragma unroll
+    for (int off = 16; off; off >>= 1) M = fmaxf(M, __shfl_xor_sync(0xffffffffu, M, off));
+    if (lane == 0) s_max[warp] = M;
+    __syncthreads();
+#pragma unroll
+    for (int w = 0; w < kWarps; ++w) M = fmaxf(M, s_max[w]);
+
+    float acc[V];
+#pragma unroll
+    for (int k = 0; k < V; ++k) acc[k] = 0.f;
+    float den = 0.f;
+    if (M != -INFINITY) {
+#pragma unroll 4
+        for (int i = warp; i < n; i += kWarps) {
+            const int64_t s = slot_of(i);
+            const float2 mlv = __ldg(&ml[s]);
+            const float w = fast_exp2(mlv.x - M) * mlv.y;
+            if constexpr (V == 4) {
+                const float4 v = __ldg(reinterpret_cast<const float4 *>(po + s * HEAD_DIM));
+                acc[0] += w * v.x;
+                acc[1] += w * v.y;
+                acc[2] += w * v.z;
+                acc[3] += w * v.w;
+            } else {
+                const float2 v = __ldg(reinterpret_cast<const float2 *>(po + s * HEAD_DIM));
+                acc[0] += w * v.x;
+                acc[1] += w * v.y;
             }
-            if (mask) __threadfence();  // the other partitions' states, seen before they are read
-            s_last = mask;
+            den += w;
         }
-        __syncthreads();
-        const unsigned int mask = s_last;
-        static_assert((16 + 8 * kMergeChunk) * 4 <= C::kRingBytes, "merge scratch reuses the ring");
-        for (int m = 0; m < nmem; ++m) {
-            if (!(mask & (1u << m))) continue;
-            const int bm = b + m;
-            const int Lm = pre ? clamp_len(__ldg(p.seq_lens + bm), p) : L;
-            merge_partials<HEAD_DIM>(p, bm, h, parts_of(shared, p.part_tokens), PREFIX ? p.num_parts : 0,
-                                     parts_of(Lm - shared, p.part_tokens), reinterpret_cast<float *>(smem));
+    }
+#pragma unroll
+    for (int k = 0; k < V; ++k) s_acc[warp][lane * V + k] = acc[k];
+    if (lane == 0) s_den[warp] = den;
+    __syncthreads();
+    for (int x = threadIdx.x; x < HEAD_DIM; x += kReduceThreads) {
+        float num = 0.f, dd = 0.f;
+#pragma unroll
+        for (int w = 0; w < kWarps; ++w) {
+            num += s_acc[w][x];
+            dd += s_den[w];
         }
+        p.out[row * HEAD_DIM + x] = dd == 0.f ? 0.f : num / dd;  // no tokens: zeros; a NaN stays NaN
     }
 }
 

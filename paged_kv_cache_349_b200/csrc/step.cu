@@ -55,9 +55,8 @@ StagingLayout staging_layout(int batch, int max_blocks_per_seq, int max_copy_pai
     l.workspace = off;
     l.workspace_bytes = pa_decode_workspace_size(batch, num_q_heads, num_kv_heads, head_dim, block_size,
                                                  max_seq_len, partition_tokens);
-    // Each chunk's slice rounds its three sections (partial states, their
-    // maxima and sums, the tickets) and itself up to kAlign.
-    if (l.workspace_bytes) l.workspace_bytes += 4 * kAlign * kMaxChunks;
+    // Each chunk's slice rounds its partial states and itself up to kAlign.
+    if (l.workspace_bytes) l.workspace_bytes += 2 * kAlign * kMaxChunks;
     off += round_up(l.workspace_bytes);
     l.total = off;
     return l;

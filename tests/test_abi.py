@@ -90,12 +90,10 @@ def test_workspace_size_explicit_partitions(pt, maxlen, parts):
         assert size == 0
         assert pa.pa_decode_partition_tokens(B, Hq, Hkv, d, 16, maxlen, pt) == -1
     else:
-        # partial outputs, then (max, sum) pairs, each 256-byte aligned, then one
-        # 8-byte arrival ticket per (sequence, kv head)
+        # partial outputs, 256-byte aligned, then the (max, sum) pairs
         rows = B * Hq * parts
         o_bytes = -(-rows * d * 4 // 256) * 256
-        ml_bytes = -(-rows * 8 // 256) * 256
-        assert size == o_bytes + ml_bytes + B * Hkv * 8
+        assert size == o_bytes + rows * 8
         assert pa.pa_decode_partition_tokens(B, Hq, Hkv, d, 16, maxlen, pt) == pt
 
 
@@ -106,7 +104,7 @@ def test_shared_prefix_workspace_size(pt, maxlen, parts):
     B, n, Hq, Hkv, d = 128, 4, 40, 40, 128
     size = pa.pa_decode_shared_prefix_workspace_size(B, n, Hq, Hkv, d, 16, maxlen, pt)
     rows = B * Hq * 2 * parts
-    assert size == -(-rows * d * 4 // 256) * 256 + -(-rows * 8 // 256) * 256 + B * Hkv * 8
+    assert size == -(-rows * d * 4 // 256) * 256 + rows * 8
     assert pa.pa_decode_shared_prefix_workspace_size(0, n, Hq, Hkv, d, 16, maxlen, pt) == 0
 
 

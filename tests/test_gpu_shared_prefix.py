@@ -73,7 +73,7 @@ def run_prefix(case, prefix, group_size, pt, fused=True, ws_fill=None):
                                group_size=group_size, max_seq_len=case.max_seq_len, scale=float(case.scale),
                                partition_tokens=pt, workspace=ws, err_flag=dc.flag,
                                k_new=bf16_dev(k_last) if fused else None, v_new=bf16_dev(v_last) if fused else None)
-    assert pa.launch_count() - before == 1
+    assert pa.launch_count() - before == 2  # decode + log-sum-exp reduce
     torch.cuda.synchronize()
     return dc, dc.out.cpu().numpy().astype(np.float64)
 

@@ -5,7 +5,7 @@ foreign runtime that only passes pointers to tensors it already owns, a
 latency-critical loop that must not call cudaMalloc) get the split decode's
 scratch from an array the library owns.  These tests call the entry point
 through the C ABI and compare it with pa_decode given a caller workspace.
-Both run the same kernel with the same partitioning on the same inputs, so
+Both run the same kernels with the same partitioning on the same inputs, so
 the outputs must agree bit for bit:
   - two calls in a row with different inputs, synchronised in between;
   - two calls queued back to back on one stream with no synchronisation, so
@@ -80,7 +80,7 @@ def test_builtin_scratch_bit_identical_to_caller_workspace_two_calls(torch_cuda)
         flag = torch.zeros(1, dtype=torch.int32, device="cuda")
         before = pa.launch_count()
         assert lib.pa_decode_builtin_scratch(*_args(case, tens, got), P(flag.data_ptr()), stream) == 0
-        assert pa.launch_count() - before == 1  # one split decode; the merge runs inside it
+        assert pa.launch_count() - before == 2  # split decode + log-sum-exp reduce
         torch.cuda.synchronize()
         assert int(flag.item()) == 0
         assert torch.equal(got, want)
