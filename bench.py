@@ -440,27 +440,30 @@ def measure_workload(cfg, args, world, rank, pa, headline):
     dec_ms = _max_over_ranks(statistics.mean(a.elapsed_time(b) for a, b in dec_ev), world)
     assert int(flag.item()) == 0, f"error flag {int(flag.item()):#x}"
 
-    # The chat mix: the other decode of the same step, and both with L2 flushed before each call.
-    alt_ms, cold = None, None
+    # The chat mix: both decodes of the same step, call by call in alternation (so both see
+    # the same clocks), with L2 warm and with L2 flushed before each call.
+    compare = None
     if has_groups:
-        kind_alt = "plain" if prefix else "shared-prefix"
+        l2 = torch.cuda.get_device_properties(torch.cuda.current_device()).L2_cache_size
 
-        def decode_ms(kind, flush=None):
-            evs = []
+        def interleaved(flush=None):
+            evs = {"plain": [], "shared-prefix": []}
             for _ in range(args.warmup):
-                step(kind=kind)
+                for kind in evs:
+                    step(kind=kind)
             torch.cuda.synchronize()
             for _ in range(args.steps):
-                if flush is not None:
-                    flush.fill_(1)
-                step(record=True, kind=kind, evs=evs)
+                for kind in evs:
+                    if flush is not None:
+                        flush.fill_(1)
+                    step(record=True, kind=kind, evs=evs[kind])
             torch.cuda.synchronize()
-            return _max_over_ranks(statistics.mean(a.elapsed_time(b) for a, b in evs), world)
+            return {kind: round(_max_over_ranks(statistics.mean(a.elapsed_time(b) for a, b in e), world), 5)
+                    for kind, e in evs.items()}
 
-        alt_ms = decode_ms(kind_alt)
-        l2 = torch.cuda.get_device_properties(torch.cuda.current_device()).L2_cache_size
+        compare = {"l2_warm": interleaved()}
         flush = torch.empty(2 * l2, dtype=torch.uint8, device="cuda")
-        cold = {kind: round(decode_ms(kind, flush), 5) for kind in ("plain", "shared-prefix")}
+        compare["l2_flushed"] = interleaved(flush)
         del flush
         assert int(flag.item()) == 0, f"error flag {int(flag.item()):#x}"
 
@@ -500,14 +503,12 @@ def measure_workload(cfg, args, world, rank, pa, headline):
         if traffic:
             roof["traffic_vs_unique"] = round(traffic / dec_b, 4)
             roof["traffic_vs_logical"] = round(traffic / dec_logical, 4)
-    if alt_ms is not None:
-        alt_name = "plain_decode" if prefix else "shared_prefix_decode"
-        roof[f"{alt_name}_launch_ms"] = round(alt_ms, 5)
-        roof[f"{alt_name}_achieved"] = round(dec_b / (alt_ms / 1e3) / 1e9, 1)
-        roof["l2_flushed_launch_ms"] = cold
-        roof["l2_flushed_note"] = (f"decode call with a {2 * l2 >> 20} MiB buffer written before each call: "
-                                   "the shared-prefix decode reads each group's shared tiles once, the plain "
-                                   "decode relies on L2 for the repeats")
+    if compare is not None:
+        roof["decode_comparison_ms"] = compare
+        roof["decode_comparison_note"] = (
+            "pa_decode_append (plain: repeated prefix rows served by L2) against pa_decode_shared_prefix "
+            "(each group's shared tiles read once), called in alternation; l2_flushed writes a "
+            f"{2 * l2 >> 20} MiB buffer before each call")
 
     entry = {
         "value": round(value, 1),
@@ -620,10 +621,11 @@ def run_e2e(args, case, pa, stream, world, k_pool, v_pool, kv_scales=None):
 
     Every step: the host allocator appends one token per sequence (and reports
     copy-on-write pairs) and exports the tables into pinned memory (one
-    ``pa_alloc_step`` call); one ``pa_decode_step_host`` call then uploads the
-    step's inputs, applies the copies and runs the fused cache write + decode,
-    whose output lands in pinned host memory; the step ends when the output is
-    on the host.  ``kv_scales`` = (k_scale, v_scale) for fp8 pools.
+    ``pa_alloc_step`` call); one ``pa_decode_step_plan_run`` call (the step is
+    prepared once) then uploads the step's inputs, applies the copies and runs
+    the fused cache write + decode, whose output lands in pinned host memory;
+    the step ends when the output is on the host.  Byte counts are taken after
+    the timed loop.  ``kv_scales`` = (k_scale, v_scale) for fp8 pools.
     """
     import torch
     bs = case.block_size
@@ -654,36 +656,45 @@ def run_e2e(args, case, pa, stream, world, k_pool, v_pool, kv_scales=None):
         raise SystemExit("--unfused applies to the device-resident step only")
     run = pa.DecodeStepHost(out_host=h_out, q_host=h_q, k_new_host=h_k, v_new_host=h_v, tables_host=h_tables,
                             lens_host=h_lens, pairs_host=h_pairs, k_cache=k_pool, v_cache=v_pool,
-                            scale=float(case.scale), partition_tokens=case.partition_tokens,
+                            scale=float(case.scale), max_seq_len_cap=max_len_cap,
+                            partition_tokens=case.partition_tokens,
                             num_chunks=args.step_chunks, staging=staging,
                             err_flag=flag, stream=stream,
                             k_scale=kv_scales[0] if kv_scales else None, v_scale=kv_scales[1] if kv_scales else None)
     elem = 1 if kv_scales else 2
-    acc = {"h2d": 0, "d2h": 0, "alg": 0, "tokens": 0}
-
     host_step = alloc.step_fn(sids, tables_np, lens_np, pairs_np)
+    # per timed step: its max length and copy-pair count (the bytes are counted after the timed loop)
+    steps_seen = []
 
-    def e2e_step(count):
+    def e2e_step():
         n_pairs, max_len = host_step()  # append one token per sequence, export tables + lengths
         run(max_len, n_pairs)
         stream.synchronize()  # the step's output is on the host
-        if count:
-            acc["h2d"] += sum(t.numel() * t.element_size() for t in (h_q, h_k, h_v, h_tables, h_lens)) + n_pairs * 8
-            acc["d2h"] += h_out.numel() * 4
-            acc["tokens"] += int(lens_np.sum())
-            c, w, d = step_bytes_from(case, lens_np, n_pairs, elem)
-            acc["alg"] += c + w + d
+        return n_pairs
 
     for _ in range(warm):
-        e2e_step(False)
+        e2e_step()
+    lens0 = lens_np.copy()  # lengths after the warm-up steps; every timed step adds one token per sequence
     _barrier(world)
     torch.cuda.synchronize()
     t0 = time.perf_counter()
     for _ in range(steps):
-        e2e_step(True)
+        steps_seen.append(e2e_step())
     dt = time.perf_counter() - t0
     dt = _max_over_ranks(dt, world)
     assert int(flag.item()) == 0
+    acc = {"h2d": 0, "d2h": 0, "alg": 0, "tokens": 0}
+    # shared prefixes (forks) count once, as in the device-resident value
+    share = (decode_bytes(case, elem, unique=True) / decode_bytes(case, elem, unique=False)
+             if case.groups is not None else 1.0)
+    for i, n_pairs in enumerate(steps_seen):
+        lens_i = lens0 + i + 1
+        acc["h2d"] += sum(t.numel() * t.element_size() for t in (h_q, h_k, h_v, h_tables, h_lens)) + n_pairs * 8
+        acc["d2h"] += h_out.numel() * 4
+        acc["tokens"] += int(lens_i.sum())
+        c, w, d = step_bytes_from(case, lens_i, n_pairs, elem)
+        acc["alg"] += c + w + d * share
+    assert np.array_equal(lens0 + len(steps_seen), lens_np), "every timed step appends one token per sequence"
     alg = _sum_over_ranks(float(acc["alg"]), world)
     alloc.close()
     return {"value": round(alg / dt / 1e9, 1), "unit": "GB/s",
@@ -692,8 +703,9 @@ def run_e2e(args, case, pa, stream, world, k_pool, v_pool, kv_scales=None):
             "kv_tokens_per_s": round(_sum_over_ranks(float(acc["tokens"]), world) / dt, 1),
             "step_chunks": args.step_chunks or "auto",
             "includes": "host allocator step (pa_alloc_step: batched append + table export into pinned memory), then one "
-                        + ("pa_decode_step_host_fp8" if kv_scales else "pa_decode_step_host")
-                        + " call: upload of q/k_new/v_new/tables/lens/copy pairs, block copies, fused cache write "
+                        "pa_decode_step_plan_run call (a step prepared once with pa_decode_step_plan_create"
+                        + (" over E4M3 pools" if kv_scales else "")
+                        + "): upload of q/k_new/v_new/tables/lens/copy pairs, block copies, fused cache write "
                           "+ decode, out stored into pinned host memory; timed until out is on the host"}
 
 

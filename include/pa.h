@@ -295,9 +295,10 @@ int pa_decode_shared_prefix(float *out, const void *q, const void *k_new, const 
  * of another.  All of them start after the work already enqueued on `stream`
  * and are joined back into `stream` before the call returns (on error paths
  * too), so synchronising `stream` covers the whole step.  0 picks the count
- * from the bytes crossing the host link: one chunk per MiB, at most 4, at
- * most one per sequence.  The output, the pools and the error flag do not
- * depend on the chunk count: the partitioning is resolved once for the whole
+ * from the bytes crossing the host link: one chunk per 512 KiB, at most 4,
+ * at most one per sequence (measured on B200: a step moving 2.6 MB took 230,
+ * 213, 208 and 205 us end to end with 1 to 4 chunks).  The output, the pools
+ * and the error flag do not depend on the chunk count: the partitioning is resolved once for the whole
  * batch (as pa_decode_partition_tokens reports it) and each chunk decodes
  * its sequences exactly as an unchunked call would.  The side streams and
  * events of a device are created by its first chunked call and kept until
@@ -342,6 +343,46 @@ int pa_decode_step_host_fp8(float *out_host, const void *q_host, const void *k_n
                             int head_dim, int block_size, int64_t num_blocks, float scale, float k_scale,
                             float v_scale, int partition_tokens, int num_chunks, void *staging,
                             size_t staging_bytes, int32_t *err_flag, void *stream);
+
+/* ------------------------------------------------------------------------
+ * Prepared host step: pa_decode_step_host with everything that stays the same
+ * from step to step resolved once -- argument checks, the staging layout,
+ * the device view of each host buffer (cudaPointerGetAttributes: page-locked
+ * buffers are read and written through their device mapping), the output
+ * path and the chunk count.  A serving loop then pays one short call per
+ * step.  No counterpart in the pages.
+ *
+ * pa_decode_step_plan_create takes the arguments of pa_decode_step_host
+ * except the per-step ones (num_pairs, err_flag, stream) and with
+ * max_seq_len_cap, the largest max_seq_len any run will pass (the staging
+ * size must have been computed with it); kv_fp8 != 0 selects E4M3 pools
+ * with k_scale / v_scale (ignored otherwise).  The plan keeps the pointers:
+ * every buffer must stay allocated, at the same address and with the same
+ * memory type (page-locked or not) until pa_decode_step_plan_destroy.  The
+ * plan owns only host memory.  Errors: as pa_decode_step_host;
+ * PA_ERR_OOM if the plan itself cannot be allocated.
+ *
+ * pa_decode_step_plan_run enqueues one step exactly as pa_decode_step_host
+ * would with the same arguments: max_seq_len <= max_seq_len_cap and
+ * num_pairs <= max_copy_pairs (else PA_ERR_INVALID_ARG, nothing enqueued).
+ * The host buffers are read when the stream reaches the step, so fill them
+ * (pa_alloc_step, the new rows) before the call and leave them unchanged
+ * until the stream has passed it.
+ * ---------------------------------------------------------------------- */
+typedef struct pa_decode_step_plan pa_decode_step_plan;
+
+int pa_decode_step_plan_create(float *out_host, const void *q_host, const void *k_new_host, const void *v_new_host,
+                               const int32_t *block_tables_host, int max_blocks_per_seq, const int32_t *seq_lens_host,
+                               const int32_t *copy_pairs_host, int max_copy_pairs, void *k_cache, void *v_cache,
+                               int batch, int max_seq_len_cap, int num_q_heads, int num_kv_heads, int head_dim,
+                               int block_size, int64_t num_blocks, float scale, int partition_tokens, int num_chunks,
+                               void *staging, size_t staging_bytes, int kv_fp8, float k_scale, float v_scale,
+                               pa_decode_step_plan **plan);
+
+int pa_decode_step_plan_run(const pa_decode_step_plan *plan, int max_seq_len, int num_pairs, int32_t *err_flag,
+                            void *stream);
+
+void pa_decode_step_plan_destroy(pa_decode_step_plan *plan);
 
 /* ------------------------------------------------------------------------
  * Decode with library-owned scratch (no workspace argument).

@@ -14,7 +14,8 @@ Device ops on fp8 (E4M3) pools:
     pa_quantize_fp8, pa_reshape_and_cache_fp8, pa_copy_blocks_fp8,
     pa_swap_blocks_fp8, pa_decode_fp8 (with k_new/v_new: the fused write)
 A whole decode step from pinned host buffers:
-    pa_decode_step_staging_size, DecodeStepHost (pa_decode_step_host[_fp8])
+    pa_decode_step_staging_size, DecodeStepHost (pa_decode_step_plan_*; the
+    one-call form is pa_decode_step_host[_fp8] in the C ABI)
 Host allocator:
     Allocator (pa_alloc_* / pa_seq_* / pa_block_refcount; step_fn = pa_alloc_step)
     validate_tables (pa_validate_tables: host-side check of decode tables)
@@ -275,19 +276,22 @@ def pa_decode_step_staging_size(batch, max_blocks_per_seq, max_copy_pairs, num_q
 
 
 class DecodeStepHost:
-    """One decode step from host buffers through ``pa_decode_step_host`` (bf16 pools) or
-    ``pa_decode_step_host_fp8`` (uint8 E4M3 pools, given ``k_scale`` and ``v_scale``).
+    """Repeated decode steps from fixed pinned host buffers: a prepared step
+    (``pa_decode_step_plan_create``) over bf16 pools, or uint8 E4M3 pools given
+    ``k_scale`` and ``v_scale``; each call is one ``pa_decode_step_plan_run``.
 
-    Holds the argument tuple for a fixed set of pinned host buffers, pools and
-    staging, so each step only marshals what changes (max_seq_len, the number of
-    copy pairs).  Host arrays are torch CPU tensors (pinned); pools and staging are
-    CUDA tensors.  ``num_chunks``: 0 lets the library pick how many chunks of
-    sequences to pipeline, 1 disables pipelining, 2..8 forces that many.
+    Host arrays are torch CPU tensors (pinned); pools and staging are CUDA
+    tensors, all kept alive by this object.  ``max_seq_len_cap`` bounds the
+    ``max_seq_len`` of every call (staging must be sized with it).
+    ``num_chunks``: 0 lets the library pick how many chunks of sequences to
+    pipeline, 1 disables pipelining, 2..8 forces that many.  ``close()`` (or
+    garbage collection) releases the plan.
     """
 
     def __init__(self, *, out_host, q_host, k_new_host, v_new_host, tables_host, lens_host, pairs_host,
-                 k_cache, v_cache, scale: float, partition_tokens: int = 0, num_chunks: int = 0, staging=None,
-                 err_flag=None, stream=None, k_scale: Optional[float] = None, v_scale: Optional[float] = None):
+                 k_cache, v_cache, scale: float, max_seq_len_cap: int, partition_tokens: int = 0,
+                 num_chunks: int = 0, staging=None, err_flag=None, stream=None, k_scale: Optional[float] = None,
+                 v_scale: Optional[float] = None):
         torch = _torch()
         B, Hq, d = q_host.shape
         NB, Hkv, bs, d2 = k_cache.shape
@@ -305,22 +309,35 @@ class DecodeStepHost:
         pool_dt = torch.uint8 if self.fp8 else torch.bfloat16
         self.max_blocks = int(tables_host.shape[1])
         self.max_pairs = int(pairs_host.shape[0])
-        self.staging = staging
-        self._head = (ctypes.c_void_p(out_host.data_ptr()), ctypes.c_void_p(q_host.data_ptr()),
-                      ctypes.c_void_p(k_new_host.data_ptr()), ctypes.c_void_p(v_new_host.data_ptr()),
-                      ctypes.c_void_p(tables_host.data_ptr()), self.max_blocks,
-                      ctypes.c_void_p(lens_host.data_ptr()), ctypes.c_void_p(pairs_host.data_ptr()))
-        self._kv = (self.max_pairs, _dev(k_cache, pool_dt, "k_cache"), _dev(v_cache, pool_dt, "v_cache"), B)
-        scales = (float(k_scale), float(v_scale)) if self.fp8 else ()
-        self._shape = (Hq, Hkv, d, bs, NB, float(scale), *scales, int(partition_tokens), int(num_chunks))
-        self._tail = (ctypes.c_void_p(staging.data_ptr()), staging.numel() * staging.element_size(),
-                      _opt_flag(err_flag), _stream(stream))
-        self._fn = lib.pa_decode_step_host_fp8 if self.fp8 else lib.pa_decode_step_host
-        self._name = "pa_decode_step_host_fp8" if self.fp8 else "pa_decode_step_host"
+        self._keep = (out_host, q_host, k_new_host, v_new_host, tables_host, lens_host, pairs_host, k_cache, v_cache,
+                      staging, err_flag)
+        self._plan = ctypes.c_void_p()
+        _check(lib.pa_decode_step_plan_create(
+            ctypes.c_void_p(out_host.data_ptr()), ctypes.c_void_p(q_host.data_ptr()),
+            ctypes.c_void_p(k_new_host.data_ptr()), ctypes.c_void_p(v_new_host.data_ptr()),
+            ctypes.c_void_p(tables_host.data_ptr()), self.max_blocks, ctypes.c_void_p(lens_host.data_ptr()),
+            ctypes.c_void_p(pairs_host.data_ptr()), self.max_pairs, _dev(k_cache, pool_dt, "k_cache"),
+            _dev(v_cache, pool_dt, "v_cache"), B, int(max_seq_len_cap), Hq, Hkv, d, bs, NB, float(scale),
+            int(partition_tokens), int(num_chunks), ctypes.c_void_p(staging.data_ptr()),
+            staging.numel() * staging.element_size(), int(self.fp8), float(k_scale or 1.0), float(v_scale or 1.0),
+            ctypes.byref(self._plan)), "pa_decode_step_plan_create")
+        self._flag = _opt_flag(err_flag)
+        self._stream = _stream(stream)
+        self._run = lib.pa_decode_step_plan_run
 
     def __call__(self, max_seq_len: int, num_pairs: int = 0) -> None:
-        _check(self._fn(*self._head, int(num_pairs), *self._kv, int(max_seq_len), *self._shape, *self._tail),
-               self._name)
+        _check(self._run(self._plan, max_seq_len, num_pairs, self._flag, self._stream), "pa_decode_step_plan_run")
+
+    def close(self) -> None:
+        if self._plan:
+            lib.pa_decode_step_plan_destroy(self._plan)
+            self._plan = ctypes.c_void_p()
+
+    def __del__(self):
+        try:
+            self.close()
+        except Exception:
+            pass
 
 
 # ---------------------------------------------------------------------------

@@ -38,6 +38,10 @@ SIGNATURES = {
     "pa_decode_shared_prefix_workspace_size": (_SZ, [_I, _I, _I, _I, _I, _I, _I, _I]),
     "pa_decode_shared_prefix": (_I, [_P, _P, _P, _P, _P, _P, _P, _I, _P, _P, _I, _I, _I, _I, _I, _I, _I, _I64, _F,
                                      _I, _P, _SZ, _P, _P]),
+    "pa_decode_step_plan_create": (_I, [_P, _P, _P, _P, _P, _I, _P, _P, _I, _P, _P, _I, _I, _I, _I, _I, _I, _I64,
+                                        _F, _I, _I, _P, _SZ, _I, _F, _F, ctypes.POINTER(_P)]),
+    "pa_decode_step_plan_run": (_I, [_P, _I, _I, _P, _P]),
+    "pa_decode_step_plan_destroy": (None, [_P]),
     "pa_decode_builtin_scratch": (_I, [_P, _P, _P, _P, _P, _I, _P, _I, _I, _I, _I, _I, _I, _I64, _F, _I, _P, _P]),
     "pa_quantize_fp8": (_I, [_P, _P, _I64, _F, _P]),
     "pa_reshape_and_cache_fp8": (_I, [_P, _P, _P, _P, _P, _I, _I64, _I, _I, _I, _F, _F, _P, _P]),

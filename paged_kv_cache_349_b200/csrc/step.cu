@@ -12,6 +12,7 @@
 // into the caller's stream before the call returns, so synchronising that
 // stream covers the whole step.
 #include <mutex>
+#include <new>
 
 #include "pa_common.cuh"
 
@@ -22,7 +23,9 @@ constexpr size_t kAlign = 256;
 constexpr int kMaxChunks = 8;
 constexpr int kMaxDevices = 64;
 // Auto chunking: one chunk per this many bytes crossing the host link, at most 4.
-constexpr size_t kAutoChunkBytes = (size_t)1 << 20;
+// (Measured on B200 with the Llama-2-7B-shaped step, 2.6 MB over the link:
+// 1, 2, 3, 4 chunks took 230, 213, 208, 205 us end to end.)
+constexpr size_t kAutoChunkBytes = (size_t)1 << 19;
 constexpr int kAutoMaxChunks = 4;
 
 inline size_t round_up(size_t x) { return (x + kAlign - 1) / kAlign * kAlign; }
@@ -247,89 +250,147 @@ size_t pa_decode_step_staging_size(int batch, int max_blocks_per_seq, int max_co
         .total;
 }
 
-// The host step for either pool type: bf16 pools, or E4M3 pools with their scales.
-static int step_host(float *out_host, const void *q_host, const void *k_new_host, const void *v_new_host,
-                     const int32_t *block_tables_host, int max_blocks_per_seq, const int32_t *seq_lens_host,
-                     const int32_t *copy_pairs_host, int num_pairs, int max_copy_pairs, void *k_cache,
-                     void *v_cache, int batch, int max_seq_len, int num_q_heads, int num_kv_heads, int head_dim,
-                     int block_size, int64_t num_blocks, float scale, int partition_tokens, int num_chunks,
-                     void *staging, size_t staging_bytes, int32_t *err_flag, void *stream, bool fp8,
-                     float k_scale, float v_scale) {
+}  // extern "C"
+
+// A host step with everything that does not change from step to step resolved
+// once: argument checks, the staging layout, the device view of each host
+// buffer (page-locked memory read through its mapping), the output path and
+// the chunk count.  pa_decode_step_host builds one per call; a
+// pa_decode_step_plan keeps one for many steps.
+struct pa_decode_step_plan {
+    float *out_host;
+    const int32_t *copy_pairs_host;
+    void *k_cache, *v_cache;
+    int batch, max_blocks_per_seq, max_copy_pairs, max_seq_len_cap;
+    int num_q_heads, num_kv_heads, head_dim, block_size;
+    int64_t num_blocks;
+    float scale;
+    int partition_tokens;
+    int chunks;
+    bool fp8;
+    float k_scale, v_scale;
+    char *st;                      // staging
+    pa::StagingLayout l;
+    pa::HostSrc hq, hk, hv, ht, hl, hp;
+    bool direct;                   // the kernels store the output into out_host
+    char *out_base;
+};
+
+namespace pa {
+namespace {
+
+int plan_init(pa_decode_step_plan &P, float *out_host, const void *q_host, const void *k_new_host,
+              const void *v_new_host, const int32_t *block_tables_host, int max_blocks_per_seq,
+              const int32_t *seq_lens_host, const int32_t *copy_pairs_host, int max_copy_pairs, void *k_cache,
+              void *v_cache, int batch, int max_seq_len_cap, int num_q_heads, int num_kv_heads, int head_dim,
+              int block_size, int64_t num_blocks, float scale, int partition_tokens, int num_chunks, void *staging,
+              size_t staging_bytes, bool fp8, float k_scale, float v_scale) {
     if (fp8 && !(k_scale > 0.f && v_scale > 0.f && k_scale < 3.0e38f && v_scale < 3.0e38f))
         return PA_ERR_INVALID_ARG;
-    if (batch < 0 || num_pairs < 0 || max_copy_pairs < 0 || max_blocks_per_seq < 0 || max_seq_len < 0 ||
-        num_chunks < 0 || num_chunks > pa::kMaxChunks)
+    if (batch < 0 || max_copy_pairs < 0 || max_blocks_per_seq < 0 || max_seq_len_cap < 0 || num_chunks < 0 ||
+        num_chunks > kMaxChunks)
         return PA_ERR_INVALID_ARG;
-    if (!pa::supported_shape(num_q_heads, num_kv_heads, head_dim, block_size)) return PA_ERR_UNSUPPORTED;
+    if (!supported_shape(num_q_heads, num_kv_heads, head_dim, block_size)) return PA_ERR_UNSUPPORTED;
+    P = pa_decode_step_plan{};
+    P.batch = batch;
     if (batch == 0) return PA_OK;
     if (!out_host || !q_host || !k_new_host || !v_new_host || !block_tables_host || !seq_lens_host || !staging ||
         !k_cache || !v_cache)
         return PA_ERR_INVALID_ARG;
-    if (num_pairs > max_copy_pairs || (num_pairs > 0 && !copy_pairs_host)) return PA_ERR_INVALID_ARG;
     if (partition_tokens > 0 && partition_tokens % block_size) return PA_ERR_INVALID_ARG;  // as pa_decode
-    const pa::StagingLayout l = pa::staging_layout(batch, max_blocks_per_seq, max_copy_pairs, num_q_heads,
-                                                   num_kv_heads, head_dim, block_size, max_seq_len,
-                                                   partition_tokens);
-    if (staging_bytes < l.total || (reinterpret_cast<uintptr_t>(staging) & (pa::kAlign - 1)))
-        return PA_ERR_INVALID_ARG;
-    // Resolve the partitioning once for the whole batch, so that every chunk
-    // splits its sequences exactly as an unchunked call would.
-    const int pt = pa_decode_partition_tokens(batch, num_q_heads, num_kv_heads, head_dim, block_size, max_seq_len,
-                                              partition_tokens);
-    char *st = static_cast<char *>(staging);
-    cudaStream_t s = static_cast<cudaStream_t>(stream);
-    // bytes per sequence of each input and of the output
-    const size_t q_row = (size_t)num_q_heads * head_dim * 2;
-    const size_t kv_row = (size_t)num_kv_heads * head_dim * 2;
-    const size_t tab_row = (size_t)max_blocks_per_seq * 4;
-    const size_t out_row = (size_t)num_q_heads * head_dim * 4;
-    const size_t link_bytes = (size_t)batch * (q_row + 2 * kv_row + tab_row + 4 + out_row) + (size_t)num_pairs * 8;
-    const int chunks = num_chunks ? (num_chunks > batch ? batch : num_chunks) : pa::auto_chunks(batch, link_bytes);
-
+    P.l = staging_layout(batch, max_blocks_per_seq, max_copy_pairs, num_q_heads, num_kv_heads, head_dim,
+                         block_size, max_seq_len_cap, partition_tokens);
+    if (staging_bytes < P.l.total || (reinterpret_cast<uintptr_t>(staging) & (kAlign - 1))) return PA_ERR_INVALID_ARG;
+    P.out_host = out_host;
+    P.copy_pairs_host = copy_pairs_host;
+    P.k_cache = k_cache;
+    P.v_cache = v_cache;
+    P.max_blocks_per_seq = max_blocks_per_seq;
+    P.max_copy_pairs = max_copy_pairs;
+    P.max_seq_len_cap = max_seq_len_cap;
+    P.num_q_heads = num_q_heads;
+    P.num_kv_heads = num_kv_heads;
+    P.head_dim = head_dim;
+    P.block_size = block_size;
+    P.num_blocks = num_blocks;
+    P.scale = scale;
+    P.partition_tokens = partition_tokens;
+    P.fp8 = fp8;
+    P.k_scale = k_scale;
+    P.v_scale = v_scale;
+    P.st = static_cast<char *>(staging);
+    // bytes per sequence crossing the host link: inputs and the fp32 output
+    const size_t link_bytes = (size_t)batch * ((size_t)num_q_heads * head_dim * 6 + (size_t)num_kv_heads * head_dim * 4 +
+                                               (size_t)max_blocks_per_seq * 4 + 4);
+    P.chunks = num_chunks ? (num_chunks > batch ? batch : num_chunks) : auto_chunks(batch, link_bytes);
+    // Host inputs as the device sees them.
+    P.hq = host_src(q_host);
+    P.hk = host_src(k_new_host);
+    P.hv = host_src(v_new_host);
+    P.ht = host_src(block_tables_host);
+    P.hl = host_src(seq_lens_host);
+    P.hp = host_src(copy_pairs_host);
     // The output goes straight into out_host when the device can address it
     // (page-locked host memory): the kernels' stores cross the host link while
     // the decode runs, and no copy stage follows.  Otherwise it is staged on the
     // device and copied back.
     void *out_mapped = nullptr;
-    const bool direct = pa::device_address(out_host, &out_mapped) == PA_OK;
-    char *out_base = direct ? static_cast<char *>(out_mapped) : st + l.out;
+    P.direct = device_address(out_host, &out_mapped) == PA_OK;
+    P.out_base = P.direct ? static_cast<char *>(out_mapped) : P.st + P.l.out;
+    return PA_OK;
+}
+
+int plan_run(const pa_decode_step_plan &P, int max_seq_len, int num_pairs, int32_t *err_flag, cudaStream_t s) {
+    if (P.batch == 0) return PA_OK;
+    if (max_seq_len < 0 || max_seq_len > P.max_seq_len_cap || num_pairs < 0 || num_pairs > P.max_copy_pairs ||
+        (num_pairs > 0 && !P.copy_pairs_host))
+        return PA_ERR_INVALID_ARG;
+    const int batch = P.batch;
+    const StagingLayout &l = P.l;
+    char *st = P.st;
+    // Resolve the partitioning once for the whole batch, so that every chunk
+    // splits its sequences exactly as an unchunked call would.
+    const int pt = pa_decode_partition_tokens(batch, P.num_q_heads, P.num_kv_heads, P.head_dim, P.block_size,
+                                              max_seq_len, P.partition_tokens);
+    // bytes per sequence of each input and of the output
+    const size_t q_row = (size_t)P.num_q_heads * P.head_dim * 2;
+    const size_t kv_row = (size_t)P.num_kv_heads * P.head_dim * 2;
+    const size_t tab_row = (size_t)P.max_blocks_per_seq * 4;
+    const size_t out_row = (size_t)P.num_q_heads * P.head_dim * 4;
+    const int chunks = P.chunks;
 
     // decode of sequences [b0, b0 + nb) with inputs in staging, on stream cs, workspace slice ws
     auto decode_rows = [&](int b0, int nb, char *ws, size_t ws_bytes, cudaStream_t cs) {
-        return pa::decode_impl(reinterpret_cast<float *>(out_base + b0 * out_row), st + l.q + b0 * q_row,
-                               st + l.k_new + b0 * kv_row, st + l.v_new + b0 * kv_row, k_cache, v_cache,
-                               reinterpret_cast<const int32_t *>(st + l.tables + b0 * tab_row), max_blocks_per_seq,
-                               reinterpret_cast<const int32_t *>(st + l.lens) + b0, nb, max_seq_len, num_q_heads,
-                               num_kv_heads, head_dim, block_size, num_blocks, scale, pt, ws, ws_bytes, err_flag,
-                               cs, fp8, k_scale, v_scale, nullptr, 0);
+        return decode_impl(reinterpret_cast<float *>(P.out_base + b0 * out_row), st + l.q + b0 * q_row,
+                           st + l.k_new + b0 * kv_row, st + l.v_new + b0 * kv_row, P.k_cache, P.v_cache,
+                           reinterpret_cast<const int32_t *>(st + l.tables + b0 * tab_row), P.max_blocks_per_seq,
+                           reinterpret_cast<const int32_t *>(st + l.lens) + b0, nb, max_seq_len, P.num_q_heads,
+                           P.num_kv_heads, P.head_dim, P.block_size, P.num_blocks, P.scale, pt, ws, ws_bytes,
+                           err_flag, cs, P.fp8, P.k_scale, P.v_scale, nullptr, 0);
     };
-    // Host inputs as the device sees them (resolved once per call).
-    const pa::HostSrc hq = pa::host_src(q_host), hk = pa::host_src(k_new_host), hv = pa::host_src(v_new_host);
-    const pa::HostSrc ht = pa::host_src(block_tables_host), hl = pa::host_src(seq_lens_host);
-    const pa::HostSrc hp = pa::host_src(num_pairs ? copy_pairs_host : nullptr);
     // q, k_new and v_new of sequences [b0, b0 + nb); with `meta`, also the copy
     // pairs, block tables and lengths of the whole batch.  One kernel launch.
     auto upload = [&](int b0, int nb, bool meta, cudaStream_t cs) {
-        pa::Upload up;
+        Upload up;
         int rc = PA_OK;
         if (meta) {
-            rc = up.add(st + l.pairs, hp, 0, (size_t)num_pairs * 8, cs);
-            if (rc == PA_OK) rc = up.add(st + l.tables, ht, 0, batch * tab_row, cs);
-            if (rc == PA_OK) rc = up.add(st + l.lens, hl, 0, (size_t)batch * 4, cs);
+            rc = up.add(st + l.pairs, P.hp, 0, (size_t)num_pairs * 8, cs);
+            if (rc == PA_OK) rc = up.add(st + l.tables, P.ht, 0, batch * tab_row, cs);
+            if (rc == PA_OK) rc = up.add(st + l.lens, P.hl, 0, (size_t)batch * 4, cs);
         }
-        if (rc == PA_OK) rc = up.add(st + l.q + b0 * q_row, hq, b0 * q_row, nb * q_row, cs);
-        if (rc == PA_OK) rc = up.add(st + l.k_new + b0 * kv_row, hk, b0 * kv_row, nb * kv_row, cs);
-        if (rc == PA_OK) rc = up.add(st + l.v_new + b0 * kv_row, hv, b0 * kv_row, nb * kv_row, cs);
+        if (rc == PA_OK) rc = up.add(st + l.q + b0 * q_row, P.hq, b0 * q_row, nb * q_row, cs);
+        if (rc == PA_OK) rc = up.add(st + l.k_new + b0 * kv_row, P.hk, b0 * kv_row, nb * kv_row, cs);
+        if (rc == PA_OK) rc = up.add(st + l.v_new + b0 * kv_row, P.hv, b0 * kv_row, nb * kv_row, cs);
         if (rc == PA_OK) rc = up.launch(cs);
         return rc;
     };
     auto copy_pairs = [&](cudaStream_t cs) {
         if (num_pairs == 0) return (int)PA_OK;
         const int32_t *pairs = reinterpret_cast<const int32_t *>(st + l.pairs);
-        return fp8 ? pa_copy_blocks_fp8(k_cache, v_cache, pairs, num_pairs, num_blocks, num_kv_heads, block_size,
-                                        head_dim, err_flag, cs)
-                   : pa_copy_blocks(k_cache, v_cache, pairs, num_pairs, num_blocks, num_kv_heads, block_size,
-                                    head_dim, err_flag, cs);
+        return P.fp8 ? pa_copy_blocks_fp8(P.k_cache, P.v_cache, pairs, num_pairs, P.num_blocks, P.num_kv_heads,
+                                          P.block_size, P.head_dim, err_flag, cs)
+                     : pa_copy_blocks(P.k_cache, P.v_cache, pairs, num_pairs, P.num_blocks, P.num_kv_heads,
+                                      P.block_size, P.head_dim, err_flag, cs);
     };
 
     if (chunks <= 1) {
@@ -337,15 +398,31 @@ static int step_host(float *out_host, const void *q_host, const void *k_new_host
         if (rc == PA_OK) rc = copy_pairs(s);
         if (rc == PA_OK)
             rc = decode_rows(0, batch, l.workspace_bytes ? st + l.workspace : nullptr, l.workspace_bytes, s);
-        if (rc == PA_OK && !direct) rc = pa::d2h(out_host, st + l.out, batch * out_row, s);
+        if (rc == PA_OK && !P.direct) rc = d2h(P.out_host, st + l.out, batch * out_row, s);
         return rc;
     }
 
+    // Chunk 0 has half the weight of the others: the first decode waits for its
+    // upload alone, while every later upload runs ahead of the decodes (the link
+    // delivers inputs faster than decode consumes them).
+    const int64_t units = 2LL * chunks - 1;
+    auto chunk_start = [&](int c) {  // at least one sequence per chunk (chunks <= batch)
+        const int b = c == 0 ? 0 : (int)((int64_t)batch * (2LL * c - 1) / units);
+        return b > c ? b : c;
+    };
+    // Without copy pairs, chunk 0's upload goes first, on the caller's stream
+    // (where chunk 0 decodes): the GPU starts while the rest is enqueued.
+    const bool early = num_pairs == 0;
+    if (early) {
+        const int rc0 = upload(0, chunk_start(1), true, s);
+        if (rc0 != PA_OK) return rc0;
+    }
+
     int dev = 0;
-    if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= pa::kMaxDevices) return PA_ERR_CUDA;
-    pa::Pipes &p = pa::g_pipes[dev];
+    if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxDevices) return PA_ERR_CUDA;
+    Pipes &p = g_pipes[dev];
     std::lock_guard<std::mutex> lock(p.mu);
-    if (!pa::make_pipes(p)) return PA_ERR_CUDA;
+    if (!make_pipes(p)) return PA_ERR_CUDA;
 
     // Fork: the side streams start after everything already on the caller's stream
     // (the previous step, which may still read this staging).
@@ -357,52 +434,68 @@ static int step_host(float *out_host, const void *q_host, const void *k_new_host
     int rc = PA_OK;
     if (num_pairs > 0) {
         rc = upload(0, 0, true, p.up);
-        if (rc == PA_OK) rc = pa::after(s, p.up, p.copied);
+        if (rc == PA_OK) rc = after(s, p.up, p.copied);
         if (rc == PA_OK) rc = copy_pairs(s);
-        if (rc == PA_OK) rc = pa::after(p.comp, s, p.copied);
+        if (rc == PA_OK) rc = after(p.comp, s, p.copied);
     }
     char *ws = l.workspace_bytes ? st + l.workspace : nullptr;
     size_t ws_left = l.workspace_bytes;
-    // Chunk 0 has half the weight of the others: the first decode waits for its
-    // upload alone, while every later upload runs ahead of the decodes (the link
-    // delivers inputs faster than decode consumes them).
-    const int64_t units = 2LL * chunks - 1;
-    auto chunk_start = [&](int c) {  // at least one sequence per chunk (chunks <= batch)
-        const int b = c == 0 ? 0 : (int)((int64_t)batch * (2LL * c - 1) / units);
-        return b > c ? b : c;
-    };
     for (int c = 0; c < chunks && rc == PA_OK; ++c) {
         const int b0 = chunk_start(c);
         const int nb = (c + 1 < chunks ? chunk_start(c + 1) : batch) - b0;
         if (nb == 0) continue;
         cudaStream_t cs = (c & 1) ? p.comp : s;
-        rc = upload(b0, nb, c == 0 && num_pairs == 0, p.up);
-        if (rc == PA_OK) rc = pa::after(cs, p.up, p.in[c]);
+        if (!(c == 0 && early)) {  // (chunk 0's early upload is already on its stream)
+            rc = upload(b0, nb, false, p.up);
+            if (rc == PA_OK) rc = after(cs, p.up, p.in[c]);
+        }
         size_t ws_bytes = 0;
         if (rc == PA_OK && ws) {
-            ws_bytes = pa_decode_workspace_size(nb, num_q_heads, num_kv_heads, head_dim, block_size, max_seq_len,
-                                                pt);
-            if (pa::round_up(ws_bytes) > ws_left) rc = PA_ERR_INVALID_ARG;
+            ws_bytes = pa_decode_workspace_size(nb, P.num_q_heads, P.num_kv_heads, P.head_dim, P.block_size,
+                                                max_seq_len, pt);
+            if (round_up(ws_bytes) > ws_left) rc = PA_ERR_INVALID_ARG;
         }
         if (rc == PA_OK) rc = decode_rows(b0, nb, ws_bytes ? ws : nullptr, ws_bytes, cs);
         if (rc == PA_OK && ws_bytes) {
-            ws += pa::round_up(ws_bytes);
-            ws_left -= pa::round_up(ws_bytes);
+            ws += round_up(ws_bytes);
+            ws_left -= round_up(ws_bytes);
         }
-        if (rc == PA_OK && !direct) {
-            rc = pa::after(p.down, cs, p.dec[c]);
+        if (rc == PA_OK && !P.direct) {
+            rc = after(p.down, cs, p.dec[c]);
             if (rc == PA_OK)
-                rc = pa::d2h(reinterpret_cast<char *>(out_host) + b0 * out_row,
-                             st + l.out + b0 * out_row, nb * out_row, p.down);
+                rc = d2h(reinterpret_cast<char *>(P.out_host) + b0 * out_row, st + l.out + b0 * out_row,
+                         nb * out_row, p.down);
         }
     }
     // Join every side stream back into the caller's stream, on error paths too.
-    const int jc = pa::after(s, p.up, p.up_done);
-    const int jp = pa::after(s, p.comp, p.comp_done);
-    const int jd = pa::after(s, p.down, p.down_done);
+    const int jc = after(s, p.up, p.up_done);
+    const int jp = after(s, p.comp, p.comp_done);
+    const int jd = after(s, p.down, p.down_done);
     if (rc == PA_OK) rc = jc != PA_OK ? jc : (jp != PA_OK ? jp : jd);
     return rc;
 }
+
+// The host step for either pool type: bf16 pools, or E4M3 pools with their scales.
+int step_host(float *out_host, const void *q_host, const void *k_new_host, const void *v_new_host,
+              const int32_t *block_tables_host, int max_blocks_per_seq, const int32_t *seq_lens_host,
+              const int32_t *copy_pairs_host, int num_pairs, int max_copy_pairs, void *k_cache, void *v_cache,
+              int batch, int max_seq_len, int num_q_heads, int num_kv_heads, int head_dim, int block_size,
+              int64_t num_blocks, float scale, int partition_tokens, int num_chunks, void *staging,
+              size_t staging_bytes, int32_t *err_flag, void *stream, bool fp8, float k_scale, float v_scale) {
+    if (num_pairs < 0 || max_seq_len < 0) return PA_ERR_INVALID_ARG;
+    pa_decode_step_plan P;
+    const int rc = plan_init(P, out_host, q_host, k_new_host, v_new_host, block_tables_host, max_blocks_per_seq,
+                             seq_lens_host, num_pairs ? copy_pairs_host : nullptr, max_copy_pairs, k_cache, v_cache,
+                             batch, max_seq_len, num_q_heads, num_kv_heads, head_dim, block_size, num_blocks, scale,
+                             partition_tokens, num_chunks, staging, staging_bytes, fp8, k_scale, v_scale);
+    if (rc != PA_OK) return rc;
+    return plan_run(P, max_seq_len, num_pairs, err_flag, static_cast<cudaStream_t>(stream));
+}
+
+}  // namespace
+}  // namespace pa
+
+extern "C" {
 
 int pa_decode_step_host(float *out_host, const void *q_host, const void *k_new_host, const void *v_new_host,
                         const int32_t *block_tables_host, int max_blocks_per_seq, const int32_t *seq_lens_host,
@@ -410,7 +503,7 @@ int pa_decode_step_host(float *out_host, const void *q_host, const void *k_new_h
                         void *v_cache, int batch, int max_seq_len, int num_q_heads, int num_kv_heads,
                         int head_dim, int block_size, int64_t num_blocks, float scale, int partition_tokens,
                         int num_chunks, void *staging, size_t staging_bytes, int32_t *err_flag, void *stream) {
-    return step_host(out_host, q_host, k_new_host, v_new_host, block_tables_host, max_blocks_per_seq,
+    return pa::step_host(out_host, q_host, k_new_host, v_new_host, block_tables_host, max_blocks_per_seq,
                      seq_lens_host, copy_pairs_host, num_pairs, max_copy_pairs, k_cache, v_cache, batch,
                      max_seq_len, num_q_heads, num_kv_heads, head_dim, block_size, num_blocks, scale,
                      partition_tokens, num_chunks, staging, staging_bytes, err_flag, stream, false, 1.f, 1.f);
@@ -423,10 +516,42 @@ int pa_decode_step_host_fp8(float *out_host, const void *q_host, const void *k_n
                             int head_dim, int block_size, int64_t num_blocks, float scale, float k_scale,
                             float v_scale, int partition_tokens, int num_chunks, void *staging,
                             size_t staging_bytes, int32_t *err_flag, void *stream) {
-    return step_host(out_host, q_host, k_new_host, v_new_host, block_tables_host, max_blocks_per_seq,
+    return pa::step_host(out_host, q_host, k_new_host, v_new_host, block_tables_host, max_blocks_per_seq,
                      seq_lens_host, copy_pairs_host, num_pairs, max_copy_pairs, k_cache, v_cache, batch,
                      max_seq_len, num_q_heads, num_kv_heads, head_dim, block_size, num_blocks, scale,
                      partition_tokens, num_chunks, staging, staging_bytes, err_flag, stream, true, k_scale, v_scale);
 }
+
+int pa_decode_step_plan_create(float *out_host, const void *q_host, const void *k_new_host, const void *v_new_host,
+                               const int32_t *block_tables_host, int max_blocks_per_seq, const int32_t *seq_lens_host,
+                               const int32_t *copy_pairs_host, int max_copy_pairs, void *k_cache, void *v_cache,
+                               int batch, int max_seq_len_cap, int num_q_heads, int num_kv_heads, int head_dim,
+                               int block_size, int64_t num_blocks, float scale, int partition_tokens, int num_chunks,
+                               void *staging, size_t staging_bytes, int kv_fp8, float k_scale, float v_scale,
+                               pa_decode_step_plan **plan) {
+    if (!plan) return PA_ERR_INVALID_ARG;
+    *plan = nullptr;
+    pa_decode_step_plan *P = new (std::nothrow) pa_decode_step_plan();
+    if (!P) return PA_ERR_OOM;
+    const int rc = pa::plan_init(*P, out_host, q_host, k_new_host, v_new_host, block_tables_host, max_blocks_per_seq,
+                                 seq_lens_host, copy_pairs_host, max_copy_pairs, k_cache, v_cache, batch,
+                                 max_seq_len_cap, num_q_heads, num_kv_heads, head_dim, block_size, num_blocks, scale,
+                                 partition_tokens, num_chunks, staging, staging_bytes, kv_fp8 != 0,
+                                 kv_fp8 ? k_scale : 1.f, kv_fp8 ? v_scale : 1.f);
+    if (rc != PA_OK) {
+        delete P;
+        return rc;
+    }
+    *plan = P;
+    return PA_OK;
+}
+
+int pa_decode_step_plan_run(const pa_decode_step_plan *plan, int max_seq_len, int num_pairs, int32_t *err_flag,
+                            void *stream) {
+    if (!plan) return PA_ERR_INVALID_ARG;
+    return pa::plan_run(*plan, max_seq_len, num_pairs, err_flag, static_cast<cudaStream_t>(stream));
+}
+
+void pa_decode_step_plan_destroy(pa_decode_step_plan *plan) { delete plan; }
 
 }  // extern "C"

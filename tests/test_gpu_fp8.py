@@ -220,6 +220,7 @@ def test_fp8_host_step_matches_device_path(torch_cuda, cfg, kw, chunks):
                              tables_host=pinned(case.block_tables, torch.int32),
                              lens_host=pinned(case.seq_lens, torch.int32), pairs_host=pinned(pairs_np, torch.int32),
                              k_cache=gk, v_cache=gv, scale=float(case.scale), k_scale=k_scale, v_scale=v_scale,
+                             max_seq_len_cap=case.max_seq_len,
                              partition_tokens=case.partition_tokens, num_chunks=chunks, staging=staging,
                              err_flag=flag)
     step(case.max_seq_len, pairs.shape[0])

@@ -122,7 +122,7 @@ def test_host_step_matches_device_path(cfg, kw, chunks, pinned_out, inputs):
                              v_new_host=pinned(v_last.view(np.int16), torch.bfloat16),
                              tables_host=pinned(case.block_tables, torch.int32),
                              lens_host=pinned(case.seq_lens, torch.int32), pairs_host=pairs_h,
-                             k_cache=dc.k, v_cache=dc.v, scale=float(case.scale),
+                             k_cache=dc.k, v_cache=dc.v, scale=float(case.scale), max_seq_len_cap=case.max_seq_len,
                              partition_tokens=case.partition_tokens, num_chunks=chunks, staging=staging,
                              err_flag=dc.flag)
     step(case.max_seq_len, pairs.shape[0])
@@ -131,3 +131,76 @@ def test_host_step_matches_device_path(cfg, kw, chunks, pinned_out, inputs):
     assert np.array_equal(got, want)
     assert np.array_equal(bits_host(dc.k), bits_host(ref.k)) and np.array_equal(bits_host(dc.v), bits_host(ref.v))
     assert int(dc.flag.item()) == 0
+
+
+@pytest.mark.parametrize("chunks", [1, 3])
+def test_one_call_host_step_matches_plan(chunks):
+    """pa_decode_step_host (everything resolved per call) and a prepared step
+    (pa_decode_step_plan_create once, pa_decode_step_plan_run per step) give the same output and
+    pools, bit for bit, over two steps; the plan refuses a run past its caps."""
+    import ctypes
+    import torch
+    import paged_kv_cache_349_b200 as pa
+    from paged_kv_cache_349_b200._lib import lib
+    case = W.make_case(3, batch=12, max_len=300, num_blocks=1024)
+    k_last, v_last, other = W.split_last_tokens(case)
+    pairs = case.copy_pairs.reshape(-1, 2)
+    P = ctypes.c_void_p
+
+    def pinned(a, dtype):
+        t = torch.from_numpy(np.ascontiguousarray(a))
+        return (t.view(dtype) if dtype is torch.bfloat16 else t.to(dtype)).pin_memory()
+
+    hq = pinned(case.q.view(np.int16), torch.bfloat16)
+    hk, hv = pinned(k_last.view(np.int16), torch.bfloat16), pinned(v_last.view(np.int16), torch.bfloat16)
+    ht, hl = pinned(case.block_tables, torch.int32), pinned(case.seq_lens, torch.int32)
+    hp = pinned(pairs, torch.int32)
+    cap = case.max_seq_len + 8
+    size = pa.pa_decode_step_staging_size(case.batch, case.max_blocks_per_seq, pairs.shape[0], case.num_q_heads,
+                                          case.num_kv_heads, case.head_dim, case.block_size, cap,
+                                          case.partition_tokens)
+    results = []
+    for use_plan in (False, True):
+        dc = DeviceCase(case)
+        if other.size:  # the copy-on-write rows other than each sequence's last, written beforehand
+            pa.pa_copy_blocks(dc.k, dc.v, dc.pairs, err_flag=dc.flag)
+            pa.pa_reshape_and_cache(dc.k_new[torch.from_numpy(other).cuda()].contiguous(),
+                                    dc.v_new[torch.from_numpy(other).cuda()].contiguous(), dc.k, dc.v,
+                                    dc.slots[torch.from_numpy(other).cuda()].contiguous(), err_flag=dc.flag)
+        staging = torch.empty(size, dtype=torch.uint8, device="cuda")
+        out_h = torch.full(case.q.shape, float("nan"), dtype=torch.float32).pin_memory()
+        stream = P(torch.cuda.current_stream().cuda_stream)
+        head = (P(out_h.data_ptr()), P(hq.data_ptr()), P(hk.data_ptr()), P(hv.data_ptr()), P(ht.data_ptr()),
+                case.max_blocks_per_seq, P(hl.data_ptr()), P(hp.data_ptr()))
+        shape = (case.num_q_heads, case.num_kv_heads, case.head_dim, case.block_size, case.num_blocks,
+                 float(case.scale), case.partition_tokens, chunks, P(staging.data_ptr()), size)
+        outs = []
+        plan = P()
+        if use_plan:
+            assert lib.pa_decode_step_plan_create(*head, pairs.shape[0], P(dc.k.data_ptr()), P(dc.v.data_ptr()),
+                                                  case.batch, cap, *shape, 0, 1.0, 1.0, ctypes.byref(plan)) == 0
+            # past the caps: refused, nothing enqueued
+            assert lib.pa_decode_step_plan_run(plan, cap + 1, 0, P(dc.flag.data_ptr()), stream) == \
+                pa.PA_ERR_INVALID_ARG
+            assert lib.pa_decode_step_plan_run(plan, cap, pairs.shape[0] + 1, P(dc.flag.data_ptr()), stream) == \
+                pa.PA_ERR_INVALID_ARG
+        for step in range(2):  # the second step re-runs on the updated pools (same inputs)
+            if use_plan:
+                rc = lib.pa_decode_step_plan_run(plan, case.max_seq_len, 0, P(dc.flag.data_ptr()), stream)
+            else:
+                rc = lib.pa_decode_step_host(*head, 0, pairs.shape[0], P(dc.k.data_ptr()), P(dc.v.data_ptr()),
+                                             case.batch, case.max_seq_len, *shape, P(dc.flag.data_ptr()), stream)
+            assert rc == 0
+            torch.cuda.synchronize()
+            outs.append(out_h.numpy().copy())
+        if use_plan:
+            lib.pa_decode_step_plan_destroy(plan)
+        assert int(dc.flag.item()) == 0
+        results.append((outs, bits_host(dc.k), bits_host(dc.v)))
+    (o1, k1, v1), (o2, k2, v2) = results
+    assert all(np.array_equal(a, b) for a, b in zip(o1, o2))
+    assert np.array_equal(k1, k2) and np.array_equal(v1, v2)
+    want, k_ref, v_ref = oracle.decode_step(case)
+    assert np.array_equal(k1, k_ref) and np.array_equal(v1, v_ref)
+    assert_close(o1[0].astype(np.float64), want, "host step")
+
