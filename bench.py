@@ -300,10 +300,10 @@ def measure_workload(cfg, args, world, rank, pa, headline):
     case = W.make_case(cfg, seed=seed, fill=W.BF16_ZERO, num_blocks=args.num_blocks)
     fp8 = args.kv_dtype == "fp8"
     elem = 1 if fp8 else 2
-    # Shared-prefix groups (the n=4 chat mix): the step decodes with the plain fused decode
-    # (on B200 the 126 MB L2 already serves the repeated prefix reads of neighbouring CTAs);
-    # the shared-prefix decode, which reads each group's shared tiles once, is timed beside it,
-    # with L2 warm and with L2 flushed before each call.
+    # Shared-prefix groups (the n=4 chat mix): the step decodes with pa_decode_shared_prefix,
+    # which reads each group's shared tiles once; the plain fused decode (whose repeated prefix
+    # reads L2 serves) is timed beside it, the two called in alternation, with L2 warm and with
+    # L2 flushed before each call.
     has_groups = case.groups is not None and not fp8 and not args.unfused
     prefix = has_groups and args.decode == "shared-prefix"
     group_size = 4
@@ -484,7 +484,7 @@ def measure_workload(cfg, args, world, rank, pa, headline):
     traffic = rec.get("traffic_bytes_per_launch") if rec else None
     split = prefix or resolved_pt > 0
     roof = {
-        "kernel": kernel + (" (split, merged in-kernel)" if split else " (single pass)"),
+        "kernel": kernel + (" (split decode + log-sum-exp reduce)" if split else " (single pass)"),
         "bound": "hbm",
         "achieved": round(achieved, 1),
         "peak": peak,
@@ -752,7 +752,7 @@ def reference_config(case, cfg, base, world):
         "partition_tokens": case.partition_tokens,
         "parallelism": f"dp{world} (independent sequences per GPU, no collective)",
         "l2": f"inputs larger than L2: {dec_b / 1e9:.2f} GB of K/V per step vs 126 MB L2; no flush",
-        "step": step_description(case, False, False, True),
+        "step": step_description(case, False, case.groups is not None, True),
     }
 
 
@@ -800,7 +800,7 @@ def main():
     ap.add_argument("--per-config", type=str, default=None,
                     help="comma-separated workloads timed after the headline into per_config "
                          "(default: 2,4,5 when --config is left at its default, none otherwise)")
-    ap.add_argument("--decode", choices=["plain", "shared-prefix"], default="plain",
+    ap.add_argument("--decode", choices=["plain", "shared-prefix"], default="shared-prefix",
                     help="the chat mix's step: pa_decode_append (plain) or pa_decode_shared_prefix; the other "
                          "is timed beside it")
     ap.add_argument("--impl", choices=["native", "reference"], default="native")

@@ -1,7 +1,8 @@
 """ctypes loader for ``libpa.so`` (the CUDA library built from ``csrc/``).
 
 There is no fallback: if the library cannot be loaded (or built with nvcc
-when it is missing), importing the package fails.
+when it is missing), importing the package fails.  ``PA_LIBRARY`` may name a
+tuning build of the same sources to load instead.
 """
 from __future__ import annotations
 
@@ -69,8 +70,10 @@ SIGNATURES = {
 
 
 def load() -> ctypes.CDLL:
-    path = _build.LIB
-    if not os.path.exists(path):
+    """Load libpa.so (building it if missing).  PA_LIBRARY may name a tuning build
+    of the same sources (build.py --define ... --out PATH) to load instead."""
+    path = os.environ.get("PA_LIBRARY") or _build.LIB
+    if path == _build.LIB and not os.path.exists(path):
         _build.build()
     lib = ctypes.CDLL(path)
     for name, (res, args) in SIGNATURES.items():

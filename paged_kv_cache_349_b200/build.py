@@ -39,25 +39,39 @@ def _stale() -> bool:
     return any(os.path.getmtime(f) > t for f in deps)
 
 
-def build(force: bool = False, verbose: bool = False) -> str:
-    """Compile the library if a source is newer than ``libpa.so``; return its path."""
-    if not force and not _stale():
+def build(force: bool = False, verbose: bool = False, defines=(), out: str = None) -> str:
+    """Compile the library if a source is newer than ``libpa.so``; return its path.
+
+    ``defines`` (``NAME=VALUE`` strings) and ``out`` make a tuning build of the
+    same sources at another path (always rebuilt); the package loads it when
+    the environment names it in ``PA_LIBRARY``."""
+    target = out or LIB
+    if not out and not defines and not force and not _stale():
         return LIB
-    tmp = LIB + f".tmp{os.getpid()}"
+    tmp = target + f".tmp{os.getpid()}"
     cmd = [_nvcc(), *ARCH, "-O3", "-lineinfo", "-std=c++17", "--expt-relaxed-constexpr",
            "-Xcompiler", "-fPIC,-O3", "-shared", "-cudart", "static", "-I", INCLUDE,
-           "-o", tmp, *sources()]
+           *[f"-D{d}" for d in defines], "-o", tmp, *sources()]
     if verbose:
         cmd.insert(1, "-Xptxas=-v")
-    out = subprocess.run(cmd, capture_output=True, text=True)
-    if out.returncode != 0:
-        sys.stderr.write(out.stdout + out.stderr)
+    res = subprocess.run(cmd, capture_output=True, text=True)
+    if res.returncode != 0:
+        sys.stderr.write(res.stdout + res.stderr)
         raise RuntimeError("nvcc failed building libpa.so")
     if verbose:
-        sys.stderr.write(out.stdout + out.stderr)
-    os.replace(tmp, LIB)
-    return LIB
+        sys.stderr.write(res.stdout + res.stderr)
+    os.replace(tmp, target)
+    return target
 
 
 if __name__ == "__main__":
-    print(build(force="--force" in sys.argv, verbose="-v" in sys.argv))
+    import argparse
+    ap = argparse.ArgumentParser(description="build libpa.so (sm_100a)")
+    ap.add_argument("--force", action="store_true")
+    ap.add_argument("-v", dest="verbose", action="store_true", help="print ptxas register and spill counts")
+    ap.add_argument("--define", action="append", default=[], help="NAME=VALUE for a tuning build")
+    ap.add_argument("--out", default=None, help="output path of a tuning build")
+    a = ap.parse_args()
+    if a.define and not a.out:
+        ap.error("a tuning build (--define) needs --out, so the library itself is left as built")
+    print(build(force=a.force, verbose=a.verbose, defines=a.define, out=a.out))

@@ -189,6 +189,15 @@ __device__ __forceinline__ void mma_16816(float (&d)[4], uint32_t a0, uint32_t a
         mma_bf16_16816(d, a0, a1, a2, a3, b0, b1);
 }
 
+// Tuning builds only: PA_DECODE_SIMT_G1=1 computes the scores and PV of bf16
+// groups of one query head on the CUDA cores (warp-shuffle dot products, fp32
+// FMA) instead of mma.sync; =2 does the same with the mma path compiled out
+// (bf16 groups of one query head only).  This is the comparison that keeps
+// tensor cores on this path.  The library is built with 0.
+#ifndef PA_DECODE_SIMT_G1
+#define PA_DECODE_SIMT_G1 0
+#endif
+
 // CTAs per SM the register allocation must allow (bf16 is limited to 3 by shared memory).
 #ifndef PA_DECODE_MIN_CTAS_FP8
 #define PA_DECODE_MIN_CTAS_FP8 3
@@ -285,6 +294,16 @@ __global__ void __launch_bounds__(kThreads, FP8 ? PA_DECODE_MIN_CTAS_FP8 : PA_DE
     // Per consumer thread: softmax state of query-head columns 2t, 2t+1.
     const int gid = lane >> 2;  // mma group id
     const int tig = lane & 3;   // thread in group
+#if PA_DECODE_SIMT_G1
+    // CUDA-core state for a group of one query head (bf16): this lane's
+    // HEAD_DIM/32 output dims, and the warp's running max and sum.
+    float so[HEAD_DIM / 32];
+#pragma unroll
+    for (int k = 0; k < HEAD_DIM / 32; ++k) so[k] = 0.f;
+    float sm = -INFINITY, sl = 0.f;
+    // 2: CUDA cores only (the mma path compiled out; groups of one query head only)
+    const bool simt = !FP8 && (PA_DECODE_SIMT_G1 == 2 || p.group == 1);
+#endif
     float m_run[2] = {-INFINITY, -INFINITY};
     float l_run[2] = {0.f, 0.f};
     float o[HEAD_DIM / 16][4];
@@ -407,6 +426,22 @@ __global__ void __launch_bounds__(kThreads, FP8 ? PA_DECODE_MIN_CTAS_FP8 : PA_DE
         // largest entry lands just below 2^14 (exact, well inside the f16 range);
         // 2^-qexp and the K dequantisation scale fold into the softmax scale.
         float s_scale = p.scale_log2;
+#if PA_DECODE_SIMT_G1
+        // this lane's half of q (token lane/2 of a tile, dims of half lane & 1), bf16 pairs
+        uint32_t sq[HEAD_DIM / 4];
+        if (simt) {
+            const uint4 *qh = reinterpret_cast<const uint4 *>(
+                p.q + ((int64_t)b * p.num_q_heads + h) * HEAD_DIM + (lane & 1) * (HEAD_DIM / 2));
+#pragma unroll
+            for (int c = 0; c < HEAD_DIM / 16; ++c) {
+                const uint4 v = __ldg(qh + c);
+                sq[4 * c] = v.x;
+                sq[4 * c + 1] = v.y;
+                sq[4 * c + 2] = v.z;
+                sq[4 * c + 3] = v.w;
+            }
+        }
+#endif
         if constexpr (FP8) {
             float amax = 0.f;
 #pragma unroll
@@ -569,6 +604,61 @@ __global__ void __launch_bounds__(kThreads, FP8 ? PA_DECODE_MIN_CTAS_FP8 : PA_DE
                     }
                     __syncwarp();
                 }
+#if PA_DECODE_SIMT_G1
+                if (simt) {
+                    // scores: lanes 2t and 2t+1 each dot half of token t's row with q
+                    const int t = lane >> 1;
+                    float acc = 0.f;
+#pragma unroll
+                    for (int c = 0; c < HEAD_DIM / 16; ++c) {
+                        const uint4 kv = lds128(kbase + tile_offset(t, (lane & 1) * (HEAD_DIM / 16) + c));
+                        const uint32_t kw[4] = {kv.x, kv.y, kv.z, kv.w};
+#pragma unroll
+                        for (int e = 0; e < 4; ++e) {
+                            acc = fmaf(bf16_lo_to_float(kw[e]), bf16_lo_to_float(sq[4 * c + e]), acc);
+                            acc = fmaf(bf16_hi_to_float(kw[e]), bf16_hi_to_float(sq[4 * c + e]), acc);
+                        }
+                    }
+                    acc += __shfl_xor_sync(0xffffffffu, acc, 1);
+                    const float sc = t < valid ? acc * s_scale : -INFINITY;
+                    float mx = sc;
+#pragma unroll
+                    for (int off = 2; off < 32; off <<= 1) mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, off));
+                    const float mn = fmaxf(sm, mx);
+                    const float alpha = fast_exp2(sm - mn);
+                    const float pt = fast_exp2(sc - mn);
+                    float ps = pt;
+#pragma unroll
+                    for (int off = 2; off < 32; off <<= 1) ps += __shfl_xor_sync(0xffffffffu, ps, off);
+                    sl = sl * alpha + ps;
+                    sm = mn;
+#pragma unroll
+                    for (int k = 0; k < HEAD_DIM / 32; ++k) so[k] *= alpha;
+                    // PV: this lane's HEAD_DIM/32 dims of every token row
+#pragma unroll
+                    for (int u = 0; u < kTileTokens; ++u) {
+                        const float pu = __shfl_sync(0xffffffffu, pt, 2 * u);
+                        if constexpr (HEAD_DIM == 128) {
+                            uint32_t v0, v1;
+                            asm volatile("ld.shared.v2.u32 {%0, %1}, [%2];"
+                                         : "=r"(v0), "=r"(v1)
+                                         : "r"(vbase + tile_offset(u, lane >> 1) + (lane & 1) * 8));
+                            so[0] = fmaf(pu, bf16_lo_to_float(v0), so[0]);
+                            so[1] = fmaf(pu, bf16_hi_to_float(v0), so[1]);
+                            so[2] = fmaf(pu, bf16_lo_to_float(v1), so[2]);
+                            so[3] = fmaf(pu, bf16_hi_to_float(v1), so[3]);
+                        } else {
+                            uint32_t v0;
+                            asm volatile("ld.shared.u32 %0, [%1];"
+                                         : "=r"(v0)
+                                         : "r"(vbase + tile_offset(u, lane >> 2) + (lane & 3) * 4));
+                            so[0] = fmaf(pu, bf16_lo_to_float(v0), so[0]);
+                            so[1] = fmaf(pu, bf16_hi_to_float(v0), so[1]);
+                        }
+                    }
+                } else
+#endif
+                {
                 // ---- S^T = K Q^T ----
                 float sacc[4] = {0.f, 0.f, 0.f, 0.f};
 #pragma unroll
@@ -687,6 +777,7 @@ __global__ void __launch_bounds__(kThreads, FP8 ? PA_DECODE_MIN_CTAS_FP8 : PA_DE
                         mma_16816<FP8>(o[mt], a0r, a1r, a2r, a3r, bl0, bl1);
                     }
                 }
+                }
                 if (!FP8 && (valid < kTileTokens || (APPEND && i == i_new))) fence_proxy_async_smem();
             } else if (FP8) {
                 __syncwarp();
@@ -731,6 +822,17 @@ __global__ void __launch_bounds__(kThreads, FP8 ? PA_DECODE_MIN_CTAS_FP8 : PA_DE
             ml[warp * 8 + 2 * tig] = l_run[0];
             ml[warp * 8 + 2 * tig + 1] = l_run[1];
         }
+#if PA_DECODE_SIMT_G1
+        if (simt) {  // column 0 holds the CUDA-core state
+            __syncwarp();
+#pragma unroll
+            for (int k = 0; k < HEAD_DIM / 32; ++k) mo[(warp * 8) * C::kMergeStride + lane * (HEAD_DIM / 32) + k] = so[k];
+            if (lane == 0) {
+                mm[warp * 8] = sm;
+                ml[warp * 8] = sl;
+            }
+        }
+#endif
     }
     __syncthreads();
     const int G = p.group;
