@@ -119,7 +119,7 @@ int launch_decode(const CUtensorMap &km, const CUtensorMap &vm, const DecodePara
     // several CTAs read (shared prefix blocks) are still in L2 when the later
     // ones reach them.
     dim3 grid((unsigned)p.num_parts, (unsigned)p.num_kv_heads, (unsigned)grid_z);
-    kern<<<grid, kThreads, C::kSmemBytes, stream>>>(km, vm, p);
+    kern<<<grid, C::kThreads, C::kSmemBytes, stream>>>(km, vm, p);
     count_launch();
     int st = launch_status();
     if (st != PA_OK || !SPLIT) return st;

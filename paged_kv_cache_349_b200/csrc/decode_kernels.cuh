@@ -20,11 +20,20 @@
 //    columns, K = head_dim), runs an online softmax in fp32 (log2 domain),
 //    and accumulates O^T += V_tile^T P^T with a second mma (M = 16 dims,
 //    N = 8 heads, K = 16 tokens).  P is split into bf16 hi + lo parts so the
-//    PV product keeps ~16 mantissa bits.
+//    PV product keeps ~16 mantissa bits (fp8 pools: one f16 part, 11 bits).
 //  * Warps merge their (max, sum, O) states through shared memory.  In the
 //    split variant each CTA writes its partition's state to the workspace
 //    and a log-sum-exp reduce kernel, launched as a programmatic dependent,
 //    combines the partitions.
+//  * fp8 (E4M3) pools: K and V codes are widened to f16 in registers and run
+//    through the same f16 mma.sync.  A tuning build (PA_DECODE_FP8_TCGEN05=1)
+//    computes the scores on the 5th-generation tensor cores instead: a sixth
+//    warp issues tcgen05.mma (kind::f8f6f4, M = 64 token rows = four ring
+//    tiles, N = 8 query-head columns, K = 32 per step) straight from the
+//    swizzled E4M3 K tiles, against q held as two E4M3 terms, with fp32
+//    scores in tensor memory; each consumer warp reads its tile's 16 rows
+//    back with tcgen05.ld, already in the mma.sync accumulator layout.  It is
+//    correct but slower on B200, so the library keeps mma.sync.
 //  * Shared-prefix variant: sequences that share their first tokens (n-way
 //    sampling of one prompt) get one extra work item per group and kv head
 //    that reads the shared tiles once and serves every member's query heads
@@ -54,8 +63,22 @@ namespace {
 #endif
 constexpr int kTileTokens = 16;
 constexpr int kConsumerWarps = PA_DECODE_CONSUMER_WARPS;
-constexpr int kThreads = (kConsumerWarps + 1) * 32;
 constexpr int kDefaultStages = PA_DECODE_STAGES;
+// fp8 pools at head_dim 128 compute the scores with mma.sync on K codes
+// widened to f16 in registers (0) or with tcgen05.mma (1, a tuning build).
+#ifndef PA_DECODE_FP8_TCGEN05
+#define PA_DECODE_FP8_TCGEN05 0
+#endif
+// fp8 pools: P enters the PV mma as one f16 part (0) or as f16 hi + lo parts
+// (1, a tuning build).  One part keeps 11 significant bits of each weight, for
+// values that carry 4 (E4M3); measured on B200 it takes 3-5 % less time.
+#ifndef PA_DECODE_FP8_P_LO
+#define PA_DECODE_FP8_P_LO 0
+#endif
+// Ring depth of fp8 pools at head_dim 128 (their tiles are half the size).
+#ifndef PA_DECODE_FP8_STAGES
+#define PA_DECODE_FP8_STAGES (2 * PA_DECODE_STAGES)
+#endif
 // Producer lanes issue tiles round-robin; lane k owns ring slots k, k+P, ...
 constexpr int kProducerLanes = PA_DECODE_PRODUCER_LANES;
 static_assert(kProducerLanes >= 1 && kProducerLanes <= 8, "window indexing assumes <= 8 lanes");
@@ -79,22 +102,46 @@ struct Cfg {
     // fp8, head_dim 64: the ring tile is unswizzled and both K and V are expanded
     // to per-warp 16-bit tiles.
     static constexpr bool kDirect = FP8 && HEAD_DIM == 128;
+    // fp8, head_dim 128, tcgen05 scores: a sixth warp issues the MMAs.  Four
+    // consecutive K tiles (a chunk) form one 64-row operand, so the ring keeps
+    // all K tiles together and all V tiles after them (otherwise slot s holds
+    // K then V).
+    static constexpr bool kTc = kDirect && PA_DECODE_FP8_TCGEN05;
+    static constexpr int kThreads = (kConsumerWarps + 1 + (kTc ? 1 : 0)) * 32;
     // Ring depth.  With K and V read from the ring, a slot stays busy until its
     // tile has gone through PV, and fp8 tiles are half the size: twice the
     // default depth keeps enough bytes in flight (measured on B200: 8-11 % less
     // time per call than the default depth).
-    static constexpr int kStages = kDirect ? 2 * kDefaultStages : kDefaultStages;
-    static_assert(kStages % kProducerLanes == 0, "each producer lane owns whole ring slots");
+    static constexpr int kStages = kDirect ? PA_DECODE_FP8_STAGES : kDefaultStages;
+    // Ring slot s is filled by one producer lane and consumed by one consumer
+    // warp, each in order: a parity wait can then never run a phase ahead.
+    static constexpr int kLanes = kStages % kProducerLanes == 0 ? kProducerLanes : kStages % 6 == 0 ? 6 : 4;
+    static_assert(kStages % kLanes == 0, "each producer lane owns whole ring slots");
+    static_assert(kStages % kConsumerWarps == 0, "each consumer warp owns whole ring slots");
     static constexpr int kRingBytes = kStages * kStageBytes;
+    __host__ __device__ static constexpr uint32_t k_off(int s) {
+        return kTc ? (uint32_t)(s * kTileBytes) : (uint32_t)(s * kStageBytes);
+    }
+    __host__ __device__ static constexpr uint32_t v_off(int s) {
+        return kTc ? (uint32_t)((kStages + s) * kTileBytes) : (uint32_t)(s * kStageBytes + kTileBytes);
+    }
+    // tcgen05 scores: q as two E4M3 terms, each 8 columns x 128 bytes (one swizzle atom)
+    static constexpr int kQTerms = 2;
+    static constexpr int kQOpBytes = kTc ? kQTerms * 1024 : 0;
+    static constexpr int kScoreBufs = 4;  // TMEM score buffers (chunks in flight)
+    static constexpr int kScoreBars = kTc ? 2 * kScoreBufs : 0;
+    static constexpr int kTmemCols = 32;  // kScoreBufs x 8 fp32 columns
     static constexpr int kTile16Bytes = (HEAD_DIM / 64) * kBox16Bytes;
     static constexpr int kStagingBytes = FP8 && !kDirect ? kConsumerWarps * 2 * kTile16Bytes : 0;
-    static constexpr int kDataBytes = kRingBytes + kStagingBytes;
+    static constexpr int kDataBytes = kRingBytes + kStagingBytes + kQOpBytes;
     static constexpr int kMergeStride = HEAD_DIM + 4;  // padded row: conflict-free merge stores
     static constexpr int kMergeBytes = kConsumerWarps * 8 * (kMergeStride + 2) * 4;
     static_assert(kMergeBytes <= kDataBytes, "merge area reuses the ring");
-    // + barriers, tile flags, the fused write's row (32 x 16 bytes) and its block id
+    // + barriers, tile flags, the fused write's row (32 x 16 bytes), its block
+    // id (twice: K and V halves with tcgen05 scores) and the TMEM address
     static constexpr int kSmemBytes =
-        1024 /*align slack*/ + kDataBytes + kStages * 8 * 2 + kStages * 4 + 32 * 16 + 16;
+        1024 /*align slack*/ + kDataBytes + 32 * 16 + kStages * 8 * 2 + kScoreBars * 8 + kStages * 4 + 16;
+    static_assert(kDataBytes % 1024 == 0, "the tail (16-byte row, then 8-byte barriers) starts 1024-aligned");
 };
 
 struct DecodeParams {
@@ -207,7 +254,8 @@ __device__ __forceinline__ void mma_16816(float (&d)[4], uint32_t a0, uint32_t a
 #endif
 
 template <int HEAD_DIM, bool SPLIT, bool APPEND, bool FP8, bool PREFIX>
-__global__ void __launch_bounds__(kThreads, FP8 ? PA_DECODE_MIN_CTAS_FP8 : PA_DECODE_MIN_CTAS_BF16) paged_decode_kernel(
+__global__ void __launch_bounds__(Cfg<HEAD_DIM, FP8>::kThreads, FP8 ? PA_DECODE_MIN_CTAS_FP8 : PA_DECODE_MIN_CTAS_BF16)
+    paged_decode_kernel(
     const __grid_constant__ CUtensorMap k_map, const __grid_constant__ CUtensorMap v_map,
     const DecodeParams p) {
     static_assert(SPLIT || !PREFIX, "shared-prefix items always merge through the split path");
@@ -215,13 +263,20 @@ __global__ void __launch_bounds__(kThreads, FP8 ? PA_DECODE_MIN_CTAS_FP8 : PA_DE
     extern __shared__ uint8_t smem_raw[];
     uint8_t *smem = reinterpret_cast<uint8_t *>(
         (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~static_cast<uintptr_t>(1023));
-    uint64_t *full = reinterpret_cast<uint64_t *>(smem + C::kDataBytes);
+    // Fused write: the new token's bf16 K/V row (16 bytes per lane), fetched
+    // asynchronously so no registers are held until the tile is reached.  It
+    // comes first in the tail: kDataBytes is a multiple of 1024, so the row is
+    // 16-byte aligned whatever the ring depth.
+    uint4 *append_row = reinterpret_cast<uint4 *>(smem + C::kDataBytes);
+    uint64_t *full = reinterpret_cast<uint64_t *>(append_row + 32);
     uint64_t *empty = full + C::kStages;
-    int *tile_ok = reinterpret_cast<int *>(empty + C::kStages);
-    // Fused write: the new token's bf16 K/V row (16 bytes per lane) and its block id,
-    // fetched asynchronously so no registers are held until the tile is reached.
-    uint4 *append_row = reinterpret_cast<uint4 *>(tile_ok + C::kStages);
-    int *append_phys = reinterpret_cast<int *>(append_row + 32);
+    // tcgen05 scores: chunk c's scores are in TMEM buffer c % kScoreBufs
+    // (score_full: its MMAs completed; score_free: the four consumer warps read them)
+    uint64_t *score_full = empty + C::kStages;
+    uint64_t *score_free = score_full + C::kScoreBars / 2;
+    int *tile_ok = reinterpret_cast<int *>(empty + C::kStages + C::kScoreBars);
+    int *append_phys = tile_ok + C::kStages;  // the new row's block id: [0], and [1] for the V half (tcgen05)
+    uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(append_phys + 2);
 
     const int part = blockIdx.x;
     const int h = blockIdx.y;
@@ -277,7 +332,7 @@ __global__ void __launch_bounds__(kThreads, FP8 ? PA_DECODE_MIN_CTAS_FP8 : PA_DE
         // Nothing to read.  An empty sequence has no partial states at all, so
         // its partition-0 CTA writes its zero rows; other empty partitions just end.
         if (!pre && part == 0 && L == 0)
-            for (int x = threadIdx.x; x < p.group * HEAD_DIM; x += kThreads)
+            for (int x = threadIdx.x; x < p.group * HEAD_DIM; x += C::kThreads)
                 p.out[((int64_t)b * p.num_q_heads + (int64_t)h * p.group) * HEAD_DIM + x] = 0.f;
         return;
     }
@@ -287,9 +342,26 @@ __global__ void __launch_bounds__(kThreads, FP8 ? PA_DECODE_MIN_CTAS_FP8 : PA_DE
             mbar_init(&full[s], 1);
             mbar_init(&empty[s], 1);
         }
+        for (int s = 0; s < C::kScoreBars / 2; ++s) {
+            mbar_init(&score_full[s], 1);  // tcgen05.commit
+            mbar_init(&score_free[s], kConsumerWarps);
+        }
         fence_mbar_init();
     }
+    if constexpr (C::kTc) {
+        static_assert(kConsumerWarps == 4, "one 64-row MMA covers one tile per consumer warp");
+        if (warp == kConsumerWarps + 1) {  // the MMA warp owns the TMEM columns
+            tmem_alloc(smem_addr(tmem_slot), C::kTmemCols);
+            tmem_relinquish();
+            tc_fence_before();
+        }
+    }
     __syncthreads();
+    uint32_t tmem = 0;
+    if constexpr (C::kTc) {
+        tc_fence_after();
+        tmem = *reinterpret_cast<volatile uint32_t *>(tmem_slot);
+    }
 
     // Per consumer thread: softmax state of query-head columns 2t, 2t+1.
     const int gid = lane >> 2;  // mma group id
@@ -310,11 +382,50 @@ __global__ void __launch_bounds__(kThreads, FP8 ? PA_DECODE_MIN_CTAS_FP8 : PA_DE
 #pragma unroll
     for (int mt = 0; mt < HEAD_DIM / 16; ++mt) o[mt][0] = o[mt][1] = o[mt][2] = o[mt][3] = 0.f;
 
+    // This CTA's query columns as mma B fragments (k = head dim, permuted; n =
+    // column gid): column n is query head n % G of member b + n / G, zero from
+    // nmem * G on.  Lane (gid, tig) holds dims 8 (4j + tig) .. +7, j < d / 32.
+    auto load_q = [&](uint32_t (&qf)[HEAD_DIM / 16][2]) {
+        const int G = p.group;
+        if (gid < nmem * G) {
+            const uint4 *qrow = reinterpret_cast<const uint4 *>(
+                p.q + ((PREFIX ? (int64_t)(b + gid / G) * p.num_q_heads + (int64_t)h * G + gid % G
+                               : (int64_t)b * p.num_q_heads + (int64_t)h * G + gid) *
+                       HEAD_DIM));
+#pragma unroll
+            for (int j = 0; j < HEAD_DIM / 32; ++j) {
+                const uint4 v = __ldg(qrow + 4 * j + tig);
+                qf[2 * j][0] = v.x;
+                qf[2 * j][1] = v.y;
+                qf[2 * j + 1][0] = v.z;
+                qf[2 * j + 1][1] = v.w;
+            }
+        } else {
+#pragma unroll
+            for (int k = 0; k < HEAD_DIM / 16; ++k) qf[k][0] = qf[k][1] = 0u;
+        }
+    };
+    // fp8 pools: the power of two 2^qexp that puts the largest |q| of the CTA's
+    // columns in [2^top, 2^(top+1)), clamped to [lo, hi] (0 for q = 0).  Every
+    // warp that calls it gets the same value.
+    auto fp8_q_exp = [&](const uint32_t (&qf)[HEAD_DIM / 16][2], int top, int lo, int hi) -> int {
+        float amax = 0.f;
+#pragma unroll
+        for (int k = 0; k < HEAD_DIM / 16; ++k) {
+            amax = fmaxf(amax, fmaxf(fabsf(bf16_lo_to_float(qf[k][0])), fabsf(bf16_hi_to_float(qf[k][0]))));
+            amax = fmaxf(amax, fmaxf(fabsf(bf16_lo_to_float(qf[k][1])), fabsf(bf16_hi_to_float(qf[k][1]))));
+        }
+#pragma unroll
+        for (int off = 16; off; off >>= 1) amax = fmaxf(amax, __shfl_xor_sync(0xffffffffu, amax, off));
+        const int e = amax > 0.f ? (int)((__float_as_uint(amax) >> 23) & 0xff) - 127 : top;
+        return max(lo, min(hi, top - e));
+    };
+
     if (warp == kConsumerWarps) {
         // ---------------- producer: block-table dereference + TMA ----------------
         // The whole warp walks the tiles so that block-table entries arrive 32 at a
         // time (one coalesced load per window, the next window loaded ahead).
-        // kProducerLanes lanes wait on the ring and issue copies in parallel:
+        // P = kLanes lanes wait on the ring and issue copies in parallel:
         // lane k handles tiles k, k+P, k+2P, ... and therefore ring slots k, k+P, ...
         const int32_t *table = p.block_tables + (int64_t)tb * p.max_blocks;
         const int j_end = (tok_end + p.block_size - 1) / p.block_size;  // blocks this CTA reads
@@ -322,7 +433,7 @@ __global__ void __launch_bounds__(kThreads, FP8 ? PA_DECODE_MIN_CTAS_FP8 : PA_DE
         int32_t cur = win + lane < j_end ? __ldg(table + win + lane) : -1;
         int32_t nxt = win + 32 + lane < j_end ? __ldg(table + win + 32 + lane) : -1;
         uint64_t policy = 0;
-        if (lane < kProducerLanes) {
+        if (lane < C::kLanes) {
             if (lane == 0) {
                 prefetch_tensormap(&k_map);
                 prefetch_tensormap(&v_map);
@@ -331,7 +442,7 @@ __global__ void __launch_bounds__(kThreads, FP8 ? PA_DECODE_MIN_CTAS_FP8 : PA_DE
         }
         int issued = 0;  // tiles issued by this lane's rounds (max over lanes below)
         bool stop = false;
-        for (int i0 = 0; i0 < n_tiles; i0 += kProducerLanes) {
+        for (int i0 = 0; i0 < n_tiles; i0 += C::kLanes) {
             const int j0 = (tok_begin + i0 * kTileTokens) / p.block_size;
             if (j0 >= win + 32) {  // warp-uniform: slide the window
                 win += 32;
@@ -339,12 +450,12 @@ __global__ void __launch_bounds__(kThreads, FP8 ? PA_DECODE_MIN_CTAS_FP8 : PA_DE
                 nxt = win + 32 + lane < j_end ? __ldg(table + win + 32 + lane) : -1;
             }
             const int i = i0 + lane;
-            const bool mine = lane < kProducerLanes && i < n_tiles;
+            const bool mine = lane < C::kLanes && i < n_tiles;
             const int tok0 = tok_begin + i * kTileTokens;
             const int j = mine ? tok0 / p.block_size : win;
             const int row = tok0 - j * p.block_size;
             // A tile is one slice of a block, or two whole 8-token blocks.
-            const int idx = j - win;  // in [0, 32 + 2 * kProducerLanes)
+            const int idx = j - win;  // in [0, 32 + 2 * C::kLanes)
             const int32_t a_cur = __shfl_sync(0xffffffffu, cur, idx & 31);
             const int32_t a_nxt = __shfl_sync(0xffffffffu, nxt, idx & 31);
             const int32_t b_cur = __shfl_sync(0xffffffffu, cur, (idx + 1) & 31);
@@ -366,25 +477,25 @@ __global__ void __launch_bounds__(kThreads, FP8 ? PA_DECODE_MIN_CTAS_FP8 : PA_DE
                     } else {
                         tile_ok[s] = 1;
                         const int y = (int)((phys * p.num_kv_heads + h) * p.block_size + row);
-                        uint8_t *dst = smem + s * C::kStageBytes;
+                        uint8_t *kdst = smem + C::k_off(s);
+                        uint8_t *vdst = smem + C::v_off(s);
                         mbar_arrive_expect_tx(&full[s], two_blocks && !second ? C::kStageBytes / 2 : C::kStageBytes);
 #pragma unroll
                         for (int bx = 0; bx < C::kBoxes; ++bx)
-                            tma_load_2d(dst + bx * C::kBoxBytes, &k_map, bx * C::kBoxCols, y, &full[s], policy);
+                            tma_load_2d(kdst + bx * C::kBoxBytes, &k_map, bx * C::kBoxCols, y, &full[s], policy);
 #pragma unroll
                         for (int bx = 0; bx < C::kBoxes; ++bx)
-                            tma_load_2d(dst + C::kTileBytes + bx * C::kBoxBytes, &v_map, bx * C::kBoxCols, y,
-                                        &full[s], policy);
+                            tma_load_2d(vdst + bx * C::kBoxBytes, &v_map, bx * C::kBoxCols, y, &full[s], policy);
                         if (second) {  // rows 8..15 of the tile come from the next 8-token block
                             const int y2 = (int)((phys2 * p.num_kv_heads + h) * p.block_size);
 #pragma unroll
                             for (int bx = 0; bx < C::kBoxes; ++bx)
-                                tma_load_2d(dst + bx * C::kBoxBytes + C::kBoxBytes / 2, &k_map, bx * C::kBoxCols, y2,
+                                tma_load_2d(kdst + bx * C::kBoxBytes + C::kBoxBytes / 2, &k_map, bx * C::kBoxCols, y2,
                                             &full[s], policy);
 #pragma unroll
                             for (int bx = 0; bx < C::kBoxes; ++bx)
-                                tma_load_2d(dst + C::kTileBytes + bx * C::kBoxBytes + C::kBoxBytes / 2, &v_map,
-                                            bx * C::kBoxCols, y2, &full[s], policy);
+                                tma_load_2d(vdst + bx * C::kBoxBytes + C::kBoxBytes / 2, &v_map, bx * C::kBoxCols, y2,
+                                            &full[s], policy);
                         }
                     }
                 }
@@ -394,37 +505,138 @@ __global__ void __launch_bounds__(kThreads, FP8 ? PA_DECODE_MIN_CTAS_FP8 : PA_DE
         // Drain: every issued tile has landed before the ring is reused or the CTA exits.
         // A tile is the last user of its slot when no tile one ring depth later was issued.
         const int issued_all = __reduce_max_sync(0xffffffffu, issued);
-        if (lane < kProducerLanes) {
-            for (int i = lane; i < issued_all; i += kProducerLanes)
+        if (lane < C::kLanes) {
+            for (int i = lane; i < issued_all; i += C::kLanes)
                 if (i + C::kStages >= issued_all && i < issued)
                     if (!mbar_wait_bounded(&full[i % C::kStages], (i / C::kStages) & 1, p.err_flag)) break;
         }
-    } else {
-        // ---------------- consumers ----------------
-        const int G = p.group;
-        // Q^T as mma B fragments (k = head dim, permuted; n = query head column gid).
-        // Column gid is query head gid % G of member b + gid / G.
-        uint32_t qf[HEAD_DIM / 16][2];
-        if (gid < nmem * G) {
-            const uint4 *qrow = reinterpret_cast<const uint4 *>(
-                p.q + ((PREFIX ? (int64_t)(b + gid / G) * p.num_q_heads + (int64_t)h * G + gid % G
-                               : (int64_t)b * p.num_q_heads + (int64_t)h * G + gid) *
-                       HEAD_DIM));
+    } else if (C::kTc && warp == kConsumerWarps + 1) {
+        if constexpr (C::kTc) {
+            // ---------------- scores on the tensor cores (fp8 pools, head_dim 128) ----------------
+            // q becomes the MMA's B operand: its 8 columns times 2^qexp (largest
+            // |q| in [2^7, 2^8)) as two E4M3 terms, hi = E4M3(x) and lo =
+            // E4M3(x - hi).  For a scaled bf16 element x with |x| >= 2^-2, x - hi
+            // is a multiple of ulp_8(x) no larger than half ulp_4(x): at most 3
+            // significant bits, an E4M3 normal, so hi + lo == x exactly.  Smaller
+            // elements fall on the E4M3 subnormal grid (2^-9) and keep an error of
+            // at most 2^-10, 2^-17 of the largest; a third term would be zero.
+            uint32_t qf[HEAD_DIM / 16][2];
+            load_q(qf);
+            const int qexp = fp8_q_exp(qf, 7, -120, 126);
+            const float up = __uint_as_float((uint32_t)(127 + qexp) << 23);
+            const uint32_t qop = smem_addr(smem + C::kRingBytes + C::kStagingBytes);
 #pragma unroll
             for (int j = 0; j < HEAD_DIM / 32; ++j) {
-                const uint4 v = __ldg(qrow + 4 * j + tig);
-                qf[2 * j][0] = v.x;
-                qf[2 * j][1] = v.y;
-                qf[2 * j + 1][0] = v.z;
-                qf[2 * j + 1][1] = v.w;
-            }
-        } else {
+                const uint32_t w[4] = {qf[2 * j][0], qf[2 * j][1], qf[2 * j + 1][0], qf[2 * j + 1][1]};
+                float x[8];
 #pragma unroll
-            for (int k = 0; k < HEAD_DIM / 16; ++k) qf[k][0] = qf[k][1] = 0u;
+                for (int e = 0; e < 4; ++e) {
+                    x[2 * e] = bf16_lo_to_float(w[e]) * up;
+                    x[2 * e + 1] = bf16_hi_to_float(w[e]) * up;
+                }
+                // dims 8 (4j + tig) .. +7 of column gid, in the 128-byte-swizzled row
+                const uint32_t off = fp8_tile_offset(gid, 8 * (4 * j + tig));
+#pragma unroll
+                for (int t = 0; t < C::kQTerms; ++t) {
+                    uint32_t codes[2] = {0u, 0u};
+#pragma unroll
+                    for (int e = 0; e < 4; ++e) {
+                        const uint32_t pair = (uint32_t)__nv_cvt_float2_to_fp8x2(
+                            make_float2(x[2 * e], x[2 * e + 1]), __NV_SATFINITE, __NV_E4M3);
+                        codes[e >> 1] |= pair << ((e & 1) * 16);
+                        const uint32_t back = e4m3x2_to_f16x2(pair);  // exact
+                        x[2 * e] -= f16_lo_to_float(back);
+                        x[2 * e + 1] -= f16_hi_to_float(back);
+                    }
+                    asm volatile("st.shared.v2.u32 [%0], {%1, %2};" ::"r"(qop + t * 1024 + off), "r"(codes[0]),
+                                 "r"(codes[1])
+                                 : "memory");
+                }
+            }
+            fence_proxy_async_smem();  // the MMAs read q through the async proxy
+            __syncwarp();
+
+            // Fused cache write, K half: the new token's K row is quantised into its
+            // ring tile (and the pool) before the MMA of its chunk reads the tile.
+            int i_new = -1;
+            if (APPEND && !pre && L == L_raw && L > 0 && L - 1 >= tok_begin && L - 1 < tok_end) {
+                i_new = (L - 1 - tok_begin) / kTileTokens;
+                if (lane < HEAD_DIM / 8)
+                    cp_async16(smem_addr(append_row + lane),
+                               p.k_new + ((int64_t)b * p.num_kv_heads + h) * HEAD_DIM + lane * 8);
+                if (lane == 0)
+                    cp_async4(smem_addr(append_phys),
+                              p.block_tables + (int64_t)b * p.max_blocks + (L - 1) / p.block_size);
+                cp_async_commit();
+            }
+
+            // Instruction descriptor: fp32 scores, E4M3 A and B, both K-major, N = 8, M = 64.
+            constexpr uint32_t kIdesc = (1u << 4) | ((8u >> 3) << 17) | ((64u >> 4) << 24);
+            const uint32_t ring = smem_addr(smem);
+            const int n_chunks = (n_tiles + kConsumerWarps - 1) / kConsumerWarps;
+            int issued = 0;
+            for (int c = 0; c < n_chunks; ++c) {
+                const int buf = c % C::kScoreBufs;
+                bool ok = true;
+#pragma unroll
+                for (int t = 0; t < kConsumerWarps; ++t) {
+                    const int i = c * kConsumerWarps + t;
+                    if (i < n_tiles) ok = ok && mbar_wait_bounded(&full[i % C::kStages], (i / C::kStages) & 1, p.err_flag);
+                }
+                if (c >= C::kScoreBufs)  // the consumers have read this buffer's previous chunk
+                    ok = ok && mbar_wait_bounded(&score_free[buf], ((c / C::kScoreBufs) - 1) & 1, p.err_flag);
+                if (!__all_sync(0xffffffffu, ok)) break;
+                if (APPEND && i_new >= 0 && i_new / kConsumerWarps == c) {
+                    cp_async_wait_all();
+                    __syncwarp();
+                    const int64_t phys = *reinterpret_cast<volatile int *>(append_phys);
+                    if (lane < HEAD_DIM / 8) {
+                        const uint2 q8 = bf16x8_to_e4m3x8(append_row[lane], p.k_inv_scale);
+                        const int r = (L - 1 - tok_begin) - i_new * kTileTokens;
+                        const uint32_t a = ring + C::k_off(i_new % C::kStages) + fp8_tile_offset(r, lane * 8);
+                        asm volatile("st.shared.v2.u32 [%0], {%1, %2};" ::"r"(a), "r"(q8.x), "r"(q8.y) : "memory");
+                        if (phys >= 0 && phys < p.num_blocks)
+                            reinterpret_cast<uint2 *>(p.k_pool)[((phys * p.num_kv_heads + h) * p.block_size +
+                                                                 (L - 1) % p.block_size) *
+                                                                    (HEAD_DIM / 8) +
+                                                                lane] = q8;
+                        fence_proxy_async_smem();
+                    }
+                    __syncwarp();
+                }
+                if (lane == 0) {
+                    tc_fence_after();
+                    // A: the chunk's four K tiles (64 token rows, contiguous in the ring);
+                    // tile 4c + w is rows 16 w .. +15, in TMEM lane quarter w: warp w's.
+                    const uint64_t a_desc = umma_desc_k_sw128(ring + C::k_off((c * kConsumerWarps) % C::kStages));
+                    const uint64_t b_desc = umma_desc_k_sw128(qop);
+                    const uint32_t d = tmem + 8 * buf;
+#pragma unroll
+                    for (int k = 0; k < HEAD_DIM / 32; ++k)
+#pragma unroll
+                        for (int t = 0; t < C::kQTerms; ++t)
+                            umma_e4m3(d, a_desc + 2 * k, b_desc + (1024 >> 4) * t + 2 * k, kIdesc, k > 0 || t > 0);
+                    umma_commit(&score_full[buf]);
+                }
+                __syncwarp();
+                issued = c + 1;
+            }
+            // Every MMA has completed (a commit tracks all earlier MMAs of its thread)
+            // before the ring is reused and TMEM is freed.
+            if (issued > 0)
+                mbar_wait_bounded(&score_full[(issued - 1) % C::kScoreBufs], ((issued - 1) / C::kScoreBufs) & 1,
+                                  p.err_flag);
+            if (APPEND && i_new >= 0) cp_async_wait_all();
         }
+    } else {
+        // ---------------- consumers ----------------
+        uint32_t qf[HEAD_DIM / 16][2];
+        load_q(qf);
         // fp8 pools run the mma in f16: q is scaled by a power of two 2^qexp so its
         // largest entry lands just below 2^14 (exact, well inside the f16 range);
         // 2^-qexp and the K dequantisation scale fold into the softmax scale.
+        // (With tcgen05 scores the MMA warp scales q by its own 2^qexp, the same
+        // value computed here.)
         float s_scale = p.scale_log2;
 #if PA_DECODE_SIMT_G1
         // this lane's half of q (token lane/2 of a tile, dims of half lane & 1), bf16 pairs
@@ -443,30 +655,25 @@ __global__ void __launch_bounds__(kThreads, FP8 ? PA_DECODE_MIN_CTAS_FP8 : PA_DE
         }
 #endif
         if constexpr (FP8) {
-            float amax = 0.f;
-#pragma unroll
-            for (int k = 0; k < HEAD_DIM / 16; ++k) {
-                amax = fmaxf(amax, fmaxf(fabsf(bf16_lo_to_float(qf[k][0])), fabsf(bf16_hi_to_float(qf[k][0]))));
-                amax = fmaxf(amax, fmaxf(fabsf(bf16_lo_to_float(qf[k][1])), fabsf(bf16_hi_to_float(qf[k][1]))));
-            }
-#pragma unroll
-            for (int off = 16; off; off >>= 1) amax = fmaxf(amax, __shfl_xor_sync(0xffffffffu, amax, off));
-            // amax in [2^e, 2^(e+1)) -> qexp = 13 - e; amax == 0 -> qexp = 0
-            const int e = amax > 0.f ? (int)((__float_as_uint(amax) >> 23) & 0xff) - 127 : 13;
-            const int qexp = max(-100, min(100, 13 - e));
-            const float up = __uint_as_float((uint32_t)(127 + qexp) << 23);
+            const int qexp = C::kTc ? fp8_q_exp(qf, 7, -120, 126) : fp8_q_exp(qf, 13, -100, 100);
             const float down = __uint_as_float((uint32_t)(127 - qexp) << 23);
+            if constexpr (!C::kTc) {
+                const float up = __uint_as_float((uint32_t)(127 + qexp) << 23);
 #pragma unroll
-            for (int k = 0; k < HEAD_DIM / 16; ++k) {
-                qf[k][0] = pack_f16x2(bf16_lo_to_float(qf[k][0]) * up, bf16_hi_to_float(qf[k][0]) * up);
-                qf[k][1] = pack_f16x2(bf16_lo_to_float(qf[k][1]) * up, bf16_hi_to_float(qf[k][1]) * up);
+                for (int k = 0; k < HEAD_DIM / 16; ++k) {
+                    qf[k][0] = pack_f16x2(bf16_lo_to_float(qf[k][0]) * up, bf16_hi_to_float(qf[k][0]) * up);
+                    qf[k][1] = pack_f16x2(bf16_lo_to_float(qf[k][1]) * up, bf16_hi_to_float(qf[k][1]) * up);
+                }
             }
             s_scale = p.scale_log2 * p.k_scale * down;
         }
         // Token row of mma row gid (gid+8 -> +8): this order keeps both the K
         // fragment loads and the V ldmatrix reads free of bank conflicts.
         // (fp8 with K read straight from the swizzled fp8 tile uses 0,2,4,6,1,3,5,7.)
-        auto token_of = [](int g) { return C::kDirect ? ((g & 3) << 1) | (g >> 2) : (g >> 1) | ((g & 1) << 2); };
+        // (tcgen05 scores: TMEM row g is token g, so the order is the identity.)
+        auto token_of = [](int g) {
+            return C::kTc ? g : C::kDirect ? ((g & 3) << 1) | (g >> 2) : (g >> 1) | ((g & 1) << 2);
+        };
         const int tau = token_of(gid);
         // ldmatrix row address pattern for V: matrix (lane>>3), row (lane&7).
         const int v_row = token_of(lane & 7) + (((lane >> 4) & 1) << 3);
@@ -484,13 +691,13 @@ __global__ void __launch_bounds__(kThreads, FP8 ? PA_DECODE_MIN_CTAS_FP8 : PA_DE
             if (it % kConsumerWarps == warp) {
                 i_new = it;
                 const int c = lane & 15;
-                if (c < HEAD_DIM / 8) {
+                if (c < HEAD_DIM / 8 && (!C::kTc || lane >= 16)) {  // tcgen05: the MMA warp writes K
                     const uint16_t *src = (lane < 16 ? p.k_new : p.v_new) +
                                           ((int64_t)b * p.num_kv_heads + h) * HEAD_DIM + c * 8;
                     cp_async16(smem_addr(append_row + lane), src);
                 }
-                if (lane == 0)
-                    cp_async4(smem_addr(append_phys),
+                if (lane == (C::kTc ? 16 : 0))
+                    cp_async4(smem_addr(append_phys + (C::kTc ? 1 : 0)),
                               p.block_tables + (int64_t)b * p.max_blocks + (L - 1) / p.block_size);
                 cp_async_commit();
             }
@@ -500,8 +707,8 @@ __global__ void __launch_bounds__(kThreads, FP8 ? PA_DECODE_MIN_CTAS_FP8 : PA_DE
         auto append_fetch = [&](uint4 &row) -> int64_t {
             cp_async_wait_all();
             __syncwarp();
-            const int64_t phys = *reinterpret_cast<volatile int *>(append_phys);
-            row = append_row[lane];
+            const int64_t phys = *reinterpret_cast<volatile int *>(append_phys + (C::kTc ? 1 : 0));
+            row = !C::kTc || lane >= 16 ? append_row[lane] : make_uint4(0u, 0u, 0u, 0u);
             if (phys < 0 || phys >= p.num_blocks) return -1;
             return ((phys * p.num_kv_heads + h) * p.block_size + (L - 1) % p.block_size) * (HEAD_DIM / 8) +
                    (lane & 15);
@@ -509,12 +716,25 @@ __global__ void __launch_bounds__(kThreads, FP8 ? PA_DECODE_MIN_CTAS_FP8 : PA_DE
 
         for (int i = warp; i < n_tiles; i += kConsumerWarps) {
             const int s = i % C::kStages;
-            const bool got = mbar_wait_bounded(&full[s], (i / C::kStages) & 1, p.err_flag);
+            const int chunk = i / kConsumerWarps;  // tcgen05 scores: the chunk of four tiles
+            const int sb = chunk % C::kScoreBufs;
+            bool got = mbar_wait_bounded(&full[s], (i / C::kStages) & 1, p.err_flag);
+            if constexpr (C::kTc)
+                got = got && mbar_wait_bounded(&score_full[sb], (chunk / C::kScoreBufs) & 1, p.err_flag);
             if (!__all_sync(0xffffffffu, got)) break;
+            float tc_s[4] = {0.f, 0.f, 0.f, 0.f};
+            if constexpr (C::kTc) {
+                // The tile's 16 rows are in TMEM lanes 32 warp .. +15, this warp's quarter.
+                tc_fence_after();
+                tmem_ld_16x256b(tmem + ((uint32_t)(32 * warp) << 16) + 8 * sb, tc_s);
+                tc_fence_before();
+                __syncwarp();
+                if (lane == 0) mbar_arrive(&score_free[sb]);
+            }
             const int valid = min(kTileTokens, tok_end - (tok_begin + i * kTileTokens));
             if (tile_ok[s]) {
-                uint32_t kbase = smem_addr(smem + s * C::kStageBytes);
-                uint32_t vbase = kbase + C::kTileBytes;
+                uint32_t kbase = smem_addr(smem + C::k_off(s));
+                uint32_t vbase = smem_addr(smem + C::v_off(s));
                 uint32_t ring_k = kbase;  // fp8 direct-K: K stays in the ring until QK is done
                 if constexpr (C::kDirect) {
                     // The fused cache write lands in the (swizzled) fp8 tile first, and in the pool.
@@ -523,10 +743,12 @@ __global__ void __launch_bounds__(kThreads, FP8 ? PA_DECODE_MIN_CTAS_FP8 : PA_DE
                         const int c = lane & 15;  // 8-byte piece of the 128-byte row
                         uint4 row;
                         const int64_t dst = append_fetch(row);
-                        const uint2 q8 = bf16x8_to_e4m3x8(row, lane < 16 ? p.k_inv_scale : p.v_inv_scale);
-                        const uint32_t a = (lane < 16 ? kbase : vbase) + fp8_tile_offset(r, c * 8);
-                        asm volatile("st.shared.v2.u32 [%0], {%1, %2};" ::"r"(a), "r"(q8.x), "r"(q8.y) : "memory");
-                        if (dst >= 0) reinterpret_cast<uint2 *>(lane < 16 ? p.k_pool : p.v_pool)[dst] = q8;
+                        if (!C::kTc || lane >= 16) {  // tcgen05: the K half is the MMA warp's
+                            const uint2 q8 = bf16x8_to_e4m3x8(row, lane < 16 ? p.k_inv_scale : p.v_inv_scale);
+                            const uint32_t a = (lane < 16 ? kbase : vbase) + fp8_tile_offset(r, c * 8);
+                            asm volatile("st.shared.v2.u32 [%0], {%1, %2};" ::"r"(a), "r"(q8.x), "r"(q8.y) : "memory");
+                            if (dst >= 0) reinterpret_cast<uint2 *>(lane < 16 ? p.k_pool : p.v_pool)[dst] = q8;
+                        }
                         __syncwarp();
                     }
                 } else if constexpr (FP8) {
@@ -660,9 +882,9 @@ __global__ void __launch_bounds__(kThreads, FP8 ? PA_DECODE_MIN_CTAS_FP8 : PA_DE
 #endif
                 {
                 // ---- S^T = K Q^T ----
-                float sacc[4] = {0.f, 0.f, 0.f, 0.f};
+                float sacc[4] = {tc_s[0], tc_s[1], tc_s[2], tc_s[3]};  // tcgen05: already computed
 #pragma unroll
-                for (int j = 0; j < HEAD_DIM / 32; ++j) {
+                for (int j = 0; j < (C::kTc ? 0 : HEAD_DIM / 32); ++j) {
                     uint4 ka, kb;
                     if constexpr (C::kDirect) {
                         // 8 fp8 codes (dims 32j+8t .. +7) of rows tau and tau+8, expanded in registers
@@ -711,13 +933,16 @@ __global__ void __launch_bounds__(kThreads, FP8 ? PA_DECODE_MIN_CTAS_FP8 : PA_DE
                         o[mt][3] *= a1;
                     }
                 }
-                // ---- P^T as B fragments: hi + lo bf16 parts ----
-                uint32_t h01, h23, l01, l23;
+                // ---- P^T as B fragments: hi + lo bf16 parts (fp8 pools: one f16 part) ----
+                constexpr bool kPLo = !FP8 || PA_DECODE_FP8_P_LO;
+                uint32_t h01, h23, l01 = 0u, l23 = 0u;
                 if constexpr (FP8) {
                     h01 = pack_f16x2(p0, p1);
                     h23 = pack_f16x2(p2, p3);
-                    l01 = pack_f16x2(p0 - f16_lo_to_float(h01), p1 - f16_hi_to_float(h01));
-                    l23 = pack_f16x2(p2 - f16_lo_to_float(h23), p3 - f16_hi_to_float(h23));
+                    if (kPLo) {
+                        l01 = pack_f16x2(p0 - f16_lo_to_float(h01), p1 - f16_hi_to_float(h01));
+                        l23 = pack_f16x2(p2 - f16_lo_to_float(h23), p3 - f16_hi_to_float(h23));
+                    }
                 } else {
                     h01 = pack_bf16x2(p0, p1);
                     h23 = pack_bf16x2(p2, p3);
@@ -725,7 +950,7 @@ __global__ void __launch_bounds__(kThreads, FP8 ? PA_DECODE_MIN_CTAS_FP8 : PA_DE
                     l23 = pack_bf16x2(p2 - bf16_lo_to_float(h23), p3 - bf16_hi_to_float(h23));
                 }
                 const uint32_t bh0 = movmatrix_trans(h01), bh1 = movmatrix_trans(h23);
-                const uint32_t bl0 = movmatrix_trans(l01), bl1 = movmatrix_trans(l23);
+                const uint32_t bl0 = kPLo ? movmatrix_trans(l01) : 0u, bl1 = kPLo ? movmatrix_trans(l23) : 0u;
                 // ---- O^T += V^T P^T ----
                 if constexpr (C::kDirect) {
                     // V^T fragments straight from the swizzled fp8 tile.  ldmatrix.trans on
@@ -760,9 +985,9 @@ __global__ void __launch_bounds__(kThreads, FP8 ? PA_DECODE_MIN_CTAS_FP8 : PA_DE
                             }
                         }
                         mma_16816<FP8>(o[2 * c], ev[0], ev[1], ev[2], ev[3], bh0, bh1);
-                        mma_16816<FP8>(o[2 * c], ev[0], ev[1], ev[2], ev[3], bl0, bl1);
+                        if (kPLo) mma_16816<FP8>(o[2 * c], ev[0], ev[1], ev[2], ev[3], bl0, bl1);
                         mma_16816<FP8>(o[2 * c + 1], od[0], od[1], od[2], od[3], bh0, bh1);
-                        mma_16816<FP8>(o[2 * c + 1], od[0], od[1], od[2], od[3], bl0, bl1);
+                        if (kPLo) mma_16816<FP8>(o[2 * c + 1], od[0], od[1], od[2], od[3], bl0, bl1);
                     }
                     // K and V have left the ring: hand the slot back to the producer.
                     if (APPEND && i == i_new) fence_proxy_async_smem();
@@ -774,7 +999,7 @@ __global__ void __launch_bounds__(kThreads, FP8 ? PA_DECODE_MIN_CTAS_FP8 : PA_DE
                         uint32_t a0r, a1r, a2r, a3r;
                         ldmatrix_x4_trans(vbase + tile_offset(v_row, 2 * mt + v_chunk_hi), a0r, a1r, a2r, a3r);
                         mma_16816<FP8>(o[mt], a0r, a1r, a2r, a3r, bh0, bh1);
-                        mma_16816<FP8>(o[mt], a0r, a1r, a2r, a3r, bl0, bl1);
+                        if (kPLo) mma_16816<FP8>(o[mt], a0r, a1r, a2r, a3r, bl0, bl1);
                     }
                 }
                 }
@@ -799,6 +1024,12 @@ __global__ void __launch_bounds__(kThreads, FP8 ? PA_DECODE_MIN_CTAS_FP8 : PA_DE
 
     // ---------------- merge the warps' states (ring memory is free now) ----------------
     __syncthreads();
+    if constexpr (C::kTc) {
+        if (warp == kConsumerWarps + 1) {  // every MMA and TMEM read is complete
+            tc_fence_after();
+            tmem_dealloc(tmem, C::kTmemCols);
+        }
+    }
     float *mo = reinterpret_cast<float *>(smem);                      // [W][8][kMergeStride]
     float *mm = mo + kConsumerWarps * 8 * C::kMergeStride;            // [W][8]
     float *ml = mm + kConsumerWarps * 8;                              // [W][8]
@@ -839,7 +1070,7 @@ __global__ void __launch_bounds__(kThreads, FP8 ? PA_DECODE_MIN_CTAS_FP8 : PA_DE
     // Column n is query head n % G of member b + n / G; in the split variant
     // its partial state goes to slot `slot` of that row.
     const int slot = PREFIX && !pre ? p.num_parts + part : part;
-    for (int x = threadIdx.x; x < (PREFIX ? nmem : 1) * G * HEAD_DIM; x += kThreads) {
+    for (int x = threadIdx.x; x < (PREFIX ? nmem : 1) * G * HEAD_DIM; x += C::kThreads) {
         const int n = x / HEAD_DIM;
         const int d = x - n * HEAD_DIM;
         float M = -INFINITY;

@@ -67,6 +67,12 @@ constexpr long long kWaitLimitCycles = 2000000000LL;
 #ifndef PA_WAIT_SPIN
 #define PA_WAIT_SPIN 0
 #endif
+// try_wait's suspend-time hint in ns (0: none, the hardware's own limit).  A
+// waiting thread sleeps until the phase completes or the hint runs out.  A
+// tuning knob: on B200 a 10 ms hint made the decode 1-3 % slower.
+#ifndef PA_WAIT_SUSPEND_NS
+#define PA_WAIT_SUSPEND_NS 0
+#endif
 
 __device__ __forceinline__ uint32_t smem_addr(const void *p) {
     return static_cast<uint32_t>(__cvta_generic_to_shared(p));
@@ -108,6 +114,18 @@ __device__ __forceinline__ bool mbar_try_wait(uint64_t *bar, uint32_t parity) {
     return done != 0;
 }
 
+__device__ __forceinline__ bool mbar_try_wait_suspend(uint64_t *bar, uint32_t parity, uint32_t ns) {
+    uint32_t done;
+    asm volatile(
+        "{\n\t.reg .pred p;\n\t"
+        "mbarrier.try_wait.parity.acquire.cta.shared::cta.b64 p, [%1], %2, %3;\n\t"
+        "selp.u32 %0, 1, 0, p;\n\t}"
+        : "=r"(done)
+        : "r"(smem_addr(bar)), "r"(parity), "r"(ns)
+        : "memory");
+    return done != 0;
+}
+
 __device__ __forceinline__ bool mbar_test_wait(uint64_t *bar, uint32_t parity) {
     uint32_t done;
     asm volatile(
@@ -121,13 +139,17 @@ __device__ __forceinline__ bool mbar_test_wait(uint64_t *bar, uint32_t parity) {
 }
 
 // Wait for the phase of `bar` with the given parity to complete.  Returns
-// false (and sets PA_FLAG_TIMEOUT) if that takes longer than kWaitLimitCycles.
-// The clock is only read every 64 polls, so the common case costs one poll.
+// false (and sets PA_FLAG_TIMEOUT) if that takes longer than kWaitLimitCycles
+// (give or take one suspend-time hint).  Without a hint the clock is only read
+// every 64 polls, so the common case costs one poll.
 __device__ __forceinline__ bool mbar_wait_bounded(uint64_t *bar, uint32_t parity, int32_t *flag) {
     const long long t0 = clock64();
     for (uint32_t it = 1;; ++it) {
 #if PA_WAIT_SPIN
         if (mbar_test_wait(bar, parity)) return true;
+#elif PA_WAIT_SUSPEND_NS > 0
+        if (mbar_try_wait_suspend(bar, parity, PA_WAIT_SUSPEND_NS)) return true;
+        it = 0;  // every poll may have slept: read the clock each time
 #else
         if (mbar_try_wait(bar, parity)) return true;
 #endif
@@ -260,6 +282,71 @@ __device__ __forceinline__ float f16_lo_to_float(uint32_t v) {
 }
 __device__ __forceinline__ float f16_hi_to_float(uint32_t v) {
     return __half2float(__ushort_as_half((unsigned short)(v >> 16)));
+}
+
+// ---- 5th-generation tensor cores (tcgen05): TMEM and single-thread MMA ----
+
+// Allocate `ncols` TMEM columns (a power of two >= 32) for this CTA; the
+// address lands in shared memory.  Whole warp; the same warp frees them.
+__device__ __forceinline__ void tmem_alloc(uint32_t smem_dst, uint32_t ncols) {
+    asm volatile("tcgen05.alloc.cta_group::1.sync.aligned.shared::cta.b32 [%0], %1;" ::"r"(smem_dst), "r"(ncols)
+                 : "memory");
+}
+__device__ __forceinline__ void tmem_relinquish() {
+    asm volatile("tcgen05.relinquish_alloc_permit.cta_group::1.sync.aligned;" ::: "memory");
+}
+__device__ __forceinline__ void tmem_dealloc(uint32_t taddr, uint32_t ncols) {
+    asm volatile("tcgen05.dealloc.cta_group::1.sync.aligned.b32 %0, %1;" ::"r"(taddr), "r"(ncols) : "memory");
+}
+// Order tcgen05 operations around a thread synchronisation (barrier, mbarrier).
+__device__ __forceinline__ void tc_fence_before() { asm volatile("tcgen05.fence::before_thread_sync;" ::: "memory"); }
+__device__ __forceinline__ void tc_fence_after() { asm volatile("tcgen05.fence::after_thread_sync;" ::: "memory"); }
+
+// Shared-memory matrix descriptor of a K-major operand stored as rows of 128
+// bytes with the 128-byte swizzle (the TMA SWIZZLE_128B layout), 8-row groups
+// 1024 bytes apart, the group base 1024-byte aligned.  Adding 2 advances the
+// start by 32 bytes: the next 32-element K step of an 8-bit operand.
+__device__ __forceinline__ uint64_t umma_desc_k_sw128(uint32_t saddr) {
+    return (uint64_t)((saddr & 0x3ffffu) >> 4)  // start address, 16-byte units
+           | ((uint64_t)1 << 16)                  // leading byte offset (16 B; unused when swizzled)
+           | ((uint64_t)(1024 >> 4) << 32)        // stride byte offset: next 8-row group
+           | ((uint64_t)1 << 46)                  // descriptor version of sm_100
+           | ((uint64_t)2 << 61);                 // 128-byte swizzle
+}
+
+// D[tmem] (+)= A * B^T, both operands E4M3 from shared memory (K-major), fp32
+// accumulate; issued by one thread.  `accumulate` false overwrites D.
+__device__ __forceinline__ void umma_e4m3(uint32_t d_tmem, uint64_t a_desc, uint64_t b_desc, uint32_t idesc,
+                                          bool accumulate) {
+    asm volatile(
+        "{\n\t.reg .pred p;\n\t"
+        "setp.ne.b32 p, %4, 0;\n\t"
+        "tcgen05.mma.cta_group::1.kind::f8f6f4 [%0], %1, %2, %3, p;\n\t}" ::"r"(d_tmem),
+        "l"(a_desc), "l"(b_desc), "r"(idesc), "r"((uint32_t)accumulate)
+        : "memory");
+}
+
+// Arrive once on `bar` when every tcgen05.mma this thread issued so far has completed.
+__device__ __forceinline__ void umma_commit(uint64_t *bar) {
+    asm volatile("tcgen05.commit.cta_group::1.mbarrier::arrive::one.shared::cluster.b64 [%0];" ::"r"(smem_addr(bar))
+                 : "memory");
+}
+
+// 16 TMEM lanes x 8 fp32 columns into the warp, in the mma.sync accumulator
+// layout: lane (g, t) gets (row g, cols 2t, 2t+1) and (row g + 8, cols 2t, 2t+1).
+// Waits for the load before returning.
+__device__ __forceinline__ void tmem_ld_16x256b(uint32_t taddr, float (&v)[4]) {
+    uint32_t r0, r1, r2, r3;
+    asm volatile(
+        "tcgen05.ld.sync.aligned.16x256b.x1.b32 {%0, %1, %2, %3}, [%4];\n\t"
+        "tcgen05.wait::ld.sync.aligned;"
+        : "=r"(r0), "=r"(r1), "=r"(r2), "=r"(r3)
+        : "r"(taddr)
+        : "memory");
+    v[0] = __uint_as_float(r0);
+    v[1] = __uint_as_float(r1);
+    v[2] = __uint_as_float(r2);
+    v[3] = __uint_as_float(r3);
 }
 
 __device__ __forceinline__ float fast_exp2(float x) {
