@@ -476,7 +476,8 @@ def measure_workload(cfg, args, world, rank, pa, headline):
 
     e2e = None
     if not (args.no_e2e or args.unfused):
-        e2e = run_e2e(args, case, pa, stream, world, k, v, (k_scale, v_scale) if fp8 else None)
+        e2e = run_e2e(args, case, pa, stream, world, k, v, (k_scale, v_scale) if fp8 else None,
+                      (case.shared_tokens[::group_size], group_size) if prefix else None)
 
     kernel = ("pa_decode_append_fp8" if fp8 else "pa_decode_shared_prefix (fused write)" if prefix else
               "pa_decode_append" if fused else "pa_decode")
@@ -616,7 +617,7 @@ def replay_allocator(pa, case):
     return alloc, sids
 
 
-def run_e2e(args, case, pa, stream, world, k_pool, v_pool, kv_scales=None):
+def run_e2e(args, case, pa, stream, world, k_pool, v_pool, kv_scales=None, prefix=None):
     """The same step through the public API with host buffers (pinned), timed end to end.
 
     Every step: the host allocator appends one token per sequence (and reports
@@ -625,7 +626,10 @@ def run_e2e(args, case, pa, stream, world, k_pool, v_pool, kv_scales=None):
     prepared once) then uploads the step's inputs, applies the copies and runs
     the fused cache write + decode, whose output lands in pinned host memory;
     the step ends when the output is on the host.  Byte counts are taken after
-    the timed loop.  ``kv_scales`` = (k_scale, v_scale) for fp8 pools.
+    the timed loop.  ``kv_scales`` = (k_scale, v_scale) for fp8 pools;
+    ``prefix`` = (prefix lengths per group, group size) makes the step decode
+    with ``pa_decode_shared_prefix`` (the replayed allocator forks each group's
+    members from its first, so their shared tokens sit in the same blocks).
     """
     import torch
     bs = case.block_size
@@ -649,8 +653,15 @@ def run_e2e(args, case, pa, stream, world, k_pool, v_pool, kv_scales=None):
     h_out = torch.empty(case.q.shape, dtype=torch.float32).pin_memory()
     tables_np, lens_np, pairs_np = h_tables.numpy(), h_lens.numpy(), h_pairs.numpy()
     flag = torch.zeros(1, dtype=torch.int32, device="cuda")
-    size = pa.pa_decode_step_staging_size(B, max_blocks, B, case.num_q_heads, case.num_kv_heads, case.head_dim, bs,
-                                          max_len_cap, case.partition_tokens)
+    if prefix is not None:
+        size = pa.pa_decode_step_staging_size_shared_prefix(B, prefix[1], max_blocks, B, case.num_q_heads,
+                                                            case.num_kv_heads, case.head_dim, bs, max_len_cap,
+                                                            case.partition_tokens)
+        h_prefix = torch.from_numpy(np.ascontiguousarray(prefix[0], dtype=np.int32)).pin_memory()
+    else:
+        size = pa.pa_decode_step_staging_size(B, max_blocks, B, case.num_q_heads, case.num_kv_heads, case.head_dim,
+                                              bs, max_len_cap, case.partition_tokens)
+        h_prefix = None
     staging = torch.empty(size, dtype=torch.uint8, device="cuda")
     if args.unfused:
         raise SystemExit("--unfused applies to the device-resident step only")
@@ -660,7 +671,8 @@ def run_e2e(args, case, pa, stream, world, k_pool, v_pool, kv_scales=None):
                             partition_tokens=case.partition_tokens,
                             num_chunks=args.step_chunks, staging=staging,
                             err_flag=flag, stream=stream,
-                            k_scale=kv_scales[0] if kv_scales else None, v_scale=kv_scales[1] if kv_scales else None)
+                            k_scale=kv_scales[0] if kv_scales else None, v_scale=kv_scales[1] if kv_scales else None,
+                            prefix_lens_host=h_prefix, group_size=prefix[1] if prefix is not None else 0)
     elem = 1 if kv_scales else 2
     host_step = alloc.step_fn(sids, tables_np, lens_np, pairs_np)
     # per timed step: its max length and copy-pair count (the bytes are counted after the timed loop)
@@ -690,6 +702,7 @@ def run_e2e(args, case, pa, stream, world, k_pool, v_pool, kv_scales=None):
     for i, n_pairs in enumerate(steps_seen):
         lens_i = lens0 + i + 1
         acc["h2d"] += sum(t.numel() * t.element_size() for t in (h_q, h_k, h_v, h_tables, h_lens)) + n_pairs * 8
+        acc["h2d"] += h_prefix.numel() * 4 if h_prefix is not None else 0
         acc["d2h"] += h_out.numel() * 4
         acc["tokens"] += int(lens_i.sum())
         c, w, d = step_bytes_from(case, lens_i, n_pairs, elem)
@@ -705,8 +718,11 @@ def run_e2e(args, case, pa, stream, world, k_pool, v_pool, kv_scales=None):
             "includes": "host allocator step (pa_alloc_step: batched append + table export into pinned memory), then one "
                         "pa_decode_step_plan_run call (a step prepared once with pa_decode_step_plan_create"
                         + (" over E4M3 pools" if kv_scales else "")
-                        + "): upload of q/k_new/v_new/tables/lens/copy pairs, block copies, fused cache write "
-                          "+ decode, out stored into pinned host memory; timed until out is on the host"}
+                        + (", in shared-prefix mode: pa_decode_step_plan_set_shared_prefix" if prefix is not None else "")
+                        + "): upload of q/k_new/v_new/tables/lens" + ("/prefix lengths" if prefix is not None else "")
+                        + "/copy pairs, block copies, fused cache write + "
+                        + ("shared-prefix decode" if prefix is not None else "decode")
+                        + ", out stored into pinned host memory; timed until out is on the host"}
 
 
 def step_bytes_from(case, lens, n_pairs, kv_elem_bytes: int = 2):

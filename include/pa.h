@@ -295,9 +295,10 @@ int pa_decode_shared_prefix(float *out, const void *q, const void *k_new, const 
  * of another.  All of them start after the work already enqueued on `stream`
  * and are joined back into `stream` before the call returns (on error paths
  * too), so synchronising `stream` covers the whole step.  0 picks the count
- * from the bytes crossing the host link: one chunk per 512 KiB, at most 4,
- * at most one per sequence (measured on B200: a step moving 2.6 MB took 230,
- * 213, 208 and 205 us end to end with 1 to 4 chunks).  The output, the pools
+ * from the bytes crossing the host link: one chunk per 512 KiB, at most 4
+ * (8 for a prepared step in shared-prefix mode), at most one per sequence
+ * (measured on B200: a step moving 2.6 MB took 230, 213, 208 and 205 us end to
+ * end with 1 to 4 chunks).  The output, the pools
  * and the error flag do not depend on the chunk count: the partitioning is resolved once for the whole
  * batch (as pa_decode_partition_tokens reports it) and each chunk decodes
  * its sequences exactly as an unchunked call would.  The side streams and
@@ -381,6 +382,29 @@ int pa_decode_step_plan_create(float *out_host, const void *q_host, const void *
 
 int pa_decode_step_plan_run(const pa_decode_step_plan *plan, int max_seq_len, int num_pairs, int32_t *err_flag,
                             void *stream);
+
+/* Makes a prepared step (bf16 pools) decode with pa_decode_shared_prefix:
+ * sequences [g*group_size, (g+1)*group_size) share their first
+ * prefix_lens_host[g] tokens (int32 [ceil(batch / group_size)], read on every
+ * run like the other host inputs), under that call's contract ("PagedAttention
+ * & vLLM", Copy-on-write sharing: the shared tokens sit in the same physical
+ * blocks in every member's table).  Each run then gives the outputs and pools
+ * of pa_decode_shared_prefix with the fused write (k_new, v_new) on the
+ * uploaded inputs.  Chunks hold whole groups.  group_size 0 returns the plan
+ * to the plain decode.
+ * The staging buffer must hold pa_decode_step_staging_size_shared_prefix(...)
+ * bytes (same arguments as at create, plus group_size): the prefix lengths
+ * and that decode's larger workspace.
+ * Errors (the plan is left unchanged): plan NULL, group_size < 0 or > 64,
+ * prefix_lens_host NULL with group_size > 0, or staging smaller than that
+ * size: PA_ERR_INVALID_ARG; a plan over fp8 pools: PA_ERR_UNSUPPORTED. */
+int pa_decode_step_plan_set_shared_prefix(pa_decode_step_plan *plan, const int32_t *prefix_lens_host,
+                                          int group_size);
+
+size_t pa_decode_step_staging_size_shared_prefix(int batch, int group_size, int max_blocks_per_seq,
+                                                 int max_copy_pairs, int num_q_heads, int num_kv_heads,
+                                                 int head_dim, int block_size, int max_seq_len,
+                                                 int partition_tokens);
 
 void pa_decode_step_plan_destroy(pa_decode_step_plan *plan);
 

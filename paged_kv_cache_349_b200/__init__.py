@@ -14,7 +14,7 @@ Device ops on fp8 (E4M3) pools:
     pa_quantize_fp8, pa_reshape_and_cache_fp8, pa_copy_blocks_fp8,
     pa_swap_blocks_fp8, pa_decode_fp8 (with k_new/v_new: the fused write)
 A whole decode step from pinned host buffers:
-    pa_decode_step_staging_size, DecodeStepHost (pa_decode_step_plan_*; the
+    pa_decode_step_staging_size[_shared_prefix], DecodeStepHost (pa_decode_step_plan_*; the
     one-call form is pa_decode_step_host[_fp8] in the C ABI)
 Host allocator:
     Allocator (pa_alloc_* / pa_seq_* / pa_block_refcount; step_fn = pa_alloc_step)
@@ -275,6 +275,14 @@ def pa_decode_step_staging_size(batch, max_blocks_per_seq, max_copy_pairs, num_q
                                                num_kv_heads, head_dim, block_size, max_seq_len, partition_tokens))
 
 
+def pa_decode_step_staging_size_shared_prefix(batch, group_size, max_blocks_per_seq, max_copy_pairs, num_q_heads,
+                                              num_kv_heads, head_dim, block_size, max_seq_len,
+                                              partition_tokens=0) -> int:
+    return int(lib.pa_decode_step_staging_size_shared_prefix(batch, group_size, max_blocks_per_seq, max_copy_pairs,
+                                                             num_q_heads, num_kv_heads, head_dim, block_size,
+                                                             max_seq_len, partition_tokens))
+
+
 class DecodeStepHost:
     """Repeated decode steps from fixed pinned host buffers: a prepared step
     (``pa_decode_step_plan_create``) over bf16 pools, or uint8 E4M3 pools given
@@ -284,14 +292,18 @@ class DecodeStepHost:
     tensors, all kept alive by this object.  ``max_seq_len_cap`` bounds the
     ``max_seq_len`` of every call (staging must be sized with it).
     ``num_chunks``: 0 lets the library pick how many chunks of sequences to
-    pipeline, 1 disables pipelining, 2..8 forces that many.  ``close()`` (or
-    garbage collection) releases the plan.
+    pipeline, 1 disables pipelining, 2..8 forces that many.  With
+    ``prefix_lens_host`` (int32, one entry per group) and ``group_size`` the
+    step decodes with ``pa_decode_shared_prefix``
+    (``pa_decode_step_plan_set_shared_prefix``; staging sized by
+    ``pa_decode_step_staging_size_shared_prefix``).  ``close()`` (or garbage
+    collection) releases the plan.
     """
 
     def __init__(self, *, out_host, q_host, k_new_host, v_new_host, tables_host, lens_host, pairs_host,
                  k_cache, v_cache, scale: float, max_seq_len_cap: int, partition_tokens: int = 0,
                  num_chunks: int = 0, staging=None, err_flag=None, stream=None, k_scale: Optional[float] = None,
-                 v_scale: Optional[float] = None):
+                 v_scale: Optional[float] = None, prefix_lens_host=None, group_size: int = 0):
         torch = _torch()
         B, Hq, d = q_host.shape
         NB, Hkv, bs, d2 = k_cache.shape
@@ -321,6 +333,17 @@ class DecodeStepHost:
             int(partition_tokens), int(num_chunks), ctypes.c_void_p(staging.data_ptr()),
             staging.numel() * staging.element_size(), int(self.fp8), float(k_scale or 1.0), float(v_scale or 1.0),
             ctypes.byref(self._plan)), "pa_decode_step_plan_create")
+        if group_size:
+            if prefix_lens_host is None or prefix_lens_host.is_cuda or prefix_lens_host.dtype != torch.int32 \
+                    or not prefix_lens_host.is_contiguous() or prefix_lens_host.numel() < -(-B // group_size):
+                self.close()
+                raise TypeError("prefix_lens_host must be a contiguous host int32 tensor, one entry per group")
+            self._keep = self._keep + (prefix_lens_host,)
+            rc = lib.pa_decode_step_plan_set_shared_prefix(self._plan, ctypes.c_void_p(prefix_lens_host.data_ptr()),
+                                                          int(group_size))
+            if rc != 0:
+                self.close()
+            _check(rc, "pa_decode_step_plan_set_shared_prefix")
         self._flag = _opt_flag(err_flag)
         self._stream = _stream(stream)
         self._run = lib.pa_decode_step_plan_run

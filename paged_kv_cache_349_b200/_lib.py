@@ -42,6 +42,8 @@ SIGNATURES = {
     "pa_decode_step_plan_create": (_I, [_P, _P, _P, _P, _P, _I, _P, _P, _I, _P, _P, _I, _I, _I, _I, _I, _I, _I64,
                                         _F, _I, _I, _P, _SZ, _I, _F, _F, ctypes.POINTER(_P)]),
     "pa_decode_step_plan_run": (_I, [_P, _I, _I, _P, _P]),
+    "pa_decode_step_plan_set_shared_prefix": (_I, [_P, _P, _I]),
+    "pa_decode_step_staging_size_shared_prefix": (_SZ, [_I, _I, _I, _I, _I, _I, _I, _I, _I, _I]),
     "pa_decode_step_plan_destroy": (None, [_P]),
     "pa_decode_builtin_scratch": (_I, [_P, _P, _P, _P, _P, _I, _P, _I, _I, _I, _I, _I, _I, _I64, _F, _I, _P, _P]),
     "pa_quantize_fp8": (_I, [_P, _P, _I64, _F, _P]),

@@ -11,6 +11,7 @@
 // chunk's first.  Every side stream is joined back
 // into the caller's stream before the call returns, so synchronising that
 // stream covers the whole step.
+#include <algorithm>
 #include <mutex>
 #include <new>
 
@@ -22,23 +23,31 @@ namespace {
 constexpr size_t kAlign = 256;
 constexpr int kMaxChunks = 8;
 constexpr int kMaxDevices = 64;
-// Auto chunking: one chunk per this many bytes crossing the host link, at most 4.
-// (Measured on B200 with the Llama-2-7B-shaped step, 2.6 MB over the link:
-// 1, 2, 3, 4 chunks took 230, 213, 208, 205 us end to end.)
+// Auto chunking: one chunk per this many bytes crossing the host link, at most
+// 4, or 8 in shared-prefix mode.  Enqueueing costs ~10 us of host time per chunk,
+// which a short step cannot hide; the shared-prefix decode writes its output at
+// each chunk's end, so it gains from more, smaller chunks.  (Measured on B200,
+// end to end: the Llama-2-7B-shaped step, 2.6 MB over the link, 230, 213, 208,
+// 205 us with 1, 2, 3, 4 chunks; the Llama-3-8B one, 7.5 MB, 0.29 ms with 4
+// chunks and 0.31-0.33 with 8; the chat mix in shared-prefix mode 0.46-0.47 ms
+// with 4 and 0.43-0.44 with 8.)
 constexpr size_t kAutoChunkBytes = (size_t)1 << 19;
 constexpr int kAutoMaxChunks = 4;
+constexpr int kAutoMaxChunksShared = 8;
 
 inline size_t round_up(size_t x) { return (x + kAlign - 1) / kAlign * kAlign; }
 
 // Device staging of one step, each section 256-byte aligned.  The workspace
 // section leaves room for every chunk to have a 256-byte aligned slice of its own.
+// group_size > 0: the step runs the shared-prefix decode, with one prefix length
+// per group of group_size sequences and that decode's partial-state workspace.
 struct StagingLayout {
-    size_t q, k_new, v_new, tables, lens, pairs, out, workspace, workspace_bytes, total;
+    size_t q, k_new, v_new, tables, lens, pairs, prefix, out, workspace, workspace_bytes, total;
 };
 
 StagingLayout staging_layout(int batch, int max_blocks_per_seq, int max_copy_pairs, int num_q_heads,
                              int num_kv_heads, int head_dim, int block_size, int max_seq_len,
-                             int partition_tokens) {
+                             int partition_tokens, int group_size = 0) {
     StagingLayout l{};
     size_t off = 0;
     l.q = off;
@@ -53,11 +62,17 @@ StagingLayout staging_layout(int batch, int max_blocks_per_seq, int max_copy_pai
     off += round_up((size_t)batch * 4);
     l.pairs = off;
     off += round_up((size_t)(max_copy_pairs > 0 ? max_copy_pairs : 0) * 8);
+    l.prefix = off;
+    if (group_size > 0) off += round_up((size_t)((batch + group_size - 1) / group_size) * 4);
     l.out = off;
     off += round_up((size_t)batch * num_q_heads * head_dim * 4);
     l.workspace = off;
-    l.workspace_bytes = pa_decode_workspace_size(batch, num_q_heads, num_kv_heads, head_dim, block_size,
-                                                 max_seq_len, partition_tokens);
+    l.workspace_bytes = group_size > 0
+                            ? pa_decode_shared_prefix_workspace_size(batch, group_size, num_q_heads, num_kv_heads,
+                                                                     head_dim, block_size, max_seq_len,
+                                                                     partition_tokens)
+                            : pa_decode_workspace_size(batch, num_q_heads, num_kv_heads, head_dim, block_size,
+                                                       max_seq_len, partition_tokens);
     // Each chunk's slice rounds its partial states and itself up to kAlign.
     if (l.workspace_bytes) l.workspace_bytes += 2 * kAlign * kMaxChunks;
     off += round_up(l.workspace_bytes);
@@ -77,7 +92,7 @@ int h2d(void *dst, const void *src, size_t bytes, cudaStream_t s) {
 // device mapping), four 16-byte loads in flight per thread, fill the link with
 // one launch for all of them.
 // ---------------------------------------------------------------------------
-constexpr int kMaxSegs = 6;
+constexpr int kMaxSegs = 8;  // copy pairs, tables, lengths, prefix lengths, q, k_new, v_new (+1 spare)
 constexpr int kUploadThreads = 256;
 constexpr int kUploadInFlight = 4;
 
@@ -229,9 +244,9 @@ int after(cudaStream_t waiter, cudaStream_t s, cudaEvent_t e) {
     return cudaStreamWaitEvent(waiter, e, 0) == cudaSuccess ? PA_OK : PA_ERR_CUDA;
 }
 
-int auto_chunks(int batch, size_t link_bytes) {
+int auto_chunks(int batch, size_t link_bytes, int max_chunks) {
     const size_t n = link_bytes / kAutoChunkBytes;
-    int c = n < 1 ? 1 : (n > (size_t)kAutoMaxChunks ? kAutoMaxChunks : (int)n);
+    int c = n < 1 ? 1 : (n > (size_t)max_chunks ? max_chunks : (int)n);
     return c > batch ? batch : c;
 }
 
@@ -247,6 +262,18 @@ size_t pa_decode_step_staging_size(int batch, int max_blocks_per_seq, int max_co
         return 0;
     return pa::staging_layout(batch, max_blocks_per_seq, max_copy_pairs, num_q_heads, num_kv_heads, head_dim,
                               block_size, max_seq_len, partition_tokens)
+        .total;
+}
+
+size_t pa_decode_step_staging_size_shared_prefix(int batch, int group_size, int max_blocks_per_seq,
+                                                 int max_copy_pairs, int num_q_heads, int num_kv_heads,
+                                                 int head_dim, int block_size, int max_seq_len,
+                                                 int partition_tokens) {
+    if (batch <= 0 || group_size < 1 || group_size > pa::kMaxGroupSize || max_blocks_per_seq < 0 ||
+        num_q_heads <= 0 || num_kv_heads <= 0 || head_dim <= 0)
+        return 0;
+    return pa::staging_layout(batch, max_blocks_per_seq, max_copy_pairs, num_q_heads, num_kv_heads, head_dim,
+                              block_size, max_seq_len, partition_tokens, group_size)
         .total;
 }
 
@@ -270,10 +297,15 @@ struct pa_decode_step_plan {
     bool fp8;
     float k_scale, v_scale;
     char *st;                      // staging
+    size_t staging_bytes;
     pa::StagingLayout l;
-    pa::HostSrc hq, hk, hv, ht, hl, hp;
+    pa::HostSrc hq, hk, hv, ht, hl, hp, hx;
     bool direct;                   // the kernels store the output into out_host
     char *out_base;
+    int group_size;                // > 0: shared-prefix decode over groups of this many sequences
+    const int32_t *prefix_lens_host;
+    bool auto_chunks;              // the chunk count is the library's choice
+    size_t link_bytes;             // bytes per step crossing the host link
 };
 
 namespace pa {
@@ -319,10 +351,13 @@ int plan_init(pa_decode_step_plan &P, float *out_host, const void *q_host, const
     P.k_scale = k_scale;
     P.v_scale = v_scale;
     P.st = static_cast<char *>(staging);
+    P.staging_bytes = staging_bytes;
     // bytes per sequence crossing the host link: inputs and the fp32 output
     const size_t link_bytes = (size_t)batch * ((size_t)num_q_heads * head_dim * 6 + (size_t)num_kv_heads * head_dim * 4 +
                                                (size_t)max_blocks_per_seq * 4 + 4);
-    P.chunks = num_chunks ? (num_chunks > batch ? batch : num_chunks) : auto_chunks(batch, link_bytes);
+    P.auto_chunks = num_chunks == 0;
+    P.link_bytes = link_bytes;
+    P.chunks = num_chunks ? (num_chunks > batch ? batch : num_chunks) : auto_chunks(batch, link_bytes, kAutoMaxChunks);
     // Host inputs as the device sees them.
     P.hq = host_src(q_host);
     P.hk = host_src(k_new_host);
@@ -357,16 +392,19 @@ int plan_run(const pa_decode_step_plan &P, int max_seq_len, int num_pairs, int32
     const size_t kv_row = (size_t)P.num_kv_heads * P.head_dim * 2;
     const size_t tab_row = (size_t)P.max_blocks_per_seq * 4;
     const size_t out_row = (size_t)P.num_q_heads * P.head_dim * 4;
-    const int chunks = P.chunks;
+    const int chunks = P.group_size > 0 ? std::min(P.chunks, (batch + P.group_size - 1) / P.group_size) : P.chunks;
 
     // decode of sequences [b0, b0 + nb) with inputs in staging, on stream cs, workspace slice ws
     auto decode_rows = [&](int b0, int nb, char *ws, size_t ws_bytes, cudaStream_t cs) {
+        // shared-prefix decode: b0 starts a group, so the chunk's groups are b0 / gs on
+        const int32_t *prefix =
+            P.group_size > 0 ? reinterpret_cast<const int32_t *>(st + l.prefix) + b0 / P.group_size : nullptr;
         return decode_impl(reinterpret_cast<float *>(P.out_base + b0 * out_row), st + l.q + b0 * q_row,
                            st + l.k_new + b0 * kv_row, st + l.v_new + b0 * kv_row, P.k_cache, P.v_cache,
                            reinterpret_cast<const int32_t *>(st + l.tables + b0 * tab_row), P.max_blocks_per_seq,
                            reinterpret_cast<const int32_t *>(st + l.lens) + b0, nb, max_seq_len, P.num_q_heads,
                            P.num_kv_heads, P.head_dim, P.block_size, P.num_blocks, P.scale, pt, ws, ws_bytes,
-                           err_flag, cs, P.fp8, P.k_scale, P.v_scale, nullptr, 0);
+                           err_flag, cs, P.fp8, P.k_scale, P.v_scale, prefix, P.group_size);
     };
     // q, k_new and v_new of sequences [b0, b0 + nb); with `meta`, also the copy
     // pairs, block tables and lengths of the whole batch.  One kernel launch.
@@ -377,6 +415,8 @@ int plan_run(const pa_decode_step_plan &P, int max_seq_len, int num_pairs, int32
             rc = up.add(st + l.pairs, P.hp, 0, (size_t)num_pairs * 8, cs);
             if (rc == PA_OK) rc = up.add(st + l.tables, P.ht, 0, batch * tab_row, cs);
             if (rc == PA_OK) rc = up.add(st + l.lens, P.hl, 0, (size_t)batch * 4, cs);
+            if (rc == PA_OK && P.group_size > 0)
+                rc = up.add(st + l.prefix, P.hx, 0, (size_t)((batch + P.group_size - 1) / P.group_size) * 4, cs);
         }
         if (rc == PA_OK) rc = up.add(st + l.q + b0 * q_row, P.hq, b0 * q_row, nb * q_row, cs);
         if (rc == PA_OK) rc = up.add(st + l.k_new + b0 * kv_row, P.hk, b0 * kv_row, nb * kv_row, cs);
@@ -404,11 +444,20 @@ int plan_run(const pa_decode_step_plan &P, int max_seq_len, int num_pairs, int32
 
     // Chunk 0 has half the weight of the others: the first decode waits for its
     // upload alone, while every later upload runs ahead of the decodes (the link
-    // delivers inputs faster than decode consumes them).
-    const int64_t units = 2LL * chunks - 1;
-    auto chunk_start = [&](int c) {  // at least one sequence per chunk (chunks <= batch)
-        const int b = c == 0 ? 0 : (int)((int64_t)batch * (2LL * c - 1) / units);
-        return b > c ? b : c;
+    // delivers inputs faster than decode consumes them).  Chunks hold whole
+    // groups of the shared-prefix decode (single sequences otherwise).  That
+    // decode writes every output row from its reduce, after the chunk's decode,
+    // so the last chunk's output crossing the link is not overlapped: its last
+    // chunk is half-size too (chat mix, 8 chunks: 0.437 against 0.460 ms a step).
+    const int gs = P.group_size > 0 ? P.group_size : 1;
+    const int groups = (batch + gs - 1) / gs;
+    const bool taper = P.group_size > 0 && chunks >= 3;
+    const int64_t units = 2LL * chunks - 1 - (taper ? 1 : 0);
+    auto chunk_start = [&](int c) {  // at least one group per chunk (chunks <= groups)
+        int g = c == 0 ? 0 : (int)((int64_t)groups * (2LL * c - 1) / units);
+        if (g < c) g = c;
+        const int b = g * gs;
+        return b < batch ? b : batch;
     };
     // Without copy pairs, chunk 0's upload goes first, on the caller's stream
     // (where chunk 0 decodes): the GPU starts while the rest is enqueued.
@@ -451,8 +500,11 @@ int plan_run(const pa_decode_step_plan &P, int max_seq_len, int num_pairs, int32
         }
         size_t ws_bytes = 0;
         if (rc == PA_OK && ws) {
-            ws_bytes = pa_decode_workspace_size(nb, P.num_q_heads, P.num_kv_heads, P.head_dim, P.block_size,
-                                                max_seq_len, pt);
+            ws_bytes = P.group_size > 0
+                           ? pa_decode_shared_prefix_workspace_size(nb, P.group_size, P.num_q_heads, P.num_kv_heads,
+                                                                    P.head_dim, P.block_size, max_seq_len, pt)
+                           : pa_decode_workspace_size(nb, P.num_q_heads, P.num_kv_heads, P.head_dim, P.block_size,
+                                                      max_seq_len, pt);
             if (round_up(ws_bytes) > ws_left) rc = PA_ERR_INVALID_ARG;
         }
         if (rc == PA_OK) rc = decode_rows(b0, nb, ws_bytes ? ws : nullptr, ws_bytes, cs);
@@ -550,6 +602,33 @@ int pa_decode_step_plan_run(const pa_decode_step_plan *plan, int max_seq_len, in
                             void *stream) {
     if (!plan) return PA_ERR_INVALID_ARG;
     return pa::plan_run(*plan, max_seq_len, num_pairs, err_flag, static_cast<cudaStream_t>(stream));
+}
+
+int pa_decode_step_plan_set_shared_prefix(pa_decode_step_plan *plan, const int32_t *prefix_lens_host,
+                                          int group_size) {
+    if (!plan) return PA_ERR_INVALID_ARG;
+    pa_decode_step_plan &P = *plan;
+    if (group_size < 0 || group_size > pa::kMaxGroupSize) return PA_ERR_INVALID_ARG;
+    if (group_size > 0 && P.fp8) return PA_ERR_UNSUPPORTED;
+    if (P.batch == 0) {  // nothing to run: remember the mode only
+        P.group_size = group_size;
+        P.prefix_lens_host = prefix_lens_host;
+        return PA_OK;
+    }
+    if (group_size > 0 && !prefix_lens_host) return PA_ERR_INVALID_ARG;
+    const pa::StagingLayout l = pa::staging_layout(P.batch, P.max_blocks_per_seq, P.max_copy_pairs, P.num_q_heads,
+                                                   P.num_kv_heads, P.head_dim, P.block_size, P.max_seq_len_cap,
+                                                   P.partition_tokens, group_size);
+    if (P.staging_bytes < l.total) return PA_ERR_INVALID_ARG;  // the plan is left as it was
+    P.l = l;
+    P.group_size = group_size;
+    P.prefix_lens_host = group_size > 0 ? prefix_lens_host : nullptr;
+    P.hx = group_size > 0 ? pa::host_src(prefix_lens_host) : pa::HostSrc{};
+    if (!P.direct) P.out_base = P.st + P.l.out;  // the staged output section moves with the layout
+    if (P.auto_chunks)
+        P.chunks = pa::auto_chunks(P.batch, P.link_bytes,
+                                   group_size > 0 ? pa::kAutoMaxChunksShared : pa::kAutoMaxChunks);
+    return PA_OK;
 }
 
 void pa_decode_step_plan_destroy(pa_decode_step_plan *plan) { delete plan; }

@@ -108,6 +108,23 @@ def test_shared_prefix_workspace_size(pt, maxlen, parts):
     assert pa.pa_decode_shared_prefix_workspace_size(0, n, Hq, Hkv, d, 16, maxlen, pt) == 0
 
 
+def test_step_staging_size_shared_prefix():
+    """The shared-prefix host step stages the plain step's sections plus one prefix length per group
+    (256-byte aligned) and the shared-prefix decode's workspace in place of the plain one's."""
+    B, n, mb, pairs, Hq, Hkv, d, bs, L = 128, 4, 160, 8, 40, 40, 128, 16, 2500
+    plain = pa.pa_decode_step_staging_size(B, mb, pairs, Hq, Hkv, d, bs, L, 0)
+    shared = pa.pa_decode_step_staging_size_shared_prefix(B, n, mb, pairs, Hq, Hkv, d, bs, L, 0)
+    slack = 2 * 256 * 8  # a 256-byte aligned workspace slice per chunk
+    ws_plain = pa.pa_decode_workspace_size(B, Hq, Hkv, d, bs, L, 0)
+    ws_shared = pa.pa_decode_shared_prefix_workspace_size(B, n, Hq, Hkv, d, bs, L, 0)
+    rnd = lambda x: -(-x // 256) * 256
+    plain_ws = rnd(ws_plain + slack) if ws_plain else 0
+    assert shared - plain == rnd(B // n * 4) + rnd(ws_shared + slack) - plain_ws
+    for g in (0, 65):
+        assert pa.pa_decode_step_staging_size_shared_prefix(B, g, mb, pairs, Hq, Hkv, d, bs, L, 0) == 0
+    assert pa.pa_decode_step_staging_size_shared_prefix(0, n, mb, pairs, Hq, Hkv, d, bs, L, 0) == 0
+
+
 def test_shared_prefix_argument_errors_need_no_gpu():
     f = lib.pa_decode_shared_prefix
     base = [_fake(), _fake(), None, None, _fake(), _fake(), _fake(), 4, _fake(), _fake(), 4, 8, 64, 8, 8, 128,

@@ -176,3 +176,106 @@ def test_full_size_chat_workload_sampled_rows():
     case = W.make_case(3)
     rows = sample_rows(case, 96, seed=33)
     check(case, case.shared_tokens[::4], 4, 0, rows=rows, what="chat full")
+
+
+def _pinned(torch, a, dtype):
+    t = torch.from_numpy(np.ascontiguousarray(a))
+    return (t.view(dtype) if dtype is torch.bfloat16 else t.to(dtype)).pin_memory()
+
+
+@pytest.mark.parametrize("kind,chunks", [("chat", 1), ("chat", 2), ("chat", 3), ("ragged", 2), ("ragged", 5)])
+def test_prepared_host_step_matches_device_path(kind, chunks):
+    """A prepared host step in shared-prefix mode (pa_decode_step_plan_set_shared_prefix): inputs
+    uploaded from pinned host memory, chunks of whole groups, output stored into pinned host memory --
+    bit-identical to pa_decode_shared_prefix on device-resident inputs, pools included."""
+    import torch
+    import paged_kv_cache_349_b200 as pa
+    if kind == "chat":
+        case = W.make_case(3, batch=12, max_len=400, num_blocks=1024)
+        n, prefix = 4, case.shared_tokens[::4]
+    else:  # 19 sequences in groups of 4: the last group has 3
+        n, prefix = 4, [35, 16, 200, 30, 94]
+        case = grouped_case(LENS_NO_EMPTY, n, prefix, Hq=8, Hkv=2, d=128, bs=16, seed=71)
+    ref, want = run_prefix(case, prefix, n, case.partition_tokens)
+    dc = DeviceCase(case)
+    k_last, v_last, other = W.split_last_tokens(case)
+    pa.pa_copy_blocks(dc.k, dc.v, dc.pairs, err_flag=dc.flag)
+    if other.size:
+        pa.pa_reshape_and_cache(bf16_dev(case.k_new[other]), bf16_dev(case.v_new[other]), dc.k, dc.v,
+                                i32_dev(case.slot_mapping[other]), err_flag=dc.flag)
+    B = case.batch
+    args = (B, n, case.max_blocks_per_seq, 1, case.num_q_heads, case.num_kv_heads, case.head_dim, case.block_size,
+            case.max_seq_len, case.partition_tokens)
+    size = pa.pa_decode_step_staging_size_shared_prefix(*args)
+    plain = pa.pa_decode_step_staging_size(B, *args[2:])
+    assert size > plain > 0
+    staging = torch.empty(size, dtype=torch.uint8, device="cuda")
+    out_h = torch.full(case.q.shape, float("nan"), dtype=torch.float32).pin_memory()
+    step = pa.DecodeStepHost(out_host=out_h, q_host=_pinned(torch, case.q.view(np.int16), torch.bfloat16),
+                             k_new_host=_pinned(torch, k_last.view(np.int16), torch.bfloat16),
+                             v_new_host=_pinned(torch, v_last.view(np.int16), torch.bfloat16),
+                             tables_host=_pinned(torch, case.block_tables, torch.int32),
+                             lens_host=_pinned(torch, case.seq_lens, torch.int32),
+                             pairs_host=_pinned(torch, np.zeros((1, 2), np.int32), torch.int32),
+                             k_cache=dc.k, v_cache=dc.v, scale=float(case.scale), max_seq_len_cap=case.max_seq_len,
+                             partition_tokens=case.partition_tokens, num_chunks=chunks, staging=staging,
+                             err_flag=dc.flag, prefix_lens_host=_pinned(torch, np.asarray(prefix), torch.int32),
+                             group_size=n)
+    step(case.max_seq_len, 0)
+    torch.cuda.synchronize()
+    assert int(dc.flag.item()) == 0 and int(ref.flag.item()) == 0
+    assert np.array_equal(out_h.numpy().astype(np.float64), want)
+    assert np.array_equal(bits_host(dc.k), bits_host(ref.k)) and np.array_equal(bits_host(dc.v), bits_host(ref.v))
+    step.close()
+
+
+def test_prepared_host_step_shared_prefix_argument_errors():
+    """set_shared_prefix refuses a bad group size, a missing prefix buffer, a staging buffer sized
+    for the plain decode (the plan stays a working plain step) and fp8 pools."""
+    import ctypes
+    import torch
+    import paged_kv_cache_349_b200 as pa
+    from paged_kv_cache_349_b200._lib import lib
+    case = W.make_case(3, batch=8, max_len=200, num_blocks=512)
+    k_last, v_last, other = W.split_last_tokens(case)
+    dc = DeviceCase(case)
+    B = case.batch
+    plain = pa.pa_decode_step_staging_size(B, case.max_blocks_per_seq, 1, case.num_q_heads, case.num_kv_heads,
+                                           case.head_dim, case.block_size, case.max_seq_len, case.partition_tokens)
+    staging = torch.empty(plain, dtype=torch.uint8, device="cuda")
+    out_h = torch.empty(case.q.shape, dtype=torch.float32).pin_memory()
+    prefix_h = _pinned(torch, case.shared_tokens[::4], torch.int32)
+    step = pa.DecodeStepHost(out_host=out_h, q_host=_pinned(torch, case.q.view(np.int16), torch.bfloat16),
+                             k_new_host=_pinned(torch, k_last.view(np.int16), torch.bfloat16),
+                             v_new_host=_pinned(torch, v_last.view(np.int16), torch.bfloat16),
+                             tables_host=_pinned(torch, case.block_tables, torch.int32),
+                             lens_host=_pinned(torch, case.seq_lens, torch.int32),
+                             pairs_host=_pinned(torch, np.zeros((1, 2), np.int32), torch.int32),
+                             k_cache=dc.k, v_cache=dc.v, scale=float(case.scale), max_seq_len_cap=case.max_seq_len,
+                             staging=staging, err_flag=dc.flag)
+    P = ctypes.c_void_p
+    setp = lib.pa_decode_step_plan_set_shared_prefix
+    assert setp(None, P(prefix_h.data_ptr()), 4) == pa.PA_ERR_INVALID_ARG
+    assert setp(step._plan, P(prefix_h.data_ptr()), 65) == pa.PA_ERR_INVALID_ARG
+    assert setp(step._plan, P(prefix_h.data_ptr()), -1) == pa.PA_ERR_INVALID_ARG
+    assert setp(step._plan, None, 4) == pa.PA_ERR_INVALID_ARG
+    assert setp(step._plan, P(prefix_h.data_ptr()), 4) == pa.PA_ERR_INVALID_ARG  # staging sized for the plain decode
+    assert setp(step._plan, None, 0) == pa.PA_OK  # back to (still) the plain decode
+    step(case.max_seq_len, 0)  # runs as the plain step
+    torch.cuda.synchronize()
+    assert int(dc.flag.item()) == 0
+    step.close()
+    # fp8 pools: no shared-prefix decode
+    k8 = torch.zeros(dc.k.shape, dtype=torch.uint8, device="cuda")
+    v8 = torch.zeros(dc.v.shape, dtype=torch.uint8, device="cuda")
+    big = torch.empty(plain * 2, dtype=torch.uint8, device="cuda")
+    step8 = pa.DecodeStepHost(out_host=out_h, q_host=_pinned(torch, case.q.view(np.int16), torch.bfloat16),
+                              k_new_host=_pinned(torch, k_last.view(np.int16), torch.bfloat16),
+                              v_new_host=_pinned(torch, v_last.view(np.int16), torch.bfloat16),
+                              tables_host=_pinned(torch, case.block_tables, torch.int32),
+                              lens_host=_pinned(torch, case.seq_lens, torch.int32),
+                              pairs_host=_pinned(torch, np.zeros((1, 2), np.int32), torch.int32),
+                              k_cache=k8, v_cache=v8, scale=float(case.scale), max_seq_len_cap=case.max_seq_len,
+                              staging=big, err_flag=dc.flag, k_scale=1.0, v_scale=1.0)
+    assert setp(step8._plan, P(prefix_h.data_ptr()), 4) == pa.PA_ERR_UNSUPPORTED
+    step8.close()
