@@ -297,7 +297,8 @@ def measure_workload(cfg, args, world, rank, pa, headline):
 
     base = 1000 + cfg if args.seed is None else args.seed
     seed = base + 7919 * rank  # weak scaling: every rank owns its own batch
-    case = W.make_case(cfg, seed=seed, fill=W.BF16_ZERO, num_blocks=args.num_blocks)
+    case = W.make_case(cfg, seed=seed, fill=W.BF16_ZERO, num_blocks=args.num_blocks,
+                       block_size=args.block_size if cfg == 2 else None)
     fp8 = args.kv_dtype == "fp8"
     elem = 1 if fp8 else 2
     # Shared-prefix groups (the n=4 chat mix): the step decodes with pa_decode_shared_prefix,
@@ -516,7 +517,7 @@ def measure_workload(cfg, args, world, rank, pa, headline):
         "unit": "GB/s",
         "ms_per_step": round(ms / args.steps, 4),
         "config": {
-            "workload": WORKLOAD_NAMES[cfg],
+            "workload": workload_name(cfg, case),
             "config_index": cfg,
             "seed": base,
             "batch_per_gpu": case.batch,
@@ -755,12 +756,20 @@ def step_description(case, fp8: bool, prefix: bool, fused: bool) -> str:
     return copies + "pa_reshape_and_cache, pa_decode"
 
 
+def workload_name(cfg: int, case) -> str:
+    """WORKLOAD_NAMES[cfg], with the block size and pool of a re-paged workload 2."""
+    name = WORKLOAD_NAMES[cfg]
+    if cfg == 2 and case.block_size != 16:
+        name = name.replace("bs=16", f"bs={case.block_size}").replace("16384-block", f"{case.num_blocks}-block")
+    return name
+
+
 def reference_config(case, cfg, base, world):
     """The reference arm's ``config``: the same keys and values as the native arm's headline."""
     prefix = case.groups is not None
     dec_b = decode_bytes(case, 2, unique=prefix)
     return {
-        "workload": WORKLOAD_NAMES[cfg],
+        "workload": workload_name(cfg, case),
         "config_index": cfg,
         "seed": base,
         "batch_per_gpu": case.batch,
@@ -779,7 +788,7 @@ def run_reference(args):
         return
     cfg = args.config
     base = 1000 + cfg if args.seed is None else args.seed
-    case = W.make_case(cfg, seed=base, fill=W.BF16_ZERO)
+    case = W.make_case(cfg, seed=base, fill=W.BF16_ZERO, block_size=args.block_size if cfg == 2 else None)
     per_step = max(1.0, args.cpu_budget / max(1, args.steps + args.warmup))
     for _ in range(args.warmup):
         cpu_baseline(case, budget_s=per_step / 4)
@@ -830,6 +839,8 @@ def main():
     ap.add_argument("--unfused", action="store_true",
                     help="time pa_reshape_and_cache + pa_decode instead of the fused pa_decode_append")
     ap.add_argument("--seed", type=int, default=None, help="input seed (default 1000 + config; + 7919 per rank)")
+    ap.add_argument("--block-size", type=int, default=None, choices=[8, 16, 32, 64],
+                    help="workload 2 only: re-page it with this block size (same lengths and pool bytes)")
     ap.add_argument("--num-blocks", type=int, default=None,
                     help="pool size override (same decode launch, smaller pool: for profiler captures)")
     args = ap.parse_args()
@@ -840,6 +851,8 @@ def main():
         args.per_config = [int(x) for x in args.per_config.split(",") if x.strip()]
     if args.warmup < 3:
         ap.error("--warmup must be at least 3")
+    if args.block_size is not None and (args.config != 2 or args.per_config):
+        ap.error("--block-size re-pages workload 2: use it with --config 2 alone")
     world = int(os.environ.get("WORLD_SIZE", "1"))
     if args.gpus != world:
         print(f"bench.py: --gpus {args.gpus} but WORLD_SIZE={world}; launch N > 1 under torchrun "

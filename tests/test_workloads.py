@@ -82,3 +82,23 @@ def test_algorithmic_bytes():
     c = W.make_case(1)
     kv = 97 * 2 * 64 * 2 * 2
     assert W.algorithmic_decode_bytes(c) == kv + 4 * 4 * 64 * 2 + 4 * 4 * 64 * 4 + 8 * 4 + 4 * 4
+
+
+@pytest.mark.parametrize("bs", [8, 32, 64])
+def test_workload_2_repaged_keeps_lengths_and_pool_bytes(bs):
+    """Re-paging the Llama-2-7B-shaped workload changes only the paging: the same lengths, the same
+    pool bytes, every sequence's blocks distinct and in range, padding never read."""
+    base = W.make_case(2, fill=W.BF16_ZERO, batch=16, max_len=600, num_blocks=2048)
+    case = W.make_case(2, fill=W.BF16_ZERO, batch=16, max_len=600, num_blocks=2048 * 16 // bs, block_size=bs)
+    assert case.block_size == bs
+    assert np.array_equal(case.seq_lens, base.seq_lens)
+    assert case.num_blocks * bs == base.num_blocks * 16
+    used = []
+    for b, L in enumerate(case.seq_lens):
+        n = -(-int(L) // bs)
+        row = case.block_tables[b, :n]
+        assert np.all((row >= 0) & (row < case.num_blocks))
+        used.extend(row.tolist())
+    assert len(used) == len(set(used))
+    with pytest.raises(ValueError):
+        W.make_case(3, block_size=8)

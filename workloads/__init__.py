@@ -215,12 +215,18 @@ def make_case(config: int, *, seed: Optional[int] = None, fill=BF16_QNAN,
               batch: Optional[int] = None, max_len: Optional[int] = None,
               num_blocks: Optional[int] = None, poison_padding: bool = True,
               num_copy_pairs: Optional[int] = None,
-              partition_tokens: Optional[int] = None) -> DecodeCase:
+              partition_tokens: Optional[int] = None,
+              block_size: Optional[int] = None) -> DecodeCase:
     """Build decode workload ``config`` (1..5).
 
     ``batch``/``max_len``/``num_blocks``/``num_copy_pairs`` shrink a workload
     (same recipe, smaller numbers) so the oracle can check every output.
+    ``block_size`` (workload 2 only) re-pages the Llama-2-7B-shaped workload
+    with another block size: the same lengths and pool bytes (the block count
+    scales inversely), the blocks dealt from a fresh permutation.
     """
+    if block_size is not None and config != 2:
+        raise ValueError("block_size applies to workload 2 only")
     if seed is None:
         seed = 1000 + config
     rng = np.random.default_rng(seed)
@@ -244,8 +250,9 @@ def make_case(config: int, *, seed: Optional[int] = None, fill=BF16_QNAN,
 
     if config == 2:
         Hq = Hkv = 32
-        d, bs = 128, 16
-        NB = 16384 if num_blocks is None else num_blocks
+        d = 128
+        bs = 16 if block_size is None else block_size
+        NB = 16384 * 16 // bs if num_blocks is None else num_blocks
         B = 64 if batch is None else batch
         hi = 2048 if max_len is None else max_len
         lo = min(128, hi)
