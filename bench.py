@@ -216,7 +216,19 @@ def _barrier(world: int):
 # CPU oracle baseline (the only place the bench runs the oracle)
 # ---------------------------------------------------------------------------
 
-def cpu_baseline(case, budget_s: float = 12.0):
+def cpu_model() -> str:
+    """The host CPU's model name (/proc/cpuinfo), or 'unknown'."""
+    try:
+        with open("/proc/cpuinfo") as f:
+            for line in f:
+                if line.startswith("model name"):
+                    return line.split(":", 1)[1].strip()
+    except OSError:
+        pass
+    return "unknown"
+
+
+def cpu_baseline(case, budget_s: float = 12.0, threads=None):
     """Time the fp64 oracle on a bounded sample of (sequence, kv head) units of ``case``.
 
     Units are taken in a seeded order, in chunks, cycling over the whole
@@ -228,7 +240,7 @@ def cpu_baseline(case, budget_s: float = 12.0):
     workload's ratio of unique to logical decode bytes.
     """
     import oracle
-    threads = len(os.sched_getaffinity(0))
+    threads = len(os.sched_getaffinity(0)) if threads is None else threads
     oracle.set_num_threads(threads)
     G = case.group_size
     rng = np.random.default_rng(7)
@@ -544,7 +556,11 @@ def measure_workload(cfg, args, world, rank, pa, headline):
     cpu = None
     if headline and rank == 0 and world == 1 and not args.no_cpu_baseline and not fp8:
         gbs, cores, sample, _, _ = cpu_baseline(case, budget_s=args.cpu_budget)
-        cpu = {"value": round(gbs, 4), "unit": "GB/s", "cores": cores, "kind": "oracle", "sample": sample}
+        cpu = {"value": round(gbs, 4), "unit": "GB/s", "cores": cores, "kind": "oracle", "sample": sample,
+               "cpu_model": cpu_model()}
+        if cores > 1:  # the same oracle on one thread, over a shorter sample
+            gbs1, _, sample1, _, _ = cpu_baseline(case, budget_s=max(1.0, args.cpu_budget / 6), threads=1)
+            cpu["single_thread"] = {"value": round(gbs1, 4), "unit": "GB/s", "sample": sample1}
     del k, v, q, ws
     torch.cuda.synchronize()
     torch.cuda.empty_cache()
