@@ -279,3 +279,45 @@ def test_prepared_host_step_shared_prefix_argument_errors():
                               staging=big, err_flag=dc.flag, k_scale=1.0, v_scale=1.0)
     assert setp(step8._plan, P(prefix_h.data_ptr()), 4) == pa.PA_ERR_UNSUPPORTED
     step8.close()
+
+
+def test_prepared_host_step_full_size_chat_sampled_rows():
+    """The chat workload at full size through a prepared host step in shared-prefix mode, in the launch
+    configuration the benchmark's end-to-end leg uses (automatic chunking: 8 chunks of whole groups,
+    first and last half-size), against the oracle on sampled rows; pools bit-exact."""
+    import torch
+    import paged_kv_cache_349_b200 as pa
+    case = W.make_case(3)
+    n, prefix = 4, case.shared_tokens[::4]
+    dc = DeviceCase(case)
+    k_last, v_last, other = W.split_last_tokens(case)
+    pa.pa_copy_blocks(dc.k, dc.v, dc.pairs, err_flag=dc.flag)
+    if other.size:
+        pa.pa_reshape_and_cache(bf16_dev(case.k_new[other]), bf16_dev(case.v_new[other]), dc.k, dc.v,
+                                i32_dev(case.slot_mapping[other]), err_flag=dc.flag)
+    B = case.batch
+    size = pa.pa_decode_step_staging_size_shared_prefix(B, n, case.max_blocks_per_seq, 1, case.num_q_heads,
+                                                        case.num_kv_heads, case.head_dim, case.block_size,
+                                                        case.max_seq_len, case.partition_tokens)
+    staging = torch.empty(size, dtype=torch.uint8, device="cuda")
+    out_h = torch.full(case.q.shape, float("nan"), dtype=torch.float32).pin_memory()
+    step = pa.DecodeStepHost(out_host=out_h, q_host=_pinned(torch, case.q.view(np.int16), torch.bfloat16),
+                             k_new_host=_pinned(torch, k_last.view(np.int16), torch.bfloat16),
+                             v_new_host=_pinned(torch, v_last.view(np.int16), torch.bfloat16),
+                             tables_host=_pinned(torch, case.block_tables, torch.int32),
+                             lens_host=_pinned(torch, case.seq_lens, torch.int32),
+                             pairs_host=_pinned(torch, np.zeros((1, 2), np.int32), torch.int32),
+                             k_cache=dc.k, v_cache=dc.v, scale=float(case.scale), max_seq_len_cap=case.max_seq_len,
+                             partition_tokens=case.partition_tokens, num_chunks=0, staging=staging,
+                             err_flag=dc.flag, prefix_lens_host=_pinned(torch, np.asarray(prefix), torch.int32),
+                             group_size=n)
+    step(case.max_seq_len, 0)
+    torch.cuda.synchronize()
+    step.close()
+    assert int(dc.flag.item()) == 0
+    rows = sample_rows(case, 96, seed=34)
+    want, k_ref, v_ref = oracle.decode_step(case, rows=rows)
+    assert np.array_equal(bits_host(dc.k), k_ref) and np.array_equal(bits_host(dc.v), v_ref)
+    got = out_h.numpy().astype(np.float64)
+    assert not np.isnan(got).any()
+    assert_close(got[rows[:, 0], rows[:, 1]], want, "chat full, prepared host step")
