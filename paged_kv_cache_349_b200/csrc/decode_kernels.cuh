@@ -90,7 +90,8 @@ constexpr float kLog2e = 1.4426950408889634f;
 template <int HEAD_DIM, bool FP8>
 struct Cfg {
     // What TMA lands in the ring: bf16 tiles in 64-column swizzled boxes, or
-    // fp8 tiles as one unswizzled box of 16 rows x HEAD_DIM bytes.
+    // fp8 tiles as one box of 16 rows x HEAD_DIM bytes (128-byte swizzle at
+    // head_dim 128, none at 64).
     static constexpr int kBoxes = FP8 ? 1 : HEAD_DIM / 64;
     static constexpr int kBoxCols = FP8 ? HEAD_DIM : 64;
     static constexpr int kBoxRowBytes = FP8 ? HEAD_DIM : 128;
